@@ -1,0 +1,322 @@
+"""Pins for the fp64 oracle, each against something other than the oracle itself.
+
+Sources: "On the Design of Qwen3.8 Next Architecture" (reading notes), section 6:
+the pooled-key equation (k̄_b), the indexer equation (I_ib), the budget sentence
+(own causal block always kept, k-1 best complete blocks), and the expansion of
+selected blocks to token indices for softmax attention.
+
+The pins: hand-worked fixtures (tests/golden), a library routine (torch SDPA in
+fp64) for the dense case, brute-force subset enumeration on tiny inputs, closed
+forms (w = 0, v = const, q = 0, r = 1, identical rows) and an independently
+ordered score computation.  Each is chosen so that a plausible slip in the oracle
+(a dropped head, a wrong sign, a missing mask, an off-by-one block) fails.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_long_09_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf16(a) -> torch.Tensor:
+    return torch.as_tensor(np.asarray(a, dtype=np.float32)).to(torch.bfloat16)
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.double().numpy()
+
+
+# --------------------------------------------------------------------------
+# Compressor
+# --------------------------------------------------------------------------
+
+def test_compress_hand_fixture():
+    rows, outs = [], []
+    with open(os.path.join(GOLDEN, "compress_hand.txt")) as f:
+        for line in f:
+            if line.startswith("in "):
+                rows.append([float(x) for x in line.split()[1:]])
+            elif line.startswith("out "):
+                outs.append([float(x) for x in line.split()[1:]])
+    kc = oracle.compress(bf16(rows), r=4, normalise=True, eps=1e-6)
+    assert kc.shape == (2, 4)
+    np.testing.assert_allclose(kc, np.array(outs), rtol=0, atol=1e-15)
+
+
+def test_compress_identical_rows_is_rmsnorm_of_row():
+    g = torch.Generator().manual_seed(3)
+    row = torch.randn(128, generator=g).to(torch.bfloat16)
+    k_idx = row[None, :].repeat(4 * 5 + 3, 1)
+    kc = oracle.compress(k_idx, r=4)
+    x = f64(row)
+    expect = x / math.sqrt(np.mean(x * x) + 1e-6)
+    assert kc.shape == (5, 128)
+    np.testing.assert_allclose(kc, np.tile(expect, (5, 1)), rtol=1e-14, atol=1e-14)
+
+
+def test_compress_without_norm_is_block_mean():
+    g = torch.Generator().manual_seed(4)
+    k_idx = torch.randn(4 * 7 + 1, 128, generator=g).to(torch.bfloat16)
+    kc = oracle.compress(k_idx, r=4, normalise=False)
+    x = f64(k_idx)[: 4 * 7].reshape(7, 4, 128)
+    np.testing.assert_allclose(kc, x.mean(axis=1), rtol=1e-15, atol=1e-15)
+
+
+def test_compress_r1_norm_of_each_row():
+    g = torch.Generator().manual_seed(5)
+    k_idx = torch.randn(9, 128, generator=g).to(torch.bfloat16)
+    kc = oracle.compress(k_idx, r=1)
+    x = f64(k_idx)
+    expect = x / np.sqrt((x * x).mean(axis=1, keepdims=True) + 1e-6)
+    np.testing.assert_allclose(kc, expect, rtol=1e-14, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# Indexer scores
+# --------------------------------------------------------------------------
+
+def _scores_by_einsum(q_idx, w, kc, Lq, Lk, r):
+    """Independent loop order: all heads' dot products as one einsum, ReLU,
+    weight, sum over heads, then the causal cut b < floor(t / r)."""
+    q = f64(q_idx)                         # [Lq, H, d]
+    dots = np.einsum("bd,ihd->ihb", kc, q)  # [Lq, H, nb]
+    s = np.einsum("ih,ihb->ib", w.double().numpy(), np.maximum(dots, 0.0))
+    t = (Lk - Lq) + np.arange(Lq)
+    bt = t // r
+    mask = np.arange(kc.shape[0])[None, :] >= bt[:, None]
+    s[mask] = -np.inf
+    return s
+
+
+@pytest.mark.parametrize("n", [37, 64, 203])
+def test_scores_match_independent_einsum(n):
+    x = inputs.make_prefill([n], seed=1)
+    kc = oracle.compress(x.k_idx, 4)
+    ld = kc.shape[0]
+    s = oracle.index_scores(x.q_idx, x.w, kc, n, n, 4, ld=ld)
+    ref = _scores_by_einsum(x.q_idx, x.w, kc, n, n, 4)
+    fin = np.isfinite(ref)
+    assert np.array_equal(fin, np.isfinite(s))
+    np.testing.assert_allclose(s[fin], ref[fin], rtol=1e-12, atol=1e-12)
+
+
+def test_scores_w_one_is_unweighted_relu_sum():
+    n = 48
+    x = inputs.make_prefill([n], seed=2)
+    w1 = torch.ones_like(x.w)
+    kc = oracle.compress(x.k_idx, 4)
+    s = oracle.index_scores(x.q_idx, w1, kc, n, n, 4, ld=kc.shape[0])
+    q = f64(x.q_idx)
+    for i in (5, 17, 47):
+        bt = i // 4
+        for b in range(bt):
+            want = sum(max(0.0, float(np.dot(q[i, h], kc[b]))) for h in range(4))
+            assert abs(s[i, b] - want) <= 1e-12 * max(1.0, abs(want))
+        assert np.all(np.isneginf(s[i, bt:]))
+
+
+def test_scores_decode_position():
+    """Lq < Lk: query row i sits at t = Lk - Lq + i."""
+    Lk, Lq = 41, 3
+    x = inputs.make_prefill([Lk], seed=6)
+    kc = oracle.compress(x.k_idx, 4)
+    s_full = oracle.index_scores(x.q_idx, x.w, kc, Lk, Lk, 4, ld=kc.shape[0])
+    s_tail = oracle.index_scores(x.q_idx[Lk - Lq:], x.w[Lk - Lq:], kc, Lq, Lk, 4, ld=kc.shape[0])
+    np.testing.assert_array_equal(s_tail, s_full[Lk - Lq:])
+
+
+# --------------------------------------------------------------------------
+# Selection
+# --------------------------------------------------------------------------
+
+def test_select_hand_fixture():
+    with open(os.path.join(GOLDEN, "select_hand.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            head, sc, want = line.split("|")
+            k, bt = (int(x) for x in head.split())
+            scores = [float(x) for x in sc.split()]
+            want = [int(x) for x in want.split()]
+            row = np.full((1, max(1, bt + 1)), -np.inf)
+            row[0, :bt] = scores
+            got = oracle.select(row, [bt], k)
+            assert got[0].tolist() == want, line
+
+
+def _brute_select(scores, bt, k):
+    """Enumerate every subset of the candidates of size min(k-1, bt); keep the
+    largest score sum, and among equal sums the lexicographically smallest
+    ascending index list; then add the own block."""
+    m = min(k - 1, bt)
+    best_sum, best = None, None
+    for comb in itertools.combinations(range(bt), m):
+        s = sum(scores[b] for b in comb)
+        if best_sum is None or s > best_sum or (s == best_sum and list(comb) < best):
+            best_sum, best = s, list(comb)
+    out = sorted(best + [bt])
+    return out + [-1] * (k - len(out))
+
+
+@pytest.mark.parametrize("k", [2, 3, 4])
+def test_select_matches_brute_force(k):
+    rng = np.random.default_rng(10 + k)
+    for bt in range(0, 9):
+        for _ in range(6):
+            # small integers make exact ties common
+            scores = rng.integers(0, 4, size=bt).astype(np.float64)
+            row = np.full((1, 9), -np.inf)
+            row[0, :bt] = scores
+            got = oracle.select(row, [bt], k)[0].tolist()
+            assert got == _brute_select(scores, bt, k), (bt, scores, got)
+
+
+def test_select_w_zero_closed_form():
+    n, k = 160, 8
+    x = inputs.make_prefill([n], seed=7)
+    kc = oracle.compress(x.k_idx, 4)
+    s = oracle.index_scores(x.q_idx, torch.zeros_like(x.w), kc, n, n, 4, ld=kc.shape[0])
+    bt = oracle.own_blocks(n, n, 4, None)
+    sel = oracle.select(s, bt, k)
+    for i in range(n):
+        b = bt[i]
+        want = sorted(set(range(min(k - 1, b))) | {b})
+        assert sel[i].tolist() == want + [-1] * (k - len(want))
+
+
+def test_select_invariants_tiny_config():
+    n, k = 512, 16
+    x = inputs.make_prefill([n], seed=0)
+    res = oracle.qsa_layer(x.q, x.k, x.v, x.q_idx, x.k_idx, x.w, n, n, 4, k,
+                           rows=np.arange(0, n, 7))
+    rows = np.arange(0, n, 7)
+    for j, i in enumerate(rows):
+        bt = i // 4
+        s = res["sel"][j]
+        valid = s[s >= 0]
+        assert np.all(s[len(valid):] == -1)
+        assert len(valid) == min(k, bt + 1)
+        assert np.all(np.diff(valid) > 0)
+        assert valid[-1] == bt and valid.max() <= bt
+        # the chosen candidates beat every unchosen one (or tie with a higher index)
+        chosen = set(valid[:-1].tolist())
+        sc = res["scores"][j]
+        worst = min(((sc[b], -b) for b in chosen), default=None)
+        for b in range(bt):
+            if b not in chosen and worst is not None:
+                assert (sc[b], -b) < worst
+
+
+# --------------------------------------------------------------------------
+# Attention
+# --------------------------------------------------------------------------
+
+def _masked_dense_numpy(q, k, v, t, tokens, scale):
+    """Separately written: full logits over keys 0..t, -inf where a key is not
+    in ``tokens``, softmax, weighted sum of v.  One query row, all heads."""
+    qn, kn, vn = f64(q), f64(k), f64(v)
+    Hq, Hkv = qn.shape[0], kn.shape[1]
+    grp = Hq // Hkv
+    mask = np.full(t + 1, -np.inf)
+    mask[sorted(tokens)] = 0.0
+    o = np.zeros((Hq, qn.shape[1]))
+    lse = np.zeros(Hq)
+    for h in range(Hq):
+        g = h // grp
+        lg = kn[: t + 1, g, :] @ qn[h] * scale + mask
+        m = lg.max()
+        p = np.exp(lg - m)
+        o[h] = p @ vn[: t + 1, g, :] / p.sum()
+        lse[h] = m + math.log(p.sum())
+    return o, lse
+
+
+def test_attend_matches_masked_dense_on_brute_force_selection():
+    n, r, k = 32, 4, 3
+    x = inputs.make_prefill([n], seed=11)
+    kc = oracle.compress(x.k_idx, r)
+    s = oracle.index_scores(x.q_idx, x.w, kc, n, n, r, ld=kc.shape[0])
+    bt = oracle.own_blocks(n, n, r, None)
+    sel = np.array([_brute_select(s[i, : bt[i]], int(bt[i]), k) for i in range(n)], dtype=np.int32)
+    np.testing.assert_array_equal(sel, oracle.select(s, bt, k))
+    rows = np.array([0, 3, 4, 9, 15, 22, 31])
+    o, lse = oracle.attend(x.q, x.k, x.v, sel[rows], n, n, r, 1 / 16, rows)
+    for j, i in enumerate(rows):
+        toks = [b * r + u for b in sel[i] if b >= 0 for u in range(r) if b * r + u <= i]
+        oref, lref = _masked_dense_numpy(x.q[i], x.k, x.v, int(i), toks, 1 / 16)
+        np.testing.assert_allclose(o[j], oref, rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(lse[j], lref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("n", [64, 101])
+def test_sparse_equals_dense_when_budget_covers_all(n):
+    x = inputs.make_prefill([n], seed=12)
+    res = oracle.qsa_layer(x.q, x.k, x.v, x.q_idx, x.k_idx, x.w, n, n, 4, budget=n // 4 + 2)
+    od, ld = oracle.dense(x.q, x.k, x.v, n, n, 1 / 16)
+    np.testing.assert_allclose(res["o"], od, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(res["lse"], ld, rtol=1e-12, atol=1e-13)
+
+
+def test_dense_matches_torch_sdpa_fp64():
+    n = 96
+    x = inputs.make_prefill([n], seed=13)
+    od, lse = oracle.dense(x.q, x.k, x.v, n, n, 1 / 16)
+    q = x.q.double().permute(1, 0, 2)[None]                     # [1, 24, n, 256]
+    k = x.k.double().repeat_interleave(12, dim=1).permute(1, 0, 2)[None]
+    v = x.v.double().repeat_interleave(12, dim=1).permute(1, 0, 2)[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True, scale=1 / 16)
+    np.testing.assert_allclose(od, ref[0].permute(1, 0, 2).numpy(), rtol=1e-11, atol=1e-12)
+    lg = torch.einsum("hid,hjd->hij", q[0], k[0]) / 16
+    lg = lg.masked_fill(torch.ones(n, n, dtype=torch.bool).triu(1), float("-inf"))
+    np.testing.assert_allclose(lse, torch.logsumexp(lg, -1).T.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_r1_full_budget_is_dense():
+    n = 40
+    x = inputs.make_prefill([n], seed=14)
+    res = oracle.qsa_layer(x.q, x.k, x.v, x.q_idx, x.k_idx, x.w, n, n, r=1, budget=n)
+    od, _ = oracle.dense(x.q, x.k, x.v, n, n, 1 / 16)
+    np.testing.assert_allclose(res["o"], od, rtol=1e-12, atol=1e-13)
+
+
+def test_constant_v_gives_constant_output():
+    n, k = 80, 4
+    x = inputs.make_prefill([n], seed=15)
+    c = torch.randn(2, 256, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16)
+    v = c[None].repeat(n, 1, 1)
+    res = oracle.qsa_layer(x.q, x.k, v, x.q_idx, x.k_idx, x.w, n, n, 4, k)
+    want = np.repeat(f64(c), 12, axis=0)  # head h uses group h // 12
+    for j in range(n):
+        np.testing.assert_allclose(res["o"][j], want, rtol=1e-13, atol=1e-13)
+
+
+def test_zero_q_gives_mean_of_selected_values():
+    n, k = 72, 3
+    x = inputs.make_prefill([n], seed=16)
+    q0 = torch.zeros_like(x.q)
+    res = oracle.qsa_layer(q0, x.k, x.v, x.q_idx, x.k_idx, x.w, n, n, 4, k)
+    vn = f64(x.v)
+    for i in range(n):
+        toks = [b * 4 + u for b in res["sel"][i] if b >= 0 for u in range(4) if b * 4 + u <= i]
+        mean = vn[toks].mean(axis=0)                   # [2, 256]
+        np.testing.assert_allclose(res["o"][i], np.repeat(mean, 12, axis=0), rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(res["lse"][i], math.log(len(toks)), rtol=1e-13, atol=1e-13)
+
+
+def test_duplicate_and_padding_entries_are_ignored():
+    n = 40
+    x = inputs.make_prefill([n], seed=17)
+    rows = np.array([39])
+    a = np.array([[1, 3, 9, -1, -1]], dtype=np.int32)
+    b = np.array([[9, 1, 1, 3, -1]], dtype=np.int32)
+    oa, la = oracle.attend(x.q, x.k, x.v, a, n, n, 4, 1 / 16, rows)
+    ob, lb = oracle.attend(x.q, x.k, x.v, b, n, n, 4, 1 / 16, rows)
+    np.testing.assert_array_equal(oa, ob)
+    np.testing.assert_array_equal(la, lb)
