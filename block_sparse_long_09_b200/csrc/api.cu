@@ -1,0 +1,282 @@
+// api.cu -- the extern "C" entry points of libqsa.so (declared in include/qsa.h):
+// host-side argument validation, tensor-map creation and kernel dispatch.
+// Nothing here allocates device memory; every buffer is the caller's.
+#include <mutex>
+
+#include "kernels.cuh"
+
+namespace qsa {
+
+__device__ int g_device_status = 0;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+bool make_tmap_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                  uint32_t box_inner, uint32_t box_outer)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr || !aligned16(base) || (row_bytes & 15u) != 0 || outer == 0) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                  uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr || !aligned16(base) || (stride1_bytes & 15u) != 0 || (stride2_bytes & 15u) != 0 || d2 == 0)
+        return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+    cuuint32_t box[3] = {b0, b1, b2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+}  // namespace qsa
+
+using namespace qsa;
+
+namespace {
+
+qsa_status check_config(const qsa_config *c)
+{
+    if (c == nullptr) return QSA_ERR_INVALID_ARG;
+    if (c->r <= 0 || c->budget_blocks <= 0 || c->n_heads_q <= 0 || c->n_heads_kv <= 0 || c->head_dim <= 0 ||
+        c->n_heads_idx <= 0 || c->idx_dim <= 0 || !(c->softmax_scale > 0.f) || !(c->rms_eps >= 0.f))
+        return QSA_ERR_INVALID_ARG;
+    if (c->r != 4 || c->budget_blocks > 2048 || c->n_heads_q != 24 || c->n_heads_kv != 2 || c->head_dim != 256 ||
+        c->n_heads_idx != 4 || c->idx_dim != 128 || (c->flags & ~QSA_COMPRESS_NO_NORM) != 0)
+        return QSA_ERR_UNSUPPORTED;
+    return QSA_OK;
+}
+
+qsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA; }
+
+const __nv_bfloat16 *bf(const qsa_bf16 *p) { return reinterpret_cast<const __nv_bfloat16 *>(p); }
+__nv_bfloat16 *bf(qsa_bf16 *p) { return reinterpret_cast<__nv_bfloat16 *>(p); }
+bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+void qsa_config_init(qsa_config *cfg)
+{
+    if (cfg == nullptr) return;
+    cfg->r = 4;
+    cfg->budget_blocks = 512;
+    cfg->n_heads_q = 24;
+    cfg->n_heads_kv = 2;
+    cfg->head_dim = 256;
+    cfg->n_heads_idx = 4;
+    cfg->idx_dim = 128;
+    cfg->softmax_scale = 0.0625f;
+    cfg->rms_eps = 1e-6f;
+    cfg->flags = 0u;
+}
+
+int32_t qsa_version(void) { return 100; }
+
+const char *qsa_status_string(qsa_status s)
+{
+    switch (s) {
+    case QSA_OK: return "QSA_OK";
+    case QSA_ERR_INVALID_ARG: return "QSA_ERR_INVALID_ARG: a pointer, size or range argument is invalid";
+    case QSA_ERR_UNSUPPORTED: return "QSA_ERR_UNSUPPORTED: configuration outside the supported model shape";
+    case QSA_ERR_WORKSPACE_TOO_SMALL: return "QSA_ERR_WORKSPACE_TOO_SMALL: workspace smaller than qsa_workspace_size()";
+    case QSA_ERR_CUDA: return "QSA_ERR_CUDA: a CUDA launch or runtime call failed";
+    case QSA_ERR_TIMEOUT: return "QSA_ERR_TIMEOUT: a bounded device-side wait gave up";
+    case QSA_ERR_DEVICE_CHECK: return "QSA_ERR_DEVICE_CHECK: a kernel found an out-of-range index and skipped it";
+    default: return "QSA: unknown status";
+    }
+}
+
+size_t qsa_workspace_size(const qsa_config *cfg, int32_t op, int32_t batch, int64_t rows, int64_t max_len_k)
+{
+    (void)max_len_k;
+    if (check_config(cfg) != QSA_OK || batch <= 0 || rows < 0) return 0;
+    if (op == QSA_OP_DECODE) {
+        // upper bound over devices: at most one split per 128-token tile
+        const int max_tiles = (cfg->budget_blocks + 31) / 32;
+        return split_workspace_bytes(batch, max_tiles > 1 ? max_tiles : 2);
+    }
+    if (op == QSA_OP_PREFILL) return split_workspace_bytes(rows, min_nsplit(cfg->budget_blocks));
+    return 0;
+}
+
+qsa_status qsa_get_device_status(void *stream, int32_t *status, int32_t clear)
+{
+    if (status == nullptr) return QSA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return QSA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return QSA_ERR_CUDA;
+    *status = v;
+    if (clear) {
+        int z = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &z, sizeof(int)) != cudaSuccess) return QSA_ERR_CUDA;
+    }
+    return QSA_OK;
+}
+
+qsa_status qsa_compress_keys(const qsa_config *cfg, const qsa_bf16 *k_idx, const int32_t *cu_seqlens_k,
+                             const int32_t *cu_blocks, int32_t batch, int64_t total_k, const int32_t *blk_begin,
+                             int32_t max_new_blocks, qsa_bf16 *kc, void *stream)
+{
+    qsa_status st = check_config(cfg);
+    if (st != QSA_OK) return st;
+    if (batch <= 0 || total_k < 0 || cu_seqlens_k == nullptr || cu_blocks == nullptr) return QSA_ERR_INVALID_ARG;
+    if (total_k == 0) return QSA_OK;
+    if (k_idx == nullptr || kc == nullptr || !al16(k_idx) || !al16(kc)) return QSA_ERR_INVALID_ARG;
+    if (blk_begin != nullptr && max_new_blocks <= 0) return QSA_ERR_INVALID_ARG;
+    return cuda_status(launch_compress(bf(k_idx), cu_seqlens_k, cu_blocks, batch, total_k, blk_begin,
+                                       max_new_blocks, cfg->r, (cfg->flags & QSA_COMPRESS_NO_NORM) == 0,
+                                       cfg->rms_eps, bf(kc), static_cast<cudaStream_t>(stream)));
+}
+
+qsa_status qsa_index_scores(const qsa_config *cfg, const qsa_bf16 *q_idx, const float *w, const qsa_bf16 *kc,
+                            int64_t kc_rows, const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                            const int32_t *cu_blocks, int32_t batch, int64_t total_q, int32_t max_len_q,
+                            int64_t row_begin, int64_t row_end, float *scores, int64_t ld, void *ws,
+                            size_t ws_bytes, void *stream)
+{
+    (void)ws;
+    (void)ws_bytes;
+    qsa_status st = check_config(cfg);
+    if (st != QSA_OK) return st;
+    if (batch <= 0 || total_q < 0 || kc_rows < 0 || ld <= 0 || max_len_q < 0) return QSA_ERR_INVALID_ARG;
+    if (row_begin < 0 || row_end < row_begin || row_end > total_q) return QSA_ERR_INVALID_ARG;
+    if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr || cu_blocks == nullptr) return QSA_ERR_INVALID_ARG;
+    if (row_end == row_begin || kc_rows == 0) return QSA_OK;
+    if (q_idx == nullptr || w == nullptr || kc == nullptr || scores == nullptr || !al16(q_idx) || !al16(kc))
+        return QSA_ERR_INVALID_ARG;
+    IndexArgs a{bf(q_idx), w, bf(kc), kc_rows, cu_seqlens_q, cu_seqlens_k, cu_blocks, batch, total_q,
+                row_begin, row_end, scores, ld, cfg->r};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (max_len_q == 1) return cuda_status(launch_index_rowwise(a, s));
+    return cuda_status(launch_index_tc(a, s));
+}
+
+qsa_status qsa_select_blocks(const qsa_config *cfg, const float *scores, int64_t ld, const int32_t *cu_seqlens_q,
+                             const int32_t *cu_seqlens_k, int32_t batch, int64_t row_begin, int64_t row_end,
+                             int32_t *sel, void *ws, size_t ws_bytes, void *stream)
+{
+    (void)ws;
+    (void)ws_bytes;
+    qsa_status st = check_config(cfg);
+    if (st != QSA_OK) return st;
+    if (batch <= 0 || ld <= 0 || row_begin < 0 || row_end < row_begin) return QSA_ERR_INVALID_ARG;
+    if (cu_seqlens_k == nullptr || cu_seqlens_q == nullptr) return QSA_ERR_INVALID_ARG;
+    if (row_end == row_begin) return QSA_OK;
+    if (scores == nullptr || sel == nullptr) return QSA_ERR_INVALID_ARG;
+    SelectArgs a{scores, ld, cu_seqlens_q, cu_seqlens_k, batch, row_begin, row_end, sel, cfg->budget_blocks, cfg->r};
+    return cuda_status(launch_select(a, static_cast<cudaStream_t>(stream)));
+}
+
+qsa_status qsa_sparse_attn_prefill(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k, const qsa_bf16 *v,
+                                   const int32_t *sel, const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                                   int32_t batch, int64_t total_q, int64_t total_k, int64_t row_begin,
+                                   int64_t row_end, qsa_bf16 *o, float *lse, void *ws, size_t ws_bytes,
+                                   void *stream)
+{
+    qsa_status st = check_config(cfg);
+    if (st != QSA_OK) return st;
+    if (batch <= 0 || total_q < 0 || total_k < 0 || row_begin < 0 || row_end < row_begin || row_end > total_q)
+        return QSA_ERR_INVALID_ARG;
+    if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr) return QSA_ERR_INVALID_ARG;
+    if (row_end == row_begin) return QSA_OK;
+    if (total_k == 0 || q == nullptr || k == nullptr || v == nullptr || sel == nullptr || o == nullptr ||
+        !al16(q) || !al16(k) || !al16(v))
+        return QSA_ERR_INVALID_ARG;
+    const int nsplit = min_nsplit(cfg->budget_blocks);
+    if (nsplit > 1) {
+        if (ws == nullptr || ws_bytes < split_workspace_bytes(row_end - row_begin, nsplit))
+            return QSA_ERR_WORKSPACE_TOO_SMALL;
+        if (!al16(ws)) return QSA_ERR_INVALID_ARG;
+    }
+    AttnArgs a{bf(q), bf(k), bf(v), sel, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, row_begin, row_end,
+               bf(o), lse, static_cast<float *>(ws), nsplit, cfg->budget_blocks, cfg->r, cfg->softmax_scale};
+    return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
+}
+
+qsa_status qsa_sparse_attn_decode(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k_cache,
+                                  const qsa_bf16 *v_cache, const int32_t *cu_seqlens_k, int32_t batch,
+                                  int64_t total_k, const int32_t *sel, qsa_bf16 *o, float *lse, void *ws,
+                                  size_t ws_bytes, void *stream)
+{
+    qsa_status st = check_config(cfg);
+    if (st != QSA_OK) return st;
+    if (batch <= 0 || total_k <= 0 || cu_seqlens_k == nullptr) return QSA_ERR_INVALID_ARG;
+    if (q == nullptr || k_cache == nullptr || v_cache == nullptr || sel == nullptr || o == nullptr ||
+        !al16(q) || !al16(k_cache) || !al16(v_cache))
+        return QSA_ERR_INVALID_ARG;
+    const int nsplit = decode_nsplit(batch, cfg->budget_blocks);
+    if (nsplit > 1) {
+        if (ws == nullptr) return QSA_ERR_WORKSPACE_TOO_SMALL;
+        if (ws_bytes < split_workspace_bytes(batch, nsplit)) return QSA_ERR_WORKSPACE_TOO_SMALL;
+        if (!al16(ws)) return QSA_ERR_INVALID_ARG;
+    }
+    AttnArgs a{bf(q), bf(k_cache), bf(v_cache), sel, nullptr, cu_seqlens_k, batch, batch, total_k, 0, batch,
+               bf(o), lse, static_cast<float *>(ws), nsplit, cfg->budget_blocks, cfg->r, cfg->softmax_scale};
+    return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
+}
+
+qsa_status qsa_dense_attn_prefill(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k, const qsa_bf16 *v,
+                                  const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int32_t batch,
+                                  int64_t total_q, int64_t total_k, int32_t max_len_q, qsa_bf16 *o, float *lse,
+                                  void *stream)
+{
+    qsa_status st = check_config(cfg);
+    if (st != QSA_OK) return st;
+    if (batch <= 0 || total_q < 0 || total_k < 0 || max_len_q < 0 || cu_seqlens_q == nullptr ||
+        cu_seqlens_k == nullptr)
+        return QSA_ERR_INVALID_ARG;
+    if (total_q == 0) return QSA_OK;
+    if (total_k == 0 || q == nullptr || k == nullptr || v == nullptr || o == nullptr || !al16(q) || !al16(k) ||
+        !al16(v))
+        return QSA_ERR_INVALID_ARG;
+    DenseArgs a{bf(q), bf(k), bf(v), cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_len_q, bf(o), lse,
+                cfg->softmax_scale};
+    return cuda_status(launch_dense_attn(a, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,267 @@
+"""Python binding of libqsa.so (the C ABI declared in include/qsa.h).
+
+Argument marshalling only: every step of the QSA path runs in the library's
+CUDA kernels.  torch supplies device memory and the current stream.  If the
+shared library is missing this module raises at import time -- there is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqsa.so")
+
+QSA_OK = 0
+QSA_ERR_INVALID_ARG = 1
+QSA_ERR_UNSUPPORTED = 2
+QSA_ERR_WORKSPACE_TOO_SMALL = 3
+QSA_ERR_CUDA = 4
+QSA_ERR_TIMEOUT = 5
+QSA_ERR_DEVICE_CHECK = 6
+QSA_COMPRESS_NO_NORM = 0x1
+OP_COMPRESS, OP_INDEX, OP_SELECT, OP_PREFILL, OP_DECODE, OP_DENSE = range(6)
+
+EXPORTED = (
+    "qsa_config_init", "qsa_compress_keys", "qsa_index_scores", "qsa_select_blocks",
+    "qsa_sparse_attn_prefill", "qsa_sparse_attn_decode", "qsa_dense_attn_prefill",
+    "qsa_workspace_size", "qsa_status_string", "qsa_get_device_status", "qsa_version",
+)
+
+
+class Config(ctypes.Structure):
+    _fields_ = [
+        ("r", ctypes.c_int32),
+        ("budget_blocks", ctypes.c_int32),
+        ("n_heads_q", ctypes.c_int32),
+        ("n_heads_kv", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("n_heads_idx", ctypes.c_int32),
+        ("idx_dim", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float),
+        ("rms_eps", ctypes.c_float),
+        ("flags", ctypes.c_uint32),
+    ]
+
+
+class QSAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s" % (where, _lib.qsa_status_string(status).decode()))
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libqsa.so is not built (python -m block_sparse_long_09_b200.build)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    CP = ctypes.POINTER(Config)
+    sig = {
+        "qsa_config_init": (None, [CP]),
+        "qsa_compress_keys": (I32, [CP, P, P, P, I32, I64, P, I32, P, P]),
+        "qsa_index_scores": (I32, [CP, P, P, P, I64, P, P, P, I32, I64, I32, I64, I64, P, I64, P, SZ, P]),
+        "qsa_select_blocks": (I32, [CP, P, I64, P, P, I32, I64, I64, P, P, SZ, P]),
+        "qsa_sparse_attn_prefill": (I32, [CP, P, P, P, P, P, P, I32, I64, I64, I64, I64, P, P, P, SZ, P]),
+        "qsa_sparse_attn_decode": (I32, [CP, P, P, P, P, I32, I64, P, P, P, P, SZ, P]),
+        "qsa_dense_attn_prefill": (I32, [CP, P, P, P, P, P, I32, I64, I64, I32, P, P, P]),
+        "qsa_workspace_size": (SZ, [CP, I32, I32, I64, I64]),
+        "qsa_status_string": (ctypes.c_char_p, [I32]),
+        "qsa_get_device_status": (I32, [P, ctypes.POINTER(I32), I32]),
+        "qsa_version": (I32, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def default_config(**overrides) -> Config:
+    c = Config()
+    _lib.qsa_config_init(ctypes.byref(c))
+    for k, v in overrides.items():
+        setattr(c, k, v)
+    return c
+
+
+def _check(status: int, where: str):
+    if status != QSA_OK:
+        raise QSAError(status, where)
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    assert t.is_cuda and t.is_contiguous(), "tensors must be contiguous CUDA tensors"
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _cfg(cfg: Optional[Config]) -> Config:
+    return cfg if cfg is not None else default_config()
+
+
+def workspace_size(op: int, batch: int, rows: int = 0, max_len_k: int = 0, cfg: Optional[Config] = None) -> int:
+    return int(_lib.qsa_workspace_size(ctypes.byref(_cfg(cfg)), op, batch, rows, max_len_k))
+
+
+def device_status(clear: bool = True) -> int:
+    st = ctypes.c_int32(0)
+    _check(_lib.qsa_get_device_status(_stream(), ctypes.byref(st), 1 if clear else 0), "qsa_get_device_status")
+    return int(st.value)
+
+
+def compress_keys(k_idx, cu_seqlens_k, cu_blocks, kc=None, blk_begin=None, max_new_blocks: int = 0,
+                  cfg: Optional[Config] = None, n_blocks: Optional[int] = None):
+    """kc[b] = RMSNorm(mean of the r indexer keys of block b) for every complete block."""
+    cfg = _cfg(cfg)
+    batch = cu_seqlens_k.numel() - 1
+    if kc is None:
+        if n_blocks is None:
+            n_blocks = int(cu_blocks[-1].item())
+        kc = torch.empty((n_blocks, cfg.idx_dim), dtype=torch.bfloat16, device=k_idx.device)
+    _check(_lib.qsa_compress_keys(ctypes.byref(cfg), _p(k_idx), _p(cu_seqlens_k), _p(cu_blocks), batch,
+                                  k_idx.shape[0], _p(blk_begin), max_new_blocks, _p(kc), _stream()),
+           "qsa_compress_keys")
+    return kc
+
+
+def index_scores(q_idx, w, kc, cu_seqlens_q, cu_seqlens_k, cu_blocks, max_len_q: int, ld: int,
+                 row_begin: int = 0, row_end: Optional[int] = None, scores=None, cfg: Optional[Config] = None):
+    """Indexer scores for packed query rows [row_begin, row_end); row i at scores[i - row_begin]."""
+    cfg = _cfg(cfg)
+    total_q = q_idx.shape[0]
+    if row_end is None:
+        row_end = total_q
+    if scores is None:
+        scores = torch.empty((max(row_end - row_begin, 1), ld), dtype=torch.float32, device=q_idx.device)
+    assert scores.shape[1] == ld
+    _check(_lib.qsa_index_scores(ctypes.byref(cfg), _p(q_idx), _p(w), _p(kc), kc.shape[0], _p(cu_seqlens_q),
+                                 _p(cu_seqlens_k), _p(cu_blocks), cu_seqlens_q.numel() - 1, total_q, max_len_q,
+                                 row_begin, row_end, _p(scores), ld, None, 0, _stream()),
+           "qsa_index_scores")
+    return scores
+
+
+def select_blocks(scores, cu_seqlens_q, cu_seqlens_k, total_q: int, row_begin: int = 0,
+                  row_end: Optional[int] = None, sel=None, cfg: Optional[Config] = None):
+    """Own block + best k-1 earlier blocks per row; sel[i] for packed rows i in [row_begin, row_end)."""
+    cfg = _cfg(cfg)
+    if row_end is None:
+        row_end = total_q
+    if sel is None:
+        sel = torch.empty((total_q, cfg.budget_blocks), dtype=torch.int32, device=scores.device)
+    _check(_lib.qsa_select_blocks(ctypes.byref(cfg), _p(scores), scores.shape[1], _p(cu_seqlens_q),
+                                  _p(cu_seqlens_k), cu_seqlens_q.numel() - 1, row_begin, row_end, _p(sel),
+                                  None, 0, _stream()),
+           "qsa_select_blocks")
+    return sel
+
+
+def sparse_attn_prefill(q, k, v, sel, cu_seqlens_q, cu_seqlens_k, row_begin: int = 0,
+                        row_end: Optional[int] = None, o=None, lse=None, want_lse: bool = False,
+                        cfg: Optional[Config] = None, ws=None):
+    cfg = _cfg(cfg)
+    total_q = q.shape[0]
+    if row_end is None:
+        row_end = total_q
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((total_q, cfg.n_heads_q), dtype=torch.float32, device=q.device)
+    batch = cu_seqlens_q.numel() - 1
+    need = workspace_size(OP_PREFILL, batch, row_end - row_begin, 0, cfg)
+    if ws is None and need > 0:
+        ws = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    _check(_lib.qsa_sparse_attn_prefill(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(sel), _p(cu_seqlens_q),
+                                        _p(cu_seqlens_k), batch, total_q, k.shape[0], row_begin, row_end,
+                                        _p(o), _p(lse), _p(ws), ws.numel() if ws is not None else 0, _stream()),
+           "qsa_sparse_attn_prefill")
+    return (o, lse) if want_lse or lse is not None else o
+
+
+def sparse_attn_decode(q, k_cache, v_cache, cu_seqlens_k, sel, o=None, lse=None, ws=None, want_lse: bool = False,
+                       cfg: Optional[Config] = None):
+    cfg = _cfg(cfg)
+    batch = q.shape[0]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((batch, cfg.n_heads_q), dtype=torch.float32, device=q.device)
+    need = workspace_size(OP_DECODE, batch, batch, 0, cfg)
+    if ws is None and need > 0:
+        ws = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    _check(_lib.qsa_sparse_attn_decode(ctypes.byref(cfg), _p(q), _p(k_cache), _p(v_cache), _p(cu_seqlens_k),
+                                       batch, k_cache.shape[0], _p(sel), _p(o), _p(lse), _p(ws),
+                                       ws.numel() if ws is not None else 0, _stream()),
+           "qsa_sparse_attn_decode")
+    return (o, lse) if want_lse or lse is not None else o
+
+
+def dense_attn_prefill(q, k, v, cu_seqlens_q, cu_seqlens_k, max_len_q: int, o=None, lse=None,
+                       want_lse: bool = False, cfg: Optional[Config] = None):
+    cfg = _cfg(cfg)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((q.shape[0], cfg.n_heads_q), dtype=torch.float32, device=q.device)
+    _check(_lib.qsa_dense_attn_prefill(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(cu_seqlens_q), _p(cu_seqlens_k),
+                                       cu_seqlens_q.numel() - 1, q.shape[0], k.shape[0], max_len_q, _p(o),
+                                       _p(lse), _stream()),
+           "qsa_dense_attn_prefill")
+    return (o, lse) if want_lse or lse is not None else o
+
+
+class Prefill:
+    """One QSA layer's prefill through the C ABI, with query rows processed in
+    chunks (the pages measure with 16K-token chunks).  Buffers are allocated
+    once and reused across calls of the same shape."""
+
+    def __init__(self, seqlens, chunk_rows: int = 16384, cfg: Optional[Config] = None, device="cuda"):
+        self.cfg = _cfg(cfg)
+        r = self.cfg.r
+        self.seqlens = [int(x) for x in seqlens]
+        self.total = sum(self.seqlens)
+        self.max_len = max(self.seqlens)
+        self.n_blocks = sum(L // r for L in self.seqlens)
+        self.ld = max(1, (self.max_len - 1) // r)
+        self.chunk = int(chunk_rows)
+        self.device = torch.device(device)
+        cu = [0]
+        for L in self.seqlens:
+            cu.append(cu[-1] + L)
+        cb = [0]
+        for L in self.seqlens:
+            cb.append(cb[-1] + L // r)
+        self.cu = torch.tensor(cu, dtype=torch.int32, device=self.device)
+        self.cu_blocks = torch.tensor(cb, dtype=torch.int32, device=self.device)
+        self.kc = torch.empty((max(self.n_blocks, 1), self.cfg.idx_dim), dtype=torch.bfloat16, device=self.device)
+        self.scores = torch.empty((min(self.chunk, self.total), self.ld), dtype=torch.float32, device=self.device)
+        self.sel = torch.empty((self.total, self.cfg.budget_blocks), dtype=torch.int32, device=self.device)
+
+    def index_select(self, q_idx, w, k_idx):
+        compress_keys(k_idx, self.cu, self.cu_blocks, kc=self.kc, cfg=self.cfg)
+        for r0 in range(0, self.total, self.chunk):
+            r1 = min(self.total, r0 + self.chunk)
+            index_scores(q_idx, w, self.kc[: self.n_blocks], self.cu, self.cu, self.cu_blocks, self.max_len,
+                         self.ld, r0, r1, scores=self.scores, cfg=self.cfg)
+            select_blocks(self.scores, self.cu, self.cu, self.total, r0, r1, sel=self.sel, cfg=self.cfg)
+        return self.sel
+
+    def __call__(self, q, k, v, q_idx, w, k_idx, o=None, lse=None):
+        self.index_select(q_idx, w, k_idx)
+        return sparse_attn_prefill(q, k, v, self.sel, self.cu, self.cu, o=o, lse=lse, cfg=self.cfg)

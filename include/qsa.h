@@ -1,0 +1,214 @@
+/*
+ * qsa.h -- C ABI of libqsa.so: Qwen Sparse Attention (QSA) on NVIDIA B200 (sm_100a).
+ *
+ * QSA replaces a full-attention layer by micro-block sparse softmax attention
+ * with a compressed lightweight indexer.  Source for every operation below:
+ * "On the Design of Qwen3.8 Next Architecture: Evaluation, Efficiency, and
+ * Training Stability" (reading notes), section 6 "GDN 连续压缩与 QSA 精确检索"
+ * (pooled-key equation, indexer equation, budget sentence, complexity
+ * equation) and its "Model Summary" table (head counts and sizes).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor pointer is DEVICE memory owned by the caller; the library
+ *    never allocates, frees or keeps a pointer after the call returns.  Host
+ *    arguments are plain integers/floats and the config struct (read during
+ *    the call only).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream) and launch on the current device.
+ *  - Return value: QSA_OK when the work was enqueued; QSA_ERR_INVALID_ARG /
+ *    QSA_ERR_UNSUPPORTED / QSA_ERR_WORKSPACE_TOO_SMALL are detected on the
+ *    host BEFORE anything is launched; QSA_ERR_CUDA reports a launch error.
+ *    Errors found on the device (an index out of range, a bounded wait that
+ *    gave up) do not abort the launch: the kernel records QSA_ERR_DEVICE_CHECK
+ *    or QSA_ERR_TIMEOUT in a sticky per-device status word and skips the
+ *    offending work; read it with qsa_get_device_status().
+ *  - bf16 tensors are raw 16-bit patterns (qsa_bf16).  Layouts are dense,
+ *    row-major, innermost dimension last, no padding.
+ *  - Variable-length batches are packed.  cu_seqlens_q / cu_seqlens_k /
+ *    cu_blocks are int32 device arrays of batch+1 prefix sums (first entry 0)
+ *    of L_q,s, L_k,s and floor(L_k,s / r).  Query row i of sequence s sits at
+ *    position t = (L_k,s - L_q,s) + (i - cu_seqlens_q[s]) (bottom-right
+ *    aligned: prefill has L_q = L_k, decode has L_q = 1).
+ *  - Notation: r = micro-block size, b_t = floor(t / r) is the query's own
+ *    block, the candidates of t are the complete blocks 0 .. b_t - 1, and
+ *    k = budget_blocks counts the own block (|Sel_t| = min(k, b_t + 1)).
+ *  - Supported configuration: the model's (r = 4, 24 query heads, 2 KV
+ *    heads, head dim 256, 4 indexer heads of dim 128) with a budget of
+ *    k <= 2048 blocks (the model uses 512); anything else returns
+ *    QSA_ERR_UNSUPPORTED.
+ *  - Thread safety: the library keeps no state besides the status word.
+ */
+#ifndef QSA_H
+#define QSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t qsa_status;
+#define QSA_OK 0
+#define QSA_ERR_INVALID_ARG 1
+#define QSA_ERR_UNSUPPORTED 2
+#define QSA_ERR_WORKSPACE_TOO_SMALL 3
+#define QSA_ERR_CUDA 4
+#define QSA_ERR_TIMEOUT 5
+#define QSA_ERR_DEVICE_CHECK 6
+
+typedef uint16_t qsa_bf16;
+
+/* flags */
+#define QSA_COMPRESS_NO_NORM 0x1u /* plain mean-pool, no RMSNorm in the compressor */
+
+typedef struct qsa_config {
+    int32_t r;             /* micro-block size (4) */
+    int32_t budget_blocks; /* k: blocks kept per query, own block included (512) */
+    int32_t n_heads_q;     /* 24 */
+    int32_t n_heads_kv;    /* 2 (GQA: head h reads KV group h / 12) */
+    int32_t head_dim;      /* 256 */
+    int32_t n_heads_idx;   /* indexer query heads (4); one shared key head */
+    int32_t idx_dim;       /* indexer head dim (128) */
+    float softmax_scale;   /* 1/sqrt(256) */
+    float rms_eps;         /* compressor RMSNorm eps (1e-6) */
+    uint32_t flags;        /* QSA_COMPRESS_NO_NORM */
+} qsa_config;
+
+/* op ids for qsa_workspace_size */
+#define QSA_OP_COMPRESS 0
+#define QSA_OP_INDEX 1
+#define QSA_OP_SELECT 2
+#define QSA_OP_PREFILL 3
+#define QSA_OP_DECODE 4
+#define QSA_OP_DENSE 5
+
+/* Fill *cfg with the model's values (r 4, k 512, 24/2/256, 4/128, scale 1/16,
+ * eps 1e-6, flags 0).  Host only. */
+void qsa_config_init(qsa_config *cfg);
+
+/*
+ * Key compressor -- pooled-key equation of section 6:
+ *   kc[b] = RMSNorm( (1/r) * sum_{j<r} k_idx[b r + j] ),   unit gain, eps cfg->rms_eps
+ * for every complete block b < floor(L_k,s / r) of every sequence (the mean
+ * alone with QSA_COMPRESS_NO_NORM).  fp32 arithmetic, bf16 round-to-nearest store.
+ *   k_idx      [total_k, idx_dim] bf16   raw indexer keys (one shared key head)
+ *   cu_seqlens_k, cu_blocks  [batch+1] int32
+ *   total_k    host: rows of k_idx (bounds the launch)
+ *   blk_begin  [batch] int32 or NULL.  NULL: every complete block is written.
+ *              Otherwise only blocks [blk_begin[s], blk_begin[s] + max_new_blocks)
+ *              that are complete (a decode step refreshes the blocks it completed).
+ *   kc         [cu_blocks[batch], idx_dim] bf16, written.
+ */
+qsa_status qsa_compress_keys(const qsa_config *cfg, const qsa_bf16 *k_idx,
+                             const int32_t *cu_seqlens_k, const int32_t *cu_blocks,
+                             int32_t batch, int64_t total_k, const int32_t *blk_begin,
+                             int32_t max_new_blocks, qsa_bf16 *kc, void *stream);
+
+/*
+ * Indexer scores -- indexer equation of section 6, with one weight per
+ * (query, indexer head) (w = 1 gives the equation as printed):
+ *   S[t, b] = sum_h w[t, h] * max(0, <q_idx[t, h, :], kc[b, :]>),   b < b_t
+ * bf16 tensor-core products, fp32 accumulation and epilogue.
+ *   q_idx   [total_q, n_heads_idx, idx_dim] bf16;  w [total_q, n_heads_idx] fp32
+ *   kc      [kc_rows, idx_dim] bf16 (the compressor's output; kc_rows = cu_blocks[batch])
+ *   rows    packed query rows [row_begin, row_end) are scored (a chunk of a prefill)
+ *   scores  fp32, row i at scores + (i - row_begin) * ld; entries b < b_t(i) are
+ *           written, entries b >= b_t(i) are left untouched.  ld >= every b_t(i).
+ *   total_q host: rows of q_idx; max_len_q host: max over s of L_q,s (a launch hint:
+ *           1 selects the one-row-per-sequence decode kernel)
+ * Workspace: none (ws may be NULL).
+ */
+qsa_status qsa_index_scores(const qsa_config *cfg, const qsa_bf16 *q_idx, const float *w,
+                            const qsa_bf16 *kc, int64_t kc_rows,
+                            const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                            const int32_t *cu_blocks, int32_t batch, int64_t total_q,
+                            int32_t max_len_q, int64_t row_begin, int64_t row_end,
+                            float *scores, int64_t ld, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Top-k block selection -- budget sentence of section 6: the own block b_t is
+ * always kept; the other min(k - 1, b_t) slots go to the highest-scoring
+ * candidates 0 .. b_t - 1, ties to the lower block index.  Exact on the fp32
+ * score bits (radix select on an order-preserving integer key; -0.0 == +0.0).
+ *   scores  as written by qsa_index_scores for rows [row_begin, row_end), stride ld
+ *   sel     [total_q, k] int32: row i at sel + i * k (absolute packed row), block ids
+ *           local to the sequence, ascending, padded with -1.
+ * NaN scores give an unspecified (but valid) selection.  Workspace: none.
+ */
+qsa_status qsa_select_blocks(const qsa_config *cfg, const float *scores, int64_t ld,
+                             const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                             int32_t batch, int64_t row_begin, int64_t row_end, int32_t *sel,
+                             void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Sparse GQA attention, prefill -- expansion + core attention of section 6:
+ * query t attends, per head h with KV group g = h / (n_heads_q / n_heads_kv), to
+ * the tokens of its selected blocks, [b r, b r + r) cut to j <= t:
+ *   o[t, h] = sum_j softmax_j(scale * <q[t, h], k[j, g]>) v[j, g]
+ * bf16 tensor-core products, fp32 softmax and accumulation, bf16 output.
+ *   q   [total_q, n_heads_q, head_dim] bf16; k, v [total_k, n_heads_kv, head_dim] bf16
+ *   sel [total_q, k] int32 as produced by qsa_select_blocks (-1 = unused slot)
+ *   rows [row_begin, row_end) of the packed queries are computed
+ *   o   [total_q, n_heads_q, head_dim] bf16 written for those rows
+ *   lse [total_q, n_heads_q] fp32 natural-log sum-exp of the scaled logits, or NULL
+ * A selected block id outside 0 .. b_t is skipped and flagged QSA_ERR_DEVICE_CHECK.
+ * Workspace: none for k <= 512.  A larger budget is processed as k/512 partial
+ * softmax states per row that a second kernel merges: pass a workspace of
+ * qsa_workspace_size(cfg, QSA_OP_PREFILL, batch, row_end - row_begin, 0) bytes.
+ */
+qsa_status qsa_sparse_attn_prefill(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k,
+                                   const qsa_bf16 *v, const int32_t *sel,
+                                   const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                                   int32_t batch, int64_t total_q, int64_t total_k,
+                                   int64_t row_begin, int64_t row_end, qsa_bf16 *o, float *lse,
+                                   void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Sparse GQA attention, decode: one new query per sequence at t = L_k,s - 1,
+ * same definition as the prefill.  The <= k*r selected tokens of a sequence
+ * are split across CTAs (split-K) and the partial softmax states (m, l, o)
+ * are merged by a second kernel.
+ *   q [batch, n_heads_q, head_dim] bf16; k_cache, v_cache [total_k, n_heads_kv,
+ *   head_dim] bf16 (packed, the new token included); sel [batch, k] int32;
+ *   o [batch, n_heads_q, head_dim] bf16; lse [batch, n_heads_q] fp32 or NULL.
+ * Workspace: qsa_workspace_size(cfg, QSA_OP_DECODE, batch, batch, 0) bytes.
+ */
+qsa_status qsa_sparse_attn_decode(const qsa_config *cfg, const qsa_bf16 *q,
+                                  const qsa_bf16 *k_cache, const qsa_bf16 *v_cache,
+                                  const int32_t *cu_seqlens_k, int32_t batch, int64_t total_k,
+                                  const int32_t *sel, qsa_bf16 *o, float *lse, void *ws,
+                                  size_t ws_bytes, void *stream);
+
+/*
+ * Dense causal GQA attention (the baseline the pages measure QSA against):
+ * query t attends to every key j <= t of its sequence.  Same layouts as the
+ * sparse prefill; max_len_q is a host launch bound.  Workspace: none.
+ */
+qsa_status qsa_dense_attn_prefill(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k,
+                                  const qsa_bf16 *v, const int32_t *cu_seqlens_q,
+                                  const int32_t *cu_seqlens_k, int32_t batch, int64_t total_q,
+                                  int64_t total_k, int32_t max_len_q, qsa_bf16 *o, float *lse,
+                                  void *stream);
+
+/* Workspace bytes an op needs (0 = none).  rows = query rows of the call,
+ * max_len_k = longest key sequence.  Host only, no CUDA calls. */
+size_t qsa_workspace_size(const qsa_config *cfg, int32_t op, int32_t batch, int64_t rows,
+                          int64_t max_len_k);
+
+/* Static string for a status code. */
+const char *qsa_status_string(qsa_status status);
+
+/* Synchronises `stream`, then copies the current device's sticky status word
+ * into *status (QSA_OK if no kernel flagged an error); clear != 0 resets it. */
+qsa_status qsa_get_device_status(void *stream, int32_t *status, int32_t clear);
+
+/* ABI version (major * 100 + minor). */
+int32_t qsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSA_H */

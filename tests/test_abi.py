@@ -1,0 +1,90 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+declared in include/qsa.h, and rejects bad arguments before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def qsa():
+    from block_sparse_long_09_b200 import build
+    build.build()
+    from block_sparse_long_09_b200 import qsa as q
+    return q
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "qsa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qsa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("qsa_compress_keys", "qsa_index_scores", "qsa_select_blocks", "qsa_sparse_attn_prefill",
+              "qsa_sparse_attn_decode"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(qsa):
+    lib = qsa.library()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(qsa.EXPORTED) >= set(declared_functions())
+
+
+def test_config_defaults_and_version(qsa):
+    c = qsa.default_config()
+    assert (c.r, c.budget_blocks, c.n_heads_q, c.n_heads_kv, c.head_dim, c.n_heads_idx, c.idx_dim) == \
+        (4, 512, 24, 2, 256, 4, 128)
+    assert abs(c.softmax_scale - 1 / 16) < 1e-9 and abs(c.rms_eps - 1e-6) < 1e-12
+    assert qsa.library().qsa_version() >= 100
+
+
+def test_status_strings(qsa):
+    lib = qsa.library()
+    for s in range(7):
+        assert lib.qsa_status_string(s).decode().startswith("QSA")
+
+
+def test_unsupported_config_rejected_on_host(qsa):
+    lib = qsa.library()
+    for field, value in (("r", 8), ("n_heads_q", 32), ("head_dim", 128), ("budget_blocks", 4096)):
+        c = qsa.default_config(**{field: value})
+        st = lib.qsa_compress_keys(ctypes.byref(c), None, None, None, 1, 0, None, 0, None, None)
+        assert st == qsa.QSA_ERR_UNSUPPORTED, field
+    c = qsa.default_config(r=0)
+    assert lib.qsa_compress_keys(ctypes.byref(c), None, None, None, 1, 0, None, 0, None, None) == \
+        qsa.QSA_ERR_INVALID_ARG
+
+
+def test_invalid_arguments_rejected_on_host(qsa):
+    lib = qsa.library()
+    c = qsa.default_config()
+    fake = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    # batch <= 0
+    assert lib.qsa_compress_keys(ctypes.byref(c), fake, fake, fake, 0, 8, None, 0, fake, None) == \
+        qsa.QSA_ERR_INVALID_ARG
+    # row range beyond total_q
+    assert lib.qsa_index_scores(ctypes.byref(c), fake, fake, fake, 4, fake, fake, fake, 1, 10, 0, 0, 11,
+                                fake, 8, None, 0, None) == qsa.QSA_ERR_INVALID_ARG
+    # ld <= 0
+    assert lib.qsa_select_blocks(ctypes.byref(c), fake, 0, fake, fake, 1, 0, 4, fake, None, 0, None) == \
+        qsa.QSA_ERR_INVALID_ARG
+    # misaligned q
+    assert lib.qsa_sparse_attn_prefill(ctypes.byref(c), ctypes.c_void_p(18), fake, fake, fake, fake, fake, 1, 4,
+                                       4, 0, 4, fake, None, None, 0, None) == qsa.QSA_ERR_INVALID_ARG
+    # empty row range is a no-op
+    assert lib.qsa_sparse_attn_prefill(ctypes.byref(c), fake, fake, fake, fake, fake, fake, 1, 4, 4, 2, 2,
+                                       fake, None, None, 0, None) == qsa.QSA_OK
+
+
+def test_workspace_sizes(qsa):
+    assert qsa.workspace_size(qsa.OP_INDEX, 1, 8192, 8192) == 0
+    assert qsa.workspace_size(qsa.OP_PREFILL, 1, 8192, 8192) == 0
+    ws = qsa.workspace_size(qsa.OP_DECODE, 64, 64, 262144)
+    assert ws >= 64 * 24 * 257 * 4
