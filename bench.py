@@ -1,0 +1,388 @@
+"""QSA benchmark: prefill tokens/s at 262,144 context and decode latency at 131,072.
+
+One step = one pass of the whole QSA hot path on synthetic inputs resident in HBM:
+  prefill  batch 1, n = 262,144: compress -> (index -> select) per 16,384-row chunk
+           -> sparse GQA attention                            (value = tokens/s of this part)
+  decode   batch 64, every cache 131,072 tokens: refresh of the last compressed block,
+           one-row indexer, top-512 select, split-K sparse attention (the "decode" object)
+Inputs are drawn by block_sparse_long_09_b200.inputs (seeded, N(0,1) / U(0,1)); every
+timed input is far larger than the 126 MB L2, so no flush is needed between steps.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl qsa|reference]
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent layer
+(weak scaling, no collective on the data path); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+N_PREFILL = 262144
+DEC_BATCH = 64
+DEC_LEN = 131072
+CHUNK = 16384
+BUDGET = 512
+METRIC = "QSA prefill tokens/s at 262K ctx; decode µs/token at 128K; % of roofline"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampler running during the timed region."""
+
+    def __init__(self, index):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % index)
+        self.index = index
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index),
+                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gather_bytes_per_query(n_tokens_selected):
+    # K and V, 2 KV heads x 256 dims x 2 bytes each
+    return n_tokens_selected * 2 * 256 * 2 * 2
+
+
+def selected_tokens(n, r=4, k=BUDGET):
+    """Sum over queries of |T_t| (tokens actually attended), by the definition."""
+    t = np.arange(n, dtype=np.int64)
+    bt = t // r
+    nblk = np.minimum(k, bt + 1)
+    # every selected block is complete except the own block, which holds t - r*bt + 1 tokens
+    return int(((nblk - 1) * r + (t - r * bt + 1)).sum())
+
+
+def run_qsa(args, rank, world, device):
+    from block_sparse_long_09_b200 import inputs, qsa
+
+    hbm, tflops, peak_kind = peaks()
+    torch.manual_seed(0)
+    x = inputs.make_prefill([N_PREFILL], seed=rank, device=device)
+    cfg = qsa.default_config(budget_blocks=BUDGET)
+    pre = qsa.Prefill([N_PREFILL], chunk_rows=CHUNK, cfg=cfg, device=device)
+    o = torch.empty_like(x.q)
+
+    d = inputs.make_decode(DEC_BATCH, DEC_LEN, None, seed=100 + rank, device=device)
+    cu_k = d.cu_seqlens_k
+    cu_b = d.cu_blocks
+    cu_q = torch.arange(DEC_BATCH + 1, dtype=torch.int32, device=device)
+    kc_dec = qsa.compress_keys(d.k_idx, cu_k, cu_b, n_blocks=int(cu_b[-1]), cfg=cfg)
+    last_blk = torch.tensor([L // 4 - 1 for L in d.seqlens], dtype=torch.int32, device=device)
+    ld_dec = (DEC_LEN - 1) // 4
+    dec_scores = torch.empty((DEC_BATCH, ld_dec), dtype=torch.float32, device=device)
+    dec_sel = torch.empty((DEC_BATCH, BUDGET), dtype=torch.int32, device=device)
+    dec_o = torch.empty_like(d.q)
+    dec_ws = torch.empty((qsa.workspace_size(qsa.OP_DECODE, DEC_BATCH, DEC_BATCH, DEC_LEN, cfg),),
+                         dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    ev = {k: [] for k in ("p0", "p1", "a0", "a1", "d0", "d1")}
+
+    def step(record):
+        e = {k: torch.cuda.Event(enable_timing=True) for k in ev} if record else None
+        if record:
+            e["p0"].record(stream)
+        pre.index_select(x.q_idx, x.w, x.k_idx)
+        if record:
+            e["a0"].record(stream)
+        qsa.sparse_attn_prefill(x.q, x.k, x.v, pre.sel, pre.cu, pre.cu, o=o, cfg=cfg)
+        if record:
+            e["a1"].record(stream)
+            e["p1"].record(stream)
+            e["d0"].record(stream)
+        qsa.compress_keys(d.k_idx, cu_k, cu_b, kc=kc_dec, blk_begin=last_blk, max_new_blocks=1, cfg=cfg)
+        qsa.index_scores(d.q_idx, d.w, kc_dec, cu_q, cu_k, cu_b, 1, ld_dec, scores=dec_scores, cfg=cfg)
+        qsa.select_blocks(dec_scores, cu_q, cu_k, DEC_BATCH, sel=dec_sel, cfg=cfg)
+        qsa.sparse_attn_decode(d.q, d.k_cache, d.v_cache, cu_k, dec_sel, o=dec_o, ws=dec_ws, cfg=cfg)
+        if record:
+            e["d1"].record(stream)
+            for k in ev:
+                ev[k].append(e[k])
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    assert qsa.device_status() == 0, "a kernel flagged a device-side error during warm-up"
+
+    clocks = Clocks(device.index if device.index is not None else 0)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step(True)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    prefill_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["p0"], ev["p1"])]))
+    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"])]))
+    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["d0"], ev["d1"])]))
+    assert qsa.device_status() == 0, "a kernel flagged a device-side error in the timed region"
+
+    def allmax(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    total_ms, prefill_ms, attn_ms, dec_ms = (allmax(v) for v in (total_ms, prefill_ms, attn_ms, dec_ms))
+
+    # end to end through the public API: pinned host inputs in, result out, every step
+    e2e = None
+    if args.e2e_steps > 0:
+        host = {k: getattr(x, k).cpu().pin_memory() for k in ("q", "k", "v", "q_idx", "k_idx", "w")}
+        o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        dev_in = {k: torch.empty_like(getattr(x, k)) for k in host}
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = o_host.numel() * o_host.element_size()
+
+        def e2e_step():
+            for k2, t in host.items():
+                dev_in[k2].copy_(t, non_blocking=True)
+            pre(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["q_idx"], dev_in["w"], dev_in["k_idx"], o=o)
+            o_host.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = allmax(e0.elapsed_time(e1) / args.e2e_steps)
+        e2e = {"value": world * N_PREFILL / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": args.e2e_steps, "scope": "prefill 262144 via qsa.Prefill"}
+
+    sel_tok = selected_tokens(N_PREFILL)
+    gather = gather_bytes_per_query(1) * sel_tok
+    achieved = gather / (attn_ms / 1e3) / 1e9
+    launches_prefill = 1 + 2 * ((N_PREFILL + CHUNK - 1) // CHUNK) + 1
+    launches_decode = 1 + 1 + 1 + 2
+    res = {
+        "metric": METRIC,
+        "value": world * N_PREFILL / (prefill_ms / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations, U(0,1) indexer weights)",
+        "config": {"workload": "QSA layer: prefill batch 1 n=262144 (16384-row chunks) + decode batch 64 ctx 131072",
+                   "budget_blocks": BUDGET, "r": 4, "heads": "24q/2kv/256, indexer 4/128",
+                   "prefill_ms": prefill_ms, "attn_prefill_ms": attn_ms, "l2": "inputs > L2, no flush",
+                   "parallelism": "independent layer per rank" if world > 1 else "1 GPU"},
+        "decode": {"batch": DEC_BATCH, "ctx": DEC_LEN, "step_us": dec_ms * 1e3, "us_per_token": dec_ms * 1e3,
+                   "us_per_token_amortized": dec_ms * 1e3 / DEC_BATCH},
+        "roofline": {"kernel": "sparse_attn_kernel (prefill)", "bound": "hbm", "achieved": achieved,
+                     "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                     "algorithmic_bytes": gather, "peak_kind": peak_kind + " (burst copy)"},
+        "gpu_launches": args.steps * (launches_prefill + launches_decode),
+        "e2e": e2e,
+        "clocks": clk,
+    }
+    return res
+
+
+def cpu_baseline(seconds: float = 12.0, rows_hint: int = 16):
+    """The fp64 oracle, as it stands, on a bounded sample of the prefill workload:
+    for each sampled query row the whole chain (scores against every earlier
+    compressed block, top-512 selection, attention over the selected tokens),
+    after one compression of all keys."""
+    import oracle
+    from block_sparse_long_09_b200 import inputs
+
+    x = inputs.make_prefill([N_PREFILL], seed=0, device="cuda" if torch.cuda.is_available() else "cpu")
+
+    def bits(t):
+        return np.ascontiguousarray(t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+    k_idx, k, v = bits(x.k_idx), bits(x.k), bits(x.v)
+    rng = np.random.default_rng(0)
+    cores = oracle.threads()
+
+    def run(rows):
+        rows = np.sort(rows)
+        q, q_idx, w = bits(x.q[rows]), bits(x.q_idx[rows]), x.w[rows].cpu().numpy()
+        t0 = time.perf_counter()
+        kc = oracle.compress(k_idx, 4)
+        ld = (N_PREFILL - 1) // 4
+        sc = np.empty((len(rows), ld))
+        for j, i in enumerate(rows):  # query row j sits at position i: Lq = 1, Lk = i + 1
+            sc[j] = oracle.index_scores(q_idx[j:j + 1], w[j:j + 1], kc, 1, int(i) + 1, 4, [0], ld=ld)[0]
+        sel = oracle.select(sc, rows // 4, BUDGET)
+        for j, i in enumerate(rows):
+            oracle.attend(q[j:j + 1], k, v, sel[j:j + 1], 1, int(i) + 1, 4, 1 / 16, [0])
+        return time.perf_counter() - t0
+
+    n = rows_hint
+    t = run(rng.integers(N_PREFILL // 2, N_PREFILL, n))
+    if t < seconds / 3:
+        n = max(n, int(n * seconds / max(t, 1e-3)))
+        t = run(rng.integers(N_PREFILL // 2, N_PREFILL, n))
+    return {"value": n / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": "%d random query rows from the second half of the 262144-token prefill: compress of all "
+                      "keys once, then per row scores, top-512 select and attention, fp64, %.1f s" % (n, t)}
+
+
+def run_profile_case(case: str, reps: int = 3):
+    """Small cases for ncu captures of one kernel (a few GB on the device, K/V larger than L2)."""
+    from block_sparse_long_09_b200 import inputs, qsa
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    cfg = qsa.default_config(budget_blocks=BUDGET)
+    if case in ("attn", "index", "select"):
+        n, rows = 131072, 8192
+        x = inputs.make_prefill([n], seed=0, device=dev)
+        pre = qsa.Prefill([n], chunk_rows=rows, cfg=cfg, device=dev)
+        qsa.compress_keys(x.k_idx, pre.cu, pre.cu_blocks, kc=pre.kc, cfg=cfg)
+        r0 = n - rows
+        for _ in range(reps):
+            if case in ("index", "select", "attn"):
+                qsa.index_scores(x.q_idx, x.w, pre.kc[: pre.n_blocks], pre.cu, pre.cu, pre.cu_blocks, n, pre.ld,
+                                 r0, n, scores=pre.scores, cfg=cfg)
+                qsa.select_blocks(pre.scores, pre.cu, pre.cu, n, r0, n, sel=pre.sel, cfg=cfg)
+            if case == "attn":
+                qsa.sparse_attn_prefill(x.q, x.k, x.v, pre.sel, pre.cu, pre.cu, r0, n, cfg=cfg)
+    elif case == "decode":
+        d = inputs.make_decode(DEC_BATCH, 16384, None, seed=1, device=dev)
+        cu_q = torch.arange(DEC_BATCH + 1, dtype=torch.int32, device=dev)
+        kc = qsa.compress_keys(d.k_idx, d.cu_seqlens_k, d.cu_blocks, n_blocks=int(d.cu_blocks[-1]), cfg=cfg)
+        ld = (16384 - 1) // 4
+        sc = torch.empty((DEC_BATCH, ld), dtype=torch.float32, device=dev)
+        for _ in range(reps):
+            qsa.index_scores(d.q_idx, d.w, kc, cu_q, d.cu_seqlens_k, d.cu_blocks, 1, ld, scores=sc, cfg=cfg)
+            sel = qsa.select_blocks(sc, cu_q, d.cu_seqlens_k, DEC_BATCH, cfg=cfg)
+            qsa.sparse_attn_decode(d.q, d.k_cache, d.v_cache, d.cu_seqlens_k, sel, cfg=cfg)
+    torch.cuda.synchronize()
+    assert qsa.device_status() == 0
+    print("profile case %s done" % case)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="qsa", choices=["qsa", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=["attn", "index", "select", "decode"], default=None,
+                    help="run one small case for an ncu capture and exit")
+    args = ap.parse_args()
+    if args.profile_case:
+        import block_sparse_long_09_b200.build as bld
+        bld.build()
+        run_profile_case(args.profile_case)
+        return
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        t0 = time.perf_counter()
+        steps = []
+        for _ in range(args.warmup + args.steps):
+            steps.append(cpu_baseline(seconds=4.0, rows_hint=8))
+        b = steps[args.warmup:]
+        val = float(np.mean([s["value"] for s in b]))
+        res = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
+               "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * (time.perf_counter() - t0) / len(steps),
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+               "data": "synthetic", "config": {"workload": "QSA prefill batch 1 n=262144, sampled rows (fp64 oracle)"},
+               "cpu_baseline": {"value": val, "unit": "tokens/s", "kind": "oracle", "cores": b[0]["cores"],
+                                "sample": b[0]["sample"]},
+               "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(res))
+        return
+
+    import block_sparse_long_09_b200.build as bld
+    bld.build()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    res = run_qsa(args, rank, world, device)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(res))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

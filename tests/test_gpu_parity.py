@@ -66,6 +66,20 @@ def check_scores(g, o, bt, k):
         assert bad.size == 0, (n, bad[:5], g[n, bad[:5]], o[n, bad[:5]])
 
 
+def check_selection_near_threshold(sel_g, sel_o, scores_o, bt, k):
+    """The GPU selects on its own scores: a block may differ from the oracle's choice
+    only where the oracle's score is within 1e-2 (relative) of the row's k-th best.
+    Returns the mask of rows whose selections agree exactly."""
+    agree = np.all(sel_g == sel_o, axis=1)
+    for n in np.nonzero(~agree)[0]:
+        s_star = kth_best(scores_o[n], int(bt[n]), k)
+        diff = set(sel_g[n].tolist()) ^ set(sel_o[n].tolist())
+        for b in diff:
+            assert 0 <= b < bt[n], (n, b)
+            assert abs(scores_o[n, b] - s_star) < 1e-2 * abs(s_star) + 1e-9, (n, b, scores_o[n, b], s_star)
+    return agree
+
+
 def check_attn(g, o):
     d = np.abs(g.astype(np.float64) - o)
     assert d.max() <= 2e-2, d.max()
@@ -294,15 +308,7 @@ def test_full_chain_tiny_config(qsa):
     pre, sel, o, lse = run_chain(qsa, x, [n], k)
     ref = oracle.qsa_layer(x.q, x.k, x.v, x.q_idx, x.k_idx, x.w, n, n, 4, k)
     sel_g = sel.cpu().numpy()
-    # selections: equal except where the oracle's own score sits within 1e-2 of the k-th best
-    agree = np.all(sel_g == ref["sel"], axis=1)
-    for i in np.nonzero(~agree)[0]:
-        bt = i // 4
-        s_star = kth_best(ref["scores"][i], bt, k)
-        diff = set(sel_g[i].tolist()) ^ set(ref["sel"][i].tolist())
-        for b in diff:
-            assert abs(ref["scores"][i, b] - s_star) < 1e-2 * abs(s_star) + 1e-9, (i, b)
-    assert agree.mean() > 0.95
+    agree = check_selection_near_threshold(sel_g, ref["sel"], ref["scores"], np.arange(n) // 4, k)
     check_attn(o.float().cpu().numpy()[agree], ref["o"][agree])
     status_ok(qsa)
 
@@ -328,8 +334,7 @@ def test_chain_n8192_budget512(qsa):
     kc = oracle.compress(x.k_idx, 4)
     sc = oracle.index_scores(x.q_idx, x.w, kc, n, n, 4, rows, ld=(n - 1) // 4)
     sel_o = oracle.select(sc, rows // 4, k)
-    agree = np.all(sel_g[rows] == sel_o, axis=1)
-    assert agree.mean() > 0.9
+    check_selection_near_threshold(sel_g[rows], sel_o, sc, rows // 4, k)
     ref_o, _ = oracle.attend(x.q, x.k, x.v, sel_g[rows], n, n, 4, SCALE, rows)
     check_attn(o.float().cpu().numpy()[rows], ref_o)
     status_ok(qsa)
