@@ -135,9 +135,8 @@ size_t qsa_workspace_size(const qsa_config *cfg, int32_t op, int32_t batch, int6
     (void)max_len_k;
     if (check_config(cfg) != QSA_OK || batch <= 0 || rows < 0) return 0;
     if (op == QSA_OP_DECODE) {
-        // upper bound over devices: at most one split per 128-token tile
-        const int max_tiles = (cfg->budget_blocks + 31) / 32;
-        return split_workspace_bytes(batch, max_tiles > 1 ? max_tiles : 2);
+        const int ns = max_nsplit(cfg->budget_blocks);
+        return split_workspace_bytes(batch, ns > 1 ? ns : 2);
     }
     if (op == QSA_OP_PREFILL) return split_workspace_bytes(rows, min_nsplit(cfg->budget_blocks));
     return 0;

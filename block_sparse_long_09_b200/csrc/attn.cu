@@ -7,25 +7,31 @@
 // group), head dim 256.  Query t sees the tokens of its selected blocks with
 // j <= t (causal inside its own block).
 //
-// Design (B200): a persistent CTA per SM walks work items = (query row, split).
-// For one item and one KV group g the 12 heads of g share every gathered key,
-// so the contraction is laid out "swap-AB": keys are the M = 128 side of the
-// tcgen05 MMA and the 12 heads (padded to N = 16) the N side, which keeps the
-// tensor-core waste at 16/12 instead of 128/12.
-//   warp 0      TMA producer: per 128-token tile and group, 32 micro-blocks x 4
-//               d-chunks are gathered as 4-row boxes straight into the 128-byte
-//               swizzled operand layout (3-slot ring of 64 KB); padding slots
-//               load an out-of-range box, i.e. zeros.
-//   warp 1      TMEM allocation + single-thread MMA issue:
-//               S^T[key, head]  = K_tile[128 x 256] . Q_g^T          (K-major A and B)
-//               O^T[d, head]   += V_tile^T[256 x 128] . P^T[128 x 16] (MN-major A)
-//   warps 2..5  softmax: S^T of all <= 16 tiles of the group stays in TMEM
-//               (16 columns each), so the exact per-head max is taken first and
-//               P = exp(S - max) needs no rescaling; P^T goes to shared memory in
-//               the swizzled K-major layout for the PV MMA; the epilogue reads O^T
-//               back from TMEM, divides by the row sums and writes bf16 (or, for
-//               split-K decode, fp32 partials + log-sum-exp for the combine kernel).
-// The kernel is bound by the gather (4 MiB of K/V per query), not by the MMAs.
+// The kernel is bound by the gather: 4 MiB of K/V per query, scattered in
+// 4 KB micro-blocks, against ~25 MFLOP of math.  Design (B200):
+//  * One TMA op per micro-block and tensor: a 3-D tensor map over K (or V)
+//    with dims (64 d, token-row, 4 d-chunks) and strides (512 B, 128 B) copies
+//    the block's 8 rows (4 tokens x 2 KV heads) x 256 d = 4 KB straight into
+//    the 128-byte-swizzled K-major UMMA layout (8-row atom per block, SBO 4 KB).
+//    Fewer, larger TMA ops is what lifts the gather rate: 512 B boxes stall at
+//    ~2.4 TB/s on B200, whole blocks stream at the HBM rate.
+//  * Both KV groups ride in one MMA: rows alternate (token, group), so
+//    S^T[128 rows, 32] = K_tile . Q^T carries all 24 heads (8 pad); entries
+//    whose head belongs to the other group are masked, and P^T keeps them at
+//    zero, so O^T[256 d, 32] += V_tile^T . P^T accumulates every head at once.
+//    Keys are the M = 128 side ("swap AB"): the tensor cores idle anyway.
+//  * Online softmax, lazy rescale: the running max is updated per 64-token
+//    tile (exact per-head tile max, one named barrier), O is rescaled in TMEM
+//    only when a new max exceeds the old by more than 2^8 in probability.
+//  * Warp roles of a persistent CTA (one per SM):
+//      warp 0      TMA producer: Q (per item), then K/V tiles in MMA order
+//                  (K0, K1, V0, K2, V1, ...) through a 3-slot ring of 64 KB;
+//                  block ids are fetched two tiles ahead
+//      warp 1      TMEM owner + single-thread tcgen05.mma issue: S(j+1) is
+//                  issued before PV(j) so QK^T overlaps the softmax
+//      warps 2..5  softmax (thread = TMEM lane = (token, group) row) and the
+//                  epilogue (thread = d); split-K decode writes fp32 partial
+//                  states that combine_kernel merges.
 #include "kernels.cuh"
 
 namespace qsa {
@@ -33,28 +39,31 @@ namespace qsa {
 namespace {
 
 constexpr int kHQ = 24, kHKV = 2, kD = 256, kGrp = kHQ / kHKV;
-constexpr int kTileTok = 128;
-constexpr int kBlkPerTile = 32;             // r = 4
-constexpr int kMaxTiles = 16;               // budget 512 blocks = 2048 tokens
-constexpr int kSlotBytes = kTileTok * kD * 2;   // 64 KB: one K or V tile of one group
-constexpr int kChunk = kTileTok * 128;      // 16 KB: 64 d-columns of a tile
+constexpr int kBlkTile = 16;                    // micro-blocks per tile (r = 4)
+constexpr int kRowsTile = 128;                  // 16 blocks x 4 tokens x 2 KV heads
+constexpr int kBlockBytes = 8 * kD * 2;         // 4 KB: one block of K (or V), both heads
+constexpr int kSlotBytes = kBlkTile * kBlockBytes;  // 64 KB
 constexpr int kNSlot = 3;
-constexpr int kQGroupBytes = 16 * kD * 2;   // 8 KB: 16 rows (12 heads + 4 pad) x 256
-constexpr int kQBytes = 2 * kQGroupBytes;
-constexpr int kPBytes = 16 * kTileTok * 2;  // 4 KB: P^T, 16 heads x 128 keys
+constexpr int kQRows = 32;                      // 24 heads + 8 pad
+constexpr int kQChunk = kQRows * 128;           // 4 KB: 64 d-columns of Q
+constexpr int kQBytes = 4 * kQChunk;            // 16 KB
+constexpr int kPChunk = kQRows * 128;           // 4 KB: P^T, 32 heads x 64 rows
+constexpr int kPBytes = 2 * kPChunk;            // 8 KB: 32 heads x 128 rows
 constexpr int kNP = 2;
 constexpr int kAttThreads = 192;
-constexpr uint32_t kSCol = 0, kOCol = 256, kTmemCols = 512;
+constexpr uint32_t kSCol = 0, kOCol = 64, kTmemCols = 128;  // S: 2 x 32 cols, O^T: 2 halves x 32
+constexpr float kRescaleLog2 = 8.f;             // lazy-rescale threshold (probability 2^8)
 
 struct AttShared {
     uint64_t slot_full[kNSlot], slot_empty[kNSlot];
     uint64_t q_full, q_empty;
-    uint64_t s_full, o_full;
+    uint64_t s_full[2], s_empty[2];
     uint64_t p_full[kNP], p_empty[kNP];
+    uint64_t pv_done;
     uint32_t tmem_base;
     int abort_flag;
-    float red_max[4][16];
-    float red_sum[4][16];
+    float red_max[2][4][2][kGrp];  // [tile parity][quad][group][head]
+    float red_sum[4][2][kGrp];
 };
 
 constexpr int kOffQ = kNSlot * kSlotBytes;
@@ -67,7 +76,6 @@ struct RowInfo {
     int s;
     int64_t t, bt, tok_base;
     int nsel, tile0, tile1;
-    bool ok;
 };
 
 __device__ __forceinline__ RowInfo row_info(int64_t item, int nsplit, int64_t row_begin,
@@ -86,18 +94,30 @@ __device__ __forceinline__ RowInfo row_info(int64_t item, int nsplit, int64_t ro
         ri.s = (int)ri.row;
         ri.t = (int64_t)cu_k[ri.s + 1] - cu_k[ri.s] - 1;
     }
-    ri.ok = ri.t >= 0;
-    ri.bt = ri.ok ? ri.t / r : 0;
+    const bool ok = ri.t >= 0;
+    ri.bt = ok ? ri.t / r : 0;
     ri.tok_base = cu_k[ri.s];
     const int64_t nsel = ri.bt + 1 < kb ? ri.bt + 1 : kb;
     ri.nsel = (int)nsel;
-    const int ntiles = (int)((nsel + kBlkPerTile - 1) / kBlkPerTile);
-    const int max_tiles = (kb + kBlkPerTile - 1) / kBlkPerTile;
+    const int ntiles = (int)((nsel + kBlkTile - 1) / kBlkTile);
+    const int max_tiles = (kb + kBlkTile - 1) / kBlkTile;
     const int tps = (max_tiles + nsplit - 1) / nsplit;
     ri.tile0 = sp * tps;
     ri.tile1 = ri.tile0 + tps < ntiles ? ri.tile0 + tps : ntiles;
-    if (!ri.ok) ri.tile1 = ri.tile0;
+    if (!ok) ri.tile1 = ri.tile0;
     return ri;
+}
+
+// block id of selection slot bi of a row: -1 for padding or an id outside 0 .. b_t
+__device__ __forceinline__ int32_t fetch_block(const int32_t *sel, const RowInfo &ri, int kb, int bi)
+{
+    if (bi >= ri.nsel) return -1;
+    const int32_t blk = __ldg(sel + ri.row * kb + bi);
+    if (blk < 0 || blk > ri.bt) {
+        set_device_status(QSA_ERR_DEVICE_CHECK);
+        return -1;
+    }
+    return blk;
 }
 
 __device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -106,6 +126,28 @@ __device__ __forceinline__ void st_shared_b16(uint32_t addr, uint16_t v)
 {
     asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0],"
+        " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16,"
+        " %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+          "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+          "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+          "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+          "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+          "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+          "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+          "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+          "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+          "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+          "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kAttThreads, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
@@ -130,15 +172,22 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         }
         mbar_init(&sh->q_full, 1);
         mbar_init(&sh->q_empty, 1);
-        mbar_init(&sh->s_full, 1);
-        mbar_init(&sh->o_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sh->s_full[i], 1);
+            mbar_init(&sh->s_empty[i], 128);
+        }
         for (int i = 0; i < kNP; ++i) {
             mbar_init(&sh->p_full[i], 128);
             mbar_init(&sh->p_empty[i], 1);
         }
+        mbar_init(&sh->pv_done, 1);
         sh->abort_flag = 0;
         fence_barrier_init();
     }
+    // P^T entries of the other KV group and of the pad heads stay zero for good
+    for (int i = threadIdx.x; i < kNP * kPBytes / 16; i += kAttThreads)
+        reinterpret_cast<uint4 *>(sP)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
     if (warp == 1) {
         tmem_alloc(&sh->tmem_base, kTmemCols);
         tmem_relinquish();
@@ -158,46 +207,50 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         }
         uint32_t slot_it = 0, q_it = 0;
         bool ok = true;
+        auto issue = [&](const CUtensorMap *map, const RowInfo &ri, int32_t blk) -> bool {
+            const uint32_t st = slot_it % kNSlot, round = slot_it / kNSlot;
+            bool good = true;
+            if (lane == 0) {
+                good = mbar_wait(&sh->slot_empty[st], (round & 1) ^ 1, abort_flag);
+                if (good) mbar_arrive_expect_tx(&sh->slot_full[st], kSlotBytes);
+            }
+            good = __shfl_sync(0xffffffffu, good, 0);
+            if (!good) return false;
+            if (lane < kBlkTile) {
+                // rows (token, group) of the block; padding reads an out-of-range box (zeros)
+                const int32_t y = blk >= 0 ? (int32_t)((ri.tok_base + (int64_t)blk * r) * kHKV) : -8;
+                tma_load_3d(sSlot + st * kSlotBytes + lane * kBlockBytes, map, &sh->slot_full[st], 0, y, 0);
+            }
+            ++slot_it;
+            return true;
+        };
         for (int64_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
             const RowInfo ri = row_info(item, nsplit, row_begin, cu_q, cu_k, batch, kb, r);
             if (ri.tile0 >= ri.tile1) continue;
+            int32_t b0 = -1, b1 = -1;
+            if (lane < kBlkTile) {
+                b0 = fetch_block(sel, ri, kb, ri.tile0 * kBlkTile + lane);
+                if (ri.tile0 + 1 < ri.tile1) b1 = fetch_block(sel, ri, kb, (ri.tile0 + 1) * kBlkTile + lane);
+            }
             if (lane == 0) {
                 ok = mbar_wait(&sh->q_empty, (q_it & 1) ^ 1, abort_flag);
                 if (ok) {
                     mbar_arrive_expect_tx(&sh->q_full, kQBytes);
-                    for (int g = 0; g < 2; ++g)
-                        for (int c = 0; c < 4; ++c)
-                            tma_load_2d(sQ + g * kQGroupBytes + c * 2048, &map_q, &sh->q_full, c * 64,
-                                        (int32_t)(ri.row * kHQ + kGrp * g));
+                    for (int c = 0; c < 4; ++c)
+                        tma_load_2d(sQ + c * kQChunk, &map_q, &sh->q_full, c * 64, (int32_t)(ri.row * kHQ));
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             ++q_it;
-            for (int g = 0; ok && g < 2; ++g) {
-                for (int phase = 0; ok && phase < 2; ++phase) {
-                    const CUtensorMap *map = phase == 0 ? &map_k : &map_v;
-                    for (int j = ri.tile0; j < ri.tile1; ++j) {
-                        const uint32_t st = slot_it % kNSlot, round = slot_it / kNSlot;
-                        if (lane == 0) {
-                            ok = mbar_wait(&sh->slot_empty[st], (round & 1) ^ 1, abort_flag);
-                            if (ok) mbar_arrive_expect_tx(&sh->slot_full[st], kSlotBytes);
-                        }
-                        ok = __shfl_sync(0xffffffffu, ok, 0);
-                        if (!ok) break;
-                        const int bi = j * kBlkPerTile + lane;
-                        int32_t blk = bi < ri.nsel ? __ldg(sel + ri.row * kb + bi) : -1;
-                        if (bi < ri.nsel && (blk < 0 || blk > ri.bt)) {
-                            set_device_status(QSA_ERR_DEVICE_CHECK);
-                            blk = -1;
-                        }
-                        const int32_t z = blk >= 0 ? (int32_t)(ri.tok_base + (int64_t)blk * r) : -4;
-                        uint8_t *dst = sSlot + st * kSlotBytes + lane * 512;
-#pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            tma_load_3d(dst + c * kChunk, map, &sh->slot_full[st], c * 64, g, z);
-                        ++slot_it;
-                    }
-                }
+            if (!ok) break;
+            ok = issue(&map_k, ri, b0);
+            for (int j = ri.tile0; ok && j < ri.tile1; ++j) {
+                int32_t b2 = -1;
+                if (lane < kBlkTile && j + 2 < ri.tile1) b2 = fetch_block(sel, ri, kb, (j + 2) * kBlkTile + lane);
+                if (j + 1 < ri.tile1) ok = issue(&map_k, ri, b1);
+                if (ok) ok = issue(&map_v, ri, b0);
+                b0 = b1;
+                b1 = b2;
             }
         }
         if (!ok && lane == 0) {
@@ -207,78 +260,80 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     } else if (warp == 1) {
         // ======================= MMA issuer (one thread) =======================
         if (elect_one()) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 16, 0, 0);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 16, 1, 0);
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, kQRows, 0, 0);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kQRows, 1, 0);
             const uint32_t slot_addr = smem_u32(sSlot), q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
-            uint32_t slot_it = 0, q_it = 0, p_it = 0;
+            uint32_t slot_it = 0, q_it = 0, s_it = 0, p_it = 0;
             bool ok = true;
+            auto do_pv = [&](bool first) -> bool {
+                const uint32_t st = slot_it % kNSlot, round = slot_it / kNSlot;
+                const uint32_t pb = p_it % kNP, pround = p_it / kNP;
+                if (!mbar_wait(&sh->slot_full[st], round & 1, abort_flag)) return false;
+                if (!mbar_wait(&sh->p_full[pb], pround & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t a0 = slot_addr + st * kSlotBytes;
+                const uint32_t b0 = p_addr + pb * kPBytes;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                    for (int ks = 0; ks < kRowsTile / 16; ++ks) {
+                        // V^T, MN-major: 64-d runs at LBO 1 KB (chunks of a block), 8-row groups at SBO 4 KB
+                        const uint64_t ad = sdesc_sw128(a0 + (2 * ks) * kBlockBytes + half * 2048, 1024, kBlockBytes);
+                        const uint64_t bd = sdesc_sw128(b0 + (ks >> 2) * kPChunk + (ks & 3) * 32, 16, 1024);
+                        mma_bf16_ss(tmem + kOCol + half * 32, ad, bd, idesc_pv, (first && ks == 0) ? 0u : 1u);
+                    }
+                }
+                mma_commit(&sh->slot_empty[st]);
+                mma_commit(&sh->p_empty[pb]);
+                mma_commit(&sh->pv_done);
+                ++slot_it;
+                ++p_it;
+                return true;
+            };
             for (int64_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
                 const RowInfo ri = row_info(item, nsplit, row_begin, cu_q, cu_k, batch, kb, r);
                 if (ri.tile0 >= ri.tile1) continue;
                 ok = mbar_wait(&sh->q_full, q_it & 1, abort_flag);
                 ++q_it;
-                for (int g = 0; ok && g < 2; ++g) {
-                    // S^T tiles
-                    for (int j = ri.tile0; ok && j < ri.tile1; ++j) {
-                        const uint32_t st = slot_it % kNSlot, round = slot_it / kNSlot;
-                        if (!(ok = mbar_wait(&sh->slot_full[st], round & 1, abort_flag))) break;
-                        tc_fence_after();
-                        const uint32_t a0 = slot_addr + st * kSlotBytes;
-                        const uint32_t b0 = q_addr + g * kQGroupBytes;
-                        const uint32_t d = tmem + kSCol + (j - ri.tile0) * 16;
+                const int nt = ri.tile1 - ri.tile0;
+                for (int jl = 0; ok && jl < nt; ++jl) {
+                    const uint32_t st = slot_it % kNSlot, round = slot_it / kNSlot;
+                    const uint32_t sb = s_it & 1, sround = s_it >> 1;
+                    if (!(ok = mbar_wait(&sh->slot_full[st], round & 1, abort_flag))) break;
+                    if (!(ok = mbar_wait(&sh->s_empty[sb], (sround & 1) ^ 1, abort_flag))) break;
+                    tc_fence_after();
+                    const uint32_t a0 = slot_addr + st * kSlotBytes;
 #pragma unroll
-                        for (int ks = 0; ks < kD / 16; ++ks) {
-                            const uint32_t off = (ks & 3) * 32;
-                            const uint64_t ad = sdesc_sw128(a0 + (ks >> 2) * kChunk + off, 16, 1024);
-                            const uint64_t bd = sdesc_sw128(b0 + (ks >> 2) * 2048 + off, 16, 1024);
-                            mma_bf16_ss(d, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
-                        }
-                        mma_commit(&sh->slot_empty[st]);
-                        ++slot_it;
+                    for (int ks = 0; ks < kD / 16; ++ks) {
+                        const uint32_t off = (ks & 3) * 32;
+                        const uint64_t ad = sdesc_sw128(a0 + (ks >> 2) * 1024 + off, 16, kBlockBytes);
+                        const uint64_t bd = sdesc_sw128(q_addr + (ks >> 2) * kQChunk + off, 16, 1024);
+                        mma_bf16_ss(tmem + kSCol + sb * 32, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
                     }
-                    if (!ok) break;
-                    if (g == 1) mma_commit(&sh->q_empty);
-                    mma_commit(&sh->s_full);
-                    // O^T += V^T P^T
-                    for (int j = ri.tile0; ok && j < ri.tile1; ++j) {
-                        const uint32_t st = slot_it % kNSlot, round = slot_it / kNSlot;
-                        const uint32_t pb = p_it % kNP, pround = p_it / kNP;
-                        if (!(ok = mbar_wait(&sh->slot_full[st], round & 1, abort_flag))) break;
-                        if (!(ok = mbar_wait(&sh->p_full[pb], pround & 1, abort_flag))) break;
-                        tc_fence_after();
-                        const uint32_t a0 = slot_addr + st * kSlotBytes;
-                        const uint32_t b0 = p_addr + pb * kPBytes;
-#pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-                            const uint32_t d = tmem + kOCol + g * 32 + half * 16;
-#pragma unroll
-                            for (int ks = 0; ks < kTileTok / 16; ++ks) {
-                                const uint64_t ad = sdesc_sw128(a0 + (2 * half) * kChunk + ks * 2048, kChunk, 1024);
-                                const uint64_t bd = sdesc_sw128(b0 + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024);
-                                mma_bf16_ss(d, ad, bd, idesc_pv, (j > ri.tile0 || ks > 0) ? 1u : 0u);
-                            }
-                        }
-                        mma_commit(&sh->slot_empty[st]);
-                        mma_commit(&sh->p_empty[pb]);
-                        ++slot_it;
-                        ++p_it;
-                    }
-                    if (!ok) break;
-                    mma_commit(&sh->o_full);
+                    mma_commit(&sh->slot_empty[st]);
+                    mma_commit(&sh->s_full[sb]);
+                    ++slot_it;
+                    ++s_it;
+                    if (jl == nt - 1) mma_commit(&sh->q_empty);
+                    if (jl >= 1) ok = do_pv(jl == 1);
                 }
+                if (ok) ok = do_pv(nt == 1);
             }
         }
     } else {
         // ======================= softmax + epilogue (warps 2..5) =======================
         const int quad = warp & 3;
-        const int key = quad * 32 + lane;           // TMEM lane = key within a tile
+        const int R = quad * 32 + lane;               // TMEM lane: row of the tile
+        const int blk_slot = R >> 3;                  // block within the tile
+        const int tok_in_blk = (R >> 1) & 3;
+        const int g = R & 1;                          // KV group of this row
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         const float c2 = scale * 1.4426950408889634f;
+        const float rescale_raw = kRescaleLog2 / c2;
         const uint32_t p_addr = smem_u32(sP);
-        const int kc64 = key & 63;
-        const uint32_t p_key_off = (key >> 6) * 2048 + (kc64 & 7) * 2;
-        const int p_unit = kc64 >> 3;
-        uint32_t p_it = 0, grp_it = 0;
+        const uint32_t p_row_off = (R >> 6) * kPChunk + (R & 7) * 2;
+        const int p_unit = (R & 63) >> 3;
+        uint32_t p_it = 0, s_it = 0, tile_it = 0;
         bool ok = true;
         for (int64_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
             const RowInfo ri = row_info(item, nsplit, row_begin, cu_q, cu_k, batch, kb, r);
@@ -287,125 +342,167 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             if (ri.tile0 >= ri.tile1) {
                 if (nsplit > 1) {  // empty split: neutral partial state
                     float *part = ws + ((row_local * nsplit + sp) * kHQ) * kD;
-                    for (int x = key; x < kHQ * kD; x += 128) part[x] = 0.f;
+                    for (int x = R; x < kHQ * kD; x += 128) part[x] = 0.f;
                     float *lp = ws + (size_t)n_items * kHQ * kD + (row_local * nsplit + sp) * kHQ;
-                    if (key < kHQ) lp[key] = -INFINITY;
+                    if (R < kHQ) lp[R] = -INFINITY;
                 }
                 continue;
             }
-            // key validity per tile (bit j - tile0): selected block present, token <= t
-            uint32_t vmask = 0;
-            for (int j = ri.tile0; j < ri.tile1; ++j) {
-                const int bi = j * kBlkPerTile + (key >> 2);
-                if (bi < ri.nsel) {
-                    const int32_t blk = __ldg(sel + ri.row * kb + bi);
-                    const int64_t tok = (int64_t)blk * r + (key & 3);
-                    if (blk >= 0 && blk <= ri.bt && tok <= ri.t) vmask |= 1u << (j - ri.tile0);
-                }
-            }
             const int nt = ri.tile1 - ri.tile0;
-            for (int g = 0; ok && g < 2; ++g) {
-                if (!(ok = mbar_wait(&sh->s_full, grp_it & 1, abort_flag))) break;
+            float m[kHQ];                             // running max per head (raw logits), identical in all threads
+            float l[kGrp];                            // this row's share of the row sums, own group's heads
+#pragma unroll
+            for (int h = 0; h < kGrp; ++h) l[h] = 0.f;
+#pragma unroll
+            for (int h = 0; h < kHQ; ++h) m[h] = 0.f;
+            int32_t blk_next = fetch_block(sel, ri, kb, ri.tile0 * kBlkTile + blk_slot);
+            for (int jl = 0; ok && jl < nt; ++jl) {
+                const int32_t blk = blk_next;
+                if (jl + 1 < nt) blk_next = fetch_block(sel, ri, kb, (ri.tile0 + jl + 1) * kBlkTile + blk_slot);
+                const bool valid = blk >= 0 && (int64_t)blk * r + tok_in_blk <= ri.t;
+                const uint32_t sb = s_it & 1, sround = s_it >> 1;
+                if (!(ok = mbar_wait(&sh->s_full[sb], sround & 1, abort_flag))) break;
                 tc_fence_after();
-                float m[16];
-#pragma unroll
-                for (int h = 0; h < 16; ++h) m[h] = -INFINITY;
-                for (int jl = 0; jl < nt; ++jl) {
-                    float s[16];
-                    tmem_ld16(tmem + lane_addr + kSCol + jl * 16, s);
-                    tmem_wait_ld();
-                    if (vmask & (1u << jl)) {
-#pragma unroll
-                        for (int h = 0; h < 16; ++h) m[h] = fmaxf(m[h], s[h]);
-                    }
-                }
-#pragma unroll
-                for (int h = 0; h < 16; ++h) {
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) m[h] = fmaxf(m[h], __shfl_xor_sync(0xffffffffu, m[h], off));
-                }
-                if (lane == 0) {
-#pragma unroll
-                    for (int h = 0; h < 16; ++h) sh->red_max[quad][h] = m[h];
-                }
-                softmax_bar();
-#pragma unroll
-                for (int h = 0; h < 16; ++h) {
-                    float x = fmaxf(fmaxf(sh->red_max[0][h], sh->red_max[1][h]), fmaxf(sh->red_max[2][h], sh->red_max[3][h]));
-                    m[h] = (x == -INFINITY) ? 0.f : x;
-                }
-                float l[16];
-#pragma unroll
-                for (int h = 0; h < 16; ++h) l[h] = 0.f;
-                for (int jl = 0; ok && jl < nt; ++jl) {
-                    const uint32_t pb = p_it % kNP, pround = p_it / kNP;
-                    if (!(ok = mbar_wait(&sh->p_empty[pb], (pround & 1) ^ 1, abort_flag))) break;
-                    float s[16];
-                    tmem_ld16(tmem + lane_addr + kSCol + jl * 16, s);
-                    tmem_wait_ld();
-                    const bool valid = vmask & (1u << jl);
-                    const uint32_t pbase = p_addr + pb * kPBytes + p_key_off;
-#pragma unroll
-                    for (int h = 0; h < 16; ++h) {
-                        const float p = valid ? exp2f((s[h] - m[h]) * c2) : 0.f;
-                        l[h] += p;
-                        const uint32_t addr = pbase + (h >> 3) * 1024 + (h & 7) * 128 + ((p_unit ^ (h & 7)) << 4);
-                        st_shared_b16(addr, __bfloat16_as_ushort(__float2bfloat16_rn(p)));
-                    }
-                    fence_proxy_async_smem();
-                    tc_fence_before();
-                    mbar_arrive(&sh->p_full[pb]);
-                    ++p_it;
-                }
-                if (!ok) break;
-#pragma unroll
-                for (int h = 0; h < 16; ++h) {
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) l[h] += __shfl_xor_sync(0xffffffffu, l[h], off);
-                }
-                if (lane == 0) {
-#pragma unroll
-                    for (int h = 0; h < 16; ++h) sh->red_sum[quad][h] = l[h];
-                }
-                softmax_bar();
-                float inv[16];
-                float my_lse = 0.f;
-#pragma unroll
-                for (int h = 0; h < 16; ++h) {
-                    const float L = sh->red_sum[0][h] + sh->red_sum[1][h] + sh->red_sum[2][h] + sh->red_sum[3][h];
-                    inv[h] = L > 0.f ? 1.f / L : 0.f;
-                    if (key == h) my_lse = m[h] * scale + logf(L);
-                }
-                if (!(ok = mbar_wait(&sh->o_full, grp_it & 1, abort_flag))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float o[16];
-                    tmem_ld16(tmem + lane_addr + kOCol + g * 32 + half * 16, o);
-                    tmem_wait_ld();
-                    const int d = half * 128 + key;
-                    if (nsplit == 1) {
-                        __nv_bfloat16 *dst = out + (ri.row * kHQ + g * kGrp) * kD + d;
-#pragma unroll
-                        for (int h = 0; h < kGrp; ++h) dst[h * kD] = __float2bfloat16_rn(o[h] * inv[h]);
-                    } else {
-                        float *dst = ws + ((row_local * nsplit + sp) * kHQ + g * kGrp) * kD + d;
-#pragma unroll
-                        for (int h = 0; h < kGrp; ++h) dst[h * kD] = o[h] * inv[h];
-                    }
-                }
-                if (key < kGrp) {
-                    if (nsplit == 1) {
-                        if (lse_out != nullptr) lse_out[ri.row * kHQ + g * kGrp + key] = my_lse;
-                    } else {
-                        float *lp = ws + (size_t)n_items * kHQ * kD + (row_local * nsplit + sp) * kHQ;
-                        lp[g * kGrp + key] = my_lse;
-                    }
-                }
+                float s[32];
+                tmem_ld32(tmem + lane_addr + kSCol + sb * 32, s);
+                tmem_wait_ld();
                 tc_fence_before();
-                softmax_bar();  // red_* reuse by the next group
-                ++grp_it;
+                mbar_arrive(&sh->s_empty[sb]);
+                ++s_it;
+                float v[kGrp];
+#pragma unroll
+                for (int h = 0; h < kGrp; ++h) v[h] = valid ? (g ? s[kGrp + h] : s[h]) : -INFINITY;
+                // exact per-head tile max: lanes of equal parity hold the same group
+                float tm[kGrp];
+#pragma unroll
+                for (int h = 0; h < kGrp; ++h) {
+                    float x = v[h];
+                    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
+                    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
+                    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 4));
+                    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));
+                    tm[h] = x;
+                }
+                const int par = tile_it & 1;
+                if (lane < 2) {
+#pragma unroll
+                    for (int h = 0; h < kGrp; ++h) sh->red_max[par][quad][lane][h] = tm[h];
+                }
+                softmax_bar();
+                float tmax[kHQ];
+#pragma unroll
+                for (int h = 0; h < kHQ; ++h) {
+                    const int gg = h / kGrp, hh = h % kGrp;
+                    tmax[h] = fmaxf(fmaxf(sh->red_max[par][0][gg][hh], sh->red_max[par][1][gg][hh]),
+                                    fmaxf(sh->red_max[par][2][gg][hh], sh->red_max[par][3][gg][hh]));
+                }
+                ++tile_it;
+                if (jl == 0) {
+#pragma unroll
+                    for (int h = 0; h < kHQ; ++h) m[h] = tmax[h] == -INFINITY ? 0.f : tmax[h];
+                } else {
+                    bool need = false;
+#pragma unroll
+                    for (int h = 0; h < kHQ; ++h) need |= tmax[h] > m[h] + rescale_raw;
+                    if (need) {  // uniform: every thread computed the same maxima
+                        float f[32];
+#pragma unroll
+                        for (int h = 0; h < 32; ++h) f[h] = 1.f;
+#pragma unroll
+                        for (int h = 0; h < kHQ; ++h) {
+                            const float mn = fmaxf(m[h], tmax[h]);
+                            f[h] = exp2f((m[h] - mn) * c2);
+                            m[h] = mn;
+                        }
+#pragma unroll
+                        for (int h = 0; h < kGrp; ++h) l[h] *= g ? f[kGrp + h] : f[h];
+                        // O^T must be stable: wait for the previous PV, then scale it in TMEM
+                        if (!(ok = mbar_wait(&sh->pv_done, (p_it - 1) & 1, abort_flag))) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            float o[32];
+                            const uint32_t ta = tmem + lane_addr + kOCol + half * 32;
+                            tmem_ld32(ta, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int h = 0; h < 32; ++h) o[h] *= f[h];
+                            tmem_st32(ta, o);
+                        }
+                        tmem_wait_st();
+                    }
+                }
+                // P = exp(S - m) for the row's own-group heads; the rest of P^T stays zero
+                const uint32_t pb = p_it % kNP, pround = p_it / kNP;
+                if (!(ok = mbar_wait(&sh->p_empty[pb], (pround & 1) ^ 1, abort_flag))) break;
+                const uint32_t pbase = p_addr + pb * kPBytes + p_row_off;
+#pragma unroll
+                for (int h = 0; h < kGrp; ++h) {
+                    const float mh = g ? m[kGrp + h] : m[h];
+                    const float p = valid ? exp2f((v[h] - mh) * c2) : 0.f;
+                    l[h] += p;
+                    const int hq = g * kGrp + h;
+                    const uint32_t addr = pbase + (hq >> 3) * 1024 + (hq & 7) * 128 + ((p_unit ^ (hq & 7)) << 4);
+                    st_shared_b16(addr, __bfloat16_as_ushort(__float2bfloat16_rn(p)));
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&sh->p_full[pb]);
+                ++p_it;
             }
+            if (!ok) break;
+            // row sums: reduce the own-group heads over rows of equal parity, then over the 4 quads
+#pragma unroll
+            for (int h = 0; h < kGrp; ++h) {
+                float x = l[h];
+                x += __shfl_xor_sync(0xffffffffu, x, 16);
+                x += __shfl_xor_sync(0xffffffffu, x, 8);
+                x += __shfl_xor_sync(0xffffffffu, x, 4);
+                x += __shfl_xor_sync(0xffffffffu, x, 2);
+                l[h] = x;
+            }
+            if (lane < 2) {
+#pragma unroll
+                for (int h = 0; h < kGrp; ++h) sh->red_sum[quad][lane][h] = l[h];
+            }
+            softmax_bar();
+            float inv[kHQ];
+            float my_lse = 0.f;
+#pragma unroll
+            for (int h = 0; h < kHQ; ++h) {
+                const int gg = h / kGrp, hh = h % kGrp;
+                const float L = sh->red_sum[0][gg][hh] + sh->red_sum[1][gg][hh] + sh->red_sum[2][gg][hh] +
+                                sh->red_sum[3][gg][hh];
+                inv[h] = L > 0.f ? 1.f / L : 0.f;
+                if (R == h) my_lse = m[h] * scale + logf(L);
+            }
+            if (!(ok = mbar_wait(&sh->pv_done, (p_it - 1) & 1, abort_flag))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float o[32];
+                tmem_ld32(tmem + lane_addr + kOCol + half * 32, o);
+                tmem_wait_ld();
+                const int d = half * 128 + R;
+                if (nsplit == 1) {
+                    __nv_bfloat16 *dst = out + ri.row * kHQ * kD + d;
+#pragma unroll
+                    for (int h = 0; h < kHQ; ++h) dst[h * kD] = __float2bfloat16_rn(o[h] * inv[h]);
+                } else {
+                    float *dst = ws + ((row_local * nsplit + sp) * kHQ) * kD + d;
+#pragma unroll
+                    for (int h = 0; h < kHQ; ++h) dst[h * kD] = o[h] * inv[h];
+                }
+            }
+            if (R < kHQ) {
+                if (nsplit == 1) {
+                    if (lse_out != nullptr) lse_out[ri.row * kHQ + R] = my_lse;
+                } else {
+                    ws[(size_t)n_items * kHQ * kD + (row_local * nsplit + sp) * kHQ + R] = my_lse;
+                }
+            }
+            tc_fence_before();
+            softmax_bar();  // red_sum reuse by the next item
         }
     }
 
@@ -443,14 +540,19 @@ combine_kernel(const float *__restrict__ ws, int64_t n_items, int nsplit, __nv_b
 
 int min_nsplit(int kb)
 {
-    const int max_tiles = (kb + kBlkPerTile - 1) / kBlkPerTile;
-    return (max_tiles + kMaxTiles - 1) / kMaxTiles;  // a split holds at most kMaxTiles tiles
+    (void)kb;
+    return 1;  // the online softmax handles any budget in one pass
+}
+
+int max_nsplit(int kb)
+{
+    return (kb + kBlkTile - 1) / kBlkTile;  // at most one split per 64-token tile
 }
 
 int decode_nsplit(int batch, int kb)
 {
-    const int max_tiles = (kb + kBlkPerTile - 1) / kBlkPerTile;
-    int ns = min_nsplit(kb);
+    const int max_tiles = (kb + kBlkTile - 1) / kBlkTile;
+    int ns = 1;
     const int target = 2 * num_sms();
     while (ns * 2 <= max_tiles && (int64_t)batch * ns < target) ns *= 2;
     return ns;
@@ -465,21 +567,18 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream)
 {
     const int64_t rows = a.row_end - a.row_begin;
     if (rows <= 0) return cudaSuccess;
+    if (a.nsplit > 1 && a.ws == nullptr) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv;
-    // q as [rows_total * 24, 256]; k, v as [total_k][2][256] with a 64 x 1 x 4 box
-    if (!make_tmap_2d(&mq, a.q, kD, (uint64_t)a.total_q * kHQ, kD * 2, 64, 16)) return cudaErrorInvalidValue;
-    if (!make_tmap_3d(&mk, a.k, kD, kHKV, (uint64_t)a.total_k, kD * 2, kHKV * kD * 2, 64, 1, 4))
-        return cudaErrorInvalidValue;
-    if (!make_tmap_3d(&mv, a.v, kD, kHKV, (uint64_t)a.total_k, kD * 2, kHKV * kD * 2, 64, 1, 4))
-        return cudaErrorInvalidValue;
+    // q as [rows_total * 24, 256], 32-row boxes (24 heads + 8 rows of padding)
+    if (!make_tmap_2d(&mq, a.q, kD, (uint64_t)a.total_q * kHQ, kD * 2, 64, kQRows)) return cudaErrorInvalidValue;
+    // k, v as (64 d, token-row, 4 d-chunks) with strides (512 B, 128 B): one box = one micro-block
+    if (!make_tmap_3d(&mk, a.k, 64, (uint64_t)a.total_k * kHKV, 4, kD * 2, 128, 64, 8, 4)) return cudaErrorInvalidValue;
+    if (!make_tmap_3d(&mv, a.v, 64, (uint64_t)a.total_k * kHKV, 4, kD * 2, 128, 64, 8, 4)) return cudaErrorInvalidValue;
     static bool attr = false;
     if (!attr) {
         cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttSmem);
         attr = true;
     }
-    const int max_tiles = (a.kb + kBlkPerTile - 1) / kBlkPerTile;
-    if ((max_tiles + a.nsplit - 1) / a.nsplit > kMaxTiles) return cudaErrorInvalidValue;
-    if (a.nsplit > 1 && a.ws == nullptr) return cudaErrorInvalidValue;
     const int64_t n_items = rows * a.nsplit;
     int64_t grid = num_sms();
     if (grid > n_items) grid = n_items;

@@ -4,9 +4,16 @@
 // notes, section 6): kc[b] = RMSNorm(AvgPool(k_idx[b r .. b r + r - 1])).
 // Unit gain; eps from the config; QSA_COMPRESS_NO_NORM keeps the plain mean.
 //
-// HBM-bound: r x 256 B read and 256 B written per block.  One warp per block,
+// Output: a compensated bf16 pair per value, kc[b] = hi + lo with hi = bf16(x)
+// and lo = bf16(x - hi) (about 16 significant bits).  A plain bf16 kc moves the
+// indexer scores by up to a few percent where a dot product is small against
+// the vectors' norms, which changes top-k selections; the pair keeps the
+// scores within ~1e-5 of the fp32 value while the indexer still runs bf16
+// tensor-core MMAs (one per plane).
+//
+// HBM-bound: r x 256 B read and 512 B written per block.  One warp per block,
 // each lane owns 4 consecutive dims (8-byte loads, 256 B per row per warp:
-// fully coalesced).  fp32 arithmetic, bf16 round-to-nearest-even store.
+// fully coalesced).  fp32 arithmetic, round-to-nearest-even stores.
 #include "kernels.cuh"
 
 namespace qsa {
@@ -71,12 +78,19 @@ compress_kernel(const __nv_bfloat16 *__restrict__ k_idx, const int32_t *__restri
 #pragma unroll
             for (int c = 0; c < 4; ++c) m[c] *= inv;
         }
-        __nv_bfloat162 o0 = __floats2bfloat162_rn(m[0], m[1]);
-        __nv_bfloat162 o1 = __floats2bfloat162_rn(m[2], m[3]);
-        uint2 packed;
-        packed.x = *reinterpret_cast<uint32_t *>(&o0);
-        packed.y = *reinterpret_cast<uint32_t *>(&o1);
-        *reinterpret_cast<uint2 *>(kc + ((int64_t)cu_blocks[s] + b) * 128 + lane * 4) = packed;
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(m[0], m[1]);
+        __nv_bfloat162 h1 = __floats2bfloat162_rn(m[2], m[3]);
+        const float2 fh0 = __bfloat1622float2(h0), fh1 = __bfloat1622float2(h1);
+        __nv_bfloat162 l0 = __floats2bfloat162_rn(m[0] - fh0.x, m[1] - fh0.y);
+        __nv_bfloat162 l1 = __floats2bfloat162_rn(m[2] - fh1.x, m[3] - fh1.y);
+        uint2 hi, lo;
+        hi.x = *reinterpret_cast<uint32_t *>(&h0);
+        hi.y = *reinterpret_cast<uint32_t *>(&h1);
+        lo.x = *reinterpret_cast<uint32_t *>(&l0);
+        lo.y = *reinterpret_cast<uint32_t *>(&l1);
+        __nv_bfloat16 *dst = kc + ((int64_t)cu_blocks[s] + b) * 256 + lane * 4;
+        *reinterpret_cast<uint2 *>(dst) = hi;
+        *reinterpret_cast<uint2 *>(dst + 128) = lo;
     }
 }
 

@@ -9,9 +9,11 @@
 // Prefill path (index_tc_kernel): a causal GEMM on the 5th-generation tensor
 // cores.  A CTA owns 32 consecutive query rows = 128 A-rows (token-major,
 // head-minor, exactly the q_idx memory order), loaded once by TMA.  It walks
-// the kc blocks below its causal bound in N-tiles of 128 blocks:
-//   warp 0      TMA producer (kc tiles, 4-stage ring, 128-byte swizzle)
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer (M128 N128 K16 x 8)
+// the kc blocks below its causal bound in N-tiles of 128 blocks; kc holds a
+// compensated bf16 pair (hi, lo) per value, and both planes are multiplied
+// into the same fp32 accumulator:
+//   warp 0      TMA producer (kc hi+lo tiles, 3-stage ring, 128-byte swizzle)
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer (M128 N128 K16 x 16)
 //   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (double-buffered in
 //               TMEM so the next tile's MMAs overlap), ReLU * w, a 4-lane
 //               butterfly that sums the heads while scattering columns, and
@@ -21,8 +23,8 @@
 // Decode path (index_rowwise_kernel): one query row per sequence is a GEMV over
 // the kc cache -- HBM-bound, so it runs on CUDA cores: each warp streams 8 kc
 // rows with coalesced 8-byte loads, keeps its 4 heads' query slice in
-// registers, and reduces the 32 (block, head) partial dots with a 5-step
-// butterfly reduce-scatter.
+// registers, adds the hi and lo planes of kc in fp32, and reduces the 32
+// (block, head) partial dots with a 5-step butterfly reduce-scatter.
 #include "kernels.cuh"
 
 namespace qsa {
@@ -34,11 +36,11 @@ constexpr int kTokTile = 32;                  // query rows per CTA
 constexpr int kBM = kTokTile * 4;             // A rows (token x head)
 constexpr int kBN = 128;                      // kc blocks per N tile
 constexpr int kIdxDim = 128;
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kChunkA = kBM * 128;            // bytes of one 64-column swizzled chunk of A
 constexpr int kChunkB = kBN * 128;
 constexpr int kABytes = 2 * kChunkA;          // 32 KB
-constexpr int kBBytes = 2 * kChunkB;          // 32 KB per stage
+constexpr int kBBytes = 4 * kChunkB;          // 64 KB per stage: hi and lo planes
 constexpr int kIdxThreads = 192;
 constexpr int kIdxSmem = kABytes + kStages * kBBytes + 1024 /*barriers*/ + 1024 /*align slack*/;
 
@@ -151,7 +153,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     if (!mbar_wait(&sh->empty[st], (round & 1) ^ 1, abort_flag)) { ok = false; break; }
                     mbar_arrive_expect_tx(&sh->full[st], kBBytes);
                     const int32_t y = (int32_t)(seg.kc_base + (int64_t)n * kBN);
-                    for (int c = 0; c < 2; ++c)
+                    for (int c = 0; c < 4; ++c)
                         tma_load_2d(sB + st * kBBytes + c * kChunkB, &map_kc, &sh->full[st], c * 64, y);
                 }
             }
@@ -179,9 +181,10 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     tc_fence_after();
                     const uint32_t d = tmem + acc * kBN;
 #pragma unroll
-                    for (int ks = 0; ks < kIdxDim / 16; ++ks) {
-                        const uint32_t koff = (ks & 3) * 32;
-                        const uint64_t ad = sdesc_sw128(a_addr + (ks >> 2) * kChunkA + koff, 16, 1024);
+                    for (int ks = 0; ks < 2 * kIdxDim / 16; ++ks) {  // hi plane, then lo plane
+                        const int ka = ks & 7;                    // k-step within the 128 dims
+                        const uint32_t koff = (ka & 3) * 32;
+                        const uint64_t ad = sdesc_sw128(a_addr + (ka >> 2) * kChunkA + koff, 16, 1024);
                         const uint64_t bd = sdesc_sw128(b_addr + st * kBBytes + (ks >> 2) * kChunkB + koff, 16, 1024);
                         mma_bf16_ss(d, ad, bd, idesc, ks > 0 ? 1u : 0u);
                     }
@@ -304,21 +307,26 @@ index_rowwise_kernel(const __nv_bfloat16 *__restrict__ q_idx, const float *__res
         q[h][0] = a.x; q[h][1] = a.y; q[h][2] = b.x; q[h][3] = b.y;
     }
     const float wv = __ldg(w + i * 4 + (lane & 3));
-    const __nv_bfloat16 *kbase = kc + (int64_t)cu_blocks[s] * 128 + lane * 4;
+    const __nv_bfloat16 *kbase = kc + (int64_t)cu_blocks[s] * 256 + lane * 4;
     float *srow = scores + (int64_t)blockIdx.y * ld;
 
     for (int64_t b0 = c0 + warp * 8; b0 < c1; b0 += kRowWarps * 8) {
-        uint2 raw[8];
+        uint2 raw[8], rlo[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int64_t b = b0 + j;
-            raw[j] = (b < c1) ? __ldg(reinterpret_cast<const uint2 *>(kbase + b * 128)) : make_uint2(0u, 0u);
+            const bool in = b < c1;
+            raw[j] = in ? __ldg(reinterpret_cast<const uint2 *>(kbase + b * 256)) : make_uint2(0u, 0u);
+            rlo[j] = in ? __ldg(reinterpret_cast<const uint2 *>(kbase + b * 256 + 128)) : make_uint2(0u, 0u);
         }
         float v[32];  // v[j * 4 + h] = partial dot of block b0 + j with head h
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw[j].x));
             float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw[j].y));
+            const float2 al = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&rlo[j].x));
+            const float2 bl = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&rlo[j].y));
+            a.x += al.x; a.y += al.y; b.x += bl.x; b.y += bl.y;
 #pragma unroll
             for (int h = 0; h < 4; ++h)
                 v[j * 4 + h] = q[h][0] * a.x + q[h][1] * a.y + q[h][2] * b.x + q[h][3] * b.y;
@@ -350,7 +358,7 @@ cudaError_t launch_index_tc(const IndexArgs &a, cudaStream_t stream)
     if (rows <= 0 || a.kc_rows <= 0) return cudaSuccess;
     CUtensorMap mq, mk;
     if (!make_tmap_2d(&mq, a.q_idx, 128, (uint64_t)a.total_q * 4, 256, 64, kBM)) return cudaErrorInvalidValue;
-    if (!make_tmap_2d(&mk, a.kc, 128, (uint64_t)a.kc_rows, 256, 64, kBN)) return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&mk, a.kc, 256, (uint64_t)a.kc_rows, 512, 64, kBN)) return cudaErrorInvalidValue;
     static bool attr = false;
     if (!attr) {
         cudaFuncSetAttribute(index_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kIdxSmem);

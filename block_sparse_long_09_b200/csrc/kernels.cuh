@@ -66,6 +66,7 @@ struct AttnArgs {
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream);
 int min_nsplit(int kb);                         // splits needed so each holds <= 16 tiles
 int decode_nsplit(int batch, int kb);           // splits used by the decode call
+int max_nsplit(int kb);                         // upper bound of decode_nsplit over devices
 size_t split_workspace_bytes(int64_t rows, int nsplit);  // partial (o, lse) states
 
 struct DenseArgs {

@@ -127,13 +127,14 @@ def device_status(clear: bool = True) -> int:
 
 def compress_keys(k_idx, cu_seqlens_k, cu_blocks, kc=None, blk_begin=None, max_new_blocks: int = 0,
                   cfg: Optional[Config] = None, n_blocks: Optional[int] = None):
-    """kc[b] = RMSNorm(mean of the r indexer keys of block b) for every complete block."""
+    """kc[b] = RMSNorm(mean of the r indexer keys of block b) for every complete block,
+    stored as a compensated bf16 pair: kc has shape [n_blocks, 2, idx_dim] (hi, lo)."""
     cfg = _cfg(cfg)
     batch = cu_seqlens_k.numel() - 1
     if kc is None:
         if n_blocks is None:
             n_blocks = int(cu_blocks[-1].item())
-        kc = torch.empty((n_blocks, cfg.idx_dim), dtype=torch.bfloat16, device=k_idx.device)
+        kc = torch.empty((n_blocks, 2, cfg.idx_dim), dtype=torch.bfloat16, device=k_idx.device)
     _check(_lib.qsa_compress_keys(ctypes.byref(cfg), _p(k_idx), _p(cu_seqlens_k), _p(cu_blocks), batch,
                                   k_idx.shape[0], _p(blk_begin), max_new_blocks, _p(kc), _stream()),
            "qsa_compress_keys")
@@ -249,7 +250,7 @@ class Prefill:
             cb.append(cb[-1] + L // r)
         self.cu = torch.tensor(cu, dtype=torch.int32, device=self.device)
         self.cu_blocks = torch.tensor(cb, dtype=torch.int32, device=self.device)
-        self.kc = torch.empty((max(self.n_blocks, 1), self.cfg.idx_dim), dtype=torch.bfloat16, device=self.device)
+        self.kc = torch.empty((max(self.n_blocks, 1), 2, self.cfg.idx_dim), dtype=torch.bfloat16, device=self.device)
         self.scores = torch.empty((min(self.chunk, self.total), self.ld), dtype=torch.float32, device=self.device)
         self.sel = torch.empty((self.total, self.cfg.budget_blocks), dtype=torch.int32, device=self.device)
 

@@ -92,14 +92,18 @@ void qsa_config_init(qsa_config *cfg);
  * Key compressor -- pooled-key equation of section 6:
  *   kc[b] = RMSNorm( (1/r) * sum_{j<r} k_idx[b r + j] ),   unit gain, eps cfg->rms_eps
  * for every complete block b < floor(L_k,s / r) of every sequence (the mean
- * alone with QSA_COMPRESS_NO_NORM).  fp32 arithmetic, bf16 round-to-nearest store.
+ * alone with QSA_COMPRESS_NO_NORM).  fp32 arithmetic.  Each value x is stored as
+ * a compensated bf16 pair, hi = bf16(x) and lo = bf16(x - hi) (round to nearest
+ * even), so kc = hi + lo carries about 16 significant bits: bf16 alone shifts
+ * small indexer scores by percents and flips top-k choices.
  *   k_idx      [total_k, idx_dim] bf16   raw indexer keys (one shared key head)
  *   cu_seqlens_k, cu_blocks  [batch+1] int32
  *   total_k    host: rows of k_idx (bounds the launch)
  *   blk_begin  [batch] int32 or NULL.  NULL: every complete block is written.
  *              Otherwise only blocks [blk_begin[s], blk_begin[s] + max_new_blocks)
  *              that are complete (a decode step refreshes the blocks it completed).
- *   kc         [cu_blocks[batch], idx_dim] bf16, written.
+ *   kc         [cu_blocks[batch], 2, idx_dim] bf16, written: per block the hi
+ *              plane, then the lo plane.
  */
 qsa_status qsa_compress_keys(const qsa_config *cfg, const qsa_bf16 *k_idx,
                              const int32_t *cu_seqlens_k, const int32_t *cu_blocks,
@@ -110,9 +114,10 @@ qsa_status qsa_compress_keys(const qsa_config *cfg, const qsa_bf16 *k_idx,
  * Indexer scores -- indexer equation of section 6, with one weight per
  * (query, indexer head) (w = 1 gives the equation as printed):
  *   S[t, b] = sum_h w[t, h] * max(0, <q_idx[t, h, :], kc[b, :]>),   b < b_t
- * bf16 tensor-core products, fp32 accumulation and epilogue.
+ * bf16 tensor-core products (q_idx . hi + q_idx . lo), fp32 accumulation and epilogue.
  *   q_idx   [total_q, n_heads_idx, idx_dim] bf16;  w [total_q, n_heads_idx] fp32
- *   kc      [kc_rows, idx_dim] bf16 (the compressor's output; kc_rows = cu_blocks[batch])
+ *   kc      [kc_rows, 2, idx_dim] bf16 hi/lo pairs (the compressor's output; kc_rows =
+ *           cu_blocks[batch]); both planes enter the products
  *   rows    packed query rows [row_begin, row_end) are scored (a chunk of a prefill)
  *   scores  fp32, row i at scores + (i - row_begin) * ld; entries b < b_t(i) are
  *           written, entries b >= b_t(i) are left untouched.  ld >= every b_t(i).
@@ -154,9 +159,7 @@ qsa_status qsa_select_blocks(const qsa_config *cfg, const float *scores, int64_t
  *   o   [total_q, n_heads_q, head_dim] bf16 written for those rows
  *   lse [total_q, n_heads_q] fp32 natural-log sum-exp of the scaled logits, or NULL
  * A selected block id outside 0 .. b_t is skipped and flagged QSA_ERR_DEVICE_CHECK.
- * Workspace: none for k <= 512.  A larger budget is processed as k/512 partial
- * softmax states per row that a second kernel merges: pass a workspace of
- * qsa_workspace_size(cfg, QSA_OP_PREFILL, batch, row_end - row_begin, 0) bytes.
+ * Workspace: none (ws may be NULL).
  */
 qsa_status qsa_sparse_attn_prefill(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k,
                                    const qsa_bf16 *v, const int32_t *sel,
