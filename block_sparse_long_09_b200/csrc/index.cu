@@ -7,17 +7,22 @@
 // cost is O(n^2 / r) (the section's complexity equation).
 //
 // Prefill path (index_tc_kernel): a causal GEMM on the 5th-generation tensor
-// cores.  A CTA owns 32 consecutive query rows = 128 A-rows (token-major,
+// cores.  A CTA owns 64 consecutive query rows = 2 x 128 A-rows (token-major,
 // head-minor, exactly the q_idx memory order), loaded once by TMA.  It walks
 // the kc blocks below its causal bound in N-tiles of 128 blocks; kc holds a
 // compensated bf16 pair (hi, lo) per value, and both planes are multiplied
 // into the same fp32 accumulator:
-//   warp 0      TMA producer (kc hi+lo tiles, 3-stage ring, 128-byte swizzle)
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer (M128 N128 K16 x 16)
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (double-buffered in
-//               TMEM so the next tile's MMAs overlap), ReLU * w, a 4-lane
-//               butterfly that sums the heads while scattering columns, and
-//               coalesced fp32 stores of the b < b_t entries.
+//   warp 0      TMA producer (kc hi+lo tiles, 2-stage ring, 128-byte swizzle)
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer: two M128 N128
+//               accumulators (one per 32-row sub-tile) share each kc tile, so the
+//               L2 traffic of kc is halved against 32-row tiles
+//   warps 2..9  epilogue: tcgen05.ld of the fp32 accumulators (double-buffered in
+//               TMEM -- all 512 columns -- so the next tile's MMAs overlap), ReLU
+//               * w, a 4-lane butterfly that sums the heads while scattering
+//               columns, 128-byte-swizzled staging in shared memory and 32 x 32
+//               TMA bulk stores of the scores (scattered per-thread stores would
+//               saturate the L1 store path).  Tiles that straddle two sequences
+//               fall back to masked per-thread stores.
 // Tiles above the diagonal are never issued; heavy (late) row tiles launch first.
 //
 // Decode path (index_rowwise_kernel): one query row per sequence is a GEMV over
@@ -32,17 +37,20 @@ namespace qsa {
 namespace {
 
 // ------------------------------------------------------------------ tcgen05 path
-constexpr int kTokTile = 32;                  // query rows per CTA
-constexpr int kBM = kTokTile * 4;             // A rows (token x head)
+constexpr int kTokTile = 64;                  // query rows per CTA
+constexpr int kSubTok = 32;                   // query rows per A sub-tile
+constexpr int kBM = kSubTok * 4;              // A rows of a sub-tile (token x head) = MMA M
 constexpr int kBN = 128;                      // kc blocks per N tile
 constexpr int kIdxDim = 128;
-constexpr int kStages = 3;
-constexpr int kChunkA = kBM * 128;            // bytes of one 64-column swizzled chunk of A
-constexpr int kChunkB = kBN * 128;
-constexpr int kABytes = 2 * kChunkA;          // 32 KB
+constexpr int kStages = 2;
+constexpr int kChunkA = kBM * 128;            // 16 KB: one 64-column swizzled chunk of a sub-tile
+constexpr int kChunkB = kBN * 128;            // 16 KB
+constexpr int kABytes = 2 * 2 * kChunkA;      // 64 KB: two sub-tiles
 constexpr int kBBytes = 4 * kChunkB;          // 64 KB per stage: hi and lo planes
-constexpr int kIdxThreads = 192;
-constexpr int kIdxSmem = kABytes + kStages * kBBytes + 1024 /*barriers*/ + 1024 /*align slack*/;
+constexpr int kStgChunk = kSubTok * 128;      // 4 KB: 32 rows x 32 fp32 scores, swizzled
+constexpr int kStgBytes = 2 * 4 * kStgChunk;  // 32 KB: 2 sub-tiles x 4 column groups
+constexpr int kIdxThreads = 320;              // producer, MMA, 8 epilogue warps
+constexpr uint32_t kAccCols = 512;            // 2 buffers x 2 sub-tiles x 128 columns
 
 struct IdxShared {
     uint64_t full[kStages];
@@ -53,6 +61,8 @@ struct IdxShared {
     uint32_t tmem_base;
     int abort_flag;
 };
+
+constexpr int kIdxSmem = kABytes + kStages * kBBytes + kStgBytes + (int)sizeof(IdxShared) + 1024;
 
 struct Segment {
     int s;
@@ -92,8 +102,20 @@ struct SegIter {
     }
 };
 
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int32_t x, int32_t y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void sub_bar(int sub) { asm volatile("bar.sync %0, 128;" ::"r"(2 + sub) : "memory"); }
+
 __global__ void __launch_bounds__(kIdxThreads, 1)
 index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kc,
+                const __grid_constant__ CUtensorMap map_s, int use_tma_store,
                 const float *__restrict__ w, const int32_t *__restrict__ cu_q,
                 const int32_t *__restrict__ cu_k, const int32_t *__restrict__ cu_blocks, int batch,
                 int64_t row_begin, int64_t row_end, float *__restrict__ scores, int64_t ld, int r)
@@ -102,7 +124,8 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + kABytes;
-    IdxShared *sh = reinterpret_cast<IdxShared *>(smem + kABytes + kStages * kBBytes);
+    uint8_t *sStg = sB + kStages * kBBytes;
+    IdxShared *sh = reinterpret_cast<IdxShared *>(sStg + kStgBytes);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t ntile_rows = (row_end - row_begin + kTokTile - 1) / kTokTile;
@@ -118,13 +141,13 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         mbar_init(&sh->a_full, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sh->acc_full[i], 1);
-            mbar_init(&sh->acc_empty[i], 4);
+            mbar_init(&sh->acc_empty[i], 8);
         }
         sh->abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(&sh->tmem_base, 2 * kBN);
+        tmem_alloc(&sh->tmem_base, kAccCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -134,6 +157,8 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     volatile int *abort_flag = &sh->abort_flag;
 
     const int s0 = find_seq(cu_q, batch, m0);
+    // one sequence covers the whole tile: whole 32 x 32 score boxes can be stored by TMA
+    const bool single = use_tma_store && (int64_t)cu_q[s0 + 1] >= m1;
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -141,8 +166,10 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             tma_prefetch_desc(&map_q);
             tma_prefetch_desc(&map_kc);
             mbar_arrive_expect_tx(&sh->a_full, kABytes);
-            for (int c = 0; c < 2; ++c)
-                tma_load_2d(sA + c * kChunkA, &map_q, &sh->a_full, c * 64, (int32_t)(m0 * 4));
+            for (int sub = 0; sub < 2; ++sub)
+                for (int c = 0; c < 2; ++c)
+                    tma_load_2d(sA + (sub * 2 + c) * kChunkA, &map_q, &sh->a_full, c * 64,
+                                (int32_t)((m0 + sub * kSubTok) * 4));
             SegIter it{cu_q, cu_k, cu_blocks, batch, r, m0, m1, s0};
             Segment seg;
             uint32_t k = 0;
@@ -158,7 +185,6 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 }
             }
             if (!ok) {
-                // drain: wait (bounded) for the copies already issued into each stage
                 for (uint32_t j = (k > kStages ? k - kStages : 0); j < k; ++j)
                     mbar_wait(&sh->full[j % kStages], (j / kStages) & 1, nullptr);
             }
@@ -179,14 +205,17 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     if (!mbar_wait(&sh->acc_empty[acc], (use & 1) ^ 1, abort_flag)) { ok = false; break; }
                     if (!mbar_wait(&sh->full[st], round & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t d = tmem + acc * kBN;
 #pragma unroll
-                    for (int ks = 0; ks < 2 * kIdxDim / 16; ++ks) {  // hi plane, then lo plane
-                        const int ka = ks & 7;                    // k-step within the 128 dims
-                        const uint32_t koff = (ka & 3) * 32;
-                        const uint64_t ad = sdesc_sw128(a_addr + (ka >> 2) * kChunkA + koff, 16, 1024);
-                        const uint64_t bd = sdesc_sw128(b_addr + st * kBBytes + (ks >> 2) * kChunkB + koff, 16, 1024);
-                        mma_bf16_ss(d, ad, bd, idesc, ks > 0 ? 1u : 0u);
+                    for (int sub = 0; sub < 2; ++sub) {
+                        const uint32_t d = tmem + (acc * 2 + sub) * kBN;
+#pragma unroll
+                        for (int ks = 0; ks < 2 * kIdxDim / 16; ++ks) {  // hi plane, then lo plane
+                            const int ka = ks & 7;                    // k-step within the 128 dims
+                            const uint32_t koff = (ka & 3) * 32;
+                            const uint64_t ad = sdesc_sw128(a_addr + (sub * 2 + (ka >> 2)) * kChunkA + koff, 16, 1024);
+                            const uint64_t bd = sdesc_sw128(b_addr + st * kBBytes + (ks >> 2) * kChunkB + koff, 16, 1024);
+                            mma_bf16_ss(d, ad, bd, idesc, ks > 0 ? 1u : 0u);
+                        }
                     }
                     mma_commit(&sh->empty[st]);
                     mma_commit(&sh->acc_full[acc]);
@@ -194,15 +223,21 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             }
         }
     } else {
-        // ---------------- epilogue (warps 2..5) ----------------
+        // ---------------- epilogue (warps 2..9) ----------------
+        const int ew = warp - 2;
+        const int sub = ew >> 2;                   // A sub-tile
         const int quad = warp & 3;                 // TMEM lane quadrant this warp may read
-        const int row_in_tile = quad * 8 + (lane >> 2);
+        const int row_in_sub = quad * 8 + (lane >> 2);
         const int head = lane & 3;
-        const int64_t i = m0 + row_in_tile;        // packed query row of this lane
+        const int64_t i = m0 + sub * kSubTok + row_in_sub;  // packed query row of this lane
         const float wv = (i < m1) ? __ldg(w + i * 4 + head) : 0.f;
         const bool b0 = lane & 1, b1 = (lane >> 1) & 1;
         const int col_sub = (b0 ? 16 : 0) + (b1 ? 8 : 0);
         const bool vec_ok = (ld & 3) == 0;
+        const bool store_thread = (ew & 3) == 0 && lane == 0;  // issues this sub-tile's TMA stores
+        uint8_t *stg = sStg + sub * 4 * kStgChunk;
+        const uint32_t stg_row = (uint32_t)row_in_sub * 128;
+        const int unit0 = col_sub >> 2;            // first 16-byte unit of the 8 values
 
         SegIter it{cu_q, cu_k, cu_blocks, batch, r, m0, m1, s0};
         Segment seg;
@@ -221,10 +256,14 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 const uint32_t acc = k & 1, use = k >> 1;
                 if (!mbar_wait(&sh->acc_full[acc], use & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
+                if (single) {
+                    if (store_thread) bulk_wait_read0();  // staging free again
+                    sub_bar(sub);
+                }
 #pragma unroll 1
                 for (int c = 0; c < kBN / 32; ++c) {
                     float v[32];
-                    tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + acc * kBN + c * 32, v);
+                    tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (acc * 2 + sub) * kBN + c * 32, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] = wv * fmaxf(v[j], 0.f);
@@ -243,8 +282,14 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                         const float keep = b1 ? h16[j + 8] : h16[j];
                         h8[j] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
                     }
-                    const int64_t bcol = (int64_t)n * kBN + c * 32 + col_sub;
-                    if (row_in_seg) {
+                    if (single) {
+                        // 128-byte swizzled staging row: 16-byte unit u lands at u ^ (row & 7)
+                        uint8_t *base = stg + c * kStgChunk + stg_row;
+                        const int sw = row_in_sub & 7;
+                        *reinterpret_cast<float4 *>(base + (((unit0) ^ sw) << 4)) = make_float4(h8[0], h8[1], h8[2], h8[3]);
+                        *reinterpret_cast<float4 *>(base + (((unit0 + 1) ^ sw) << 4)) = make_float4(h8[4], h8[5], h8[6], h8[7]);
+                    } else if (row_in_seg) {
+                        const int64_t bcol = (int64_t)n * kBN + c * 32 + col_sub;
                         if (vec_ok && bcol + 8 <= bt) {
                             float4 *dst = reinterpret_cast<float4 *>(srow + bcol);
                             dst[0] = make_float4(h8[0], h8[1], h8[2], h8[3]);
@@ -259,15 +304,26 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh->acc_empty[acc]);
+                if (single) {
+                    fence_proxy_async_smem();
+                    sub_bar(sub);
+                    if (store_thread) {
+                        const int32_t y = (int32_t)(m0 + sub * kSubTok - row_begin);
+                        for (int c = 0; c < 4; ++c)
+                            tma_store_2d(&map_s, stg + c * kStgChunk, n * kBN + c * 32, y);
+                        bulk_commit();
+                    }
+                }
             }
         }
+        if (store_thread) bulk_wait0();
     }
 
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 2 * kBN);
+        tmem_dealloc(tmem, kAccCols);
     }
 }
 
@@ -356,9 +412,13 @@ cudaError_t launch_index_tc(const IndexArgs &a, cudaStream_t stream)
 {
     const int64_t rows = a.row_end - a.row_begin;
     if (rows <= 0 || a.kc_rows <= 0) return cudaSuccess;
-    CUtensorMap mq, mk;
+    CUtensorMap mq, mk, ms;
     if (!make_tmap_2d(&mq, a.q_idx, 128, (uint64_t)a.total_q * 4, 256, 64, kBM)) return cudaErrorInvalidValue;
     if (!make_tmap_2d(&mk, a.kc, 256, (uint64_t)a.kc_rows, 512, 64, kBN)) return cudaErrorInvalidValue;
+    // the scores of this call as an fp32 [rows, ld] tensor for 32 x 32 TMA stores (needs ld % 4 == 0)
+    int use_tma = ((a.ld & 3) == 0) && make_tmap_2d_f32(&ms, a.scores, (uint64_t)a.ld, (uint64_t)rows,
+                                                       (uint64_t)a.ld * 4, 32, 32);
+    if (!use_tma) ms = mq;  // unused
     static bool attr = false;
     if (!attr) {
         cudaFuncSetAttribute(index_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kIdxSmem);
@@ -366,7 +426,8 @@ cudaError_t launch_index_tc(const IndexArgs &a, cudaStream_t stream)
     }
     const int64_t tiles = (rows + kTokTile - 1) / kTokTile;
     index_tc_kernel<<<(unsigned)tiles, kIdxThreads, kIdxSmem, stream>>>(
-        mq, mk, a.w, a.cu_q, a.cu_k, a.cu_blocks, a.batch, a.row_begin, a.row_end, a.scores, a.ld, a.r);
+        mq, mk, ms, use_tma, a.w, a.cu_q, a.cu_k, a.cu_blocks, a.batch, a.row_begin, a.row_end, a.scores, a.ld,
+        a.r);
     return cudaGetLastError();
 }
 

@@ -84,6 +84,8 @@ cudaError_t launch_dense_attn(const DenseArgs &a, cudaStream_t stream);
 // tensor-map creation (host), defined in api.cu
 bool make_tmap_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
+bool make_tmap_2d_f32(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                      uint32_t box_inner, uint32_t box_outer);
 bool make_tmap_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
 int num_sms();

@@ -239,7 +239,7 @@ class Prefill:
         self.total = sum(self.seqlens)
         self.max_len = max(self.seqlens)
         self.n_blocks = sum(L // r for L in self.seqlens)
-        self.ld = max(1, (self.max_len - 1) // r)
+        self.ld = max(4, ((self.max_len - 1) // r + 3) // 4 * 4)  # a multiple of 4: whole-tile score stores
         self.chunk = int(chunk_rows)
         self.device = torch.device(device)
         cu = [0]

@@ -119,8 +119,9 @@ qsa_status qsa_compress_keys(const qsa_config *cfg, const qsa_bf16 *k_idx,
  *   kc      [kc_rows, 2, idx_dim] bf16 hi/lo pairs (the compressor's output; kc_rows =
  *           cu_blocks[batch]); both planes enter the products
  *   rows    packed query rows [row_begin, row_end) are scored (a chunk of a prefill)
- *   scores  fp32, row i at scores + (i - row_begin) * ld; entries b < b_t(i) are
- *           written, entries b >= b_t(i) are left untouched.  ld >= every b_t(i).
+ *   scores  fp32, row i at scores + (i - row_begin) * ld; entries b < b_t(i) hold
+ *           the scores, entries b_t(i) <= b < ld are unspecified (whole tiles are
+ *           stored when ld % 4 == 0).  ld >= every b_t(i).
  *   total_q host: rows of q_idx; max_len_q host: max over s of L_q,s (a launch hint:
  *           1 selects the one-row-per-sequence decode kernel)
  * Workspace: none (ws may be NULL).
