@@ -217,6 +217,34 @@ def run_qsa(args, rank, world, device):
         e2e = {"value": world * N_PREFILL / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps, "scope": "prefill 262144 via qsa.Prefill"}
 
+    # the build's dense causal attention on the same inputs (the pages' comparison)
+    dense = None
+    if args.dense:
+        cu_dec_q = torch.arange(DEC_BATCH + 1, dtype=torch.int32, device=device)
+        qsa.dense_attn_prefill(x.q, x.k, x.v, pre.cu, pre.cu, N_PREFILL, o=o, cfg=cfg, max_len_k=N_PREFILL)
+        dws = torch.empty((qsa.workspace_size(qsa.OP_DENSE, DEC_BATCH, DEC_BATCH, DEC_LEN, cfg),),
+                          dtype=torch.uint8, device=device)
+        qsa.dense_attn_prefill(d.q, d.k_cache, d.v_cache, cu_dec_q, cu_k, 1, o=dec_o, cfg=cfg, max_len_k=DEC_LEN,
+                               ws=dws)
+        torch.cuda.synchronize()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record(stream)
+        qsa.dense_attn_prefill(x.q, x.k, x.v, pre.cu, pre.cu, N_PREFILL, o=o, cfg=cfg, max_len_k=N_PREFILL)
+        e[1].record(stream)
+        for _ in range(5):
+            qsa.dense_attn_prefill(d.q, d.k_cache, d.v_cache, cu_dec_q, cu_k, 1, o=dec_o, cfg=cfg,
+                                   max_len_k=DEC_LEN, ws=dws)
+        e[2].record(stream)
+        torch.cuda.synchronize()
+        dp_ms = allmax(e[0].elapsed_time(e[1]))
+        dd_us = allmax(e[1].elapsed_time(e[2]) / 5 * 1e3)
+        dense_flops = 4.0 * 24 * 256 * (N_PREFILL * (N_PREFILL + 1) / 2)
+        dense = {"prefill_ms": dp_ms, "prefill_tokens_per_s": N_PREFILL / (dp_ms / 1e3),
+                 "prefill_tflops": dense_flops / (dp_ms / 1e3) / 1e12,
+                 "qsa_layer_speedup": dp_ms / prefill_ms, "qsa_attention_only_speedup": dp_ms / attn_ms,
+                 "decode_step_us": dd_us, "qsa_decode_speedup": dd_us / (dec_ms * 1e3),
+                 "pages_context": "7.6x prefill / 4.9x decode at 1M context, kernel level, hardware not stated"}
+
     sel_tok = selected_tokens(N_PREFILL)
     gather = gather_bytes_per_query(1) * sel_tok
     achieved = gather / (attn_ms / 1e3) / 1e9
@@ -245,6 +273,7 @@ def run_qsa(args, rank, world, device):
                      "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
                      "algorithmic_bytes": gather, "peak_kind": peak_kind + " (burst copy)"},
         "gpu_launches": args.steps * (launches_prefill + launches_decode),
+        "dense": dense,
         "e2e": e2e,
         "clocks": clk,
     }
@@ -335,6 +364,8 @@ def main():
     ap.add_argument("--impl", default="qsa", choices=["qsa", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", dest="dense", action="store_false",
+                    help="skip the dense causal-attention comparison")
     ap.add_argument("--profile-case", choices=["attn", "index", "select", "decode"], default=None,
                     help="run one small case for an ncu capture and exit")
     args = ap.parse_args()

@@ -146,13 +146,13 @@ const char *qsa_status_string(qsa_status s)
 
 size_t qsa_workspace_size(const qsa_config *cfg, int32_t op, int32_t batch, int64_t rows, int64_t max_len_k)
 {
-    (void)max_len_k;
     if (check_config(cfg) != QSA_OK || batch <= 0 || rows < 0) return 0;
     if (op == QSA_OP_DECODE) {
         const int ns = max_nsplit(cfg->budget_blocks);
         return split_workspace_bytes(batch, ns > 1 ? ns : 2);
     }
     if (op == QSA_OP_PREFILL) return split_workspace_bytes(rows, min_nsplit(cfg->budget_blocks));
+    if (op == QSA_OP_DENSE) return split_workspace_bytes(rows, dense_decode_nsplit(max_len_k, cfg->r));
     return 0;
 }
 
@@ -275,21 +275,33 @@ qsa_status qsa_sparse_attn_decode(const qsa_config *cfg, const qsa_bf16 *q, cons
 
 qsa_status qsa_dense_attn_prefill(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k, const qsa_bf16 *v,
                                   const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int32_t batch,
-                                  int64_t total_q, int64_t total_k, int32_t max_len_q, qsa_bf16 *o, float *lse,
-                                  void *stream)
+                                  int64_t total_q, int64_t total_k, int32_t max_len_q, int64_t max_len_k,
+                                  qsa_bf16 *o, float *lse, void *ws, size_t ws_bytes, void *stream)
 {
     qsa_status st = check_config(cfg);
     if (st != QSA_OK) return st;
-    if (batch <= 0 || total_q < 0 || total_k < 0 || max_len_q < 0 || cu_seqlens_q == nullptr ||
+    if (batch <= 0 || total_q < 0 || total_k < 0 || max_len_q < 0 || max_len_k < 0 || cu_seqlens_q == nullptr ||
         cu_seqlens_k == nullptr)
         return QSA_ERR_INVALID_ARG;
     if (total_q == 0) return QSA_OK;
     if (total_k == 0 || q == nullptr || k == nullptr || v == nullptr || o == nullptr || !al16(q) || !al16(k) ||
         !al16(v))
         return QSA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (max_len_q == 1) {
+        // one query per sequence: split-K flash decoding over every block (HBM-bound)
+        const int nsplit = dense_decode_nsplit(max_len_k, cfg->r);
+        if (nsplit > 1 && (ws == nullptr || ws_bytes < split_workspace_bytes(total_q, nsplit)))
+            return QSA_ERR_WORKSPACE_TOO_SMALL;
+        if (nsplit > 1 && !al16(ws)) return QSA_ERR_INVALID_ARG;
+        const int kb = (int)((max_len_k + cfg->r - 1) / cfg->r);
+        AttnArgs a{bf(q), bf(k), bf(v), nullptr, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, 0, total_q,
+                   bf(o), lse, static_cast<float *>(ws), nsplit, kb > 0 ? kb : 1, cfg->r, cfg->softmax_scale};
+        return cuda_status(launch_sparse_attn(a, s));
+    }
     DenseArgs a{bf(q), bf(k), bf(v), cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_len_q, bf(o), lse,
                 cfg->softmax_scale};
-    return cuda_status(launch_dense_attn(a, static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_dense_attn(a, s));
 }
 
 }  // extern "C"

@@ -32,6 +32,8 @@
 //      warps 2..5  softmax (thread = TMEM lane = (token, group) row) and the
 //                  epilogue (thread = d); split-K decode writes fp32 partial
 //                  states that combine_kernel merges.
+// Without a selection array the kernel attends to every block j <= t: that is
+// the dense flash-decoding baseline (one query per sequence, split-K).
 #include "kernels.cuh"
 
 namespace qsa {
@@ -108,10 +110,12 @@ __device__ __forceinline__ RowInfo row_info(int64_t item, int nsplit, int64_t ro
     return ri;
 }
 
-// block id of selection slot bi of a row: -1 for padding or an id outside 0 .. b_t
+// block id of selection slot bi of a row: -1 for padding or an id outside 0 .. b_t;
+// without a selection (sel == nullptr, dense attention) slot bi is block bi
 __device__ __forceinline__ int32_t fetch_block(const int32_t *sel, const RowInfo &ri, int kb, int bi)
 {
     if (bi >= ri.nsel) return -1;
+    if (sel == nullptr) return bi;
     const int32_t blk = __ldg(sel + ri.row * kb + bi);
     if (blk < 0 || blk > ri.bt) {
         set_device_status(QSA_ERR_DEVICE_CHECK);
@@ -547,6 +551,14 @@ int min_nsplit(int kb)
 int max_nsplit(int kb)
 {
     return (kb + kBlkTile - 1) / kBlkTile;  // at most one split per 64-token tile
+}
+
+int dense_decode_nsplit(int64_t max_len_k, int r)
+{
+    const int64_t blocks = (max_len_k + r - 1) / r;
+    const int64_t tiles = (blocks + kBlkTile - 1) / kBlkTile;
+    const int64_t ns = (tiles + 31) / 32;  // about 2048 tokens per split, as a QSA query
+    return (int)(ns > 0 ? ns : 1);
 }
 
 int decode_nsplit(int batch, int kb)

@@ -50,7 +50,7 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t stream);
 
 struct AttnArgs {
     const __nv_bfloat16 *q, *k, *v;  // q [rows_total, 24, 256]; k, v [total_k, 2, 256]
-    const int32_t *sel;              // [rows_total, kb]
+    const int32_t *sel;              // [rows_total, kb]; nullptr = every block (dense)
     const int32_t *cu_q;             // nullptr = decode: row i is sequence i, L_q = 1
     const int32_t *cu_k;
     int batch;
@@ -67,6 +67,7 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream);
 int min_nsplit(int kb);                         // splits needed so each holds <= 16 tiles
 int decode_nsplit(int batch, int kb);           // splits used by the decode call
 int max_nsplit(int kb);                         // upper bound of decode_nsplit over devices
+int dense_decode_nsplit(int64_t max_len_k, int r);  // splits of the dense flash-decoding path
 size_t split_workspace_bytes(int64_t rows, int nsplit);  // partial (o, lse) states
 
 struct DenseArgs {

@@ -67,7 +67,7 @@ def _load():
         "qsa_select_blocks": (I32, [CP, P, I64, P, P, I32, I64, I64, P, P, SZ, P]),
         "qsa_sparse_attn_prefill": (I32, [CP, P, P, P, P, P, P, I32, I64, I64, I64, I64, P, P, P, SZ, P]),
         "qsa_sparse_attn_decode": (I32, [CP, P, P, P, P, I32, I64, P, P, P, P, SZ, P]),
-        "qsa_dense_attn_prefill": (I32, [CP, P, P, P, P, P, I32, I64, I64, I32, P, P, P]),
+        "qsa_dense_attn_prefill": (I32, [CP, P, P, P, P, P, I32, I64, I64, I32, I64, P, P, P, SZ, P]),
         "qsa_workspace_size": (SZ, [CP, I32, I32, I64, I64]),
         "qsa_status_string": (ctypes.c_char_p, [I32]),
         "qsa_get_device_status": (I32, [P, ctypes.POINTER(I32), I32]),
@@ -214,15 +214,23 @@ def sparse_attn_decode(q, k_cache, v_cache, cu_seqlens_k, sel, o=None, lse=None,
 
 
 def dense_attn_prefill(q, k, v, cu_seqlens_q, cu_seqlens_k, max_len_q: int, o=None, lse=None,
-                       want_lse: bool = False, cfg: Optional[Config] = None):
+                       want_lse: bool = False, cfg: Optional[Config] = None, max_len_k: Optional[int] = None,
+                       ws=None):
+    """Dense causal attention; max_len_q == 1 runs split-K flash decoding."""
     cfg = _cfg(cfg)
     if o is None:
         o = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty((q.shape[0], cfg.n_heads_q), dtype=torch.float32, device=q.device)
+    if max_len_k is None:
+        max_len_k = int((cu_seqlens_k[1:] - cu_seqlens_k[:-1]).max().item())
+    batch = cu_seqlens_q.numel() - 1
+    need = workspace_size(OP_DENSE, batch, q.shape[0], max_len_k, cfg) if max_len_q == 1 else 0
+    if ws is None and need > 0:
+        ws = torch.empty((need,), dtype=torch.uint8, device=q.device)
     _check(_lib.qsa_dense_attn_prefill(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(cu_seqlens_q), _p(cu_seqlens_k),
-                                       cu_seqlens_q.numel() - 1, q.shape[0], k.shape[0], max_len_q, _p(o),
-                                       _p(lse), _stream()),
+                                       batch, q.shape[0], k.shape[0], max_len_q, max_len_k, _p(o), _p(lse),
+                                       _p(ws), ws.numel() if ws is not None else 0, _stream()),
            "qsa_dense_attn_prefill")
     return (o, lse) if want_lse or lse is not None else o
 

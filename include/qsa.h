@@ -188,13 +188,16 @@ qsa_status qsa_sparse_attn_decode(const qsa_config *cfg, const qsa_bf16 *q,
 /*
  * Dense causal GQA attention (the baseline the pages measure QSA against):
  * query t attends to every key j <= t of its sequence.  Same layouts as the
- * sparse prefill; max_len_q is a host launch bound.  Workspace: none.
+ * sparse prefill.  max_len_q and max_len_k are host bounds of L_q,s and L_k,s.
+ * max_len_q == 1 (one query per sequence, decode) runs split-K flash decoding
+ * over all blocks and needs qsa_workspace_size(cfg, QSA_OP_DENSE, batch,
+ * total_q, max_len_k) bytes of workspace; otherwise no workspace (ws may be NULL).
  */
 qsa_status qsa_dense_attn_prefill(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k,
                                   const qsa_bf16 *v, const int32_t *cu_seqlens_q,
                                   const int32_t *cu_seqlens_k, int32_t batch, int64_t total_q,
-                                  int64_t total_k, int32_t max_len_q, qsa_bf16 *o, float *lse,
-                                  void *stream);
+                                  int64_t total_k, int32_t max_len_q, int64_t max_len_k,
+                                  qsa_bf16 *o, float *lse, void *ws, size_t ws_bytes, void *stream);
 
 /* Workspace bytes an op needs (0 = none).  rows = query rows of the call,
  * max_len_k = longest key sequence.  Host only, no CUDA calls. */

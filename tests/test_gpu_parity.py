@@ -377,3 +377,55 @@ def test_decode_chain(qsa, batch, lo, hi, k):
         check_attn(o_g[s:s + 1], ref_o)
         np.testing.assert_allclose(lse_g[s], ref_lse[0], rtol=0, atol=2e-3)
     status_ok(qsa)
+
+
+# ---------------------------------------------------------------------------------------------
+# dense causal attention (the comparison baseline)
+# ---------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("lengths", [[1], [77], [512], [1, 3, 130, 129, 700, 64]])
+def test_dense_attention(qsa, lengths):
+    x = inputs.make_prefill(lengths, seed=28)
+    cu_q = torch.tensor(np.r_[0, np.cumsum(lengths)], dtype=torch.int32, device="cuda")
+    o, lse = qsa.dense_attn_prefill(x.q.cuda(), x.k.cuda(), x.v.cuda(), cu_q, cu_q, max(lengths), want_lse=True)
+    torch.cuda.synchronize()
+    og, lg = o.float().cpu().numpy(), lse.cpu().numpy()
+    for s, (a, b) in enumerate(seq_slices(lengths)):
+        L = b - a
+        rows = sample_rows(L)
+        ref_o, ref_l = oracle.dense(x.q[a:b], x.k[a:b], x.v[a:b], L, L, SCALE, rows)
+        check_attn(og[a + rows], ref_o)
+        np.testing.assert_allclose(lg[a + rows], ref_l, rtol=0, atol=2e-3)
+    status_ok(qsa)
+
+
+def test_dense_attention_decode_shape(qsa):
+    """One query per sequence against its whole cache (L_q = 1 < L_k)."""
+    d = inputs.make_decode(4, 100, 3000, seed=29)
+    cu_k, _ = cu(d.seqlens)
+    cu_q = torch.arange(5, dtype=torch.int32, device="cuda")
+    o = qsa.dense_attn_prefill(d.q.cuda(), d.k_cache.cuda(), d.v_cache.cuda(), cu_q, cu_k, 1)
+    torch.cuda.synchronize()
+    og = o.float().cpu().numpy()
+    for s, (a, b) in enumerate(seq_slices(d.seqlens)):
+        L = b - a
+        ref_o, _ = oracle.dense(d.q[s:s + 1], d.k_cache[a:b], d.v_cache[a:b], 1, L, SCALE, [0])
+        check_attn(og[s:s + 1], ref_o)
+    status_ok(qsa)
+
+
+def test_dense_n8192_matches_full_budget_sparse(qsa):
+    """Two independent GPU paths to the same number: dense causal attention and QSA with
+    a budget covering every block; both against the oracle on sampled rows."""
+    n = 8192
+    x = inputs.make_prefill([n], seed=0)
+    cu_q = torch.tensor([0, n], dtype=torch.int32, device="cuda")
+    od = qsa.dense_attn_prefill(x.q.cuda(), x.k.cuda(), x.v.cuda(), cu_q, cu_q, n)
+    _, _, osp, _ = run_chain(qsa, x, [n], 2048)
+    torch.cuda.synchronize()
+    d = (od.float() - osp.float()).abs()
+    assert d.max().item() <= 2e-2 and d.mean().item() <= 1e-3
+    rows = sample_rows(n, 64)
+    ref_o, _ = oracle.dense(x.q, x.k, x.v, n, n, SCALE, rows)
+    check_attn(od.float().cpu().numpy()[rows], ref_o)
+    status_ok(qsa)
