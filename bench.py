@@ -34,6 +34,11 @@ CHUNK = 16384
 BUDGET = 512
 METRIC = "QSA prefill tokens/s at 262K ctx; decode µs/token at 128K; % of roofline"
 
+# DRAM traffic (read + write bytes) of one full prefill launch of sparse_attn_kernel, from the
+# 1-pass ncu capture summarised in profiles/sparse_attn_prefill262k_traffic.md; valid only for
+# the kernel source it was taken on (checked by hash), null otherwise.
+ATTN_TRAFFIC = {"src_sha256_16": "ab6d73155f361a17", "bytes": 613.42e9}
+
 
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -119,15 +124,11 @@ def run_qsa(args, rank, world, device):
     d = inputs.make_decode(DEC_BATCH, DEC_LEN, None, seed=100 + rank, device=device)
     cu_k = d.cu_seqlens_k
     cu_b = d.cu_blocks
-    cu_q = torch.arange(DEC_BATCH + 1, dtype=torch.int32, device=device)
     kc_dec = qsa.compress_keys(d.k_idx, cu_k, cu_b, n_blocks=int(cu_b[-1]), cfg=cfg)
     last_blk = torch.tensor([L // 4 - 1 for L in d.seqlens], dtype=torch.int32, device=device)
-    ld_dec = (DEC_LEN - 1) // 4
-    dec_scores = torch.empty((DEC_BATCH, ld_dec), dtype=torch.float32, device=device)
-    dec_sel = torch.empty((DEC_BATCH, BUDGET), dtype=torch.int32, device=device)
-    dec_o = torch.empty_like(d.q)
-    dec_ws = torch.empty((qsa.workspace_size(qsa.OP_DECODE, DEC_BATCH, DEC_BATCH, DEC_LEN, cfg),),
-                         dtype=torch.uint8, device=device)
+    dec = qsa.DecodeStep(d.q, d.q_idx, d.w, d.k_cache, d.v_cache, d.k_idx, kc_dec, cu_k, cu_b, DEC_LEN,
+                         refresh_blocks=last_blk, cfg=cfg, graph=True)
+    dec_o = dec.o
     stream = torch.cuda.current_stream()
 
     ev = {k: [] for k in ("p0", "p1", "a0", "a1", "d0", "d1")}
@@ -144,10 +145,7 @@ def run_qsa(args, rank, world, device):
             e["a1"].record(stream)
             e["p1"].record(stream)
             e["d0"].record(stream)
-        qsa.compress_keys(d.k_idx, cu_k, cu_b, kc=kc_dec, blk_begin=last_blk, max_new_blocks=1, cfg=cfg)
-        qsa.index_scores(d.q_idx, d.w, kc_dec, cu_q, cu_k, cu_b, 1, ld_dec, scores=dec_scores, cfg=cfg)
-        qsa.select_blocks(dec_scores, cu_q, cu_k, DEC_BATCH, sel=dec_sel, cfg=cfg)
-        qsa.sparse_attn_decode(d.q, d.k_cache, d.v_cache, cu_k, dec_sel, o=dec_o, ws=dec_ws, cfg=cfg)
+        dec()  # decode step: one CUDA-graph replay of its five launches
         if record:
             e["d1"].record(stream)
             for k in ev:
@@ -245,6 +243,11 @@ def run_qsa(args, rank, world, device):
                  "decode_step_us": dd_us, "qsa_decode_speedup": dd_us / (dec_ms * 1e3),
                  "pages_context": "7.6x prefill / 4.9x decode at 1M context, kernel level, hardware not stated"}
 
+    import hashlib
+    src = os.path.join(ROOT, "block_sparse_long_09_b200", "csrc", "attn.cu")
+    same_src = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] == ATTN_TRAFFIC["src_sha256_16"]
+    traffic = ATTN_TRAFFIC["bytes"] if (same_src and world == 1) else None
+
     sel_tok = selected_tokens(N_PREFILL)
     gather = gather_bytes_per_query(1) * sel_tok
     achieved = gather / (attn_ms / 1e3) / 1e9
@@ -270,7 +273,7 @@ def run_qsa(args, rank, world, device):
         "decode": {"batch": DEC_BATCH, "ctx": DEC_LEN, "step_us": dec_ms * 1e3, "us_per_token": dec_ms * 1e3,
                    "us_per_token_amortized": dec_ms * 1e3 / DEC_BATCH},
         "roofline": {"kernel": "sparse_attn_kernel (prefill)", "bound": "hbm", "achieved": achieved,
-                     "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                     "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
                      "algorithmic_bytes": gather, "peak_kind": peak_kind + " (burst copy)"},
         "gpu_launches": args.steps * (launches_prefill + launches_decode),
         "dense": dense,

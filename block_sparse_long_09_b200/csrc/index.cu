@@ -329,7 +329,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
 
 // ------------------------------------------------------------------ row-wise path
 constexpr int kRowWarps = 8;
-constexpr int kRowChunk = 4096;  // kc blocks per CTA
+constexpr int kRowChunk = 1024;  // kc blocks per CTA
 
 __global__ void __launch_bounds__(kRowWarps * 32)
 index_rowwise_kernel(const __nv_bfloat16 *__restrict__ q_idx, const float *__restrict__ w,

@@ -222,8 +222,32 @@ select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__res
         }
         if (tid == 0) sc.cand_n = 0;
         __syncthreads();
-        // pass 1: histogram of the top 12 key bits
-        {
+        // pass 1: histogram of the top 12 key bits (16 keys in flight per thread)
+        if ((reinterpret_cast<uintptr_t>(srow) & 15u) == 0) {
+            const float4 *s4 = reinterpret_cast<const float4 *>(srow);
+            const int n4 = n >> 2;
+            int j = tid;
+            for (; j + 3 * kSelThreads < n4; j += 4 * kSelThreads) {
+                float4 v[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) v[q] = __ldg(s4 + j + q * kSelThreads);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    atomicAdd(&hist[order_key(v[q].x) >> 20], 1u);
+                    atomicAdd(&hist[order_key(v[q].y) >> 20], 1u);
+                    atomicAdd(&hist[order_key(v[q].z) >> 20], 1u);
+                    atomicAdd(&hist[order_key(v[q].w) >> 20], 1u);
+                }
+            }
+            for (; j < n4; j += kSelThreads) {
+                const float4 v = __ldg(s4 + j);
+                atomicAdd(&hist[order_key(v.x) >> 20], 1u);
+                atomicAdd(&hist[order_key(v.y) >> 20], 1u);
+                atomicAdd(&hist[order_key(v.z) >> 20], 1u);
+                atomicAdd(&hist[order_key(v.w) >> 20], 1u);
+            }
+            for (int e = (n4 << 2) + tid; e < n; e += kSelThreads) atomicAdd(&hist[order_key(__ldg(srow + e)) >> 20], 1u);
+        } else {
             int j = tid;
             for (; j + 3 * kSelThreads < n; j += 4 * kSelThreads) {
                 const float a0 = __ldg(srow + j), a1 = __ldg(srow + j + kSelThreads);
@@ -245,25 +269,36 @@ select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__res
             // pass 2: bitmap of keys whose top digit is above d1; collect the d1 bin
             const bool take_bin = (need == cnt1);
             const int words = (n + 31) >> 5;
-            for (int w = wid; w < words; w += kSelWarps) {
-                const int j = w * 32 + lane;
-                const bool in = j < n;
-                const uint32_t u = in ? order_key(__ldg(srow + j)) : 0u;
-                const uint32_t dg = u >> 20;
-                const bool gt = in && (dg > d1u || (take_bin && dg == d1u));
-                const bool inbin = in && !take_bin && dg == d1u;
-                const uint32_t gb = __ballot_sync(0xffffffffu, gt);
-                const uint32_t cb = __ballot_sync(0xffffffffu, inbin);
-                int base = 0;
-                if (lane == 0) {
-                    gtw[w] = gb;
-                    if (cb) base = atomicAdd(&sc.cand_n, __popc(cb));
+            for (int w0 = wid; w0 < words; w0 += 4 * kSelWarps) {
+                uint32_t uu[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {  // four words' loads in flight
+                    const int j = (w0 + q * kSelWarps) * 32 + lane;
+                    uu[q] = (w0 + q * kSelWarps < words && j < n) ? order_key(__ldg(srow + j)) : 0u;
                 }
-                base = __shfl_sync(0xffffffffu, base, 0);
-                if (inbin) {
-                    const int p = base + __popc(cb & ((1u << lane) - 1u));
-                    cand_key[p] = u;
-                    cand_idx[p] = (uint32_t)j;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int w = w0 + q * kSelWarps;
+                    if (w >= words) break;  // uniform across the warp
+                    const int j = w * 32 + lane;
+                    const bool in = j < n;
+                    const uint32_t u = uu[q];
+                    const uint32_t dg = u >> 20;
+                    const bool gt = in && (dg > d1u || (take_bin && dg == d1u));
+                    const bool inbin = in && !take_bin && dg == d1u;
+                    const uint32_t gb = __ballot_sync(0xffffffffu, gt);
+                    const uint32_t cb = __ballot_sync(0xffffffffu, inbin);
+                    int base = 0;
+                    if (lane == 0) {
+                        gtw[w] = gb;
+                        if (cb) base = atomicAdd(&sc.cand_n, __popc(cb));
+                    }
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    if (inbin) {
+                        const int p = base + __popc(cb & ((1u << lane) - 1u));
+                        cand_key[p] = u;
+                        cand_idx[p] = (uint32_t)j;
+                    }
                 }
             }
             __syncthreads();

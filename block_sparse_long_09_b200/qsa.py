@@ -274,3 +274,54 @@ class Prefill:
     def __call__(self, q, k, v, q_idx, w, k_idx, o=None, lse=None):
         self.index_select(q_idx, w, k_idx)
         return sparse_attn_prefill(q, k, v, self.sel, self.cu, self.cu, o=o, lse=lse, cfg=self.cfg)
+
+
+class DecodeStep:
+    """One QSA decode step for a fixed batch, one new query per sequence: refresh
+    the compressed block each sequence just completed, score every earlier block,
+    select the top k, and run split-K sparse attention.  The five launches can be
+    captured once in a CUDA graph and replayed (graph=True): the tensors passed
+    here are the graph's fixed inputs, so a caller refreshes them in place."""
+
+    def __init__(self, q, q_idx, w, k_cache, v_cache, k_idx, kc, cu_seqlens_k, cu_blocks, max_len_k: int,
+                 refresh_blocks=None, cfg: Optional[Config] = None, graph: bool = True):
+        self.cfg = _cfg(cfg)
+        r = self.cfg.r
+        self.q, self.q_idx, self.w = q, q_idx, w
+        self.k_cache, self.v_cache, self.k_idx, self.kc = k_cache, v_cache, k_idx, kc
+        self.cu_k, self.cu_b = cu_seqlens_k, cu_blocks
+        self.batch = q.shape[0]
+        dev = q.device
+        self.cu_q = torch.arange(self.batch + 1, dtype=torch.int32, device=dev)
+        self.refresh = refresh_blocks  # [batch] int32 block ids to recompute, or None
+        self.ld = max(4, ((max_len_k - 1) // r + 3) // 4 * 4)
+        self.scores = torch.empty((self.batch, self.ld), dtype=torch.float32, device=dev)
+        self.sel = torch.empty((self.batch, self.cfg.budget_blocks), dtype=torch.int32, device=dev)
+        self.o = torch.empty_like(q)
+        self.ws = torch.empty((max(workspace_size(OP_DECODE, self.batch, self.batch, max_len_k, self.cfg), 16),),
+                              dtype=torch.uint8, device=dev)
+        self.graph = None
+        self.run()  # first call outside any capture (one-time kernel attribute setup)
+        if graph:
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.run()
+            self.graph = g
+
+    def run(self):
+        if self.refresh is not None:
+            compress_keys(self.k_idx, self.cu_k, self.cu_b, kc=self.kc, blk_begin=self.refresh, max_new_blocks=1,
+                          cfg=self.cfg)
+        index_scores(self.q_idx, self.w, self.kc, self.cu_q, self.cu_k, self.cu_b, 1, self.ld, scores=self.scores,
+                     cfg=self.cfg)
+        select_blocks(self.scores, self.cu_q, self.cu_k, self.batch, sel=self.sel, cfg=self.cfg)
+        sparse_attn_decode(self.q, self.k_cache, self.v_cache, self.cu_k, self.sel, o=self.o, ws=self.ws,
+                           cfg=self.cfg)
+        return self.o
+
+    def __call__(self):
+        if self.graph is not None:
+            self.graph.replay()
+            return self.o
+        return self.run()

@@ -429,3 +429,28 @@ def test_dense_n8192_matches_full_budget_sparse(qsa):
     ref_o, _ = oracle.dense(x.q, x.k, x.v, n, n, SCALE, rows)
     check_attn(od.float().cpu().numpy()[rows], ref_o)
     status_ok(qsa)
+
+
+def test_decode_step_cuda_graph(qsa):
+    """The CUDA-graph replay of a decode step equals the eager launches, bit for bit,
+    and matches the oracle on the selection it made."""
+    d = inputs.make_decode(8, 2000, 9000, seed=30)
+    cu_k, cu_b = cu(d.seqlens)
+    args = [t.cuda() for t in (d.q, d.q_idx, d.w, d.k_cache, d.v_cache, d.k_idx)]
+    kc = qsa.compress_keys(args[5], cu_k, cu_b, n_blocks=int(cu_b[-1]))
+    last = torch.tensor([L // 4 - 1 for L in d.seqlens], dtype=torch.int32, device="cuda")
+    eager = qsa.DecodeStep(*args, kc, cu_k, cu_b, max(d.seqlens), refresh_blocks=last, graph=False)
+    o_eager = eager().clone()
+    sel_eager = eager.sel.clone()
+    graphed = qsa.DecodeStep(*args, kc, cu_k, cu_b, max(d.seqlens), refresh_blocks=last, graph=True)
+    for _ in range(3):
+        o_graph = graphed()
+    torch.cuda.synchronize()
+    assert torch.equal(graphed.sel, sel_eager)
+    assert torch.equal(o_graph, o_eager)
+    sel_g = sel_eager.cpu().numpy()
+    for s in (0, 7):
+        a, b = int(cu_k[s]), int(cu_k[s + 1])
+        ref_o, _ = oracle.attend(d.q[s:s + 1], d.k_cache[a:b], d.v_cache[a:b], sel_g[s:s + 1], 1, b - a, 4, SCALE, [0])
+        check_attn(o_eager.float().cpu().numpy()[s:s + 1], ref_o)
+    status_ok(qsa)
