@@ -140,7 +140,7 @@ def run_qsa(args, rank, world, device):
         pre.index_select(x.q_idx, x.w, x.k_idx)
         if record:
             e["a0"].record(stream)
-        qsa.sparse_attn_prefill(x.q, x.k, x.v, pre.sel, pre.cu, pre.cu, o=o, cfg=cfg)
+        pre.attend(x.q, x.k, x.v, o=o)  # one pass per query
         if record:
             e["a1"].record(stream)
             e["p1"].record(stream)
@@ -251,7 +251,8 @@ def run_qsa(args, rank, world, device):
     sel_tok = selected_tokens(N_PREFILL)
     gather = gather_bytes_per_query(1) * sel_tok
     achieved = gather / (attn_ms / 1e3) / 1e9
-    launches_prefill = 1 + 2 * ((N_PREFILL + CHUNK - 1) // CHUNK) + 1
+    n_chunks = (N_PREFILL + CHUNK - 1) // CHUNK
+    launches_prefill = 1 + 2 * n_chunks + n_chunks  # compress; index + select per chunk; attention per chunk
     launches_decode = 1 + 1 + 1 + 2
     res = {
         "metric": METRIC,
@@ -343,7 +344,7 @@ def run_profile_case(case: str, reps: int = 3):
                                  r0, n, scores=pre.scores, cfg=cfg)
                 qsa.select_blocks(pre.scores, pre.cu, pre.cu, n, r0, n, sel=pre.sel, cfg=cfg)
             if case == "attn":
-                qsa.sparse_attn_prefill(x.q, x.k, x.v, pre.sel, pre.cu, pre.cu, r0, n, cfg=cfg)
+                qsa.sparse_attn_prefill(x.q, x.k, x.v, pre.sel, pre.cu, pre.cu, r0, n, cfg=cfg, max_len_k=n)
     elif case == "decode":
         d = inputs.make_decode(DEC_BATCH, 16384, None, seed=1, device=dev)
         cu_q = torch.arange(DEC_BATCH + 1, dtype=torch.int32, device=dev)

@@ -95,7 +95,8 @@ qsa_status check_config(const qsa_config *c)
 {
     if (c == nullptr) return QSA_ERR_INVALID_ARG;
     if (c->r <= 0 || c->budget_blocks <= 0 || c->n_heads_q <= 0 || c->n_heads_kv <= 0 || c->head_dim <= 0 ||
-        c->n_heads_idx <= 0 || c->idx_dim <= 0 || !(c->softmax_scale > 0.f) || !(c->rms_eps >= 0.f))
+        c->n_heads_idx <= 0 || c->idx_dim <= 0 || !(c->softmax_scale > 0.f) || !(c->rms_eps >= 0.f) ||
+        c->kv_chunk_blocks < 0)
         return QSA_ERR_INVALID_ARG;
     if (c->r != 4 || c->budget_blocks > 2048 || c->n_heads_q != 24 || c->n_heads_kv != 2 || c->head_dim != 256 ||
         c->n_heads_idx != 4 || c->idx_dim != 128 || (c->flags & ~QSA_COMPRESS_NO_NORM) != 0)
@@ -104,6 +105,16 @@ qsa_status check_config(const qsa_config *c)
 }
 
 qsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA; }
+
+// key-chunked (L2-blocked) prefill schedule: opt-in through cfg->kv_chunk_blocks > 0
+int nchunks_of(const qsa_config *c, int64_t max_len_k)
+{
+    if (c->kv_chunk_blocks <= 0) return 1;
+    const int64_t blocks = (max_len_k + c->r - 1) / c->r;
+    const int64_t cb = c->kv_chunk_blocks;
+    const int64_t n = (blocks + cb - 1) / cb;
+    return (int)(n > 0 ? (n < 4096 ? n : 4096) : 1);
+}
 
 const __nv_bfloat16 *bf(const qsa_bf16 *p) { return reinterpret_cast<const __nv_bfloat16 *>(p); }
 __nv_bfloat16 *bf(qsa_bf16 *p) { return reinterpret_cast<__nv_bfloat16 *>(p); }
@@ -126,6 +137,7 @@ void qsa_config_init(qsa_config *cfg)
     cfg->softmax_scale = 0.0625f;
     cfg->rms_eps = 1e-6f;
     cfg->flags = 0u;
+    cfg->kv_chunk_blocks = 0;
 }
 
 int32_t qsa_version(void) { return 100; }
@@ -151,7 +163,10 @@ size_t qsa_workspace_size(const qsa_config *cfg, int32_t op, int32_t batch, int6
         const int ns = max_nsplit(cfg->budget_blocks);
         return split_workspace_bytes(batch, ns > 1 ? ns : 2);
     }
-    if (op == QSA_OP_PREFILL) return split_workspace_bytes(rows, min_nsplit(cfg->budget_blocks));
+    if (op == QSA_OP_PREFILL) {
+        const int nc = nchunks_of(cfg, max_len_k);
+        return nc > 1 ? chunked_workspace_bytes(rows, nc) : 0;
+    }
     if (op == QSA_OP_DENSE) return split_workspace_bytes(rows, dense_decode_nsplit(max_len_k, cfg->r));
     return 0;
 }
@@ -227,27 +242,29 @@ qsa_status qsa_select_blocks(const qsa_config *cfg, const float *scores, int64_t
 
 qsa_status qsa_sparse_attn_prefill(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k, const qsa_bf16 *v,
                                    const int32_t *sel, const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
-                                   int32_t batch, int64_t total_q, int64_t total_k, int64_t row_begin,
-                                   int64_t row_end, qsa_bf16 *o, float *lse, void *ws, size_t ws_bytes,
-                                   void *stream)
+                                   int32_t batch, int64_t total_q, int64_t total_k, int64_t max_len_k,
+                                   int64_t row_begin, int64_t row_end, qsa_bf16 *o, float *lse, void *ws,
+                                   size_t ws_bytes, void *stream)
 {
     qsa_status st = check_config(cfg);
     if (st != QSA_OK) return st;
-    if (batch <= 0 || total_q < 0 || total_k < 0 || row_begin < 0 || row_end < row_begin || row_end > total_q)
+    if (batch <= 0 || total_q < 0 || total_k < 0 || max_len_k < 0 || row_begin < 0 || row_end < row_begin ||
+        row_end > total_q)
         return QSA_ERR_INVALID_ARG;
     if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr) return QSA_ERR_INVALID_ARG;
     if (row_end == row_begin) return QSA_OK;
     if (total_k == 0 || q == nullptr || k == nullptr || v == nullptr || sel == nullptr || o == nullptr ||
         !al16(q) || !al16(k) || !al16(v))
         return QSA_ERR_INVALID_ARG;
-    const int nsplit = min_nsplit(cfg->budget_blocks);
-    if (nsplit > 1) {
-        if (ws == nullptr || ws_bytes < split_workspace_bytes(row_end - row_begin, nsplit))
-            return QSA_ERR_WORKSPACE_TOO_SMALL;
-        if (!al16(ws)) return QSA_ERR_INVALID_ARG;
-    }
     AttnArgs a{bf(q), bf(k), bf(v), sel, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, row_begin, row_end,
-               bf(o), lse, static_cast<float *>(ws), nsplit, cfg->budget_blocks, cfg->r, cfg->softmax_scale};
+               bf(o), lse, nullptr, 1, cfg->budget_blocks, cfg->r, cfg->softmax_scale};
+    // the L2-blocked schedule when the keys span several chunks and the workspace allows it
+    const int nc = nchunks_of(cfg, max_len_k);
+    if (nc > 1 && ws != nullptr && al16(ws) && ws_bytes >= chunked_workspace_bytes(row_end - row_begin, nc)) {
+        a.ws = static_cast<float *>(ws);
+        a.nchunks = nc;
+        a.chunk_blocks = cfg->kv_chunk_blocks;
+    }
     return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
 }
 

@@ -61,7 +61,7 @@ struct AttShared {
     uint64_t q_full, q_empty;
     uint64_t s_full[2], s_empty[2];
     uint64_t p_full[kNP], p_empty[kNP];
-    uint64_t pv_done;
+    uint64_t o_full;               // once per item: every PV of the item has completed
     uint32_t tmem_base;
     int abort_flag;
     float red_max[2][4][2][kGrp];  // [tile parity][quad][group][head]
@@ -75,18 +75,34 @@ constexpr int kAttSmem = kOffShared + (int)sizeof(AttShared) + 1024;
 
 struct RowInfo {
     int64_t row;    // packed query row
+    int64_t rl;     // row within the call (row - row_begin)
     int s;
+    int sp;         // split (or key chunk) of this item
     int64_t t, bt, tok_base;
-    int nsel, tile0, tile1;
+    int nsel;       // valid selection slots of the row
+    int p0, p1;     // selection positions [p0, p1) handled by this item
+    int nt;         // 16-block tiles covering [p0, p1)
 };
 
-__device__ __forceinline__ RowInfo row_info(int64_t item, int nsplit, int64_t row_begin,
+// Work item -> (row, selection range).  Three schedules:
+//  * nsplit == 1: one item per row, the whole selection;
+//  * split-K (bounds == nullptr, nsplit > 1): item = rl * nsplit + sp, split sp takes
+//    tiles [sp * tps, (sp + 1) * tps) of the row's selection;
+//  * key-chunked (bounds != nullptr): item = sp * rows + rl (chunk-major, so all CTAs
+//    gather from the same L2-resident key chunk sp); the range comes from bounds.
+__device__ __forceinline__ RowInfo row_info(int64_t item, int nsplit, int64_t rows, int64_t row_begin,
                                             const int32_t *cu_q, const int32_t *cu_k, int batch,
-                                            int kb, int r)
+                                            int kb, int r, const int32_t *bounds)
 {
     RowInfo ri;
-    ri.row = row_begin + item / nsplit;
-    const int sp = (int)(item % nsplit);
+    if (bounds != nullptr) {
+        ri.rl = item % rows;
+        ri.sp = (int)(item / rows);
+    } else {
+        ri.rl = item / nsplit;
+        ri.sp = (int)(item % nsplit);
+    }
+    ri.row = row_begin + ri.rl;
     if (cu_q != nullptr) {
         ri.s = find_seq(cu_q, batch, ri.row);
         const int64_t Lq = (int64_t)cu_q[ri.s + 1] - cu_q[ri.s];
@@ -101,22 +117,30 @@ __device__ __forceinline__ RowInfo row_info(int64_t item, int nsplit, int64_t ro
     ri.tok_base = cu_k[ri.s];
     const int64_t nsel = ri.bt + 1 < kb ? ri.bt + 1 : kb;
     ri.nsel = (int)nsel;
-    const int ntiles = (int)((nsel + kBlkTile - 1) / kBlkTile);
-    const int max_tiles = (kb + kBlkTile - 1) / kBlkTile;
-    const int tps = (max_tiles + nsplit - 1) / nsplit;
-    ri.tile0 = sp * tps;
-    ri.tile1 = ri.tile0 + tps < ntiles ? ri.tile0 + tps : ntiles;
-    if (!ok) ri.tile1 = ri.tile0;
+    if (bounds != nullptr) {
+        ri.p0 = bounds[ri.rl * (nsplit + 1) + ri.sp];
+        ri.p1 = bounds[ri.rl * (nsplit + 1) + ri.sp + 1];
+        if (ri.p1 > ri.nsel) ri.p1 = ri.nsel;
+    } else {
+        const int max_tiles = (kb + kBlkTile - 1) / kBlkTile;
+        const int tps = (max_tiles + nsplit - 1) / nsplit;
+        ri.p0 = ri.sp * tps * kBlkTile;
+        const int e = (ri.sp + 1) * tps * kBlkTile;
+        ri.p1 = e < ri.nsel ? e : ri.nsel;
+    }
+    if (!ok || ri.p0 < 0 || ri.p1 < ri.p0) ri.p1 = ri.p0 = 0;
+    ri.nt = (ri.p1 - ri.p0 + kBlkTile - 1) / kBlkTile;
     return ri;
 }
 
-// block id of selection slot bi of a row: -1 for padding or an id outside 0 .. b_t;
-// without a selection (sel == nullptr, dense attention) slot bi is block bi
-__device__ __forceinline__ int32_t fetch_block(const int32_t *sel, const RowInfo &ri, int kb, int bi)
+// block id at selection position pos of an item: -1 outside [p0, p1) or for an id
+// outside 0 .. b_t; without a selection (sel == nullptr, dense attention) position
+// pos is block pos
+__device__ __forceinline__ int32_t fetch_block(const int32_t *sel, const RowInfo &ri, int kb, int pos)
 {
-    if (bi >= ri.nsel) return -1;
-    if (sel == nullptr) return bi;
-    const int32_t blk = __ldg(sel + ri.row * kb + bi);
+    if (pos >= ri.p1) return -1;
+    if (sel == nullptr) return pos;
+    const int32_t blk = __ldg(sel + ri.row * kb + pos);
     if (blk < 0 || blk > ri.bt) {
         set_device_status(QSA_ERR_DEVICE_CHECK);
         return -1;
@@ -157,9 +181,9 @@ __global__ void __launch_bounds__(kAttThreads, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_v, const int32_t *__restrict__ sel,
                    const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k, int batch,
-                   int64_t row_begin, int64_t n_items, int nsplit, int kb, int r, float scale,
+                   int64_t row_begin, int64_t rows, int nsplit, int kb, int r, float scale,
                    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse_out,
-                   float *__restrict__ ws)
+                   float *__restrict__ ws, const int32_t *__restrict__ bounds)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -184,7 +208,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             mbar_init(&sh->p_full[i], 128);
             mbar_init(&sh->p_empty[i], 1);
         }
-        mbar_init(&sh->pv_done, 1);
+        mbar_init(&sh->o_full, 1);
         sh->abort_flag = 0;
         fence_barrier_init();
     }
@@ -201,6 +225,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     tc_fence_after();
     const uint32_t tmem = sh->tmem_base;
     volatile int *abort_flag = &sh->abort_flag;
+    const int64_t n_items = rows * nsplit;
 
     if (warp == 0) {
         // ======================= TMA producer (whole warp) =======================
@@ -211,6 +236,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         }
         uint32_t slot_it = 0, q_it = 0;
         bool ok = true;
+        const uint64_t kv_policy = make_policy_evict_last();  // K/V stay in L2 while reused
         auto issue = [&](const CUtensorMap *map, const RowInfo &ri, int32_t blk) -> bool {
             const uint32_t st = slot_it % kNSlot, round = slot_it / kNSlot;
             bool good = true;
@@ -223,18 +249,19 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             if (lane < kBlkTile) {
                 // rows (token, group) of the block; padding reads an out-of-range box (zeros)
                 const int32_t y = blk >= 0 ? (int32_t)((ri.tok_base + (int64_t)blk * r) * kHKV) : -8;
-                tma_load_3d(sSlot + st * kSlotBytes + lane * kBlockBytes, map, &sh->slot_full[st], 0, y, 0);
+                tma_load_3d_hint(sSlot + st * kSlotBytes + lane * kBlockBytes, map, &sh->slot_full[st], 0, y, 0,
+                                 kv_policy);
             }
             ++slot_it;
             return true;
         };
         for (int64_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
-            const RowInfo ri = row_info(item, nsplit, row_begin, cu_q, cu_k, batch, kb, r);
-            if (ri.tile0 >= ri.tile1) continue;
+            const RowInfo ri = row_info(item, nsplit, rows, row_begin, cu_q, cu_k, batch, kb, r, bounds);
+            if (ri.nt == 0) continue;
             int32_t b0 = -1, b1 = -1;
             if (lane < kBlkTile) {
-                b0 = fetch_block(sel, ri, kb, ri.tile0 * kBlkTile + lane);
-                if (ri.tile0 + 1 < ri.tile1) b1 = fetch_block(sel, ri, kb, (ri.tile0 + 1) * kBlkTile + lane);
+                b0 = fetch_block(sel, ri, kb, ri.p0 + lane);
+                if (ri.nt > 1) b1 = fetch_block(sel, ri, kb, ri.p0 + kBlkTile + lane);
             }
             if (lane == 0) {
                 ok = mbar_wait(&sh->q_empty, (q_it & 1) ^ 1, abort_flag);
@@ -248,10 +275,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             ++q_it;
             if (!ok) break;
             ok = issue(&map_k, ri, b0);
-            for (int j = ri.tile0; ok && j < ri.tile1; ++j) {
+            for (int jl = 0; ok && jl < ri.nt; ++jl) {
                 int32_t b2 = -1;
-                if (lane < kBlkTile && j + 2 < ri.tile1) b2 = fetch_block(sel, ri, kb, (j + 2) * kBlkTile + lane);
-                if (j + 1 < ri.tile1) ok = issue(&map_k, ri, b1);
+                if (lane < kBlkTile && jl + 2 < ri.nt) b2 = fetch_block(sel, ri, kb, ri.p0 + (jl + 2) * kBlkTile + lane);
+                if (jl + 1 < ri.nt) ok = issue(&map_k, ri, b1);
                 if (ok) ok = issue(&map_v, ri, b0);
                 b0 = b1;
                 b1 = b2;
@@ -289,17 +316,16 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                 }
                 mma_commit(&sh->slot_empty[st]);
                 mma_commit(&sh->p_empty[pb]);
-                mma_commit(&sh->pv_done);
                 ++slot_it;
                 ++p_it;
                 return true;
             };
             for (int64_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
-                const RowInfo ri = row_info(item, nsplit, row_begin, cu_q, cu_k, batch, kb, r);
-                if (ri.tile0 >= ri.tile1) continue;
+                const RowInfo ri = row_info(item, nsplit, rows, row_begin, cu_q, cu_k, batch, kb, r, bounds);
+                if (ri.nt == 0) continue;
                 ok = mbar_wait(&sh->q_full, q_it & 1, abort_flag);
                 ++q_it;
-                const int nt = ri.tile1 - ri.tile0;
+                const int nt = ri.nt;
                 for (int jl = 0; ok && jl < nt; ++jl) {
                     const uint32_t st = slot_it % kNSlot, round = slot_it / kNSlot;
                     const uint32_t sb = s_it & 1, sround = s_it >> 1;
@@ -322,6 +348,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                     if (jl >= 1) ok = do_pv(jl == 1);
                 }
                 if (ok) ok = do_pv(nt == 1);
+                if (ok) mma_commit(&sh->o_full);
             }
         }
     } else {
@@ -337,32 +364,30 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         const uint32_t p_addr = smem_u32(sP);
         const uint32_t p_row_off = (R >> 6) * kPChunk + (R & 7) * 2;
         const int p_unit = (R & 63) >> 3;
-        uint32_t p_it = 0, s_it = 0, tile_it = 0;
+        uint32_t p_it = 0, s_it = 0, tile_it = 0, o_it = 0;
         bool ok = true;
         for (int64_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
-            const RowInfo ri = row_info(item, nsplit, row_begin, cu_q, cu_k, batch, kb, r);
-            const int sp = (int)(item % nsplit);
-            const int64_t row_local = item / nsplit;
-            if (ri.tile0 >= ri.tile1) {
-                if (nsplit > 1) {  // empty split: neutral partial state
-                    float *part = ws + ((row_local * nsplit + sp) * kHQ) * kD;
+            const RowInfo ri = row_info(item, nsplit, rows, row_begin, cu_q, cu_k, batch, kb, r, bounds);
+            const int64_t slot = ri.rl * nsplit + ri.sp;  // partial-state slot (split schedules)
+            if (ri.nt == 0) {
+                if (nsplit > 1 && bounds == nullptr) {  // empty split: neutral partial state
+                    float *part = ws + slot * kHQ * kD;
                     for (int x = R; x < kHQ * kD; x += 128) part[x] = 0.f;
-                    float *lp = ws + (size_t)n_items * kHQ * kD + (row_local * nsplit + sp) * kHQ;
-                    if (R < kHQ) lp[R] = -INFINITY;
+                    if (R < kHQ) ws[(size_t)n_items * kHQ * kD + slot * kHQ + R] = -INFINITY;
                 }
                 continue;
             }
-            const int nt = ri.tile1 - ri.tile0;
+            const int nt = ri.nt;
             float m[kHQ];                             // running max per head (raw logits), identical in all threads
             float l[kGrp];                            // this row's share of the row sums, own group's heads
 #pragma unroll
             for (int h = 0; h < kGrp; ++h) l[h] = 0.f;
 #pragma unroll
             for (int h = 0; h < kHQ; ++h) m[h] = 0.f;
-            int32_t blk_next = fetch_block(sel, ri, kb, ri.tile0 * kBlkTile + blk_slot);
+            int32_t blk_next = fetch_block(sel, ri, kb, ri.p0 + blk_slot);
             for (int jl = 0; ok && jl < nt; ++jl) {
                 const int32_t blk = blk_next;
-                if (jl + 1 < nt) blk_next = fetch_block(sel, ri, kb, (ri.tile0 + jl + 1) * kBlkTile + blk_slot);
+                if (jl + 1 < nt) blk_next = fetch_block(sel, ri, kb, ri.p0 + (jl + 1) * kBlkTile + blk_slot);
                 const bool valid = blk >= 0 && (int64_t)blk * r + tok_in_blk <= ri.t;
                 const uint32_t sb = s_it & 1, sround = s_it >> 1;
                 if (!(ok = mbar_wait(&sh->s_full[sb], sround & 1, abort_flag))) break;
@@ -420,8 +445,12 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                         }
 #pragma unroll
                         for (int h = 0; h < kGrp; ++h) l[h] *= g ? f[kGrp + h] : f[h];
-                        // O^T must be stable: wait for the previous PV, then scale it in TMEM
-                        if (!(ok = mbar_wait(&sh->pv_done, (p_it - 1) & 1, abort_flag))) break;
+                        // O^T must be stable: wait for the previous PV (the completion of the
+                        // last use of its P buffer), then scale it in TMEM
+                        {
+                            const uint32_t x = p_it - 1;
+                            if (!(ok = mbar_wait(&sh->p_empty[x % kNP], (x / kNP) & 1, abort_flag))) break;
+                        }
                         tc_fence_after();
 #pragma unroll
                         for (int half = 0; half < 2; ++half) {
@@ -480,7 +509,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                 inv[h] = L > 0.f ? 1.f / L : 0.f;
                 if (R == h) my_lse = m[h] * scale + logf(L);
             }
-            if (!(ok = mbar_wait(&sh->pv_done, (p_it - 1) & 1, abort_flag))) break;
+            if (!(ok = mbar_wait(&sh->o_full, o_it & 1, abort_flag))) break;
+            ++o_it;
             tc_fence_after();
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
@@ -493,16 +523,16 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
 #pragma unroll
                     for (int h = 0; h < kHQ; ++h) dst[h * kD] = __float2bfloat16_rn(o[h] * inv[h]);
                 } else {
-                    float *dst = ws + ((row_local * nsplit + sp) * kHQ) * kD + d;
+                    float *dst = ws + (slot * kHQ) * kD + d;
 #pragma unroll
-                    for (int h = 0; h < kHQ; ++h) dst[h * kD] = o[h] * inv[h];
+                    for (int h = 0; h < kHQ; ++h) __stcs(dst + h * kD, o[h] * inv[h]);
                 }
             }
             if (R < kHQ) {
                 if (nsplit == 1) {
                     if (lse_out != nullptr) lse_out[ri.row * kHQ + R] = my_lse;
                 } else {
-                    ws[(size_t)n_items * kHQ * kD + (row_local * nsplit + sp) * kHQ + R] = my_lse;
+                    ws[(size_t)n_items * kHQ * kD + slot * kHQ + R] = my_lse;
                 }
             }
             tc_fence_before();
@@ -518,26 +548,70 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     }
 }
 
-// merge split-K partials: lse = logsumexp_s lse_s, o = sum_s exp(lse_s - lse) o_s
+// merge split-K partials: lse = logsumexp_s lse_s, o = sum_s exp(lse_s - lse) o_s;
+// with bounds, splits (key chunks) whose selection range is empty hold no state
 __global__ void __launch_bounds__(256)
-combine_kernel(const float *__restrict__ ws, int64_t n_items, int nsplit, __nv_bfloat16 *__restrict__ out,
-               float *__restrict__ lse_out)
+combine_kernel(const float *__restrict__ ws, int64_t n_items, int nsplit, const int32_t *__restrict__ bounds,
+               __nv_bfloat16 *__restrict__ out, float *__restrict__ lse_out)
 {
     const int64_t row = blockIdx.x;
     const int h = blockIdx.y;
     const int d = threadIdx.x;
     const float *lp = ws + (size_t)n_items * kHQ * kD + row * nsplit * kHQ + h;
+    const int32_t *bd = bounds ? bounds + row * (nsplit + 1) : nullptr;
     float mx = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) mx = fmaxf(mx, lp[s * kHQ]);
+    for (int s = 0; s < nsplit; ++s)
+        if (bd == nullptr || bd[s + 1] > bd[s]) mx = fmaxf(mx, lp[s * kHQ]);
     float tot = 0.f, acc = 0.f;
     for (int s = 0; s < nsplit; ++s) {
+        if (bd != nullptr && bd[s + 1] <= bd[s]) continue;
         const float l = lp[s * kHQ];
         const float wgt = (l == -INFINITY) ? 0.f : __expf(l - mx);
         tot += wgt;
-        acc += wgt * ws[((row * nsplit + s) * kHQ + h) * kD + d];
+        acc += wgt * __ldcs(ws + ((row * nsplit + s) * kHQ + h) * kD + d);
     }
     out[(row * kHQ + h) * kD + d] = __float2bfloat16_rn(tot > 0.f ? acc / tot : 0.f);
     if (lse_out != nullptr && d == 0) lse_out[row * kHQ + h] = mx + logf(tot);
+}
+
+// key-chunk boundaries of each row's (ascending) selection: bounds[rl][c] = number of
+// selected blocks below c * chunk_blocks, c = 0 .. nchunks (one warp per row)
+__global__ void __launch_bounds__(256)
+chunk_bounds_kernel(const int32_t *__restrict__ sel, const int32_t *__restrict__ cu_q,
+                    const int32_t *__restrict__ cu_k, int batch, int64_t row_begin, int64_t rows, int kb, int r,
+                    int chunk_blocks, int nchunks, int32_t *__restrict__ bounds)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t rl = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (rl >= rows) return;
+    const int64_t row = row_begin + rl;
+    const int s = find_seq(cu_q, batch, row);
+    const int64_t Lq = (int64_t)cu_q[s + 1] - cu_q[s];
+    const int64_t Lk = (int64_t)cu_k[s + 1] - cu_k[s];
+    const int64_t t = (Lk - Lq) + (row - cu_q[s]);
+    int32_t *bd = bounds + rl * (nchunks + 1);
+    if (t < 0) {
+        for (int c = lane; c <= nchunks; c += 32) bd[c] = 0;
+        return;
+    }
+    const int64_t bt = t / r;
+    const int nsel = (int)(bt + 1 < kb ? bt + 1 : kb);
+    const int32_t *srow = sel + row * kb;
+    auto chunk_of = [&](int j) -> int {
+        const int32_t b = __ldg(srow + j);
+        if (b < 0) return 0;
+        const int c = b / chunk_blocks;
+        return c < nchunks ? c : nchunks - 1;
+    };
+    // position j starts its chunk when the previous entry lies in a lower chunk:
+    // bounds[c] = j for every c in (chunk(j - 1), chunk(j)]
+    for (int j = lane; j < nsel; j += 32) {
+        const int cj = chunk_of(j);
+        const int cprev = j > 0 ? chunk_of(j - 1) : -1;
+        for (int c = cprev + 1; c <= cj; ++c) bd[c] = j;
+        if (j == nsel - 1)
+            for (int c = cj + 1; c <= nchunks; ++c) bd[c] = nsel;
+    }
 }
 
 }  // namespace
@@ -575,11 +649,19 @@ size_t split_workspace_bytes(int64_t rows, int nsplit)
     return nsplit > 1 ? (size_t)rows * nsplit * kHQ * (kD + 1) * sizeof(float) : 0;
 }
 
+size_t chunked_workspace_bytes(int64_t rows, int nchunks)
+{
+    const size_t b = ((size_t)rows * (nchunks + 1) * sizeof(int32_t) + 255) & ~(size_t)255;
+    return b + split_workspace_bytes(rows, nchunks);
+}
+
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream)
 {
     const int64_t rows = a.row_end - a.row_begin;
     if (rows <= 0) return cudaSuccess;
-    if (a.nsplit > 1 && a.ws == nullptr) return cudaErrorInvalidValue;
+    const bool chunked = a.nchunks > 1;
+    const int nsplit = chunked ? a.nchunks : a.nsplit;
+    if (nsplit > 1 && a.ws == nullptr) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv;
     // q as [rows_total * 24, 256], 32-row boxes (24 heads + 8 rows of padding)
     if (!make_tmap_2d(&mq, a.q, kD, (uint64_t)a.total_q * kHQ, kD * 2, 64, kQRows)) return cudaErrorInvalidValue;
@@ -591,16 +673,25 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream)
         cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttSmem);
         attr = true;
     }
-    const int64_t n_items = rows * a.nsplit;
+    float *ws = a.ws;
+    int32_t *bounds = nullptr;
+    if (chunked) {
+        bounds = reinterpret_cast<int32_t *>(a.ws);
+        const size_t bb = ((size_t)rows * (a.nchunks + 1) * sizeof(int32_t) + 255) & ~(size_t)255;
+        ws = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(a.ws) + bb);
+        chunk_bounds_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+            a.sel, a.cu_q, a.cu_k, a.batch, a.row_begin, rows, a.kb, a.r, a.chunk_blocks, a.nchunks, bounds);
+    }
+    const int64_t n_items = rows * nsplit;
     int64_t grid = num_sms();
     if (grid > n_items) grid = n_items;
     sparse_attn_kernel<<<(unsigned)grid, kAttThreads, kAttSmem, stream>>>(
-        mq, mk, mv, a.sel, a.cu_q, a.cu_k, a.batch, a.row_begin, n_items, a.nsplit, a.kb, a.r, a.scale,
-        a.o, a.lse, a.ws);
+        mq, mk, mv, a.sel, a.cu_q, a.cu_k, a.batch, a.row_begin, rows, nsplit, a.kb, a.r, a.scale, a.o, a.lse,
+        ws, bounds);
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess || a.nsplit == 1) return e;
+    if (e != cudaSuccess || nsplit == 1) return e;
     dim3 cg((unsigned)rows, kHQ);
-    combine_kernel<<<cg, kD, 0, stream>>>(a.ws, n_items, a.nsplit, a.o + a.row_begin * kHQ * kD,
+    combine_kernel<<<cg, kD, 0, stream>>>(ws, n_items, nsplit, bounds, a.o + a.row_begin * kHQ * kD,
                                           a.lse ? a.lse + a.row_begin * kHQ : nullptr);
     return cudaGetLastError();
 }

@@ -38,7 +38,7 @@ struct DenseShared {
     uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
     uint64_t s_full[2], s_empty[2];
     uint64_t p_full[2], p_empty[2];
-    uint64_t pv_done;
+    uint64_t o_full;  // every PV of the tile has completed
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -143,7 +143,7 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             mbar_init(&sh->p_full[i], 128);
             mbar_init(&sh->p_empty[i], 1);
         }
-        mbar_init(&sh->pv_done, 1);
+        mbar_init(&sh->o_full, 1);
         sh->abort_flag = 0;
         fence_barrier_init();
     }
@@ -202,7 +202,6 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 }
                 mma_commit(&sh->v_empty[b]);
                 mma_commit(&sh->p_empty[b]);
-                mma_commit(&sh->pv_done);
                 return true;
             };
             for (int j = 0; ok && j < nkt; ++j) {
@@ -222,7 +221,7 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 mma_commit(&sh->s_full[b]);
                 if (j >= 1) ok = do_pv(j - 1);
             }
-            if (ok) do_pv(nkt - 1);
+            if (ok && do_pv(nkt - 1)) mma_commit(&sh->o_full);
         }
     } else {
         // ---------------- softmax + epilogue (warps 2..5) ----------------
@@ -260,7 +259,8 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 const float f = exp2f((m - mx) * c2);
                 m = mx;
                 l *= f;
-                if (!(ok = mbar_wait(&sh->pv_done, (j - 1) & 1, abort_flag))) break;
+                // the previous PV has completed once its P buffer's last use is released
+                if (!(ok = mbar_wait(&sh->p_empty[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag))) break;
                 tc_fence_after();
 #pragma unroll 1
                 for (int c = 0; c < kD / 32; ++c) {
@@ -299,7 +299,7 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             tc_fence_before();
             mbar_arrive(&sh->p_full[b]);
         }
-        if (ok) ok = mbar_wait(&sh->pv_done, (nkt - 1) & 1, abort_flag);
+        if (ok) ok = mbar_wait(&sh->o_full, 0, abort_flag);
         if (ok) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;

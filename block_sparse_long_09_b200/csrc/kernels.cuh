@@ -58,10 +58,12 @@ struct AttnArgs {
     int64_t row_begin, row_end;
     __nv_bfloat16 *o;
     float *lse;
-    float *ws;                       // split partials (nsplit > 1)
+    float *ws;                       // split partials (nsplit > 1), or bounds + partials (chunked)
     int nsplit;
     int kb, r;
     float scale;
+    int nchunks = 0;                 // > 1: key-chunked (L2-blocked) schedule
+    int chunk_blocks = 0;            // micro-blocks per key chunk
 };
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream);
 int min_nsplit(int kb);                         // splits needed so each holds <= 16 tiles
@@ -69,6 +71,7 @@ int decode_nsplit(int batch, int kb);           // splits used by the decode cal
 int max_nsplit(int kb);                         // upper bound of decode_nsplit over devices
 int dense_decode_nsplit(int64_t max_len_k, int r);  // splits of the dense flash-decoding path
 size_t split_workspace_bytes(int64_t rows, int nsplit);  // partial (o, lse) states
+size_t chunked_workspace_bytes(int64_t rows, int nchunks);  // bounds + partial states
 
 struct DenseArgs {
     const __nv_bfloat16 *q, *k, *v;

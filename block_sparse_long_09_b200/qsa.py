@@ -45,6 +45,7 @@ class Config(ctypes.Structure):
         ("softmax_scale", ctypes.c_float),
         ("rms_eps", ctypes.c_float),
         ("flags", ctypes.c_uint32),
+        ("kv_chunk_blocks", ctypes.c_int32),
     ]
 
 
@@ -65,7 +66,7 @@ def _load():
         "qsa_compress_keys": (I32, [CP, P, P, P, I32, I64, P, I32, P, P]),
         "qsa_index_scores": (I32, [CP, P, P, P, I64, P, P, P, I32, I64, I32, I64, I64, P, I64, P, SZ, P]),
         "qsa_select_blocks": (I32, [CP, P, I64, P, P, I32, I64, I64, P, P, SZ, P]),
-        "qsa_sparse_attn_prefill": (I32, [CP, P, P, P, P, P, P, I32, I64, I64, I64, I64, P, P, P, SZ, P]),
+        "qsa_sparse_attn_prefill": (I32, [CP, P, P, P, P, P, P, I32, I64, I64, I64, I64, I64, P, P, P, SZ, P]),
         "qsa_sparse_attn_decode": (I32, [CP, P, P, P, P, I32, I64, P, P, P, P, SZ, P]),
         "qsa_dense_attn_prefill": (I32, [CP, P, P, P, P, P, I32, I64, I64, I32, I64, P, P, P, SZ, P]),
         "qsa_workspace_size": (SZ, [CP, I32, I32, I64, I64]),
@@ -175,7 +176,9 @@ def select_blocks(scores, cu_seqlens_q, cu_seqlens_k, total_q: int, row_begin: i
 
 def sparse_attn_prefill(q, k, v, sel, cu_seqlens_q, cu_seqlens_k, row_begin: int = 0,
                         row_end: Optional[int] = None, o=None, lse=None, want_lse: bool = False,
-                        cfg: Optional[Config] = None, ws=None):
+                        cfg: Optional[Config] = None, ws=None, max_len_k: Optional[int] = None):
+    """Sparse attention over the selected blocks.  With a workspace (allocated here
+    when ws is None) long contexts run the L2-blocked key-chunk schedule."""
     cfg = _cfg(cfg)
     total_q = q.shape[0]
     if row_end is None:
@@ -184,12 +187,14 @@ def sparse_attn_prefill(q, k, v, sel, cu_seqlens_q, cu_seqlens_k, row_begin: int
         o = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty((total_q, cfg.n_heads_q), dtype=torch.float32, device=q.device)
+    if max_len_k is None:
+        max_len_k = int((cu_seqlens_k[1:] - cu_seqlens_k[:-1]).max().item())
     batch = cu_seqlens_q.numel() - 1
-    need = workspace_size(OP_PREFILL, batch, row_end - row_begin, 0, cfg)
+    need = workspace_size(OP_PREFILL, batch, row_end - row_begin, max_len_k, cfg)
     if ws is None and need > 0:
         ws = torch.empty((need,), dtype=torch.uint8, device=q.device)
     _check(_lib.qsa_sparse_attn_prefill(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(sel), _p(cu_seqlens_q),
-                                        _p(cu_seqlens_k), batch, total_q, k.shape[0], row_begin, row_end,
+                                        _p(cu_seqlens_k), batch, total_q, k.shape[0], max_len_k, row_begin, row_end,
                                         _p(o), _p(lse), _p(ws), ws.numel() if ws is not None else 0, _stream()),
            "qsa_sparse_attn_prefill")
     return (o, lse) if want_lse or lse is not None else o
@@ -261,6 +266,19 @@ class Prefill:
         self.kc = torch.empty((max(self.n_blocks, 1), 2, self.cfg.idx_dim), dtype=torch.bfloat16, device=self.device)
         self.scores = torch.empty((min(self.chunk, self.total), self.ld), dtype=torch.float32, device=self.device)
         self.sel = torch.empty((self.total, self.cfg.budget_blocks), dtype=torch.int32, device=self.device)
+        rows = min(self.chunk, self.total)
+        need = workspace_size(OP_PREFILL, len(self.seqlens), rows, self.max_len, self.cfg)
+        self.ws = torch.empty((need,), dtype=torch.uint8, device=self.device) if need > 0 else None
+
+    def attend(self, q, k, v, o=None, lse=None):
+        """Sparse attention of every row, chunk of rows by chunk of rows."""
+        if o is None:
+            o = torch.empty_like(q)
+        for r0 in range(0, self.total, self.chunk):
+            r1 = min(self.total, r0 + self.chunk)
+            sparse_attn_prefill(q, k, v, self.sel, self.cu, self.cu, r0, r1, o=o, lse=lse, cfg=self.cfg, ws=self.ws,
+                                max_len_k=self.max_len)
+        return o
 
     def index_select(self, q_idx, w, k_idx):
         compress_keys(k_idx, self.cu, self.cu_blocks, kc=self.kc, cfg=self.cfg)
@@ -273,7 +291,7 @@ class Prefill:
 
     def __call__(self, q, k, v, q_idx, w, k_idx, o=None, lse=None):
         self.index_select(q_idx, w, k_idx)
-        return sparse_attn_prefill(q, k, v, self.sel, self.cu, self.cu, o=o, lse=lse, cfg=self.cfg)
+        return self.attend(q, k, v, o=o, lse=lse)
 
 
 class DecodeStep:

@@ -74,6 +74,8 @@ typedef struct qsa_config {
     float softmax_scale;   /* 1/sqrt(256) */
     float rms_eps;         /* compressor RMSNorm eps (1e-6) */
     uint32_t flags;        /* QSA_COMPRESS_NO_NORM */
+    int32_t kv_chunk_blocks; /* > 0: key-chunk size (micro-blocks) of the L2-blocked prefill
+                                schedule; 0 (default): one pass per query */
 } qsa_config;
 
 /* op ids for qsa_workspace_size */
@@ -85,7 +87,7 @@ typedef struct qsa_config {
 #define QSA_OP_DENSE 5
 
 /* Fill *cfg with the model's values (r 4, k 512, 24/2/256, 4/128, scale 1/16,
- * eps 1e-6, flags 0).  Host only. */
+ * eps 1e-6, flags 0, kv_chunk_blocks 0).  Host only. */
 void qsa_config_init(qsa_config *cfg);
 
 /*
@@ -155,17 +157,24 @@ qsa_status qsa_select_blocks(const qsa_config *cfg, const float *scores, int64_t
  *   o[t, h] = sum_j softmax_j(scale * <q[t, h], k[j, g]>) v[j, g]
  * bf16 tensor-core products, fp32 softmax and accumulation, bf16 output.
  *   q   [total_q, n_heads_q, head_dim] bf16; k, v [total_k, n_heads_kv, head_dim] bf16
- *   sel [total_q, k] int32 as produced by qsa_select_blocks (-1 = unused slot)
+ *   sel [total_q, k] int32 as produced by qsa_select_blocks (ascending, -1 = unused)
  *   rows [row_begin, row_end) of the packed queries are computed
  *   o   [total_q, n_heads_q, head_dim] bf16 written for those rows
  *   lse [total_q, n_heads_q] fp32 natural-log sum-exp of the scaled logits, or NULL
+ *   max_len_k host: max over s of L_k,s
  * A selected block id outside 0 .. b_t is skipped and flagged QSA_ERR_DEVICE_CHECK.
- * Workspace: none (ws may be NULL).
+ * Workspace: none by default.  With cfg->kv_chunk_blocks > 0 and
+ * qsa_workspace_size(cfg, QSA_OP_PREFILL, batch, row_end - row_begin, max_len_k)
+ * bytes, the rows are processed key chunk by key chunk (chunk-major, so the
+ * gathers of a chunk hit L2) and the per-chunk softmax states are merged by a
+ * second kernel; with less (or NULL) one pass per query is used.  Both compute
+ * the same function.  (On B200 at 262144 tokens the single pass is faster: the
+ * gather is bound by the per-SM pipeline, not by DRAM, and the merge costs.)
  */
 qsa_status qsa_sparse_attn_prefill(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k,
                                    const qsa_bf16 *v, const int32_t *sel,
                                    const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
-                                   int32_t batch, int64_t total_q, int64_t total_k,
+                                   int32_t batch, int64_t total_q, int64_t total_k, int64_t max_len_k,
                                    int64_t row_begin, int64_t row_end, qsa_bf16 *o, float *lse,
                                    void *ws, size_t ws_bytes, void *stream);
 

@@ -77,14 +77,19 @@ def test_invalid_arguments_rejected_on_host(qsa):
         qsa.QSA_ERR_INVALID_ARG
     # misaligned q
     assert lib.qsa_sparse_attn_prefill(ctypes.byref(c), ctypes.c_void_p(18), fake, fake, fake, fake, fake, 1, 4,
-                                       4, 0, 4, fake, None, None, 0, None) == qsa.QSA_ERR_INVALID_ARG
+                                       4, 4, 0, 4, fake, None, None, 0, None) == qsa.QSA_ERR_INVALID_ARG
     # empty row range is a no-op
-    assert lib.qsa_sparse_attn_prefill(ctypes.byref(c), fake, fake, fake, fake, fake, fake, 1, 4, 4, 2, 2,
+    assert lib.qsa_sparse_attn_prefill(ctypes.byref(c), fake, fake, fake, fake, fake, fake, 1, 4, 4, 4, 2, 2,
                                        fake, None, None, 0, None) == qsa.QSA_OK
 
 
 def test_workspace_sizes(qsa):
     assert qsa.workspace_size(qsa.OP_INDEX, 1, 8192, 8192) == 0
-    assert qsa.workspace_size(qsa.OP_PREFILL, 1, 8192, 8192) == 0
+    assert qsa.workspace_size(qsa.OP_PREFILL, 1, 8192, 8192) == 0     # single-pass schedule (default)
+    assert qsa.workspace_size(qsa.OP_PREFILL, 1, 16384, 262144) == 0
+    big = qsa.workspace_size(qsa.OP_PREFILL, 1, 16384, 262144, qsa.default_config(kv_chunk_blocks=8192))
+    assert big >= 16384 * 8 * 24 * 257 * 4                             # 8 key chunks of 32768 tokens
+    small = qsa.workspace_size(qsa.OP_PREFILL, 1, 1000, 8192, qsa.default_config(kv_chunk_blocks=64))
+    assert small >= 1000 * 32 * 24 * 257 * 4
     ws = qsa.workspace_size(qsa.OP_DECODE, 64, 64, 262144)
     assert ws >= 64 * 24 * 257 * 4

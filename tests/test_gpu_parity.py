@@ -269,8 +269,8 @@ def test_select_short_rows_and_ragged_batch(qsa):
 # attention
 # ---------------------------------------------------------------------------------------------
 
-def run_chain(qsa, x, lengths, k, chunk=None, want_lse=True):
-    cfg = qsa.default_config(budget_blocks=k)
+def run_chain(qsa, x, lengths, k, chunk=None, want_lse=True, kv_chunk=0):
+    cfg = qsa.default_config(budget_blocks=k, kv_chunk_blocks=kv_chunk)
     pre = qsa.Prefill(lengths, chunk_rows=chunk or 16384, cfg=cfg)
     q, kk, v = x.q.cuda(), x.k.cuda(), x.v.cuda()
     sel = pre.index_select(x.q_idx.cuda(), x.w.cuda(), x.k_idx.cuda())
@@ -288,11 +288,13 @@ def sample_rows(L, n_rand=128, seed=0):
     return np.unique(r[(r >= 0) & (r < L)])
 
 
-@pytest.mark.parametrize("lengths,k", [([512], 16), ([1, 3, 4, 5, 37, 130, 701, 2], 16), ([3000], 512),
-                                       ([100, 2100], 64)])
-def test_attention_on_gpu_selection(qsa, lengths, k):
+@pytest.mark.parametrize("lengths,k,kv_chunk", [([512], 16, 0), ([1, 3, 4, 5, 37, 130, 701, 2], 16, 0),
+                                                ([3000], 512, 0), ([100, 2100], 64, 0),
+                                                ([3000], 512, 64), ([1, 130, 701, 2100], 64, 37)])
+def test_attention_on_gpu_selection(qsa, lengths, k, kv_chunk):
+    """kv_chunk > 0 runs the L2-blocked schedule with tiny key chunks (many chunks per row)."""
     x = inputs.make_prefill(lengths, seed=26)
-    pre, sel, o, lse = run_chain(qsa, x, lengths, k)
+    pre, sel, o, lse = run_chain(qsa, x, lengths, k, kv_chunk=kv_chunk)
     sel_g, o_g, lse_g = sel.cpu().numpy(), o.float().cpu().numpy(), lse.cpu().numpy()
     for s, (a, b) in enumerate(seq_slices(lengths)):
         L = b - a
@@ -334,10 +336,11 @@ def test_full_budget_equals_dense_n8192(qsa):
     status_ok(qsa)
 
 
-def test_chain_n8192_budget512(qsa):
+@pytest.mark.parametrize("kv_chunk", [0, 256])
+def test_chain_n8192_budget512(qsa, kv_chunk):
     n, k = 8192, 512
     x = inputs.make_prefill([n], seed=0)
-    pre, sel, o, lse = run_chain(qsa, x, [n], k, chunk=3000)
+    pre, sel, o, lse = run_chain(qsa, x, [n], k, chunk=3000, kv_chunk=kv_chunk)
     rows = sample_rows(n, 160)
     sel_g = sel.cpu().numpy()
     kc = oracle.compress(x.k_idx, 4)
