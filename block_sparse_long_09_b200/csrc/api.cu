@@ -152,6 +152,9 @@ const char *qsa_status_string(qsa_status s)
     case QSA_ERR_CUDA: return "QSA_ERR_CUDA: a CUDA launch or runtime call failed";
     case QSA_ERR_TIMEOUT: return "QSA_ERR_TIMEOUT: a bounded device-side wait gave up";
     case QSA_ERR_DEVICE_CHECK: return "QSA_ERR_DEVICE_CHECK: a kernel found an out-of-range index and skipped it";
+    case QSA_ERR_SCRATCH_LIMIT:
+        return "QSA_ERR_SCRATCH_LIMIT: the call needs more than the library's fixed 16 MiB decode scratch "
+               "(QSA_STATIC_SCRATCH_BYTES); use qsa_sparse_attn_decode with a workspace";
     default: return "QSA: unknown status";
     }
 }
@@ -319,6 +322,69 @@ qsa_status qsa_dense_attn_prefill(const qsa_config *cfg, const qsa_bf16 *q, cons
     DenseArgs a{bf(q), bf(k), bf(v), cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_len_q, bf(o), lse,
                 cfg->softmax_scale};
     return cuda_status(launch_dense_attn(a, s));
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode with library-held scratch.  For callers that cannot allocate device
+// memory while decoding (a pool that has reserved all free memory up front, a
+// plain C host without a device allocator): the split-K partial states live in
+// a fixed array of the library's device image instead of a caller workspace.
+// Every GPU that loads the library holds the array until the process exits;
+// every call on a device shares it, so calls whose kernels overlap on the GPU
+// race.  Nothing in it needs to start at zero: each call writes every partial
+// state (a neutral one for an empty split) before the merge kernel reads it.
+
+static __device__ __align__(256) float g_decode_scratch[QSA_STATIC_SCRATCH_BYTES / sizeof(float)];
+
+namespace {
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mu;
+void *g_scratch_ptr[kMaxScratchDevices];  // device address of g_decode_scratch, per device ordinal
+
+// Set-up, once per device, with that device current: the array's device
+// address.  The first call on a device therefore does this lookup, which
+// belongs before any stream capture.
+qsa_status decode_scratch(float **out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return QSA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxScratchDevices) return QSA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return QSA_ERR_CUDA;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = static_cast<float *>(g_scratch_ptr[dev]);
+    return QSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+qsa_status qsa_sparse_attn_decode_static_scratch(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k_cache,
+                                                 const qsa_bf16 *v_cache, const int32_t *cu_seqlens_k, int32_t batch,
+                                                 int64_t total_k, const int32_t *sel, qsa_bf16 *o, float *lse,
+                                                 void *stream)
+{
+    qsa_status st = check_config(cfg);
+    if (st != QSA_OK) return st;
+    if (batch <= 0 || total_k <= 0 || cu_seqlens_k == nullptr) return QSA_ERR_INVALID_ARG;
+    if (q == nullptr || k_cache == nullptr || v_cache == nullptr || sel == nullptr || o == nullptr ||
+        !al16(q) || !al16(k_cache) || !al16(v_cache))
+        return QSA_ERR_INVALID_ARG;
+    float *scratch = nullptr;
+    st = decode_scratch(&scratch);
+    if (st != QSA_OK) return st;
+    const int nsplit = decode_nsplit(batch, cfg->budget_blocks);
+    if (split_workspace_bytes(batch, nsplit) > (size_t)QSA_STATIC_SCRATCH_BYTES) return QSA_ERR_SCRATCH_LIMIT;
+    AttnArgs a{bf(q), bf(k_cache), bf(v_cache), sel, nullptr, cu_seqlens_k, batch, batch, total_k, 0, batch,
+               bf(o), lse, nsplit > 1 ? scratch : nullptr, nsplit, cfg->budget_blocks, cfg->r, cfg->softmax_scale};
+    return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

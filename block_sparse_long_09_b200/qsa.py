@@ -23,12 +23,15 @@ QSA_ERR_WORKSPACE_TOO_SMALL = 3
 QSA_ERR_CUDA = 4
 QSA_ERR_TIMEOUT = 5
 QSA_ERR_DEVICE_CHECK = 6
+QSA_ERR_SCRATCH_LIMIT = 7
+STATIC_SCRATCH_BYTES = 16 * 1024 * 1024  # QSA_STATIC_SCRATCH_BYTES
 QSA_COMPRESS_NO_NORM = 0x1
 OP_COMPRESS, OP_INDEX, OP_SELECT, OP_PREFILL, OP_DECODE, OP_DENSE = range(6)
 
 EXPORTED = (
     "qsa_config_init", "qsa_compress_keys", "qsa_index_scores", "qsa_select_blocks",
-    "qsa_sparse_attn_prefill", "qsa_sparse_attn_decode", "qsa_dense_attn_prefill",
+    "qsa_sparse_attn_prefill", "qsa_sparse_attn_decode", "qsa_sparse_attn_decode_static_scratch",
+    "qsa_dense_attn_prefill",
     "qsa_workspace_size", "qsa_status_string", "qsa_get_device_status", "qsa_version",
 )
 
@@ -68,6 +71,7 @@ def _load():
         "qsa_select_blocks": (I32, [CP, P, I64, P, P, I32, I64, I64, P, P, SZ, P]),
         "qsa_sparse_attn_prefill": (I32, [CP, P, P, P, P, P, P, I32, I64, I64, I64, I64, I64, P, P, P, SZ, P]),
         "qsa_sparse_attn_decode": (I32, [CP, P, P, P, P, I32, I64, P, P, P, P, SZ, P]),
+        "qsa_sparse_attn_decode_static_scratch": (I32, [CP, P, P, P, P, I32, I64, P, P, P, P]),
         "qsa_dense_attn_prefill": (I32, [CP, P, P, P, P, P, I32, I64, I64, I32, I64, P, P, P, SZ, P]),
         "qsa_workspace_size": (SZ, [CP, I32, I32, I64, I64]),
         "qsa_status_string": (ctypes.c_char_p, [I32]),
@@ -216,6 +220,19 @@ def sparse_attn_decode(q, k_cache, v_cache, cu_seqlens_k, sel, o=None, lse=None,
                                        ws.numel() if ws is not None else 0, _stream()),
            "qsa_sparse_attn_decode")
     return (o, lse) if want_lse or lse is not None else o
+
+
+def sparse_attn_decode_static_scratch(q, k_cache, v_cache, cu_seqlens_k, sel, o, lse=None,
+                                      cfg: Optional[Config] = None):
+    """Decode attention into the caller's `o` (and `lse`), using the library's fixed
+    device scratch: neither this wrapper nor the call allocates device memory.
+    Calls that overlap on the GPU share that scratch and race."""
+    cfg = _cfg(cfg)
+    _check(_lib.qsa_sparse_attn_decode_static_scratch(ctypes.byref(cfg), _p(q), _p(k_cache), _p(v_cache),
+                                                      _p(cu_seqlens_k), q.shape[0], k_cache.shape[0], _p(sel),
+                                                      _p(o), _p(lse), _stream()),
+           "qsa_sparse_attn_decode_static_scratch")
+    return o
 
 
 def dense_attn_prefill(q, k, v, cu_seqlens_q, cu_seqlens_k, max_len_q: int, o=None, lse=None,

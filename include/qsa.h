@@ -57,6 +57,7 @@ typedef int32_t qsa_status;
 #define QSA_ERR_CUDA 4
 #define QSA_ERR_TIMEOUT 5
 #define QSA_ERR_DEVICE_CHECK 6
+#define QSA_ERR_SCRATCH_LIMIT 7 /* the call needs more than QSA_STATIC_SCRATCH_BYTES */
 
 typedef uint16_t qsa_bf16;
 
@@ -193,6 +194,39 @@ qsa_status qsa_sparse_attn_decode(const qsa_config *cfg, const qsa_bf16 *q,
                                   const int32_t *cu_seqlens_k, int32_t batch, int64_t total_k,
                                   const int32_t *sel, qsa_bf16 *o, float *lse, void *ws,
                                   size_t ws_bytes, void *stream);
+
+/*
+ * Sparse GQA attention, decode, with library-held scratch instead of a caller
+ * workspace.  Computes exactly what qsa_sparse_attn_decode computes, with the
+ * same split-K schedule, and takes the same arguments minus ws / ws_bytes.
+ * The reading notes describe no counterpart of this call: it exists for
+ * callers that cannot allocate device memory at decode time, e.g. a serving
+ * loop whose pool has reserved all free device memory up front, or a plain C
+ * host with no device allocator of its own to hand a workspace from.
+ *
+ * Scratch: a fixed array of QSA_STATIC_SCRATCH_BYTES in the library's device
+ * image; every GPU that loads libqsa.so holds it until the process exits.  The
+ * call allocates and frees nothing (no cudaMalloc / cudaFree, no allocating
+ * library routine).  The first call on a device, with that device current,
+ * looks up the array's device address once (cudaGetSymbolAddress); make that
+ * first call before any stream capture.
+ * Sharing: every call on a device uses the SAME array, so two calls whose
+ * kernels overlap on the GPU (different streams without ordering between them,
+ * or concurrent host threads) race and corrupt each other's results; order
+ * them on one stream.  Nothing in the array has to start at zero: each call
+ * writes every partial state before the merge reads it.
+ * Limit: a call whose split-K partial states need more than
+ * QSA_STATIC_SCRATCH_BYTES returns QSA_ERR_SCRATCH_LIMIT before launching
+ * anything (use qsa_sparse_attn_decode with a workspace there).  With 148 SMs
+ * the schedule keeps batch * splits below 592, i.e. under 14.6 MB, so no batch
+ * size reaches the limit on B200.
+ */
+#define QSA_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+qsa_status qsa_sparse_attn_decode_static_scratch(const qsa_config *cfg, const qsa_bf16 *q,
+                                                 const qsa_bf16 *k_cache, const qsa_bf16 *v_cache,
+                                                 const int32_t *cu_seqlens_k, int32_t batch,
+                                                 int64_t total_k, const int32_t *sel, qsa_bf16 *o,
+                                                 float *lse, void *stream);
 
 /*
  * Dense causal GQA attention (the baseline the pages measure QSA against):

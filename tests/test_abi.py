@@ -47,7 +47,7 @@ def test_config_defaults_and_version(qsa):
 
 def test_status_strings(qsa):
     lib = qsa.library()
-    for s in range(7):
+    for s in range(8):
         assert lib.qsa_status_string(s).decode().startswith("QSA")
 
 
