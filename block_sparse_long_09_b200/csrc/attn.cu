@@ -26,7 +26,8 @@
 //  * Warp roles of a persistent CTA (one per SM):
 //      warp 0      TMA producer: Q (per item), then K/V tiles in MMA order
 //                  (K0, K1, V0, K2, V1, ...) through a 3-slot ring of 64 KB;
-//                  block ids are fetched two tiles ahead
+//                  block ids are loaded three tiles ahead (across items) and
+//                  checked at use, so their latency stays off the issue path
 //      warp 1      TMEM owner + single-thread tcgen05.mma issue: S(j+1) is
 //                  issued before PV(j) so QK^T overlaps the softmax
 //      warps 2..5  softmax (thread = TMEM lane = (token, group) row) and the
@@ -133,22 +134,46 @@ __device__ __forceinline__ RowInfo row_info(int64_t item, int nsplit, int64_t ro
     return ri;
 }
 
-// block id at selection position pos of an item: -1 outside [p0, p1) or for an id
-// outside 0 .. b_t; without a selection (sel == nullptr, dense attention) position
-// pos is block pos
-__device__ __forceinline__ int32_t fetch_block(const int32_t *sel, const RowInfo &ri, int kb, int pos)
+constexpr int32_t kNoBlock = INT32_MIN;  // a position past the item's selection range
+
+// raw block id at selection position pos of an item, unchecked (so that the load's
+// latency is paid only where the id is used): kNoBlock outside [p0, p1); without a
+// selection (sel == nullptr, dense attention) position pos is block pos
+__device__ __forceinline__ int32_t load_block(const int32_t *sel, const RowInfo &ri, int kb, int pos)
 {
-    if (pos >= ri.p1) return -1;
+    if (pos >= ri.p1) return kNoBlock;
     if (sel == nullptr) return pos;
-    const int32_t blk = __ldg(sel + ri.row * kb + pos);
-    if (blk < 0 || blk > ri.bt) {
+    return __ldg(sel + ri.row * kb + pos);
+}
+
+// the id to gather, or -1 (nothing: past the range, or an id outside 0 .. b_t,
+// which is flagged)
+__device__ __forceinline__ int32_t check_block(int32_t raw, const RowInfo &ri)
+{
+    if (raw == kNoBlock) return -1;
+    if (raw < 0 || raw > ri.bt) {
         set_device_status(QSA_ERR_DEVICE_CHECK);
         return -1;
     }
-    return blk;
+    return raw;
 }
 
 __device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// barrier of the 128 softmax threads that also ORs a predicate over them
+__device__ __forceinline__ bool softmax_any(bool x)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)x)
+        : "memory");
+    return r != 0;
+}
 
 __device__ __forceinline__ void st_shared_b16(uint32_t addr, uint16_t v)
 {
@@ -255,14 +280,38 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             ++slot_it;
             return true;
         };
+        // Block ids stream through a window w0..w3 of raw loads that runs three tiles
+        // ahead of the issue point, across item boundaries (the same item order as the
+        // issue loop); an id is checked only when its tile is issued.
+        int64_t pf_item = blockIdx.x;
+        RowInfo pf_ri;
+        pf_ri.nt = 0;
+        int pf_tile = 0;
+        auto pf_seek = [&]() {  // the cursor's next item with tiles, or past the end
+            for (; pf_item < n_items; pf_item += gridDim.x) {
+                pf_ri = row_info(pf_item, nsplit, rows, row_begin, cu_q, cu_k, batch, kb, r, bounds);
+                if (pf_ri.nt > 0) return;
+            }
+        };
+        auto pf_next = [&]() -> int32_t {  // this lane's raw id of the cursor's tile; advance
+            int32_t v = kNoBlock;
+            if (pf_item < n_items) {
+                if (lane < kBlkTile) v = load_block(sel, pf_ri, kb, pf_ri.p0 + pf_tile * kBlkTile + lane);
+                if (++pf_tile == pf_ri.nt) {
+                    pf_tile = 0;
+                    pf_item += gridDim.x;
+                    pf_seek();
+                }
+            }
+            return v;
+        };
+        pf_seek();
+        int32_t w0 = pf_next();
+        int32_t w1 = pf_next();
+        int32_t w2 = pf_next();
         for (int64_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
             const RowInfo ri = row_info(item, nsplit, rows, row_begin, cu_q, cu_k, batch, kb, r, bounds);
             if (ri.nt == 0) continue;
-            int32_t b0 = -1, b1 = -1;
-            if (lane < kBlkTile) {
-                b0 = fetch_block(sel, ri, kb, ri.p0 + lane);
-                if (ri.nt > 1) b1 = fetch_block(sel, ri, kb, ri.p0 + kBlkTile + lane);
-            }
             if (lane == 0) {
                 ok = mbar_wait(&sh->q_empty, (q_it & 1) ^ 1, abort_flag);
                 if (ok) {
@@ -274,14 +323,14 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             ok = __shfl_sync(0xffffffffu, ok, 0);
             ++q_it;
             if (!ok) break;
-            ok = issue(&map_k, ri, b0);
+            ok = issue(&map_k, ri, check_block(w0, ri));
             for (int jl = 0; ok && jl < ri.nt; ++jl) {
-                int32_t b2 = -1;
-                if (lane < kBlkTile && jl + 2 < ri.nt) b2 = fetch_block(sel, ri, kb, ri.p0 + (jl + 2) * kBlkTile + lane);
-                if (jl + 1 < ri.nt) ok = issue(&map_k, ri, b1);
-                if (ok) ok = issue(&map_v, ri, b0);
-                b0 = b1;
-                b1 = b2;
+                const int32_t w3 = pf_next();
+                if (jl + 1 < ri.nt) ok = issue(&map_k, ri, check_block(w1, ri));
+                if (ok) ok = issue(&map_v, ri, check_block(w0, ri));
+                w0 = w1;
+                w1 = w2;
+                w2 = w3;
             }
         }
         if (!ok && lane == 0) {
@@ -380,20 +429,25 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             const int nt = ri.nt;
             float m[kHQ];                             // running max per head (raw logits), identical in all threads
             float l[kGrp];                            // this row's share of the row sums, own group's heads
+            float mc[kGrp];                           // own group: m * scale * log2(e)
 #pragma unroll
             for (int h = 0; h < kGrp; ++h) l[h] = 0.f;
 #pragma unroll
             for (int h = 0; h < kHQ; ++h) m[h] = 0.f;
-            int32_t blk_next = fetch_block(sel, ri, kb, ri.p0 + blk_slot);
+            // raw ids two tiles ahead, checked at use (the producer flags bad ids)
+            int32_t raw0 = load_block(sel, ri, kb, ri.p0 + blk_slot);
+            int32_t raw1 = nt > 1 ? load_block(sel, ri, kb, ri.p0 + kBlkTile + blk_slot) : kNoBlock;
             for (int jl = 0; ok && jl < nt; ++jl) {
-                const int32_t blk = blk_next;
-                if (jl + 1 < nt) blk_next = fetch_block(sel, ri, kb, ri.p0 + (jl + 1) * kBlkTile + blk_slot);
+                const int32_t blk = check_block(raw0, ri);
+                raw0 = raw1;
+                raw1 = jl + 2 < nt ? load_block(sel, ri, kb, ri.p0 + (jl + 2) * kBlkTile + blk_slot) : kNoBlock;
                 const bool valid = blk >= 0 && (int64_t)blk * r + tok_in_blk <= ri.t;
                 const uint32_t sb = s_it & 1, sround = s_it >> 1;
                 if (!(ok = mbar_wait(&sh->s_full[sb], sround & 1, abort_flag))) break;
                 tc_fence_after();
-                float s[32];
-                tmem_ld32(tmem + lane_addr + kSCol + sb * 32, s);
+                float s[kHQ];  // columns 0..23: the real heads (24..31 pad)
+                tmem_ld16(tmem + lane_addr + kSCol + sb * 32, s);
+                tmem_ld8(tmem + lane_addr + kSCol + sb * 32 + 16, s + 16);
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&sh->s_empty[sb]);
@@ -401,68 +455,85 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                 float v[kGrp];
 #pragma unroll
                 for (int h = 0; h < kGrp; ++h) v[h] = valid ? (g ? s[kGrp + h] : s[h]) : -INFINITY;
-                // exact per-head tile max: lanes of equal parity hold the same group
-                float tm[kGrp];
+                // The running max only moves when some logit of the tile exceeds it by the
+                // lazy-rescale margin (or on the item's first tile).  Every row tests its own
+                // heads and one barrier ORs the answers; only then is the exact per-head tile
+                // max reduced over the 128 rows.
+                bool full = jl == 0;
+                if (!full) {
+                    bool ex = false;
 #pragma unroll
-                for (int h = 0; h < kGrp; ++h) {
-                    float x = v[h];
-                    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
-                    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
-                    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 4));
-                    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));
-                    tm[h] = x;
+                    for (int h = 0; h < kGrp; ++h) ex |= fmaf(v[h], c2, -mc[h]) > kRescaleLog2;
+                    full = softmax_any(ex);
                 }
-                const int par = tile_it & 1;
-                if (lane < 2) {
+                if (full) {
+                    // exact per-head tile max: lanes of equal parity hold the same group
+                    float tm[kGrp];
 #pragma unroll
-                    for (int h = 0; h < kGrp; ++h) sh->red_max[par][quad][lane][h] = tm[h];
-                }
-                softmax_bar();
-                float tmax[kHQ];
+                    for (int h = 0; h < kGrp; ++h) {
+                        float x = v[h];
+                        x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
+                        x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
+                        x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 4));
+                        x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));
+                        tm[h] = x;
+                    }
+                    const int par = tile_it & 1;
+                    if (lane < 2) {
 #pragma unroll
-                for (int h = 0; h < kHQ; ++h) {
-                    const int gg = h / kGrp, hh = h % kGrp;
-                    tmax[h] = fmaxf(fmaxf(sh->red_max[par][0][gg][hh], sh->red_max[par][1][gg][hh]),
-                                    fmaxf(sh->red_max[par][2][gg][hh], sh->red_max[par][3][gg][hh]));
-                }
-                ++tile_it;
-                if (jl == 0) {
+                        for (int h = 0; h < kGrp; ++h) sh->red_max[par][quad][lane][h] = tm[h];
+                    }
+                    softmax_bar();
+                    float tmax[kHQ];
 #pragma unroll
-                    for (int h = 0; h < kHQ; ++h) m[h] = tmax[h] == -INFINITY ? 0.f : tmax[h];
-                } else {
-                    bool need = false;
+                    for (int h = 0; h < kHQ; ++h) {
+                        const int gg = h / kGrp, hh = h % kGrp;
+                        tmax[h] = fmaxf(fmaxf(sh->red_max[par][0][gg][hh], sh->red_max[par][1][gg][hh]),
+                                        fmaxf(sh->red_max[par][2][gg][hh], sh->red_max[par][3][gg][hh]));
+                    }
+                    ++tile_it;
+                    if (jl == 0) {
 #pragma unroll
-                    for (int h = 0; h < kHQ; ++h) need |= tmax[h] > m[h] + rescale_raw;
-                    if (need) {  // uniform: every thread computed the same maxima
-                        float f[32];
+                        for (int h = 0; h < kHQ; ++h) m[h] = tmax[h] == -INFINITY ? 0.f : tmax[h];
+                    } else {
+                        bool need = false;
 #pragma unroll
-                        for (int h = 0; h < 32; ++h) f[h] = 1.f;
+                        for (int h = 0; h < kHQ; ++h) need |= tmax[h] > m[h] + rescale_raw;
+                        if (need) {  // uniform: every thread computed the same maxima
+                            float f[32];
 #pragma unroll
-                        for (int h = 0; h < kHQ; ++h) {
-                            const float mn = fmaxf(m[h], tmax[h]);
-                            f[h] = exp2f((m[h] - mn) * c2);
-                            m[h] = mn;
+                            for (int h = 0; h < 32; ++h) f[h] = 1.f;
+#pragma unroll
+                            for (int h = 0; h < kHQ; ++h) {
+                                const float mn = fmaxf(m[h], tmax[h]);
+                                f[h] = exp2f((m[h] - mn) * c2);
+                                m[h] = mn;
+                            }
+#pragma unroll
+                            for (int h = 0; h < kGrp; ++h) l[h] *= g ? f[kGrp + h] : f[h];
+                            // O^T must be stable: wait for the previous PV (the completion of the
+                            // last use of its P buffer), then scale it in TMEM
+                            {
+                                const uint32_t x = p_it - 1;
+                                if (!(ok = mbar_wait(&sh->p_empty[x % kNP], (x / kNP) & 1, abort_flag))) break;
+                            }
+                            tc_fence_after();
+#pragma unroll
+                            for (int half = 0; half < 2; ++half) {
+                                float o[32];
+                                const uint32_t ta = tmem + lane_addr + kOCol + half * 32;
+                                tmem_ld32(ta, o);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int h = 0; h < 32; ++h) o[h] *= f[h];
+                                tmem_st32(ta, o);
+                            }
+                            tmem_wait_st();
                         }
+                    }
 #pragma unroll
-                        for (int h = 0; h < kGrp; ++h) l[h] *= g ? f[kGrp + h] : f[h];
-                        // O^T must be stable: wait for the previous PV (the completion of the
-                        // last use of its P buffer), then scale it in TMEM
-                        {
-                            const uint32_t x = p_it - 1;
-                            if (!(ok = mbar_wait(&sh->p_empty[x % kNP], (x / kNP) & 1, abort_flag))) break;
-                        }
-                        tc_fence_after();
-#pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-                            float o[32];
-                            const uint32_t ta = tmem + lane_addr + kOCol + half * 32;
-                            tmem_ld32(ta, o);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int h = 0; h < 32; ++h) o[h] *= f[h];
-                            tmem_st32(ta, o);
-                        }
-                        tmem_wait_st();
+                    for (int h = 0; h < kGrp; ++h) {
+                        mc[h] = (g ? m[kGrp + h] : m[h]) * c2;
                     }
                 }
                 // P = exp(S - m) for the row's own-group heads; the rest of P^T stays zero
@@ -471,8 +542,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                 const uint32_t pbase = p_addr + pb * kPBytes + p_row_off;
 #pragma unroll
                 for (int h = 0; h < kGrp; ++h) {
-                    const float mh = g ? m[kGrp + h] : m[h];
-                    const float p = valid ? exp2f((v[h] - mh) * c2) : 0.f;
+                    const float p = exp2f(fmaf(v[h], c2, -mc[h]));  // v = -inf (masked) gives 0
                     l[h] += p;
                     const int hq = g * kGrp + h;
                     const uint32_t addr = pbase + (hq >> 3) * 1024 + (hq & 7) * 128 + ((p_unit ^ (hq & 7)) << 4);

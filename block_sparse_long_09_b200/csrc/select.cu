@@ -6,25 +6,30 @@
 // blocks 0 .. b_t - 1.  Ties go to the lower block index; the output lists the
 // chosen blocks in ascending order, padded with -1.
 //
-// One CTA per query row, about 41 KB of shared memory: 128 threads when there
-// are many rows (prefill), so several rows are in flight on every SM and their
+// One CTA per query row, about 21 KB of shared memory: 128 threads when there
+// are many rows (prefill), so eight rows are in flight on every SM and their
 // memory latency overlaps; 512 threads when rows are few (decode).  The fp32
 // scores become order-preserving 32-bit keys (sign-flip trick, -0.0 folded
 // into +0.0).
-//  * Fast path (rows of up to 65536 candidates): a strided sample of 1024 keys
-//    yields a conservative lower bound on the threshold (its rank in the
-//    sample is 4 sigma above the expected one); one pass over the row (32 keys
-//    in flight per thread, a float compare per key and a warp vote per four)
-//    lists every key at or above the bound with warp-aggregated appends; the exact (k-1)-th key is then found on that
-//    short list by an MSD radix select with 8-bit digits.  Each score is read
-//    from global memory once.
-//  * General path (the bound missed, the list overflowed, or a longer row):
-//    the same radix select over every key, read from global memory per digit.
-// Winners land in two bitmaps -- "above the threshold" and "equal to it" -- and
-// only when the threshold value is shared by more keys than slots left does a
-// scan of the "equal" bitmap pick the lowest indices; one block scan of the
-// bitmap popcounts gives every winner its output position, so the list comes
-// out ascending without a sort.
+//  * Fast path (16-byte aligned rows of up to 65536 candidates):
+//    - bound: a sample of 1024..2048 keys spread over the row; two 8-bit
+//      digits of a radix select over the sample keys relative to their minimum
+//      locate the sample of rank r_lo (4 sigma above the expected rank of the
+//      threshold), and the smallest sample of that bin is a conservative lower
+//      bound;
+//    - one pass over the row (32 keys in flight per thread): every warp votes
+//      key >= bound, and right after its loads lists its own candidates (index
+//      and score, the score re-read from L1) in a private list;
+//    - an MSD radix select with 8-bit digits over the candidates' keys relative
+//      to the bound, started at their highest differing bit, finds the exact
+//      (k-1)-th key; the winners' bits are set in a bitmap, a block scan of its
+//      word popcounts gives every winner its output slot, so the list comes out
+//      ascending without a sort.
+//  * General path (the bound missed, a list overflowed, the threshold value is
+//    shared by more keys than slots left, an unaligned or a longer row): a
+//    radix select with 11-bit digits over every key, read from global memory
+//    per digit, then bitmaps of the keys above and equal to the threshold per
+//    65536-key segment; the lowest indices win among equal keys.
 #include "kernels.cuh"
 
 namespace qsa {
@@ -32,12 +37,22 @@ namespace qsa {
 namespace {
 
 constexpr int kMaxSelWarps = 16;
-constexpr int kBins = 256;                   // 8-bit digits
+constexpr int kBins = 2048;                  // 11-bit digits (sample pass, general path)
+constexpr int kCandBits = 8;                 // digits of the exact select over the candidates
 constexpr int kSegWords = 2048;              // bitmap segment: 65536 candidates
 constexpr int kSegElems = kSegWords * 32;
-constexpr int kCandCap = 3072;               // fast-path list
-constexpr int kSampleMax = 1024;             // strided sample that bounds the threshold
-constexpr int kSelSmem = (kBins + 2 * kSegWords + 2 * kCandCap) * 4;  // 41 KB
+constexpr int kCandCap = 2048;               // candidate lists (and the sample)
+constexpr int kSampleMin = 1024;
+
+// shared memory: region A (kSegWords words: histogram, then the winner bitmap),
+// region B (kCandCap words: sample keys, then candidate scores, then bitmap word
+// prefixes), 16-bit candidate indices, and a 32-word ballot stage per warp
+template <int kSelThreads>
+constexpr int sel_smem_bytes()
+{
+    return kSegWords * 4 + kCandCap * 4 + kCandCap * 2 + (kSelThreads / 32) * 32 * 4;
+}
+static_assert(kBins <= kSegWords, "the histogram lives in region A");
 
 __device__ __forceinline__ uint32_t order_key(float x)
 {
@@ -54,8 +69,9 @@ __device__ __forceinline__ float key_value(uint32_t k)
 
 struct SelScratch {
     int warp_tot[kMaxSelWarps];
+    uint32_t warp_val[kMaxSelWarps];
+    int warp_cnt[kMaxSelWarps];  // candidates listed per warp
     int digit, above;
-    int cand_n;
 };
 
 // block-wide exclusive scan of one int per thread; every thread gets the total
@@ -84,29 +100,48 @@ __device__ __forceinline__ int block_exclusive_scan(int v, SelScratch *sc, int *
     return before + incl - v;
 }
 
-// hist[0 .. 256) counts the keys still in play by digit: find the digit whose bin
-// holds the need-th largest key.  *above = keys in higher bins.
-template <int kSelThreads>
-__device__ __forceinline__ int find_digit(const uint32_t *hist, int need, SelScratch *sc, int *above_out)
+// block-wide sum (or max) of one value per thread (warp-uniform inputs allowed)
+template <int kSelThreads, bool kMax>
+__device__ __forceinline__ uint32_t block_reduce(uint32_t v, SelScratch *sc)
 {
+    constexpr int kSelWarps = kSelThreads / 32;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    v = kMax ? __reduce_max_sync(0xffffffffu, v) : __reduce_add_sync(0xffffffffu, v);
+    if (lane == 0) sc->warp_val[wid] = v;
+    __syncthreads();
+    uint32_t r = 0u;
+#pragma unroll
+    for (int w = 0; w < kSelWarps; ++w) r = kMax ? (r > sc->warp_val[w] ? r : sc->warp_val[w]) : r + sc->warp_val[w];
+    __syncthreads();
+    return r;
+}
+
+// hist[0 .. nb) counts the keys still in play by digit (nb a power of two <=
+// 2^kBitsMax): find the digit whose bin holds the need-th largest key (1 <= need
+// <= keys in play).  *above = keys in higher bins.
+template <int kSelThreads, int kBitsMax>
+__device__ __forceinline__ int find_digit(const uint32_t *hist, int nb, int need, SelScratch *sc, int *above_out)
+{
+    constexpr int kPer = (1 << kBitsMax) >= kSelThreads ? (1 << kBitsMax) / kSelThreads : 1;
     const int tid = threadIdx.x;
-    constexpr int per = kBins >= kSelThreads ? kBins / kSelThreads : 1;  // digits per thread, highest first
-    const int top = kBins - tid * per;                                  // owns digits [top - per, top)
-    const bool owns = top > 0;
+    const int per = (nb + kSelThreads - 1) / kSelThreads;
+    const int top = nb - tid * per;  // this thread owns bins [top - per, top), highest first
     int mine = 0;
 #pragma unroll
-    for (int q = 1; q <= per; ++q) mine += owns ? (int)hist[top - q] : 0;
+    for (int q = 1; q <= kPer; ++q)
+        if (q <= per && top - q >= 0) mine += (int)hist[top - q];
     int tot;
     int above = block_exclusive_scan<kSelThreads>(mine, sc, &tot);
 #pragma unroll
-    for (int q = 1; q <= per; ++q) {
-        if (!owns) break;
-        const int h = (int)hist[top - q];
-        if (above < need && above + h >= need) {
-            sc->digit = top - q;
-            sc->above = above;
+    for (int q = 1; q <= kPer; ++q) {
+        if (q <= per && top - q >= 0) {
+            const int h = (int)hist[top - q];
+            if (above < need && above + h >= need) {
+                sc->digit = top - q;
+                sc->above = above;
+            }
+            above += h;
         }
-        above += h;
     }
     __syncthreads();
     const int d = sc->digit;
@@ -115,34 +150,41 @@ __device__ __forceinline__ int find_digit(const uint32_t *hist, int need, SelScr
     return d;
 }
 
-// MSD radix select over keys get(0 .. count): locate the need-th largest key.
-// Returns the resolved digits as prefix/mask; *need_left = keys equal to the
-// prefix still needed, *in_bin = keys equal to the prefix.
-template <int kSelThreads, typename Get>
-__device__ __forceinline__ void radix_select(Get get, int count, int need, uint32_t *hist, SelScratch *sc,
-                                             uint32_t *prefix_out, uint32_t *mask_out, int *need_left,
-                                             int *in_bin_out)
+// MSD radix select over the keys that visit(f) hands to f (each thread its own
+// share), whose bits above `top` are all zero: locate the need-th largest key
+// (1 <= need <= count) with kBits-bit digits from bit `top` down, at most
+// max_passes digits.  Returns the resolved bits as prefix/mask (the prefix alone
+// is a lower bound on the key); *need_left = keys equal to the prefix still
+// needed, *in_bin = keys equal to it.
+template <int kSelThreads, int kBits, typename Visit>
+__device__ __forceinline__ void radix_select(Visit visit, int count, int need, int top, uint32_t *hist,
+                                             SelScratch *sc, uint32_t *prefix_out, uint32_t *mask_out,
+                                             int *need_left, int *in_bin_out, int max_passes = 32)
 {
     const int tid = threadIdx.x;
-    uint32_t prefix = 0u, mask = 0u;
+    uint32_t prefix = 0u;
+    uint32_t mask = top >= 31 ? 0u : ~((2u << top) - 1u);
     int in_bin = count;
+    int hi = top;
 #pragma unroll 1
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int b = tid; b < kBins; b += kSelThreads) hist[b] = 0u;
+    while (true) {
+        const int lo = hi - (kBits - 1) > 0 ? hi - (kBits - 1) : 0;
+        const int nb = 1 << (hi - lo + 1);
+        for (int b = tid; b < nb; b += kSelThreads) hist[b] = 0u;
         __syncthreads();
-        for (int i = tid; i < count; i += kSelThreads) {
-            const uint32_t u = get(i);
-            if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 0xFFu], 1u);
-        }
+        visit([&](uint32_t u) {
+            if ((u & mask) == prefix) atomicAdd(&hist[(u >> lo) & (uint32_t)(nb - 1)], 1u);
+        });
         __syncthreads();
         int ab;
-        const int d = find_digit<kSelThreads>(hist, need, sc, &ab);
+        const int d = find_digit<kSelThreads, kBits>(hist, nb, need, sc, &ab);
         need -= ab;
-        prefix |= (uint32_t)d << shift;
-        mask |= 0xFFu << shift;
+        prefix |= (uint32_t)d << lo;
+        mask |= (uint32_t)(nb - 1) << lo;
         in_bin = (int)hist[d];
         __syncthreads();
-        if (need == in_bin) break;  // the whole bin is taken: no finer digit matters
+        if (need == in_bin || lo == 0 || --max_passes == 0) break;  // bin taken whole, or resolved
+        hi = lo - 1;
     }
     *prefix_out = prefix;
     *mask_out = mask;
@@ -152,7 +194,8 @@ __device__ __forceinline__ void radix_select(Get get, int count, int need, uint3
 
 // Ordered emission of one bitmap segment: winners are gtw bits plus, when
 // `partial`, the lowest-index eqw bits while the running equal-rank stays below
-// `need`; otherwise all eqw bits.  Writes out[pos] = seg0 + bit index.
+// `need` (otherwise gtw already holds the equal keys).  Writes out[pos] = seg0 +
+// bit index.
 template <int kSelThreads>
 __device__ __forceinline__ void emit_segment(const uint32_t *gtw, const uint32_t *eqw, int words, int seg0,
                                              bool partial, int need, int need_total, int *out_base,
@@ -182,9 +225,9 @@ __device__ __forceinline__ void emit_segment(const uint32_t *gtw, const uint32_t
             wsel[q] = ((w0 + q < words) ? gtw[w0 + q] : 0u) | taken;
         }
         *eq_base += etot;
-    } else {
+    } else {  // every key equal to the threshold wins: they are in gtw already
 #pragma unroll
-        for (int q = 0; q < kWordsPerThread; ++q) wsel[q] = (w0 + q < words) ? (gtw[w0 + q] | eqw[w0 + q]) : 0u;
+        for (int q = 0; q < kWordsPerThread; ++q) wsel[q] = (w0 + q < words) ? gtw[w0 + q] : 0u;
     }
     int cnt = 0;
 #pragma unroll
@@ -205,19 +248,19 @@ __device__ __forceinline__ void emit_segment(const uint32_t *gtw, const uint32_t
 }
 
 template <int kSelThreads>
-__global__ void __launch_bounds__(kSelThreads)
+__global__ void __launch_bounds__(kSelThreads, kSelThreads == 128 ? 8 : 2)
 select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ cu_q,
               const int32_t *__restrict__ cu_k, int batch, int64_t row_begin, int k, int r,
               int32_t *__restrict__ sel)
 {
-    extern __shared__ uint32_t smem_sel[];
-    uint32_t *hist = smem_sel;                     // kBins
-    uint32_t *gtw = hist + kBins;                  // kSegWords: key above the threshold
-    uint32_t *eqw = gtw + kSegWords;               // kSegWords: key equal to the threshold
-    uint32_t *cand_key = eqw + kSegWords;          // kCandCap (the sample first)
-    uint32_t *cand_idx = cand_key + kCandCap;      // kCandCap
-    __shared__ SelScratch sc;
     constexpr int kSelWarps = kSelThreads / 32;
+    constexpr int kCapW = kCandCap / kSelWarps;         // candidate list of one warp
+    extern __shared__ uint32_t smem_sel[];
+    uint32_t *regA = smem_sel;                          // kSegWords
+    uint32_t *regB = regA + kSegWords;                  // kCandCap
+    uint16_t *cidx = reinterpret_cast<uint16_t *>(regB + kCandCap);  // kCandCap
+    uint32_t *stage = reinterpret_cast<uint32_t *>(cidx + kCandCap);  // 32 words per warp
+    __shared__ SelScratch sc;
 
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int64_t i = row_begin + blockIdx.x;
@@ -254,120 +297,198 @@ select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__res
 
     // ============================ fast path ============================
     bool done = false;
-    if (n <= kSegElems) {
-        const int ns = n < kSampleMax ? n : kSampleMax;
-        for (int w = tid; w < kSegWords; w += kSelThreads) {
-            gtw[w] = 0u;
-            eqw[w] = 0u;
+    if (n <= kSegElems && (reinterpret_cast<uintptr_t>(srow) & 15u) == 0) {
+        // ---- bound from a sample: about 16 expected winners, 1024..2048 keys ----
+        int ns = (int)min((int64_t)kCandCap, max((int64_t)kSampleMin, (int64_t)16 * n / need_total));
+        if (ns > n) ns = n;
+        uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+        for (int q = tid; q < ns; q += kSelThreads) {
+            const uint32_t u = order_key(__ldg(srow + (int)(((int64_t)q * n) / ns)));
+            regB[q] = u;
+            kmin = u < kmin ? u : kmin;
+            kmax = u > kmax ? u : kmax;
         }
-        const int stride = n / ns;
-        for (int q = tid; q < ns; q += kSelThreads) cand_key[q] = order_key(__ldg(srow + q * stride));
-        if (tid == 0) sc.cand_n = 0;
-        __syncthreads();
-        // bound: the r_lo-th largest sample key, r_lo = mean + 4 sigma + 8 ranks.  When
-        // the radix select stops on a bin taken whole, the prefix (the bin's smallest
-        // possible key) is a bound as well.
+        kmin = ~block_reduce<kSelThreads, true>(~kmin, &sc);
+        kmax = block_reduce<kSelThreads, true>(kmax, &sc);
+        // r_lo = mean + 4 sigma + 8 ranks
         const float mu = (float)need_total * (float)ns / (float)n;
         int r_lo = (int)ceilf(mu + 4.f * sqrtf(mu) + 8.f);
         if (r_lo > ns) r_lo = ns;
         uint32_t lo_key;
         {
+            const uint32_t sspan = kmax - kmin;
             uint32_t mk;
             int nl, ib;
-            radix_select<kSelThreads>([&](int q) { return cand_key[q]; }, ns, r_lo, hist, &sc, &lo_key, &mk, &nl, &ib);
-        }
-        __syncthreads();
-        // one pass over the row: list every key >= lo_key.  Most keys are below the
-        // bound, so the test is a float compare (lo_val is the bound's value; -0.0
-        // compares equal to +0.0, like the keys) with one vote per 4 keys, and only a
-        // warp that holds a candidate pays for the ballots and appends.
-        const float lo_val = key_value(lo_key);
-        auto append = [&](float x, int j, bool c) {
-            const uint32_t cb = __ballot_sync(0xffffffffu, c);
-            if (cb == 0u) return;
-            int base = 0;
-            if (lane == 0) base = atomicAdd(&sc.cand_n, __popc(cb));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            const int p = base + __popc(cb & ((1u << lane) - 1u));
-            if (c && p < kCandCap) {
-                cand_key[p] = order_key(x);
-                cand_idx[p] = (uint32_t)j;
+            radix_select<kSelThreads, 8>(
+                [&](auto f) {
+                    for (int q = tid; q < ns; q += kSelThreads) f(regB[q] - kmin);
+                },
+                ns, r_lo, sspan != 0u ? 31 - __clz(sspan) : 0, regA, &sc, &lo_key, &mk, &nl, &ib, 2);
+            if (mk != 0xFFFFFFFFu) {
+                // stopped on a bin with the sample of rank r_lo in it: its smallest key
+                // ranks r_lo or a little below (the bin's floor would be a looser bound)
+                uint32_t mn = 0xFFFFFFFFu;
+                for (int q = tid; q < ns; q += kSelThreads) {
+                    const uint32_t u = regB[q] - kmin;
+                    if ((u & mk) == lo_key && u < mn) mn = u;
+                }
+                lo_key = ~block_reduce<kSelThreads, true>(~mn, &sc);
             }
-        };
-        if ((reinterpret_cast<uintptr_t>(srow) & 15u) == 0) {
-            const float4 *s4 = reinterpret_cast<const float4 *>(srow);
-            const int n4 = (n + 3) >> 2;
-            const int n4full = n >> 2;
-            constexpr float kNeg = -INFINITY;
-            for (int j0 = tid; j0 - tid < n4; j0 += 8 * kSelThreads) {  // uniform trip count
-                float4 v[8];
+            lo_key += kmin;
+        }
+        // ---- one pass over the row; every warp lists its own candidates ----
+        // A float compare against the bound's value is the same test as the key
+        // compare (-0.0 compares equal to +0.0, like the keys).
+        const float lo_val = key_value(lo_key);
+        const float4 *s4 = reinterpret_cast<const float4 *>(srow);
+        const int n4 = (n + 3) >> 2;
+        const int n4full = n >> 2;
+        constexpr float kNeg = -INFINITY;
+        float *craw = reinterpret_cast<float *>(regB) + wid * kCapW;
+        uint16_t *cix = cidx + wid * kCapW;
+        uint32_t *wst = stage + wid * 32;
+        int wc = 0;  // this warp's list length (warp-uniform)
+        for (int j0 = tid; j0 - tid < n4; j0 += 8 * kSelThreads) {  // uniform trip count
+            float4 v[8];
+            if ((j0 - tid) + 8 * kSelThreads <= n4full) {
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {  // 32 keys in flight per thread
+                for (int q = 0; q < 8; ++q) v[q] = __ldg(s4 + j0 + q * kSelThreads);  // 32 keys in flight
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
                     const int j4 = j0 + q * kSelThreads;
-                    v[q] = j4 < n4full ? __ldg(s4 + j4) : make_float4(kNeg, kNeg, kNeg, kNeg);
-                    if (j4 == n4full && j4 < n4) {  // ragged tail, element by element
+                    if (j4 < n4full) {
+                        v[q] = __ldg(s4 + j4);
+                    } else {  // ragged tail, element by element
                         const int e = j4 * 4;
                         v[q].x = e < n ? __ldg(srow + e) : kNeg;
                         v[q].y = e + 1 < n ? __ldg(srow + e + 1) : kNeg;
                         v[q].z = e + 2 < n ? __ldg(srow + e + 2) : kNeg;
+                        v[q].w = kNeg;
                     }
                 }
+            }
+            // stage word 4 q + c: bit l says key 4 (j + l) + c >= bound, j = the warp's
+            // first float4 of step q
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const bool cx = v[q].x >= lo_val, cy = v[q].y >= lo_val;
-                    const bool cz = v[q].z >= lo_val, cw = v[q].w >= lo_val;
-                    if (!__any_sync(0xffffffffu, cx || cy || cz || cw)) continue;
-                    const int e = (j0 + q * kSelThreads) * 4;
-                    append(v[q].x, e, cx);
-                    append(v[q].y, e + 1, cy);
-                    append(v[q].z, e + 2, cz);
-                    append(v[q].w, e + 3, cw);
+            for (int q = 0; q < 8; ++q) {
+                const uint32_t b0 = __ballot_sync(0xffffffffu, v[q].x >= lo_val);
+                const uint32_t b1 = __ballot_sync(0xffffffffu, v[q].y >= lo_val);
+                const uint32_t b2 = __ballot_sync(0xffffffffu, v[q].z >= lo_val);
+                const uint32_t b3 = __ballot_sync(0xffffffffu, v[q].w >= lo_val);
+                if (lane == 0) *reinterpret_cast<uint4 *>(wst + 4 * q) = make_uint4(b0, b1, b2, b3);
+            }
+            __syncwarp();
+            uint32_t word = wst[lane];
+            __syncwarp();
+            const int cnt = __popc(word);
+            int incl = cnt;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += y;
+            }
+            const int tot = __shfl_sync(0xffffffffu, incl, 31);
+            if (wc + tot <= kCapW) {
+                int pos = wc + incl - cnt;
+                const int q = lane >> 2, c = lane & 3;
+                const int jb = (j0 - tid) + q * kSelThreads + wid * 32;
+                while (word != 0u) {
+                    const int l = __ffs(word) - 1;
+                    word &= word - 1u;
+                    const int key = 4 * (jb + l) + c;
+                    craw[pos] = __ldg(srow + key);  // loaded by this warp just now: an L1 hit
+                    cix[pos] = (uint16_t)key;
+                    ++pos;
                 }
             }
-        } else {
-            for (int j0 = tid; j0 - tid < n; j0 += 4 * kSelThreads) {  // uniform trip count
-                float v[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int j = j0 + q * kSelThreads;
-                    v[q] = j < n ? __ldg(srow + j) : -INFINITY;
-                }
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const bool c = v[q] >= lo_val;
-                    if (!__any_sync(0xffffffffu, c)) continue;
-                    append(v[q], j0 + q * kSelThreads, c);
-                }
-            }
+            wc += tot;
         }
+        if (lane == 0) sc.warp_cnt[wid] = wc;
         __syncthreads();
-        const int nc = sc.cand_n;
-        if (nc >= need_total && nc <= kCandCap) {
+        int nc = 0;
+        bool overflow = false;
+#pragma unroll
+        for (int w = 0; w < kSelWarps; ++w) {
+            nc += sc.warp_cnt[w];
+            overflow |= sc.warp_cnt[w] > kCapW;
+        }
+        if (!overflow && nc >= need_total) {
+            // every candidate c of every list, as (list slot, key relative to the bound)
+            auto each_cand = [&](auto f) {
+#pragma unroll 1
+                for (int w = 0; w < kSelWarps; ++w) {
+                    const int cw = sc.warp_cnt[w];
+                    const float *cr = reinterpret_cast<const float *>(regB) + w * kCapW;
+                    for (int c = tid; c < cw; c += kSelThreads) f(w * kCapW + c, order_key(cr[c]) - lo_key);
+                }
+            };
+            uint32_t mx = 0u;
+            each_cand([&](int, uint32_t u) { mx = u > mx ? u : mx; });
+            const uint32_t span = block_reduce<kSelThreads, true>(mx, &sc);
+            const int top = span != 0u ? 31 - __clz(span) : 0;
             // exact threshold among the listed keys (every key above it is listed)
             uint32_t prefix, mask;
             int need, in_bin;
-            radix_select<kSelThreads>([&](int c) { return cand_key[c]; }, nc, need_total, hist, &sc, &prefix, &mask, &need,
-                         &in_bin);
-            const bool partial = need < in_bin;
-            for (int c = tid; c < nc; c += kSelThreads) {
-                const uint32_t u = cand_key[c] & mask;
-                const uint32_t j = cand_idx[c];
-                if (u > prefix) atomicOr(&gtw[j >> 5], 1u << (j & 31));
-                else if (u == prefix) atomicOr(&eqw[j >> 5], 1u << (j & 31));
+            radix_select<kSelThreads, kCandBits>(
+                [&](auto f) { each_cand([&](int, uint32_t u) { f(u); }); }, nc, need_total, top, regA, &sc,
+                &prefix, &mask, &need, &in_bin);
+            // a threshold value shared by more keys than slots left goes to the general
+            // path (the lowest indices among them win there)
+            if (need == in_bin) {
+                const int nwn = (n + 31) >> 5;
+                for (int w = tid; w < nwn; w += kSelThreads) regA[w] = 0u;
+                __syncthreads();
+                each_cand([&](int slot, uint32_t u) {
+                    if ((u & mask) >= prefix) {
+                        const uint32_t j = cidx[slot];
+                        atomicOr(&regA[j >> 5], 1u << (j & 31));
+                    }
+                });
+                __syncthreads();
+                // output slot of word w's first winner: block scan of the word popcounts
+                // (region B: the scores are no longer needed)
+                const int wpt = (nwn + kSelThreads - 1) / kSelThreads;
+                const int w0 = tid * wpt;
+                int cnt = 0;
+                for (int q = 0; q < wpt; ++q)
+                    if (w0 + q < nwn) cnt += __popc(regA[w0 + q]);
+                int tot;
+                int base = block_exclusive_scan<kSelThreads>(cnt, &sc, &tot);
+                for (int q = 0; q < wpt; ++q) {
+                    if (w0 + q < nwn) {
+                        regB[w0 + q] = (uint32_t)base;
+                        base += __popc(regA[w0 + q]);
+                    }
+                }
+                __syncthreads();
+#pragma unroll 1
+                for (int w = 0; w < kSelWarps; ++w) {
+                    const int cw = sc.warp_cnt[w];
+                    for (int c = tid; c < cw; c += kSelThreads) {
+                        const uint32_t j = cidx[w * kCapW + c];
+                        const uint32_t word = regA[j >> 5];
+                        const uint32_t bit = 1u << (j & 31);
+                        if (word & bit) out[regB[j >> 5] + __popc(word & (bit - 1u))] = (int32_t)j;
+                    }
+                }
+                out_base = tot;
+                done = true;
             }
-            __syncthreads();
-            emit_segment<kSelThreads>(gtw, eqw, (n + 31) >> 5, 0, partial, need, need_total, &out_base, &eq_base, out, &sc);
-            done = true;
         }
         __syncthreads();
     }
 
     // ============================ general path ============================
     if (!done) {
+        uint32_t *gtw = regA, *eqw = regB;
         uint32_t prefix, mask;
         int need, in_bin;
-        radix_select<kSelThreads>([&](int j) { return order_key(__ldg(srow + j)); }, n, need_total, hist, &sc, &prefix, &mask,
-                     &need, &in_bin);
+        radix_select<kSelThreads, 11>(
+            [&](auto f) {
+                for (int j = tid; j < n; j += kSelThreads) f(order_key(__ldg(srow + j)));
+            },
+            n, need_total, 31, regA, &sc, &prefix, &mask, &need, &in_bin);
         const bool partial = need < in_bin;
         for (int seg0 = 0; seg0 < n; seg0 += kSegElems) {
             const int seg_n = n - seg0 < kSegElems ? n - seg0 : kSegElems;
@@ -376,7 +497,7 @@ select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__res
                 const int j = seg0 + w * 32 + lane;
                 const bool in = j < n;
                 const uint32_t u = in ? (order_key(__ldg(srow + j)) & mask) : 0u;
-                const uint32_t g = __ballot_sync(0xffffffffu, in && u > prefix);
+                const uint32_t g = __ballot_sync(0xffffffffu, in && (u > prefix || (u == prefix && !partial)));
                 const uint32_t e = __ballot_sync(0xffffffffu, in && u == prefix);
                 if (lane == 0) {
                     gtw[w] = g;
@@ -405,10 +526,10 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t stream)
     for (int64_t done = 0; done < rows; done += 0x7FFFFFFF) {
         const int64_t chunk = rows - done < 0x7FFFFFFF ? rows - done : 0x7FFFFFFF;
         if (wide)
-            select_kernel<512><<<(unsigned)chunk, 512, kSelSmem, stream>>>(
+            select_kernel<512><<<(unsigned)chunk, 512, sel_smem_bytes<512>(), stream>>>(
                 a.scores + done * a.ld, a.ld, a.cu_q, a.cu_k, a.batch, a.row_begin + done, a.k, a.r, a.sel);
         else
-            select_kernel<128><<<(unsigned)chunk, 128, kSelSmem, stream>>>(
+            select_kernel<128><<<(unsigned)chunk, 128, sel_smem_bytes<128>(), stream>>>(
                 a.scores + done * a.ld, a.ld, a.cu_q, a.cu_k, a.batch, a.row_begin + done, a.k, a.r, a.sel);
     }
     return cudaGetLastError();
