@@ -112,16 +112,17 @@ def selected_tokens(n, r=4, k=BUDGET):
 
 
 def run_qsa(args, rank, world, device):
-    from block_sparse_long_09_b200 import inputs, qsa
+    from block_sparse_long_09_b200 import inputs, qsa, ranks
 
     hbm, tflops, peak_kind = peaks()
     torch.manual_seed(0)
-    x = inputs.make_prefill([N_PREFILL], seed=rank, device=device)
+    seeds = ranks.rank_seeds(rank)
+    x = inputs.make_prefill([N_PREFILL], seed=seeds["prefill"], device=device)
     cfg = qsa.default_config(budget_blocks=BUDGET)
     pre = qsa.Prefill([N_PREFILL], chunk_rows=CHUNK, cfg=cfg, device=device)
     o = torch.empty_like(x.q)
 
-    d = inputs.make_decode(DEC_BATCH, DEC_LEN, None, seed=100 + rank, device=device)
+    d = inputs.make_decode(DEC_BATCH, DEC_LEN, None, seed=seeds["decode"], device=device)
     cu_k = d.cu_seqlens_k
     cu_b = d.cu_blocks
     kc_dec = qsa.compress_keys(d.k_idx, cu_k, cu_b, n_blocks=int(cu_b[-1]), cfg=cfg)
@@ -157,8 +158,7 @@ def run_qsa(args, rank, world, device):
     assert qsa.device_status() == 0, "a kernel flagged a device-side error during warm-up"
 
     clocks = Clocks(device.index if device.index is not None else 0)
-    if world > 1:
-        torch.distributed.barrier()
+    ranks.barrier(world)
     torch.cuda.synchronize()
     clocks.start()
     t_start = torch.cuda.Event(enable_timing=True)
@@ -168,8 +168,7 @@ def run_qsa(args, rank, world, device):
         step(True)
     t_end.record(stream)
     torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    ranks.barrier(world)
     clk = clocks.stop()
     total_ms = t_start.elapsed_time(t_end)
     prefill_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["p0"], ev["p1"])]))
@@ -178,13 +177,10 @@ def run_qsa(args, rank, world, device):
     assert qsa.device_status() == 0, "a kernel flagged a device-side error in the timed region"
 
     def allmax(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+        return ranks.max_over_ranks([v], world, device)[0]
 
-    total_ms, prefill_ms, attn_ms, dec_ms = (allmax(v) for v in (total_ms, prefill_ms, attn_ms, dec_ms))
+    total_ms, prefill_ms, attn_ms, dec_ms = ranks.max_over_ranks([total_ms, prefill_ms, attn_ms, dec_ms], world,
+                                                                 device)
 
     # end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
@@ -203,8 +199,7 @@ def run_qsa(args, rank, world, device):
 
         e2e_step()
         torch.cuda.synchronize()
-        if world > 1:
-            torch.distributed.barrier()
+        ranks.barrier(world)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.e2e_steps):
@@ -212,7 +207,7 @@ def run_qsa(args, rank, world, device):
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = allmax(e0.elapsed_time(e1) / args.e2e_steps)
-        e2e = {"value": world * N_PREFILL / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": ranks.job_throughput(world, N_PREFILL, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps, "scope": "prefill 262144 via qsa.Prefill"}
 
     # the build's dense causal attention on the same inputs (the pages' comparison)
@@ -256,7 +251,7 @@ def run_qsa(args, rank, world, device):
     launches_decode = 1 + 1 + 1 + 2
     res = {
         "metric": METRIC,
-        "value": world * N_PREFILL / (prefill_ms / 1e3),
+        "value": ranks.job_throughput(world, N_PREFILL, prefill_ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -379,9 +374,9 @@ def main():
         run_profile_case(args.profile_case)
         return
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from block_sparse_long_09_b200 import ranks
+    env = ranks.env_ranks()
+    world, rank, local = env["world"], env["rank"], env["local"]
 
     if args.impl == "reference":
         if rank != 0:
@@ -406,17 +401,13 @@ def main():
     bld.build()
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=device)
+    ranks.init("nccl", world, device)
     res = run_qsa(args, rank, world, device)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline()
     if rank == 0:
         print(json.dumps(res))
-    if world > 1:
-        torch.distributed.destroy_process_group()
+    ranks.finish(world)
 
 
 if __name__ == "__main__":
