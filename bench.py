@@ -247,7 +247,7 @@ def run_qsa(args, rank, world, device):
     gather = gather_bytes_per_query(1) * sel_tok
     achieved = gather / (attn_ms / 1e3) / 1e9
     n_chunks = (N_PREFILL + CHUNK - 1) // CHUNK
-    launches_prefill = 1 + 2 * n_chunks + n_chunks  # compress; index + select per chunk; attention per chunk
+    launches_prefill = 1 + 2 * n_chunks + 1  # compress; index + select per chunk; attention over all rows
     launches_decode = 1 + 1 + 1 + 2
     res = {
         "metric": METRIC,

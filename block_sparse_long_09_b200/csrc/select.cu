@@ -6,20 +6,21 @@
 // blocks 0 .. b_t - 1.  Ties go to the lower block index; the output lists the
 // chosen blocks in ascending order, padded with -1.
 //
-// One CTA per query row, about 21 KB of shared memory: 128 threads when there
+// One CTA per query row, about 25 KB of shared memory: 128 threads when there
 // are many rows (prefill), so eight rows are in flight on every SM and their
 // memory latency overlaps; 512 threads when rows are few (decode).  The fp32
 // scores become order-preserving 32-bit keys (sign-flip trick, -0.0 folded
 // into +0.0).
 //  * Fast path (16-byte aligned rows of up to 65536 candidates):
-//    - bound: a sample of 1024..2048 keys spread over the row; two 8-bit
-//      digits of a radix select over the sample keys relative to their minimum
-//      locate the sample of rank r_lo (4 sigma above the expected rank of the
-//      threshold), and the smallest sample of that bin is a conservative lower
-//      bound;
-//    - one pass over the row (32 keys in flight per thread): every warp votes
-//      key >= bound, and right after its loads lists its own candidates (index
-//      and score, the score re-read from L1) in a private list;
+//    - bound: a sample of 1024..2048 keys in runs of 8 spread over the row (a
+//      run is one 32-byte sector); two 8-bit digits of a radix select over the
+//      sample keys relative to their minimum locate the sample of rank r_lo (4
+//      sigma above the expected rank of the threshold), and the smallest sample
+//      of that bin is a conservative lower bound;
+//    - one pass over the row (32 keys in flight per thread): for every key slot
+//      a warp ballot of key >= bound gives each candidate its place in the
+//      warp's private list, and the lane that holds it writes score and index
+//      there from its registers (nothing is read twice);
 //    - an MSD radix select with 8-bit digits over the candidates' keys relative
 //      to the bound, started at their highest differing bit, finds the exact
 //      (k-1)-th key; the winners' bits are set in a bitmap, a block scan of its
@@ -44,15 +45,16 @@ constexpr int kSegElems = kSegWords * 32;
 constexpr int kCandCap = 2048;               // candidate lists (and the sample)
 constexpr int kSampleMin = 1024;
 
-// shared memory: region A (kSegWords words: histogram, then the winner bitmap),
-// region B (kCandCap words: sample keys, then candidate scores, then bitmap word
-// prefixes), 16-bit candidate indices, and a 32-word ballot stage per warp
+// shared memory: region A (kSegWords words: histogram, then the winner bitmap)
+// and region C (kCandCap (score bits, index) pairs; before them the sample keys,
+// after them the bitmap word prefixes; in the general path the "equal" bitmap)
 template <int kSelThreads>
 constexpr int sel_smem_bytes()
 {
-    return kSegWords * 4 + kCandCap * 4 + kCandCap * 2 + (kSelThreads / 32) * 32 * 4;
+    return kSegWords * 4 + kCandCap * 8;
 }
 static_assert(kBins <= kSegWords, "the histogram lives in region A");
+static_assert(kCandCap * 2 >= kSegWords && kCandCap * 2 >= kCandCap, "samples, prefixes and eqw fit region C");
 
 __device__ __forceinline__ uint32_t order_key(float x)
 {
@@ -71,6 +73,7 @@ struct SelScratch {
     int warp_tot[kMaxSelWarps];
     uint32_t warp_val[kMaxSelWarps];
     int warp_cnt[kMaxSelWarps];  // candidates listed per warp
+    int grp_pre[kSegWords / 32];  // winners before each group of 32 bitmap words
     int digit, above;
 };
 
@@ -256,10 +259,9 @@ select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__res
     constexpr int kSelWarps = kSelThreads / 32;
     constexpr int kCapW = kCandCap / kSelWarps;         // candidate list of one warp
     extern __shared__ uint32_t smem_sel[];
-    uint32_t *regA = smem_sel;                          // kSegWords
-    uint32_t *regB = regA + kSegWords;                  // kCandCap
-    uint16_t *cidx = reinterpret_cast<uint16_t *>(regB + kCandCap);  // kCandCap
-    uint32_t *stage = reinterpret_cast<uint32_t *>(cidx + kCandCap);  // 32 words per warp
+    uint32_t *regA = smem_sel;                          // kSegWords words
+    uint2 *cand = reinterpret_cast<uint2 *>(regA + kSegWords);  // kCandCap (score bits, index)
+    uint32_t *regB = reinterpret_cast<uint32_t *>(cand);         // the same bytes, as words
     __shared__ SelScratch sc;
 
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -300,13 +302,31 @@ select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__res
     if (n <= kSegElems && (reinterpret_cast<uintptr_t>(srow) & 15u) == 0) {
         // ---- bound from a sample: about 16 expected winners, 1024..2048 keys ----
         int ns = (int)min((int64_t)kCandCap, max((int64_t)kSampleMin, (int64_t)16 * n / need_total));
-        if (ns > n) ns = n;
         uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-        for (int q = tid; q < ns; q += kSelThreads) {
-            const uint32_t u = order_key(__ldg(srow + (int)(((int64_t)q * n) / ns)));
-            regB[q] = u;
-            kmin = u < kmin ? u : kmin;
-            kmax = u > kmax ? u : kmax;
+        if (n <= kCandCap) {  // short row: the sample is the whole row
+            ns = n;
+            for (int q = tid; q < ns; q += kSelThreads) {
+                const uint32_t u = order_key(__ldg(srow + q));
+                regB[q] = u;
+                kmin = u < kmin ? u : kmin;
+                kmax = u > kmax ? u : kmax;
+            }
+        } else {  // runs of 8 keys (two float4, one sector) at ns / 8 spread places
+            const int runs = ns >> 3;
+            ns = runs << 3;
+            for (int g = tid; g < runs; g += kSelThreads) {
+                const int at = (int)(((int64_t)g * n) / runs) & ~3;  // 16-byte aligned, at + 8 <= n
+                const float4 a = __ldg(reinterpret_cast<const float4 *>(srow + at));
+                const float4 b = __ldg(reinterpret_cast<const float4 *>(srow + at + 4));
+                const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const uint32_t u = order_key(x[e]);
+                    regB[g * 8 + e] = u;
+                    kmin = u < kmin ? u : kmin;
+                    kmax = u > kmax ? u : kmax;
+                }
+            }
         }
         kmin = ~block_reduce<kSelThreads, true>(~kmin, &sc);
         kmax = block_reduce<kSelThreads, true>(kmax, &sc);
@@ -344,9 +364,8 @@ select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__res
         const int n4 = (n + 3) >> 2;
         const int n4full = n >> 2;
         constexpr float kNeg = -INFINITY;
-        float *craw = reinterpret_cast<float *>(regB) + wid * kCapW;
-        uint16_t *cix = cidx + wid * kCapW;
-        uint32_t *wst = stage + wid * 32;
+        uint2 *wlist = cand + wid * kCapW;
+        const uint32_t lt = (1u << lane) - 1u;
         int wc = 0;  // this warp's list length (warp-uniform)
         for (int j0 = tid; j0 - tid < n4; j0 += 8 * kSelThreads) {  // uniform trip count
             float4 v[8];
@@ -368,41 +387,21 @@ select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__res
                     }
                 }
             }
-            // stage word 4 q + c: bit l says key 4 (j + l) + c >= bound, j = the warp's
-            // first float4 of step q
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                const uint32_t b0 = __ballot_sync(0xffffffffu, v[q].x >= lo_val);
-                const uint32_t b1 = __ballot_sync(0xffffffffu, v[q].y >= lo_val);
-                const uint32_t b2 = __ballot_sync(0xffffffffu, v[q].z >= lo_val);
-                const uint32_t b3 = __ballot_sync(0xffffffffu, v[q].w >= lo_val);
-                if (lane == 0) *reinterpret_cast<uint4 *>(wst + 4 * q) = make_uint4(b0, b1, b2, b3);
-            }
-            __syncwarp();
-            uint32_t word = wst[lane];
-            __syncwarp();
-            const int cnt = __popc(word);
-            int incl = cnt;
+                const float x[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+                const uint32_t key0 = 4u * (uint32_t)(j0 + q * kSelThreads);
 #pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += y;
-            }
-            const int tot = __shfl_sync(0xffffffffu, incl, 31);
-            if (wc + tot <= kCapW) {
-                int pos = wc + incl - cnt;
-                const int q = lane >> 2, c = lane & 3;
-                const int jb = (j0 - tid) + q * kSelThreads + wid * 32;
-                while (word != 0u) {
-                    const int l = __ffs(word) - 1;
-                    word &= word - 1u;
-                    const int key = 4 * (jb + l) + c;
-                    craw[pos] = __ldg(srow + key);  // loaded by this warp just now: an L1 hit
-                    cix[pos] = (uint16_t)key;
-                    ++pos;
+                for (int c = 0; c < 4; ++c) {
+                    const bool hit = x[c] >= lo_val;
+                    const uint32_t bal = __ballot_sync(0xffffffffu, hit);
+                    if (bal != 0u) {
+                        const int pos = wc + __popc(bal & lt);
+                        if (hit && pos < kCapW) wlist[pos] = make_uint2(__float_as_uint(x[c]), key0 + c);
+                        wc += __popc(bal);
+                    }
                 }
             }
-            wc += tot;
         }
         if (lane == 0) sc.warp_cnt[wid] = wc;
         __syncthreads();
@@ -419,8 +418,10 @@ select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__res
 #pragma unroll 1
                 for (int w = 0; w < kSelWarps; ++w) {
                     const int cw = sc.warp_cnt[w];
-                    const float *cr = reinterpret_cast<const float *>(regB) + w * kCapW;
-                    for (int c = tid; c < cw; c += kSelThreads) f(w * kCapW + c, order_key(cr[c]) - lo_key);
+                    for (int c = tid; c < cw; c += kSelThreads) {
+                        const uint2 e = cand[w * kCapW + c];
+                        f(e.y, order_key(__uint_as_float(e.x)) - lo_key);
+                    }
                 }
             };
             uint32_t mx = 0u;
@@ -439,39 +440,51 @@ select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__res
                 const int nwn = (n + 31) >> 5;
                 for (int w = tid; w < nwn; w += kSelThreads) regA[w] = 0u;
                 __syncthreads();
-                each_cand([&](int slot, uint32_t u) {
-                    if ((u & mask) >= prefix) {
-                        const uint32_t j = cidx[slot];
-                        atomicOr(&regA[j >> 5], 1u << (j & 31));
-                    }
+                each_cand([&](uint32_t j, uint32_t u) {
+                    if ((u & mask) >= prefix) atomicOr(&regA[j >> 5], 1u << (j & 31));
                 });
                 __syncthreads();
-                // output slot of word w's first winner: block scan of the word popcounts
-                // (region B: the scores are no longer needed)
-                const int wpt = (nwn + kSelThreads - 1) / kSelThreads;
-                const int w0 = tid * wpt;
-                int cnt = 0;
-                for (int q = 0; q < wpt; ++q)
-                    if (w0 + q < nwn) cnt += __popc(regA[w0 + q]);
-                int tot;
-                int base = block_exclusive_scan<kSelThreads>(cnt, &sc, &tot);
-                for (int q = 0; q < wpt; ++q) {
-                    if (w0 + q < nwn) {
-                        regB[w0 + q] = (uint32_t)base;
-                        base += __popc(regA[w0 + q]);
-                    }
+                // output slot of a winner: the winners before its group of 32 bitmap
+                // words (a scan over at most 64 groups) plus those before it in the group
+                const int ngrp = (nwn + 31) >> 5;
+                for (int gi = wid; gi < ngrp; gi += kSelWarps) {
+                    const int w = gi * 32 + lane;
+                    const int c = w < nwn ? __popc(regA[w]) : 0;
+                    const int sum = __reduce_add_sync(0xffffffffu, c);
+                    if (lane == 0) sc.grp_pre[gi] = sum;
                 }
                 __syncthreads();
-#pragma unroll 1
-                for (int w = 0; w < kSelWarps; ++w) {
-                    const int cw = sc.warp_cnt[w];
-                    for (int c = tid; c < cw; c += kSelThreads) {
-                        const uint32_t j = cidx[w * kCapW + c];
-                        const uint32_t word = regA[j >> 5];
-                        const uint32_t bit = 1u << (j & 31);
-                        if (word & bit) out[regB[j >> 5] + __popc(word & (bit - 1u))] = (int32_t)j;
+                int tot = 0;
+                if (wid == 0) {
+                    const int a0 = lane < ngrp ? sc.grp_pre[lane] : 0;
+                    const int a1 = lane + 32 < ngrp ? sc.grp_pre[lane + 32] : 0;
+                    int i0 = a0, i1 = a1;
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const int y0 = __shfl_up_sync(0xffffffffu, i0, off);
+                        const int y1 = __shfl_up_sync(0xffffffffu, i1, off);
+                        if (lane >= off) {
+                            i0 += y0;
+                            i1 += y1;
+                        }
                     }
+                    const int t0 = __shfl_sync(0xffffffffu, i0, 31);
+                    const int t1 = __shfl_sync(0xffffffffu, i1, 31);  // every lane: a full-mask shuffle
+                    if (lane < ngrp) sc.grp_pre[lane] = i0 - a0;
+                    if (lane + 32 < ngrp) sc.grp_pre[lane + 32] = t0 + i1 - a1;
+                    if (lane == 0) sc.warp_tot[0] = t0 + t1;
                 }
+                __syncthreads();
+                tot = sc.warp_tot[0];
+                each_cand([&](uint32_t j, uint32_t) {
+                    const uint32_t w = j >> 5, bit = 1u << (j & 31);
+                    const uint32_t word = regA[w];
+                    if (word & bit) {
+                        int pos = sc.grp_pre[w >> 5] + __popc(word & (bit - 1u));
+                        for (uint32_t w2 = w & ~31u; w2 < w; ++w2) pos += __popc(regA[w2]);
+                        out[pos] = (int32_t)j;
+                    }
+                });
                 out_base = tot;
                 done = true;
             }

@@ -288,11 +288,13 @@ class Prefill:
         self.ws = torch.empty((need,), dtype=torch.uint8, device=self.device) if need > 0 else None
 
     def attend(self, q, k, v, o=None, lse=None):
-        """Sparse attention of every row, chunk of rows by chunk of rows."""
+        """Sparse attention of every row: one launch over all rows (persistent CTAs), or,
+        with the key-chunked schedule (its workspace is sized per chunk), chunk by chunk."""
         if o is None:
             o = torch.empty_like(q)
-        for r0 in range(0, self.total, self.chunk):
-            r1 = min(self.total, r0 + self.chunk)
+        step = self.chunk if self.ws is not None else self.total
+        for r0 in range(0, self.total, step):
+            r1 = min(self.total, r0 + step)
             sparse_attn_prefill(q, k, v, self.sel, self.cu, self.cu, r0, r1, o=o, lse=lse, cfg=self.cfg, ws=self.ws,
                                 max_len_k=self.max_len)
         return o
