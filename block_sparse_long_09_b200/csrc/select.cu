@@ -23,9 +23,9 @@
 //      there from its registers (nothing is read twice);
 //    - an MSD radix select with 8-bit digits over the candidates' keys relative
 //      to the bound, started at their highest differing bit, finds the exact
-//      (k-1)-th key; the winners' bits are set in a bitmap, a block scan of its
-//      word popcounts gives every winner its output slot, so the list comes out
-//      ascending without a sort.
+//      (k-1)-th key; the winners' bits are set in a bitmap, and a block scan of
+//      its word popcounts gives every winner its output slot, so the list comes
+//      out ascending without a sort.
 //  * General path (the bound missed, a list overflowed, the threshold value is
 //    shared by more keys than slots left, an unaligned or a longer row): a
 //    radix select with 11-bit digits over every key, read from global memory
@@ -69,11 +69,21 @@ __device__ __forceinline__ float key_value(uint32_t k)
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
+// st.shared.v2 of (a, b) at addr when p holds: a predicated store, no branch
+__device__ __forceinline__ void st_shared_v2_if(bool p, uint32_t addr, uint32_t a, uint32_t b)
+{
+    asm volatile(
+        "{\n\t.reg .pred q;\n\t"
+        "setp.ne.u32 q, %0, 0;\n\t"
+        "@q st.shared.v2.u32 [%1], {%2, %3};\n\t}" ::"r"((uint32_t)p),
+        "r"(addr), "r"(a), "r"(b)
+        : "memory");
+}
+
 struct SelScratch {
     int warp_tot[kMaxSelWarps];
     uint32_t warp_val[kMaxSelWarps];
     int warp_cnt[kMaxSelWarps];  // candidates listed per warp
-    int grp_pre[kSegWords / 32];  // winners before each group of 32 bitmap words
     int digit, above;
 };
 
@@ -117,6 +127,27 @@ __device__ __forceinline__ uint32_t block_reduce(uint32_t v, SelScratch *sc)
     for (int w = 0; w < kSelWarps; ++w) r = kMax ? (r > sc->warp_val[w] ? r : sc->warp_val[w]) : r + sc->warp_val[w];
     __syncthreads();
     return r;
+}
+
+// block-wide max of two values per thread, in one round
+template <int kSelThreads>
+__device__ __forceinline__ void block_max2(uint32_t &a, uint32_t &b, SelScratch *sc)
+{
+    constexpr int kSelWarps = kSelThreads / 32;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    a = __reduce_max_sync(0xffffffffu, a);
+    b = __reduce_max_sync(0xffffffffu, b);
+    if (lane == 0) {
+        sc->warp_val[wid] = a;
+        sc->warp_tot[wid] = (int)b;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kSelWarps; ++w) {
+        a = a > sc->warp_val[w] ? a : sc->warp_val[w];
+        b = b > (uint32_t)sc->warp_tot[w] ? b : (uint32_t)sc->warp_tot[w];
+    }
+    __syncthreads();
 }
 
 // hist[0 .. nb) counts the keys still in play by digit (nb a power of two <=
@@ -204,19 +235,21 @@ __device__ __forceinline__ void emit_segment(const uint32_t *gtw, const uint32_t
                                              bool partial, int need, int need_total, int *out_base,
                                              int *eq_base, int32_t *out, SelScratch *sc)
 {
-    constexpr int kWordsPerThread = kSegWords / kSelThreads;
+    constexpr int kWordsPerThread = kSegWords / kSelThreads;  // at most
     const int tid = threadIdx.x;
     uint32_t wsel[kWordsPerThread];
-    const int w0 = tid * kWordsPerThread;
+    const int wpt = (words + kSelThreads - 1) / kSelThreads;  // spread the words over every thread
+    const int w0 = tid * wpt;
+    const int wend = min(w0 + wpt, words);
     if (partial) {
         int ecnt = 0;
 #pragma unroll
-        for (int q = 0; q < kWordsPerThread; ++q) ecnt += (w0 + q < words) ? __popc(eqw[w0 + q]) : 0;
+        for (int q = 0; q < kWordsPerThread; ++q) ecnt += (w0 + q < wend) ? __popc(eqw[w0 + q]) : 0;
         int etot;
         int epos = *eq_base + block_exclusive_scan<kSelThreads>(ecnt, sc, &etot);
 #pragma unroll
         for (int q = 0; q < kWordsPerThread; ++q) {
-            uint32_t e = (w0 + q < words) ? eqw[w0 + q] : 0u;
+            uint32_t e = (w0 + q < wend) ? eqw[w0 + q] : 0u;
             uint32_t taken = 0u;
             while (e != 0u && epos < need) {  // keep the lowest set bits while rank < need
                 const uint32_t lowbit = e & (~e + 1u);
@@ -225,12 +258,12 @@ __device__ __forceinline__ void emit_segment(const uint32_t *gtw, const uint32_t
                 ++epos;
             }
             epos += __popc(e);
-            wsel[q] = ((w0 + q < words) ? gtw[w0 + q] : 0u) | taken;
+            wsel[q] = ((w0 + q < wend) ? gtw[w0 + q] : 0u) | taken;
         }
         *eq_base += etot;
     } else {  // every key equal to the threshold wins: they are in gtw already
 #pragma unroll
-        for (int q = 0; q < kWordsPerThread; ++q) wsel[q] = (w0 + q < words) ? gtw[w0 + q] : 0u;
+        for (int q = 0; q < kWordsPerThread; ++q) wsel[q] = (w0 + q < wend) ? gtw[w0 + q] : 0u;
     }
     int cnt = 0;
 #pragma unroll
@@ -328,8 +361,9 @@ select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__res
                 }
             }
         }
-        kmin = ~block_reduce<kSelThreads, true>(~kmin, &sc);
-        kmax = block_reduce<kSelThreads, true>(kmax, &sc);
+        kmin = ~kmin;
+        block_max2<kSelThreads>(kmin, kmax, &sc);
+        kmin = ~kmin;
         // r_lo = mean + 4 sigma + 8 ranks
         const float mu = (float)need_total * (float)ns / (float)n;
         int r_lo = (int)ceilf(mu + 4.f * sqrtf(mu) + 8.f);
@@ -364,7 +398,7 @@ select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__res
         const int n4 = (n + 3) >> 2;
         const int n4full = n >> 2;
         constexpr float kNeg = -INFINITY;
-        uint2 *wlist = cand + wid * kCapW;
+        const uint32_t wlist = smem_u32(cand + wid * kCapW);
         const uint32_t lt = (1u << lane) - 1u;
         int wc = 0;  // this warp's list length (warp-uniform)
         for (int j0 = tid; j0 - tid < n4; j0 += 8 * kSelThreads) {  // uniform trip count
@@ -389,18 +423,29 @@ select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__res
             }
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
+                // the four key slots of the step: their ballots order the hits of the warp
+                // (slot c of every lane after slot c - 1 of every lane)
                 const float x[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
                 const uint32_t key0 = 4u * (uint32_t)(j0 + q * kSelThreads);
+                bool hit[4];
+                uint32_t bal[4];
+                int cnt[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const bool hit = x[c] >= lo_val;
-                    const uint32_t bal = __ballot_sync(0xffffffffu, hit);
-                    if (bal != 0u) {
-                        const int pos = wc + __popc(bal & lt);
-                        if (hit && pos < kCapW) wlist[pos] = make_uint2(__float_as_uint(x[c]), key0 + c);
-                        wc += __popc(bal);
-                    }
+                    hit[c] = x[c] >= lo_val;
+                    bal[c] = __ballot_sync(0xffffffffu, hit[c]);
+                    cnt[c] = __popc(bal[c]);
                 }
+                // a list that overflows keeps writing its last slot (the row then takes
+                // the general path)
+                int base = wc;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int pos = min(base + __popc(bal[c] & lt), kCapW - 1);
+                    st_shared_v2_if(hit[c], wlist + 8u * (uint32_t)pos, __float_as_uint(x[c]), key0 + c);
+                    base += cnt[c];
+                }
+                wc = base;
             }
         }
         if (lane == 0) sc.warp_cnt[wid] = wc;
@@ -413,19 +458,29 @@ select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__res
             overflow |= sc.warp_cnt[w] > kCapW;
         }
         if (!overflow && nc >= need_total) {
-            // every candidate c of every list, as (list slot, key relative to the bound)
+            // scores -> keys relative to the bound, in place (every candidate key is >= lo_key)
+            uint32_t mx = 0u;
+#pragma unroll 1
+            for (int w = 0; w < kSelWarps; ++w) {
+                const int cw = sc.warp_cnt[w];
+                for (int c = tid; c < cw; c += kSelThreads) {
+                    uint32_t *e = &cand[w * kCapW + c].x;
+                    const uint32_t u = order_key(__uint_as_float(*e)) - lo_key;
+                    *e = u;
+                    mx = u > mx ? u : mx;
+                }
+            }
+            // every candidate of every list, as (block index, relative key)
             auto each_cand = [&](auto f) {
 #pragma unroll 1
                 for (int w = 0; w < kSelWarps; ++w) {
                     const int cw = sc.warp_cnt[w];
                     for (int c = tid; c < cw; c += kSelThreads) {
                         const uint2 e = cand[w * kCapW + c];
-                        f(e.y, order_key(__uint_as_float(e.x)) - lo_key);
+                        f(e.y, e.x);
                     }
                 }
             };
-            uint32_t mx = 0u;
-            each_cand([&](int, uint32_t u) { mx = u > mx ? u : mx; });
             const uint32_t span = block_reduce<kSelThreads, true>(mx, &sc);
             const int top = span != 0u ? 31 - __clz(span) : 0;
             // exact threshold among the listed keys (every key above it is listed)
@@ -444,48 +499,8 @@ select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__res
                     if ((u & mask) >= prefix) atomicOr(&regA[j >> 5], 1u << (j & 31));
                 });
                 __syncthreads();
-                // output slot of a winner: the winners before its group of 32 bitmap
-                // words (a scan over at most 64 groups) plus those before it in the group
-                const int ngrp = (nwn + 31) >> 5;
-                for (int gi = wid; gi < ngrp; gi += kSelWarps) {
-                    const int w = gi * 32 + lane;
-                    const int c = w < nwn ? __popc(regA[w]) : 0;
-                    const int sum = __reduce_add_sync(0xffffffffu, c);
-                    if (lane == 0) sc.grp_pre[gi] = sum;
-                }
-                __syncthreads();
-                int tot = 0;
-                if (wid == 0) {
-                    const int a0 = lane < ngrp ? sc.grp_pre[lane] : 0;
-                    const int a1 = lane + 32 < ngrp ? sc.grp_pre[lane + 32] : 0;
-                    int i0 = a0, i1 = a1;
-#pragma unroll
-                    for (int off = 1; off < 32; off <<= 1) {
-                        const int y0 = __shfl_up_sync(0xffffffffu, i0, off);
-                        const int y1 = __shfl_up_sync(0xffffffffu, i1, off);
-                        if (lane >= off) {
-                            i0 += y0;
-                            i1 += y1;
-                        }
-                    }
-                    const int t0 = __shfl_sync(0xffffffffu, i0, 31);
-                    const int t1 = __shfl_sync(0xffffffffu, i1, 31);  // every lane: a full-mask shuffle
-                    if (lane < ngrp) sc.grp_pre[lane] = i0 - a0;
-                    if (lane + 32 < ngrp) sc.grp_pre[lane + 32] = t0 + i1 - a1;
-                    if (lane == 0) sc.warp_tot[0] = t0 + t1;
-                }
-                __syncthreads();
-                tot = sc.warp_tot[0];
-                each_cand([&](uint32_t j, uint32_t) {
-                    const uint32_t w = j >> 5, bit = 1u << (j & 31);
-                    const uint32_t word = regA[w];
-                    if (word & bit) {
-                        int pos = sc.grp_pre[w >> 5] + __popc(word & (bit - 1u));
-                        for (uint32_t w2 = w & ~31u; w2 < w; ++w2) pos += __popc(regA[w2]);
-                        out[pos] = (int32_t)j;
-                    }
-                });
-                out_base = tot;
+                // ordered emission: a block scan of the word popcounts places every winner
+                emit_segment<kSelThreads>(regA, regA, nwn, 0, false, need, need_total, &out_base, &eq_base, out, &sc);
                 done = true;
             }
         }
