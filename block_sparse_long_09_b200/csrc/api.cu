@@ -162,10 +162,8 @@ const char *qsa_status_string(qsa_status s)
 size_t qsa_workspace_size(const qsa_config *cfg, int32_t op, int32_t batch, int64_t rows, int64_t max_len_k)
 {
     if (check_config(cfg) != QSA_OK || batch <= 0 || rows < 0) return 0;
-    if (op == QSA_OP_DECODE) {
-        const int ns = max_nsplit(cfg->budget_blocks);
-        return split_workspace_bytes(batch, ns > 1 ? ns : 2);
-    }
+    if (op == QSA_OP_DECODE)  // the even schedule runs below two rows per CTA
+        return batch < 2 * kMaxEvenCtas ? even_workspace_bytes(batch, kMaxEvenCtas) : 0;
     if (op == QSA_OP_PREFILL) {
         const int nc = nchunks_of(cfg, max_len_k);
         return nc > 1 ? chunked_workspace_bytes(rows, nc) : 0;
@@ -282,14 +280,19 @@ qsa_status qsa_sparse_attn_decode(const qsa_config *cfg, const qsa_bf16 *q, cons
     if (q == nullptr || k_cache == nullptr || v_cache == nullptr || sel == nullptr || o == nullptr ||
         !al16(q) || !al16(k_cache) || !al16(v_cache))
         return QSA_ERR_INVALID_ARG;
-    const int nsplit = decode_nsplit(batch, cfg->budget_blocks);
-    if (nsplit > 1) {
+    // below two rows per CTA the batch's tiles are spread evenly over the CTAs (rows cut
+    // in pieces, merged by a second kernel); above, one CTA per row at a time balances
+    const int grid = even_grid();
+    const bool even = batch < 2 * grid;
+    if (even) {
         if (ws == nullptr) return QSA_ERR_WORKSPACE_TOO_SMALL;
-        if (ws_bytes < split_workspace_bytes(batch, nsplit)) return QSA_ERR_WORKSPACE_TOO_SMALL;
+        if (ws_bytes < even_workspace_bytes(batch, grid)) return QSA_ERR_WORKSPACE_TOO_SMALL;
         if (!al16(ws)) return QSA_ERR_INVALID_ARG;
     }
     AttnArgs a{bf(q), bf(k_cache), bf(v_cache), sel, nullptr, cu_seqlens_k, batch, batch, total_k, 0, batch,
-               bf(o), lse, static_cast<float *>(ws), nsplit, cfg->budget_blocks, cfg->r, cfg->softmax_scale};
+               bf(o), lse, even ? static_cast<float *>(ws) : nullptr, 1, cfg->budget_blocks, cfg->r,
+               cfg->softmax_scale};
+    a.even = even ? 1 : 0;
     return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -380,10 +383,12 @@ qsa_status qsa_sparse_attn_decode_static_scratch(const qsa_config *cfg, const qs
     float *scratch = nullptr;
     st = decode_scratch(&scratch);
     if (st != QSA_OK) return st;
-    const int nsplit = decode_nsplit(batch, cfg->budget_blocks);
-    if (split_workspace_bytes(batch, nsplit) > (size_t)QSA_STATIC_SCRATCH_BYTES) return QSA_ERR_SCRATCH_LIMIT;
+    const int grid = even_grid();
+    const bool even = batch < 2 * grid;
+    if (even && even_workspace_bytes(batch, grid) > (size_t)QSA_STATIC_SCRATCH_BYTES) return QSA_ERR_SCRATCH_LIMIT;
     AttnArgs a{bf(q), bf(k_cache), bf(v_cache), sel, nullptr, cu_seqlens_k, batch, batch, total_k, 0, batch,
-               bf(o), lse, nsplit > 1 ? scratch : nullptr, nsplit, cfg->budget_blocks, cfg->r, cfg->softmax_scale};
+               bf(o), lse, even ? scratch : nullptr, 1, cfg->budget_blocks, cfg->r, cfg->softmax_scale};
+    a.even = even ? 1 : 0;
     return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
 }
 

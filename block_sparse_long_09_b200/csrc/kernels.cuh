@@ -64,12 +64,14 @@ struct AttnArgs {
     float scale;
     int nchunks = 0;                 // > 1: key-chunked (L2-blocked) schedule
     int chunk_blocks = 0;            // micro-blocks per key chunk
+    int even = 0;                    // decode: tiles spread evenly over the CTAs (ws: partial states)
 };
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream);
 int min_nsplit(int kb);                         // splits needed so each holds <= 16 tiles
-int decode_nsplit(int batch, int kb);           // splits used by the decode call
-int max_nsplit(int kb);                         // upper bound of decode_nsplit over devices
 int dense_decode_nsplit(int64_t max_len_k, int r);  // splits of the dense flash-decoding path
+constexpr int kMaxEvenCtas = 256;               // CTAs of the even decode schedule, at most
+int even_grid();                                // CTAs of the even decode schedule on this device
+size_t even_workspace_bytes(int64_t rows, int grid);  // its partial states (rows + grid slots)
 size_t split_workspace_bytes(int64_t rows, int nsplit);  // partial (o, lse) states
 size_t chunked_workspace_bytes(int64_t rows, int nchunks);  // bounds + partial states
 

@@ -181,9 +181,10 @@ qsa_status qsa_sparse_attn_prefill(const qsa_config *cfg, const qsa_bf16 *q, con
 
 /*
  * Sparse GQA attention, decode: one new query per sequence at t = L_k,s - 1,
- * same definition as the prefill.  The <= k*r selected tokens of a sequence
- * are split across CTAs (split-K) and the partial softmax states (m, l, o)
- * are merged by a second kernel.
+ * same definition as the prefill.  Below two sequences per SM the batch's
+ * 64-token tiles are spread evenly over the CTAs, cutting sequences into
+ * pieces whose partial softmax states (m, l, o) a second kernel merges; from
+ * two sequences per SM on, every CTA attends whole sequences.
  *   q [batch, n_heads_q, head_dim] bf16; k_cache, v_cache [total_k, n_heads_kv,
  *   head_dim] bf16 (packed, the new token included); sel [batch, k] int32;
  *   o [batch, n_heads_q, head_dim] bf16; lse [batch, n_heads_q] fp32 or NULL.
@@ -218,8 +219,8 @@ qsa_status qsa_sparse_attn_decode(const qsa_config *cfg, const qsa_bf16 *q,
  * Limit: a call whose split-K partial states need more than
  * QSA_STATIC_SCRATCH_BYTES returns QSA_ERR_SCRATCH_LIMIT before launching
  * anything (use qsa_sparse_attn_decode with a workspace there).  With 148 SMs
- * the schedule keeps batch * splits below 592, i.e. under 14.6 MB, so no batch
- * size reaches the limit on B200.
+ * the partial states take (batch + 148) x 24.7 KB below batch 296 and nothing
+ * from there on, 10.9 MB at most, so no batch size reaches the limit on B200.
  */
 #define QSA_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
 qsa_status qsa_sparse_attn_decode_static_scratch(const qsa_config *cfg, const qsa_bf16 *q,
