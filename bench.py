@@ -37,7 +37,7 @@ METRIC = "QSA prefill tokens/s at 262K ctx; decode µs/token at 128K; % of roofl
 # DRAM traffic (read + write bytes) of one full prefill launch of sparse_attn_kernel, from the
 # 1-pass ncu capture summarised in profiles/sparse_attn_prefill262k_traffic.md; valid only for
 # the kernel source it was taken on (checked by hash), null otherwise.
-ATTN_TRAFFIC = {"src_sha256_16": "dc26282f3ec95059", "bytes": 448.99e9}
+ATTN_TRAFFIC = {"src_sha256_16": "26e5acf14acc2ec6", "bytes": 412.45e9}
 
 
 def peaks():

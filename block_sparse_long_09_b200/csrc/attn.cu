@@ -325,7 +325,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                    const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k, int batch,
                    int64_t row_begin, int64_t rows, int nsplit, int kb, int r, float scale,
                    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse_out,
-                   float *__restrict__ ws, const int32_t *__restrict__ bounds, int even)
+                   float *__restrict__ ws, const int32_t *__restrict__ bounds)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -362,23 +362,17 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         tmem_alloc(&sh->tmem_base, kTmemCols);
         tmem_relinquish();
     }
-    if (even && warp == 2)
-        even_setup(sh, cu_k, row_begin, rows, kb, r, lane,
-                   reinterpret_cast<int64_t *>(ws + ((size_t)gridDim.x + rows) * kHQ * (kD + 1)));
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sh->tmem_base;
     volatile int *abort_flag = &sh->abort_flag;
     // this CTA's work items, in the same order for every role
-    const int64_t it_begin = even ? 0 : (int64_t)blockIdx.x;
-    const int64_t it_end = even ? (int64_t)sh->ev_nseg : rows * nsplit;
-    const int64_t it_step = even ? 1 : (int64_t)gridDim.x;
-    const bool partials = even || nsplit > 1;
-    const int64_t n_slots = even ? (int64_t)gridDim.x + rows : rows * nsplit;  // partial-state slots
+    const int64_t it_begin = blockIdx.x, it_end = rows * nsplit, it_step = gridDim.x;
+    const bool partials = nsplit > 1;
+    const int64_t n_slots = rows * nsplit;  // partial-state slots
     auto item_info = [&](int64_t item) -> RowInfo {
-        return even ? row_info_even(item, sh, cu_k, row_begin, kb, r)
-                    : row_info(item, nsplit, rows, row_begin, cu_q, cu_k, batch, kb, r, bounds);
+        return row_info(item, nsplit, rows, row_begin, cu_q, cu_k, batch, kb, r, bounds);
     };
 
     if (warp == 0) {
@@ -699,15 +693,19 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             }
             softmax_bar();
             float inv[kHQ];
-            float my_lse = 0.f;
+            float mR = 0.f, LR = 1.f;  // thread R < 24 writes head R's log-sum-exp
 #pragma unroll
             for (int h = 0; h < kHQ; ++h) {
                 const int gg = h / kGrp, hh = h % kGrp;
                 const float L = sh->red_sum[0][gg][hh] + sh->red_sum[1][gg][hh] + sh->red_sum[2][gg][hh] +
                                 sh->red_sum[3][gg][hh];
                 inv[h] = L > 0.f ? 1.f / L : 0.f;
-                if (R == h) my_lse = m[h] * scale + logf(L);
+                if (R == h) {
+                    mR = m[h];
+                    LR = L;
+                }
             }
+            const float my_lse = mR * scale + logf(LR);
             if (!(ok = mbar_wait(&sh->o_full, o_it & 1, abort_flag))) break;
             ++o_it;
             tc_fence_after();
@@ -1366,7 +1364,7 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream)
     if (grid > n_items) grid = n_items;
     sparse_attn_kernel<<<(unsigned)grid, kAttThreads, kAttSmem, stream>>>(
         mq, mk, mv, a.sel, a.cu_q, a.cu_k, a.batch, a.row_begin, rows, nsplit, a.kb, a.r, a.scale, a.o, a.lse,
-        ws, bounds, 0);
+        ws, bounds);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || nsplit == 1) return e;
     dim3 cg((unsigned)rows, kHQ);
