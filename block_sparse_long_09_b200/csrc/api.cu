@@ -164,6 +164,7 @@ size_t qsa_workspace_size(const qsa_config *cfg, int32_t op, int32_t batch, int6
     if (check_config(cfg) != QSA_OK || batch <= 0 || rows < 0) return 0;
     if (op == QSA_OP_DECODE)  // the even schedule runs below two rows per CTA
         return batch < 2 * kMaxEvenCtas ? even_workspace_bytes(batch, kMaxEvenCtas) : 0;
+    if (op == QSA_OP_DECODE_PAGED) return even_workspace_bytes(batch, kMaxEvenCtas);
     if (op == QSA_OP_PREFILL) {
         const int nc = nchunks_of(cfg, max_len_k);
         return nc > 1 ? chunked_workspace_bytes(rows, nc) : 0;
@@ -293,6 +294,34 @@ qsa_status qsa_sparse_attn_decode(const qsa_config *cfg, const qsa_bf16 *q, cons
                bf(o), lse, even ? static_cast<float *>(ws) : nullptr, 1, cfg->budget_blocks, cfg->r,
                cfg->softmax_scale};
     a.even = even ? 1 : 0;
+    return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
+}
+
+qsa_status qsa_sparse_attn_decode_paged(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k_pages,
+                                        const qsa_bf16 *v_pages, int64_t num_pages, int32_t page_size,
+                                        const int32_t *block_table, int32_t max_pages,
+                                        const int32_t *cu_seqlens_k, int32_t batch, const int32_t *sel,
+                                        qsa_bf16 *o, float *lse, void *ws, size_t ws_bytes, void *stream)
+{
+    qsa_status st = check_config(cfg);
+    if (st != QSA_OK) return st;
+    if (batch <= 0 || num_pages <= 0 || page_size <= 0 || max_pages <= 0 || cu_seqlens_k == nullptr ||
+        block_table == nullptr)
+        return QSA_ERR_INVALID_ARG;
+    if (page_size % cfg->r != 0) return QSA_ERR_INVALID_ARG;
+    if (num_pages * (int64_t)page_size * cfg->n_heads_kv >= ((int64_t)1 << 31)) return QSA_ERR_UNSUPPORTED;
+    if (q == nullptr || k_pages == nullptr || v_pages == nullptr || sel == nullptr || o == nullptr || !al16(q) ||
+        !al16(k_pages) || !al16(v_pages))
+        return QSA_ERR_INVALID_ARG;
+    const int grid = even_grid();
+    if (ws == nullptr || ws_bytes < even_workspace_bytes(batch, grid)) return QSA_ERR_WORKSPACE_TOO_SMALL;
+    if (!al16(ws)) return QSA_ERR_INVALID_ARG;
+    AttnArgs a{bf(q), bf(k_pages), bf(v_pages), sel, nullptr, cu_seqlens_k, batch, batch, num_pages * page_size, 0,
+               batch, bf(o), lse, static_cast<float *>(ws), 1, cfg->budget_blocks, cfg->r, cfg->softmax_scale};
+    a.even = 1;
+    a.block_table = block_table;
+    a.page_size = page_size;
+    a.max_pages = max_pages;
     return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
 }
 

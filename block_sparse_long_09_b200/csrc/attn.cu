@@ -767,7 +767,8 @@ __global__ void __launch_bounds__(kAttThreads, 1)
 sparse_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                      const __grid_constant__ CUtensorMap map_v, const int32_t *__restrict__ sel,
                      const int32_t *__restrict__ cu_k, int64_t rows, int kb, int r, float scale,
-                     float *__restrict__ ws)
+                     float *__restrict__ ws, const int32_t *__restrict__ block_table, int page_size,
+                     int max_pages, int64_t num_pages)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -835,7 +836,21 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
             good = __shfl_sync(0xffffffffu, good, 0);
             if (!good) return false;
             if (lane < kBlkTile) {
-                const int32_t y = blk >= 0 ? (int32_t)((ri.tok_base + (int64_t)blk * r) * kHKV) : -8;
+                // the block's first token row (token, group) in the cache; -8 reads zeros
+                int32_t y = -8;
+                if (blk >= 0) {
+                    const int64_t tok = (int64_t)blk * r;  // position in the sequence
+                    if (block_table == nullptr) {
+                        y = (int32_t)((ri.tok_base + tok) * kHKV);
+                    } else {
+                        const int64_t j = tok / page_size;
+                        const int32_t page = j < max_pages ? __ldg(block_table + ri.row * max_pages + j) : -1;
+                        if (page >= 0 && page < num_pages)
+                            y = (int32_t)(((int64_t)page * page_size + tok % page_size) * kHKV);
+                        else
+                            set_device_status(QSA_ERR_DEVICE_CHECK);
+                    }
+                }
                 tma_load_3d(sSlot + st * kSlotBytes + lane * kBlockBytes, map, &sh->slot_full[st], 0, y, 0);
             }
             ++slot_it;
@@ -1351,8 +1366,11 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream)
             dattr = true;
         }
         if (a.row_begin != 0) return cudaErrorInvalidValue;
-        sparse_decode_kernel<<<(unsigned)grid, kAttThreads, kAttSmem, stream>>>(mq, mk, mv, a.sel, a.cu_k, rows,
-                                                                               a.kb, a.r, a.scale, ws);
+        if (a.block_table != nullptr && (a.page_size <= 0 || a.page_size % a.r != 0 || a.max_pages <= 0))
+            return cudaErrorInvalidValue;
+        sparse_decode_kernel<<<(unsigned)grid, kAttThreads, kAttSmem, stream>>>(
+            mq, mk, mv, a.sel, a.cu_k, rows, a.kb, a.r, a.scale, ws, a.block_table, a.page_size, a.max_pages,
+            a.block_table != nullptr ? a.total_k / a.page_size : 0);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         even_combine_kernel<<<dim3((unsigned)rows, kHQ), kD, 0, stream>>>(ws, grid, a.row_begin, rows, a.o,

@@ -65,6 +65,10 @@ struct AttnArgs {
     int nchunks = 0;                 // > 1: key-chunked (L2-blocked) schedule
     int chunk_blocks = 0;            // micro-blocks per key chunk
     int even = 0;                    // decode: tiles spread evenly over the CTAs (ws: partial states)
+    // decode over a paged K/V cache: k, v are [num_pages * page_size, 2, 256] (total_k rows);
+    // block_table [batch, max_pages] maps page j of sequence s to a page of the pool
+    const int32_t *block_table = nullptr;
+    int page_size = 0, max_pages = 0;
 };
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream);
 int min_nsplit(int kb);                         // splits needed so each holds <= 16 tiles

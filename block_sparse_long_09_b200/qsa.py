@@ -26,11 +26,12 @@ QSA_ERR_DEVICE_CHECK = 6
 QSA_ERR_SCRATCH_LIMIT = 7
 STATIC_SCRATCH_BYTES = 16 * 1024 * 1024  # QSA_STATIC_SCRATCH_BYTES
 QSA_COMPRESS_NO_NORM = 0x1
-OP_COMPRESS, OP_INDEX, OP_SELECT, OP_PREFILL, OP_DECODE, OP_DENSE = range(6)
+OP_COMPRESS, OP_INDEX, OP_SELECT, OP_PREFILL, OP_DECODE, OP_DENSE, OP_DECODE_PAGED = range(7)
 
 EXPORTED = (
     "qsa_config_init", "qsa_compress_keys", "qsa_index_scores", "qsa_select_blocks",
-    "qsa_sparse_attn_prefill", "qsa_sparse_attn_decode", "qsa_sparse_attn_decode_static_scratch",
+    "qsa_sparse_attn_prefill", "qsa_sparse_attn_decode", "qsa_sparse_attn_decode_paged",
+    "qsa_sparse_attn_decode_static_scratch",
     "qsa_dense_attn_prefill",
     "qsa_workspace_size", "qsa_status_string", "qsa_get_device_status", "qsa_version",
 )
@@ -72,6 +73,7 @@ def _load():
         "qsa_sparse_attn_prefill": (I32, [CP, P, P, P, P, P, P, I32, I64, I64, I64, I64, I64, P, P, P, SZ, P]),
         "qsa_sparse_attn_decode": (I32, [CP, P, P, P, P, I32, I64, P, P, P, P, SZ, P]),
         "qsa_sparse_attn_decode_static_scratch": (I32, [CP, P, P, P, P, I32, I64, P, P, P, P]),
+        "qsa_sparse_attn_decode_paged": (I32, [CP, P, P, P, I64, I32, P, I32, P, I32, P, P, P, P, SZ, P]),
         "qsa_dense_attn_prefill": (I32, [CP, P, P, P, P, P, I32, I64, I64, I32, I64, P, P, P, SZ, P]),
         "qsa_workspace_size": (SZ, [CP, I32, I32, I64, I64]),
         "qsa_status_string": (ctypes.c_char_p, [I32]),
@@ -219,6 +221,26 @@ def sparse_attn_decode(q, k_cache, v_cache, cu_seqlens_k, sel, o=None, lse=None,
                                        batch, k_cache.shape[0], _p(sel), _p(o), _p(lse), _p(ws),
                                        ws.numel() if ws is not None else 0, _stream()),
            "qsa_sparse_attn_decode")
+    return (o, lse) if want_lse or lse is not None else o
+
+
+def sparse_attn_decode_paged(q, k_pages, v_pages, block_table, cu_seqlens_k, sel, o=None, lse=None, ws=None,
+                             want_lse: bool = False, cfg: Optional[Config] = None):
+    """Decode attention over a paged K/V pool [num_pages, page_size, 2, 256] with a
+    block table [batch, max_pages]; cu_seqlens_k gives the sequence lengths."""
+    cfg = _cfg(cfg)
+    batch = q.shape[0]
+    num_pages, page_size = k_pages.shape[0], k_pages.shape[1]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((batch, cfg.n_heads_q), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = torch.empty((workspace_size(OP_DECODE_PAGED, batch, batch, 0, cfg),), dtype=torch.uint8, device=q.device)
+    _check(_lib.qsa_sparse_attn_decode_paged(ctypes.byref(cfg), _p(q), _p(k_pages), _p(v_pages), num_pages, page_size,
+                                             _p(block_table), block_table.shape[1], _p(cu_seqlens_k), batch, _p(sel),
+                                             _p(o), _p(lse), _p(ws), ws.numel(), _stream()),
+           "qsa_sparse_attn_decode_paged")
     return (o, lse) if want_lse or lse is not None else o
 
 

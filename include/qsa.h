@@ -86,6 +86,7 @@ typedef struct qsa_config {
 #define QSA_OP_PREFILL 3
 #define QSA_OP_DECODE 4
 #define QSA_OP_DENSE 5
+#define QSA_OP_DECODE_PAGED 6 /* qsa_sparse_attn_decode_paged */
 
 /* Fill *cfg with the model's values (r 4, k 512, 24/2/256, 4/128, scale 1/16,
  * eps 1e-6, flags 0, kv_chunk_blocks 0).  Host only. */
@@ -195,6 +196,29 @@ qsa_status qsa_sparse_attn_decode(const qsa_config *cfg, const qsa_bf16 *q,
                                   const int32_t *cu_seqlens_k, int32_t batch, int64_t total_k,
                                   const int32_t *sel, qsa_bf16 *o, float *lse, void *ws,
                                   size_t ws_bytes, void *stream);
+
+/*
+ * Sparse GQA attention, decode, over a paged K/V cache: the same result as
+ * qsa_sparse_attn_decode, with the K/V rows of sequence s found through its
+ * block table instead of a packed cache.  Only the attention reads pages; the
+ * compressed keys, the indexer and the selector keep their packed layout.
+ *   k_pages, v_pages [num_pages, page_size, n_heads_kv, head_dim] bf16: the pool
+ *   block_table [batch, max_pages] int32 (device): page j of sequence s holds its
+ *     tokens [j page_size, (j + 1) page_size); page ids in 0 .. num_pages - 1
+ *   cu_seqlens_k [batch + 1] int32 (device): only the lengths L_s = cu[s+1] - cu[s]
+ *     are used here (t = L_s - 1)
+ *   page_size: a multiple of r (a micro-block never straddles pages);
+ *     num_pages * page_size * n_heads_kv < 2^31.
+ * The batch's tiles are always spread evenly over the CTAs (pieces merged by a
+ * second kernel).  Workspace: qsa_workspace_size(cfg, QSA_OP_DECODE_PAGED, batch,
+ * batch, 0) bytes.  A page id out of range reads zeros and flags
+ * QSA_ERR_DEVICE_CHECK.  The pages' own dense baseline uses a paged GQA cache.
+ */
+qsa_status qsa_sparse_attn_decode_paged(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k_pages,
+                                        const qsa_bf16 *v_pages, int64_t num_pages, int32_t page_size,
+                                        const int32_t *block_table, int32_t max_pages,
+                                        const int32_t *cu_seqlens_k, int32_t batch, const int32_t *sel,
+                                        qsa_bf16 *o, float *lse, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * Sparse GQA attention, decode, with library-held scratch instead of a caller

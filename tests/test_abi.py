@@ -45,6 +45,27 @@ def test_config_defaults_and_version(qsa):
     assert qsa.library().qsa_version() >= 100
 
 
+def test_paged_decode_args_rejected_on_host(qsa):
+    import ctypes
+    lib = qsa.library()
+    cfg = qsa.default_config()
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the call returns before any device work
+    P = lambda: fake  # noqa: E731
+    # page size not a multiple of r = 4
+    st = lib.qsa_sparse_attn_decode_paged(ctypes.byref(cfg), P(), P(), P(), 8, 6, P(), 4, P(), 2, P(), P(), None,
+                                          P(), 1 << 20, None)
+    assert st == qsa.QSA_ERR_INVALID_ARG
+    # no block table
+    st = lib.qsa_sparse_attn_decode_paged(ctypes.byref(cfg), P(), P(), P(), 8, 16, None, 4, P(), 2, P(), P(), None,
+                                          P(), 1 << 20, None)
+    assert st == qsa.QSA_ERR_INVALID_ARG
+    # a pool whose rows overflow 32-bit tensor coordinates
+    st = lib.qsa_sparse_attn_decode_paged(ctypes.byref(cfg), P(), P(), P(), 1 << 30, 16, P(), 4, P(), 2, P(), P(),
+                                          None, P(), 1 << 20, None)
+    assert st == qsa.QSA_ERR_UNSUPPORTED
+    assert qsa.workspace_size(qsa.OP_DECODE_PAGED, 1000, 1000) >= 1000 * 24 * 257 * 4
+
+
 def test_status_strings(qsa):
     lib = qsa.library()
     for s in range(8):

@@ -356,7 +356,10 @@ def test_chain_n8192_budget512(qsa, kv_chunk):
 # decode
 # ---------------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("batch,lo,hi,k", [(5, 1, 3000, 512), (64, 2000, 9000, 512), (3, 5000, 5000, 2048)])
+# batches below two per SM take the even schedule (rows cut in pieces: 200 rows of a few
+# tiles put several rows in every CTA's share); from 296 rows on every CTA attends whole rows
+@pytest.mark.parametrize("batch,lo,hi,k", [(5, 1, 3000, 512), (64, 2000, 9000, 512), (3, 5000, 5000, 2048),
+                                           (200, 1, 600, 64), (300, 1, 600, 64)])
 def test_decode_chain(qsa, batch, lo, hi, k):
     d = inputs.make_decode(batch, lo, hi, seed=27)
     cfg = qsa.default_config(budget_blocks=k)
@@ -379,6 +382,62 @@ def test_decode_chain(qsa, batch, lo, hi, k):
         ref_o, ref_lse = oracle.attend(d.q[s:s + 1], d.k_cache[a:b], d.v_cache[a:b], srow[None], 1, L, 4, SCALE, [0])
         check_attn(o_g[s:s + 1], ref_o)
         np.testing.assert_allclose(lse_g[s], ref_lse[0], rtol=0, atol=2e-3)
+    status_ok(qsa)
+
+
+def paged_cache(kv, seqlens, page, seed, spare=5):
+    """Scatter a packed [sum L, 2, 256] cache into a pool of pages in a seeded random
+    order; returns the pool [n_pages, page, 2, 256] and the block table [B, max_pages]."""
+    npg = [(L + page - 1) // page for L in seqlens]
+    total = sum(npg) + spare
+    perm = torch.randperm(total, generator=torch.Generator().manual_seed(seed))
+    pool = torch.zeros((total, page) + tuple(kv.shape[1:]), dtype=kv.dtype)
+    table = torch.full((len(seqlens), max(npg)), -1, dtype=torch.int32)
+    a, nxt = 0, 0
+    for s, L in enumerate(seqlens):
+        for j in range(npg[s]):
+            pid = int(perm[nxt])
+            nxt += 1
+            t0, t1 = j * page, min((j + 1) * page, L)
+            pool[pid, : t1 - t0] = kv[a + t0 : a + t1]
+            table[s, j] = pid
+        a += L
+    return pool, table
+
+
+@pytest.mark.parametrize("batch,lo,hi,k,page", [(5, 1, 3000, 512, 16), (64, 2000, 9000, 512, 64),
+                                                (300, 1, 600, 64, 4)])
+def test_decode_paged(qsa, batch, lo, hi, k, page):
+    """The paged decode reads the same K/V through a block table: equal to the packed
+    decode (bit for bit where both run the even schedule) and to the oracle."""
+    d = inputs.make_decode(batch, lo, hi, seed=31)
+    cfg = qsa.default_config(budget_blocks=k)
+    cu_k, cu_b = cu(d.seqlens)
+    cu_q = torch.arange(batch + 1, dtype=torch.int32, device="cuda")
+    kc = qsa.compress_keys(d.k_idx.cuda(), cu_k, cu_b, n_blocks=max(int(cu_b[-1]), 1), cfg=cfg)
+    ld = max(1, (max(d.seqlens) - 1) // 4)
+    scores = torch.empty((batch, ld), dtype=torch.float32, device="cuda")
+    qsa.index_scores(d.q_idx.cuda(), d.w.cuda(), kc[: int(cu_b[-1])], cu_q, cu_k, cu_b, 1, ld, scores=scores, cfg=cfg)
+    sel = qsa.select_blocks(scores, cu_q, cu_k, batch, cfg=cfg)
+    o_p, lse_p = qsa.sparse_attn_decode(d.q.cuda(), d.k_cache.cuda(), d.v_cache.cuda(), cu_k, sel, want_lse=True,
+                                        cfg=cfg)
+    kp, table = paged_cache(d.k_cache, d.seqlens, page, seed=32)
+    vp, _ = paged_cache(d.v_cache, d.seqlens, page, seed=32)
+    o_g, lse_g = qsa.sparse_attn_decode_paged(d.q.cuda(), kp.cuda(), vp.cuda(), table.cuda(), cu_k, sel,
+                                              want_lse=True, cfg=cfg)
+    torch.cuda.synchronize()
+    og, lg = o_g.float().cpu().numpy(), lse_g.cpu().numpy()
+    if batch < 296:  # both ran the even-schedule decode kernel on the same values
+        assert torch.equal(o_g, o_p) and torch.equal(lse_g, lse_p)
+    else:
+        check_attn(og, o_p.float().cpu().numpy().astype(np.float64))
+    sel_g = sel.cpu().numpy()
+    for s, (a, b) in list(enumerate(seq_slices(d.seqlens)))[:: max(1, batch // 16)]:
+        L = b - a
+        ref_o, ref_lse = oracle.attend(d.q[s:s + 1], d.k_cache[a:b], d.v_cache[a:b], sel_g[s][None], 1, L, 4, SCALE,
+                                       [0])
+        check_attn(og[s:s + 1], ref_o)
+        np.testing.assert_allclose(lg[s], ref_lse[0], rtol=0, atol=2e-3)
     status_ok(qsa)
 
 
