@@ -15,6 +15,7 @@ Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent laye
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import subprocess
@@ -36,8 +37,16 @@ METRIC = "QSA prefill tokens/s at 262K ctx; decode µs/token at 128K; % of roofl
 
 # DRAM traffic (read + write bytes) of one full prefill launch of sparse_attn_kernel, from the
 # 1-pass ncu capture summarised in profiles/sparse_attn_prefill262k_traffic.md; valid only for
-# the kernel source it was taken on (checked by hash), null otherwise.
-ATTN_TRAFFIC = {"src_sha256_16": "26e5acf14acc2ec6", "bytes": 412.45e9}
+# the kernel sources it was taken on (attn.cu + attn_common.cuh, checked by hash), null otherwise.
+ATTN_TRAFFIC = {"src_sha256_16": "0ff7f8844c9810a1", "bytes": 411.57e9}
+
+
+def attn_src_hash() -> str:
+    """Hash of the prefill attention kernel's sources (the traffic figure is valid only for them)."""
+    h = hashlib.sha256()
+    for f in ("attn.cu", "attn_common.cuh"):
+        h.update(open(os.path.join(ROOT, "block_sparse_long_09_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def peaks():
@@ -238,9 +247,7 @@ def run_qsa(args, rank, world, device):
                  "decode_step_us": dd_us, "qsa_decode_speedup": dd_us / (dec_ms * 1e3),
                  "pages_context": "7.6x prefill / 4.9x decode at 1M context, kernel level, hardware not stated"}
 
-    import hashlib
-    src = os.path.join(ROOT, "block_sparse_long_09_b200", "csrc", "attn.cu")
-    same_src = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] == ATTN_TRAFFIC["src_sha256_16"]
+    same_src = attn_src_hash() == ATTN_TRAFFIC["src_sha256_16"]
     traffic = ATTN_TRAFFIC["bytes"] if (same_src and world == 1) else None
 
     sel_tok = selected_tokens(N_PREFILL)
