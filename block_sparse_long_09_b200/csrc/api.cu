@@ -361,7 +361,7 @@ qsa_status qsa_dense_attn_prefill(const qsa_config *cfg, const qsa_bf16 *q, cons
 // ---------------------------------------------------------------------------
 // Decode with library-held scratch.  For callers that cannot allocate device
 // memory while decoding (a pool that has reserved all free memory up front, a
-// plain C host without a device allocator): the split-K partial states live in
+// plain C host without a device allocator): the partial softmax states live in
 // a fixed array of the library's device image instead of a caller workspace.
 // Every GPU that loads the library holds the array until the process exits;
 // every call on a device shares it, so calls whose kernels overlap on the GPU

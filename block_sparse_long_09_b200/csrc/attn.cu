@@ -31,8 +31,9 @@
 //      warp 1      TMEM owner + single-thread tcgen05.mma issue: S(j+1) is
 //                  issued before PV(j) so QK^T overlaps the softmax
 //      warps 2..5  softmax (thread = TMEM lane = (token, group) row) and the
-//                  epilogue (thread = d); split-K decode writes fp32 partial
-//                  states that combine_kernel merges.
+//                  epilogue (thread = d); the split-K dense decode and the
+//                  key-chunked schedule write fp32 partial states that
+//                  combine_kernel merges.
 // Without a selection array the kernel attends to every block j <= t: that is
 // the dense flash-decoding baseline (one query per sequence, split-K).
 #include "attn_common.cuh"
@@ -534,12 +535,6 @@ chunk_bounds_kernel(const int32_t *__restrict__ sel, const int32_t *__restrict__
 }
 
 }  // namespace
-
-int min_nsplit(int kb)
-{
-    (void)kb;
-    return 1;  // the online softmax handles any budget in one pass
-}
 
 int dense_decode_nsplit(int64_t max_len_k, int r)
 {

@@ -72,7 +72,6 @@ struct AttnArgs {
 };
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream);
 cudaError_t launch_sparse_decode(const AttnArgs &a, cudaStream_t stream);  // a.even: the decode kernel
-int min_nsplit(int kb);                         // splits needed so each holds <= 16 tiles
 int dense_decode_nsplit(int64_t max_len_k, int r);  // splits of the dense flash-decoding path
 constexpr int kMaxEvenCtas = 256;               // CTAs of the even decode schedule, at most
 int even_grid();                                // CTAs of the even decode schedule on this device

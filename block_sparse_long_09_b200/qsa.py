@@ -338,7 +338,8 @@ class Prefill:
 class DecodeStep:
     """One QSA decode step for a fixed batch, one new query per sequence: refresh
     the compressed block each sequence just completed, score every earlier block,
-    select the top k, and run split-K sparse attention.  The five launches can be
+    select the top k, and run the decode attention (the batch's tiles spread evenly
+    over the CTAs) and the merge of the row pieces.  The five launches can be
     captured once in a CUDA graph and replayed (graph=True): the tensors passed
     here are the graph's fixed inputs, so a caller refreshes them in place."""
 

@@ -223,7 +223,7 @@ qsa_status qsa_sparse_attn_decode_paged(const qsa_config *cfg, const qsa_bf16 *q
 /*
  * Sparse GQA attention, decode, with library-held scratch instead of a caller
  * workspace.  Computes exactly what qsa_sparse_attn_decode computes, with the
- * same split-K schedule, and takes the same arguments minus ws / ws_bytes.
+ * same schedule, and takes the same arguments minus ws / ws_bytes.
  * The reading notes describe no counterpart of this call: it exists for
  * callers that cannot allocate device memory at decode time, e.g. a serving
  * loop whose pool has reserved all free device memory up front, or a plain C
@@ -240,7 +240,7 @@ qsa_status qsa_sparse_attn_decode_paged(const qsa_config *cfg, const qsa_bf16 *q
  * or concurrent host threads) race and corrupt each other's results; order
  * them on one stream.  Nothing in the array has to start at zero: each call
  * writes every partial state before the merge reads it.
- * Limit: a call whose split-K partial states need more than
+ * Limit: a call whose partial softmax states need more than
  * QSA_STATIC_SCRATCH_BYTES returns QSA_ERR_SCRATCH_LIMIT before launching
  * anything (use qsa_sparse_attn_decode with a workspace there).  With 148 SMs
  * the partial states take (batch + 148) x 24.7 KB below batch 296 and nothing
