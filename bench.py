@@ -38,7 +38,7 @@ METRIC = "QSA prefill tokens/s at 262K ctx; decode µs/token at 128K; % of roofl
 # DRAM traffic (read + write bytes) of one full prefill launch of sparse_attn_kernel, from the
 # 1-pass ncu capture summarised in profiles/sparse_attn_prefill262k_traffic.md; valid only for
 # the kernel sources it was taken on (attn.cu + attn_common.cuh, checked by hash), null otherwise.
-ATTN_TRAFFIC = {"src_sha256_16": "0ff7f8844c9810a1", "bytes": 411.57e9}
+ATTN_TRAFFIC = {"src_sha256_16": "07dc3c02b1842d7d", "bytes": 474.22e9}
 
 
 def attn_src_hash() -> str:
