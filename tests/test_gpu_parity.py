@@ -357,9 +357,11 @@ def test_chain_n8192_budget512(qsa, kv_chunk):
 # ---------------------------------------------------------------------------------------------
 
 # batches below two per SM take the even schedule (rows cut in pieces: 200 rows of a few
-# tiles put several rows in every CTA's share); from 296 rows on every CTA attends whole rows
+# tiles put several rows in every CTA's share; one row of 125 tiles or two rows of one tile
+# leave most shares empty); from 296 rows on every CTA attends whole rows
 @pytest.mark.parametrize("batch,lo,hi,k", [(5, 1, 3000, 512), (64, 2000, 9000, 512), (3, 5000, 5000, 2048),
-                                           (200, 1, 600, 64), (300, 1, 600, 64)])
+                                           (200, 1, 600, 64), (300, 1, 600, 64), (1, 8000, 8000, 2048),
+                                           (2, 1, 50, 512)])
 def test_decode_chain(qsa, batch, lo, hi, k):
     d = inputs.make_decode(batch, lo, hi, seed=27)
     cfg = qsa.default_config(budget_blocks=k)
