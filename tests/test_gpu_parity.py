@@ -237,9 +237,10 @@ def test_select_bit_exact_on_oracle_scores(qsa, case):
     status_ok(qsa)
 
 
-@pytest.mark.parametrize("bt,mod", [(40000, 7), (65535, 3), (65535, 0)])
+@pytest.mark.parametrize("bt,mod", [(40000, 7), (65535, 3), (65535, 0), (70000, 0), (70000, 3), (131071, 5)])
 def test_select_long_rows(qsa, bt, mod):
-    """Rows longer than the shared-memory staging limit, with heavy ties."""
+    """Long rows, with heavy ties; beyond 65536 candidates the general path runs, its
+    threshold ties spread over more than one 65536-key bitmap segment."""
     rng = np.random.default_rng(bt + mod)
     L = bt * 4 + 1
     row = rng.standard_normal(bt).astype(np.float32)
