@@ -327,6 +327,58 @@ def cpu_baseline(seconds: float = 12.0, rows_hint: int = 16):
                       "keys once, then per row scores, top-512 select and attention, fp64, %.1f s" % (n, t)}
 
 
+def run_extra_configs(steps: int = 5, warmup: int = 3):
+    """The other workloads of the measurement plan, one line each on stderr (the bench's
+    own JSON line on stdout is unchanged): prefill of 2 x 65536 tokens with peaked indexer
+    keys, and decode steps at 262144 tokens and at mixed lengths U{32768 .. 262144}."""
+    from block_sparse_long_09_b200 import inputs, qsa
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    cfg = qsa.default_config(budget_blocks=BUDGET)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        assert qsa.device_status() == 0
+        return e0.elapsed_time(e1) / steps
+
+    # prefill, 2 sequences of 65536 tokens, per-block offsets in k_I (peaked selections)
+    lens = [65536, 65536]
+    x = inputs.make_prefill(lens, seed=0, peaked=True, device=dev)
+    pre = qsa.Prefill(lens, chunk_rows=CHUNK, cfg=cfg, device=dev)
+    o = torch.empty_like(x.q)
+    ms = timed(lambda: pre(x.q, x.k, x.v, x.q_idx, x.w, x.k_idx, o=o))
+    att = timed(lambda: pre.attend(x.q, x.k, x.v, o=o))
+    sel_tok = sum(selected_tokens(L) for L in lens)
+    print(json.dumps({"workload": "prefill 2 x 65536, peaked k_I (one c_b ~ N(0, 0.5^2) per block)",
+                      "prefill_ms": ms, "tokens_per_s": sum(lens) / (ms / 1e3), "attn_ms": att,
+                      "attn_gather_TBps": gather_bytes_per_query(1) * sel_tok / (att / 1e3) / 1e12}),
+          file=sys.stderr)
+    del x, pre, o
+    torch.cuda.empty_cache()
+    # decode, batch 64, every sequence at 262144 tokens and at mixed lengths
+    for name, lo, hi in (("decode batch 64, all L = 262144", 262144, None),
+                         ("decode batch 64, L ~ U{32768 .. 262144}", 32768, 262144)):
+        d = inputs.make_decode(DEC_BATCH, lo, hi, seed=0, device=dev)
+        kc = qsa.compress_keys(d.k_idx, d.cu_seqlens_k, d.cu_blocks, n_blocks=int(d.cu_blocks[-1]), cfg=cfg)
+        last = torch.tensor([L // 4 - 1 for L in d.seqlens], dtype=torch.int32, device=dev)
+        dec = qsa.DecodeStep(d.q, d.q_idx, d.w, d.k_cache, d.v_cache, d.k_idx, kc, d.cu_seqlens_k, d.cu_blocks,
+                             max(d.seqlens), refresh_blocks=last, cfg=cfg, graph=True)
+        us = timed(dec) * 1e3
+        print(json.dumps({"workload": name, "step_us": us, "us_per_token_amortized": us / DEC_BATCH}),
+              file=sys.stderr)
+        del d, kc, dec
+        torch.cuda.empty_cache()
+
+
 def run_profile_case(case: str, reps: int = 3):
     """Small cases for ncu captures of one kernel (a few GB on the device, K/V larger than L2)."""
     from block_sparse_long_09_b200 import inputs, qsa
@@ -372,6 +424,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", dest="dense", action="store_false",
                     help="skip the dense causal-attention comparison")
+    ap.add_argument("--extra-configs", action="store_true",
+                    help="also time the other workloads (peaked 2 x 65536 prefill, decode at 262144 and mixed "
+                         "lengths) and print them on stderr")
     ap.add_argument("--profile-case", choices=["attn", "index", "select", "decode"], default=None,
                     help="run one small case for an ncu capture and exit")
     args = ap.parse_args()
@@ -379,6 +434,11 @@ def main():
         import block_sparse_long_09_b200.build as bld
         bld.build()
         run_profile_case(args.profile_case)
+        return
+    if args.extra_configs:
+        import block_sparse_long_09_b200.build as bld
+        bld.build()
+        run_extra_configs(args.steps, args.warmup)
         return
 
     from block_sparse_long_09_b200 import ranks
