@@ -19,6 +19,7 @@ import hashlib
 import json
 import os
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -62,7 +63,7 @@ class Clocks:
 
     def __init__(self, index):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % index)
+        self.path = os.path.join(tempfile.gettempdir(), "qsa_clocks_rank%d.csv" % index)
         self.index = index
 
     def start(self):

@@ -54,7 +54,7 @@ def kth_best(scores_row, bt, k):
 
 
 def check_scores(g, o, bt, k):
-    """The benchmark spec bound, relative where it matters and floored at the row's k-th score."""
+    """The score tolerance: relative where it matters, floored at the row's k-th score."""
     for n in range(g.shape[0]):
         b = bt[n]
         if b == 0:
