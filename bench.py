@@ -36,10 +36,12 @@ CHUNK = 16384
 BUDGET = 512
 METRIC = "QSA prefill tokens/s at 262K ctx; decode µs/token at 128K; % of roofline"
 
-# DRAM traffic (read + write bytes) of one full prefill launch of sparse_attn_kernel, from the
-# 1-pass ncu capture summarised in profiles/sparse_attn_prefill262k_traffic.md; valid only for
-# the kernel sources it was taken on (attn.cu + attn_common.cuh, checked by hash), null otherwise.
-ATTN_TRAFFIC = {"src_sha256_16": "07dc3c02b1842d7d", "bytes": 474.22e9}
+# DRAM traffic (read + write) of sparse_attn_kernel on the small profiling case
+# (`bench.py --profile-case attn`: rows 122880..131071 of a 131072-token prefill,
+# 8192 queries x 4 MiB = 34.36 GB gathered), from a one-kernel ncu capture; the
+# full launch's traffic is estimated by scaling with the gathered bytes.  Valid
+# only for the kernel sources it was taken on (checked by hash), null otherwise.
+ATTN_SMALL_TRAFFIC = {"src_sha256_16": "afa9165f2aa7e996", "bytes": 14.44e9, "gather_bytes": 34.36e9}
 
 
 def attn_src_hash() -> str:
@@ -51,11 +53,12 @@ def attn_src_hash() -> str:
 
 
 def peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, bf16 TFLOP/s sustained, kind)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return d["hbm_gbs"], d["bf16_tflops"], "measured"
-    return 6650.0, 1590.0, "fallback"
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
 
 
 class Clocks:
@@ -121,10 +124,29 @@ def selected_tokens(n, r=4, k=BUDGET):
     return int(((nblk - 1) * r + (t - r * bt + 1)).sum())
 
 
+def index_pairs(n, r=4):
+    """Sum over queries of b_t = floor(t / r): the (row, candidate block) pairs the indexer scores."""
+    t = np.arange(n, dtype=np.int64)
+    return int((t // r).sum())
+
+
+def decode_bytes(seqlens, kc_bytes_per_block, k=BUDGET, r=4):
+    """Bytes one decode step must move: the kc scan, the scores written and read once
+    by the selector, and the selected K/V tokens (2 KV heads x 256 x bf16, K and V)."""
+    kc = sum((L // r) * kc_bytes_per_block for L in seqlens)
+    scores = sum(((L - 1) // r) * 4 * 2 for L in seqlens)
+    tok = sum(min(k - 1, (L - 1) // r) * r + ((L - 1) % r + 1) for L in seqlens)
+    return kc + scores + gather_bytes_per_query(tok), kc, gather_bytes_per_query(tok)
+
+
+def ev_ms(pairs):
+    return float(np.mean([a.elapsed_time(b) for a, b in pairs])) if pairs else 0.0
+
+
 def run_qsa(args, rank, world, device):
     from block_sparse_long_09_b200 import inputs, qsa, ranks
 
-    hbm, tflops, peak_kind = peaks()
+    hbm, tflops, tflops_sus, peak_kind = peaks()
     torch.manual_seed(0)
     seeds = ranks.rank_seeds(rank)
     x = inputs.make_prefill([N_PREFILL], seed=seeds["prefill"], device=device)
@@ -136,19 +158,39 @@ def run_qsa(args, rank, world, device):
     cu_k = d.cu_seqlens_k
     cu_b = d.cu_blocks
     kc_dec = qsa.compress_keys(d.k_idx, cu_k, cu_b, n_blocks=int(cu_b[-1]), cfg=cfg)
+    kc_bpb = kc_dec[0].numel() * kc_dec.element_size()  # bytes of one compressed key
     last_blk = torch.tensor([L // 4 - 1 for L in d.seqlens], dtype=torch.int32, device=device)
     dec = qsa.DecodeStep(d.q, d.q_idx, d.w, d.k_cache, d.v_cache, d.k_idx, kc_dec, cu_k, cu_b, DEC_LEN,
                          refresh_blocks=last_blk, cfg=cfg, graph=True)
     dec_o = dec.o
     stream = torch.cuda.current_stream()
+    n_chunks = (N_PREFILL + CHUNK - 1) // CHUNK
 
-    ev = {k: [] for k in ("p0", "p1", "a0", "a1", "d0", "d1")}
+    ev = {k: [] for k in ("p0", "p1", "a0", "a1", "d0", "d1", "ix", "sl")}
+
+    def mk():
+        return torch.cuda.Event(enable_timing=True)
 
     def step(record):
-        e = {k: torch.cuda.Event(enable_timing=True) for k in ev} if record else None
+        e = {k: mk() for k in ("p0", "p1", "a0", "a1", "d0", "d1")} if record else None
         if record:
             e["p0"].record(stream)
-        pre.index_select(x.q_idx, x.w, x.k_idx)
+        # compress, then index and select per chunk (qsa.Prefill.index_select, with events)
+        qsa.compress_keys(x.k_idx, pre.cu, pre.cu_blocks, kc=pre.kc, cfg=cfg)
+        for r0 in range(0, N_PREFILL, CHUNK):
+            r1 = min(N_PREFILL, r0 + CHUNK)
+            e0, e1, e2 = (mk(), mk(), mk()) if record else (None, None, None)
+            if record:
+                e0.record(stream)
+            qsa.index_scores(x.q_idx, x.w, pre.kc[: pre.n_blocks], pre.cu, pre.cu, pre.cu_blocks, pre.max_len,
+                             pre.ld, r0, r1, scores=pre.scores, cfg=cfg)
+            if record:
+                e1.record(stream)
+            qsa.select_blocks(pre.scores, pre.cu, pre.cu, pre.total, r0, r1, sel=pre.sel, cfg=cfg)
+            if record:
+                e2.record(stream)
+                ev["ix"].append((e0, e1))
+                ev["sl"].append((e1, e2))
         if record:
             e["a0"].record(stream)
         pre.attend(x.q, x.k, x.v, o=o)  # one pass per query
@@ -159,7 +201,7 @@ def run_qsa(args, rank, world, device):
         dec()  # decode step: one CUDA-graph replay of its five launches
         if record:
             e["d1"].record(stream)
-            for k in ev:
+            for k in ("p0", "p1", "a0", "a1", "d0", "d1"):
                 ev[k].append(e[k])
 
     for _ in range(args.warmup):
@@ -181,16 +223,56 @@ def run_qsa(args, rank, world, device):
     ranks.barrier(world)
     clk = clocks.stop()
     total_ms = t_start.elapsed_time(t_end)
-    prefill_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["p0"], ev["p1"])]))
-    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"])]))
-    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["d0"], ev["d1"])]))
+    prefill_ms = ev_ms(list(zip(ev["p0"], ev["p1"])))
+    attn_ms = ev_ms(list(zip(ev["a0"], ev["a1"])))
+    dec_ms = ev_ms(list(zip(ev["d0"], ev["d1"])))
+    index_ms = ev_ms(ev["ix"]) * n_chunks  # per step: all chunks
+    select_ms = ev_ms(ev["sl"]) * n_chunks
     assert qsa.device_status() == 0, "a kernel flagged a device-side error in the timed region"
 
     def allmax(v):
         return ranks.max_over_ranks([v], world, device)[0]
 
-    total_ms, prefill_ms, attn_ms, dec_ms = ranks.max_over_ranks([total_ms, prefill_ms, attn_ms, dec_ms], world,
-                                                                 device)
+    total_ms, prefill_ms, attn_ms, dec_ms, index_ms, select_ms = ranks.max_over_ranks(
+        [total_ms, prefill_ms, attn_ms, dec_ms, index_ms, select_ms], world, device)
+
+    def timed(fn, reps=5):
+        fn()
+        torch.cuda.synchronize()
+        a, b = mk(), mk()
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return allmax(a.elapsed_time(b) / reps)
+
+    # decode kernels one by one at 131072 (eager launches of the step's calls)
+    dec_index_us = timed(lambda: qsa.index_scores(dec.q_idx, dec.w, dec.kc, dec.cu_q, dec.cu_k, dec.cu_b, 1, dec.ld,
+                                                  scores=dec.scores, cfg=cfg)) * 1e3
+    dec_select_us = timed(lambda: qsa.select_blocks(dec.scores, dec.cu_q, dec.cu_k, DEC_BATCH, sel=dec.sel,
+                                                    cfg=cfg)) * 1e3
+    dec_attn_us = timed(lambda: qsa.sparse_attn_decode(d.q, d.k_cache, d.v_cache, cu_k, dec.sel, o=dec_o, ws=dec.ws,
+                                                       cfg=cfg)) * 1e3
+    step_bytes, kc_scan, dec_gather = decode_bytes(d.seqlens, kc_bpb)
+
+    # decode at 262144 tokens per sequence: the step, and the attention kernel alone
+    del d, dec
+    torch.cuda.empty_cache()
+    d2 = inputs.make_decode(DEC_BATCH, 262144, None, seed=seeds["decode"] + 1, device=device)
+    kc2 = qsa.compress_keys(d2.k_idx, d2.cu_seqlens_k, d2.cu_blocks, n_blocks=int(d2.cu_blocks[-1]), cfg=cfg)
+    last2 = torch.tensor([L // 4 - 1 for L in d2.seqlens], dtype=torch.int32, device=device)
+    dec2 = qsa.DecodeStep(d2.q, d2.q_idx, d2.w, d2.k_cache, d2.v_cache, d2.k_idx, kc2, d2.cu_seqlens_k,
+                          d2.cu_blocks, 262144, refresh_blocks=last2, cfg=cfg, graph=True)
+    step262_us = timed(dec2, reps=10) * 1e3
+    attn262_us = timed(lambda: qsa.sparse_attn_decode(d2.q, d2.k_cache, d2.v_cache, d2.cu_seqlens_k, dec2.sel,
+                                                      o=dec2.o, ws=dec2.ws, cfg=cfg), reps=10) * 1e3
+    index262_us = timed(lambda: qsa.index_scores(dec2.q_idx, dec2.w, dec2.kc, dec2.cu_q, dec2.cu_k, dec2.cu_b, 1,
+                                                 dec2.ld, scores=dec2.scores, cfg=cfg), reps=10) * 1e3
+    step262_bytes, kc262, gather262 = decode_bytes(d2.seqlens, kc_bpb)
+    assert qsa.device_status() == 0
+    del d2, kc2, dec2
+    torch.cuda.empty_cache()
 
     # end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
@@ -219,23 +301,26 @@ def run_qsa(args, rank, world, device):
         e2e_ms = allmax(e0.elapsed_time(e1) / args.e2e_steps)
         e2e = {"value": ranks.job_throughput(world, N_PREFILL, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps, "scope": "prefill 262144 via qsa.Prefill"}
+        del host, o_host, dev_in
 
     # the build's dense causal attention on the same inputs (the pages' comparison)
     dense = None
     if args.dense:
+        dd = inputs.make_decode(DEC_BATCH, DEC_LEN, None, seed=seeds["decode"], device=device)
         cu_dec_q = torch.arange(DEC_BATCH + 1, dtype=torch.int32, device=device)
+        dec_o = torch.empty_like(dd.q)
         qsa.dense_attn_prefill(x.q, x.k, x.v, pre.cu, pre.cu, N_PREFILL, o=o, cfg=cfg, max_len_k=N_PREFILL)
         dws = torch.empty((qsa.workspace_size(qsa.OP_DENSE, DEC_BATCH, DEC_BATCH, DEC_LEN, cfg),),
                           dtype=torch.uint8, device=device)
-        qsa.dense_attn_prefill(d.q, d.k_cache, d.v_cache, cu_dec_q, cu_k, 1, o=dec_o, cfg=cfg, max_len_k=DEC_LEN,
-                               ws=dws)
+        qsa.dense_attn_prefill(dd.q, dd.k_cache, dd.v_cache, cu_dec_q, dd.cu_seqlens_k, 1, o=dec_o, cfg=cfg,
+                               max_len_k=DEC_LEN, ws=dws)
         torch.cuda.synchronize()
         e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         e[0].record(stream)
         qsa.dense_attn_prefill(x.q, x.k, x.v, pre.cu, pre.cu, N_PREFILL, o=o, cfg=cfg, max_len_k=N_PREFILL)
         e[1].record(stream)
         for _ in range(5):
-            qsa.dense_attn_prefill(d.q, d.k_cache, d.v_cache, cu_dec_q, cu_k, 1, o=dec_o, cfg=cfg,
+            qsa.dense_attn_prefill(dd.q, dd.k_cache, dd.v_cache, cu_dec_q, dd.cu_seqlens_k, 1, o=dec_o, cfg=cfg,
                                    max_len_k=DEC_LEN, ws=dws)
         e[2].record(stream)
         torch.cuda.synchronize()
@@ -247,16 +332,50 @@ def run_qsa(args, rank, world, device):
                  "qsa_layer_speedup": dp_ms / prefill_ms, "qsa_attention_only_speedup": dp_ms / attn_ms,
                  "decode_step_us": dd_us, "qsa_decode_speedup": dd_us / (dec_ms * 1e3),
                  "pages_context": "7.6x prefill / 4.9x decode at 1M context, kernel level, hardware not stated"}
-
-    same_src = attn_src_hash() == ATTN_TRAFFIC["src_sha256_16"]
-    traffic = ATTN_TRAFFIC["bytes"] if (same_src and world == 1) else None
+        del dd
 
     sel_tok = selected_tokens(N_PREFILL)
     gather = gather_bytes_per_query(1) * sel_tok
-    achieved = gather / (attn_ms / 1e3) / 1e9
-    n_chunks = (N_PREFILL + CHUNK - 1) // CHUNK
+    attn_flops = 24 * 256 * 4 * sel_tok
+    pairs = index_pairs(N_PREFILL)
+    traffic = None
+    if attn_src_hash() == ATTN_SMALL_TRAFFIC["src_sha256_16"] and world == 1:
+        traffic = ATTN_SMALL_TRAFFIC["bytes"] * gather / ATTN_SMALL_TRAFFIC["gather_bytes"]
+    attn_tflops = attn_flops / (attn_ms / 1e3) / 1e12
     launches_prefill = 1 + 2 * n_chunks + 1  # compress; index + select per chunk; attention over all rows
-    launches_decode = 1 + 1 + 1 + 2
+    launches_decode = 1 + 1 + 1 + 2           # refresh, indexer, select, attention + merge
+    kern = {
+        "sparse_attn_prefill": {
+            "ms": attn_ms, "bound": "tensor", "flop": attn_flops, "achieved_tflops": attn_tflops,
+            "peak_tflops": tflops_sus, "frac": attn_tflops / tflops_sus,
+            "gather_bytes": gather, "effective_gather_TBps": gather / (attn_ms / 1e3) / 1e12,
+            "dram_traffic_est": traffic,
+            "dram_frac": (traffic / (attn_ms / 1e3) / 1e9 / hbm) if traffic else None},
+        "index_tc": {
+            "ms_per_step": index_ms, "bound": "tensor", "method_flop": 1024.0 * pairs,
+            "achieved_tflops": 1024.0 * pairs / (index_ms / 1e3) / 1e12, "peak_tflops": tflops_sus,
+            "frac": 1024.0 * pairs / (index_ms / 1e3) / 1e12 / tflops_sus,
+            "score_bytes_written": 4.0 * pairs},
+        "select": {
+            "ms_per_step": select_ms, "bound": "hbm", "bytes": 4.0 * pairs,
+            "achieved_gbs": 4.0 * pairs / (select_ms / 1e3) / 1e9, "peak_gbs": hbm,
+            "frac": 4.0 * pairs / (select_ms / 1e3) / 1e9 / hbm},
+        "decode_131k": {
+            "step_us": dec_ms * 1e3, "step_bytes": step_bytes,
+            "step_frac": step_bytes / (dec_ms / 1e3) / 1e9 / hbm,
+            "index_us": dec_index_us, "kc_scan_bytes": kc_scan,
+            "index_frac": kc_scan / (dec_index_us / 1e6) / 1e9 / hbm,
+            "select_us": dec_select_us,
+            "attn_us": dec_attn_us, "attn_bytes": dec_gather,
+            "attn_frac": dec_gather / (dec_attn_us / 1e6) / 1e9 / hbm},
+        "decode_262k": {
+            "step_us": step262_us, "step_bytes": step262_bytes,
+            "step_frac": step262_bytes / (step262_us / 1e6) / 1e9 / hbm,
+            "index_us": index262_us, "kc_scan_bytes": kc262,
+            "index_frac": kc262 / (index262_us / 1e6) / 1e9 / hbm,
+            "attn_us": attn262_us, "attn_bytes": gather262,
+            "attn_frac": gather262 / (attn262_us / 1e6) / 1e9 / hbm},
+    }
     res = {
         "metric": METRIC,
         "value": ranks.job_throughput(world, N_PREFILL, prefill_ms),
@@ -276,9 +395,11 @@ def run_qsa(args, rank, world, device):
                    "parallelism": "independent layer per rank" if world > 1 else "1 GPU"},
         "decode": {"batch": DEC_BATCH, "ctx": DEC_LEN, "step_us": dec_ms * 1e3, "us_per_token": dec_ms * 1e3,
                    "us_per_token_amortized": dec_ms * 1e3 / DEC_BATCH},
-        "roofline": {"kernel": "sparse_attn_kernel (prefill)", "bound": "hbm", "achieved": achieved,
-                     "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
-                     "algorithmic_bytes": gather, "peak_kind": peak_kind + " (burst copy)"},
+        "roofline": {"kernel": "sparse_attn_kernel (prefill)", "bound": "tensor", "achieved": attn_tflops,
+                     "peak": tflops_sus, "unit": "TFLOP/s", "frac": attn_tflops / tflops_sus, "traffic": traffic,
+                     "peak_kind": peak_kind + " (sustained bf16: the kernel runs inside a long step)",
+                     "note": "gather-bound: 4 MiB of K/V per query against 25 MFLOP; see kernels"},
+        "kernels": kern,
         "gpu_launches": args.steps * (launches_prefill + launches_decode),
         "dense": dense,
         "e2e": e2e,
@@ -421,7 +542,7 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="qsa", choices=["qsa", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", dest="dense", action="store_false",
                     help="skip the dense causal-attention comparison")

@@ -2,6 +2,7 @@
 // host-side argument validation, tensor-map creation and kernel dispatch.
 // Nothing here allocates device memory; every buffer is the caller's.
 #include <mutex>
+#include <vector>
 
 #include "kernels.cuh"
 
@@ -75,6 +76,25 @@ bool make_tmap_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, 
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t set_smem_attr_once(const void *func, int bytes)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    struct Done {
+        const void *func;
+        int dev, bytes;
+    };
+    static std::mutex mu;
+    static std::vector<Done> done;
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Done &d : done)
+        if (d.func == func && d.dev == dev && d.bytes >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.push_back(Done{func, dev, bytes});
+    return e;
 }
 
 int num_sms()

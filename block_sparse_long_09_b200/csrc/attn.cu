@@ -580,10 +580,9 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream)
     // k, v as (64 d, token-row, 4 d-chunks) with strides (512 B, 128 B): one box = one micro-block
     if (!make_tmap_3d(&mk, a.k, 64, (uint64_t)a.total_k * kHKV, 4, kD * 2, 128, 64, 8, 4)) return cudaErrorInvalidValue;
     if (!make_tmap_3d(&mv, a.v, 64, (uint64_t)a.total_k * kHKV, 4, kD * 2, 128, 64, 8, 4)) return cudaErrorInvalidValue;
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttSmem);
-        attr = true;
+    {
+        const cudaError_t e = set_smem_attr_once(reinterpret_cast<const void *>(sparse_attn_kernel), kAttSmem);
+        if (e != cudaSuccess) return e;
     }
     float *ws = a.ws;
     int32_t *bounds = nullptr;

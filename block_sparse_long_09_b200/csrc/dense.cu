@@ -350,10 +350,9 @@ cudaError_t launch_dense_attn(const DenseArgs &a, cudaStream_t stream)
         return cudaErrorInvalidValue;
     if (!make_tmap_3d(&mv, a.v, kD, kHKV, (uint64_t)a.total_k, kD * 2, (uint64_t)kHKV * kD * 2, 64, 1, kBK))
         return cudaErrorInvalidValue;
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(dense_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDenseSmem);
-        attr = true;
+    {
+        const cudaError_t e = set_smem_attr_once(reinterpret_cast<const void *>(dense_attn_kernel), kDenseSmem);
+        if (e != cudaSuccess) return e;
     }
     // upper bound on tiles: every sequence may add one partial tile
     const int64_t max_tiles = (a.total_q + kBQ - 1) / kBQ + a.batch;

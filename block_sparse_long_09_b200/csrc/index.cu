@@ -419,10 +419,9 @@ cudaError_t launch_index_tc(const IndexArgs &a, cudaStream_t stream)
     int use_tma = ((a.ld & 3) == 0) && make_tmap_2d_f32(&ms, a.scores, (uint64_t)a.ld, (uint64_t)rows,
                                                        (uint64_t)a.ld * 4, 32, 32);
     if (!use_tma) ms = mq;  // unused
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(index_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kIdxSmem);
-        attr = true;
+    {
+        const cudaError_t e = set_smem_attr_once(reinterpret_cast<const void *>(index_tc_kernel), kIdxSmem);
+        if (e != cudaSuccess) return e;
     }
     const int64_t tiles = (rows + kTokTile - 1) / kTokTile;
     index_tc_kernel<<<(unsigned)tiles, kIdxThreads, kIdxSmem, stream>>>(

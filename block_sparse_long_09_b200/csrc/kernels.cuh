@@ -24,7 +24,7 @@ cudaError_t launch_compress(const __nv_bfloat16 *k_idx, const int32_t *cu_k, con
 struct IndexArgs {
     const __nv_bfloat16 *q_idx;  // [total_q, 4, 128]
     const float *w;              // [total_q, 4]
-    const __nv_bfloat16 *kc;     // [kc_rows, 128]
+    const __nv_bfloat16 *kc;     // [kc_rows, 2, 128]: hi plane, then lo plane
     int64_t kc_rows;
     const int32_t *cu_q, *cu_k, *cu_blocks;
     int batch;
@@ -99,5 +99,8 @@ bool make_tmap_2d_f32(CUtensorMap *map, const void *base, uint64_t inner, uint64
 bool make_tmap_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
 int num_sms();
+// Opt-in dynamic shared memory of `func` on the current device, set once per device
+// (thread-safe; later calls on that device only look it up).
+cudaError_t set_smem_attr_once(const void *func, int bytes);
 
 }  // namespace qsa

@@ -37,7 +37,13 @@
  *    heads, head dim 256, 4 indexer heads of dim 128) with a budget of
  *    k <= 2048 blocks (the model uses 512); anything else returns
  *    QSA_ERR_UNSUPPORTED.
- *  - Thread safety: the library keeps no state besides the status word.
+ *  - Thread safety: calls may come from several host threads.  Host-side
+ *    state is set up once and guarded by locks: the driver's tensor-map
+ *    encoder, each kernel's shared-memory opt-in (once per device) and the
+ *    static-scratch address (once per device).  The device keeps one sticky
+ *    status word per device.  Work on the GPU is ordered by the caller's
+ *    streams; only qsa_sparse_attn_decode_static_scratch shares memory
+ *    between calls (see there).
  */
 #ifndef QSA_H
 #define QSA_H

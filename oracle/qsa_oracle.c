@@ -17,7 +17,7 @@
  *   [table]  same page, "Model Summary" table: QSA 24 query / 2 KV heads, head
  *            dim 256; indexer 4 query heads, 1 key head, dim 128, ratio 4.
  *
- * Readings where the pages are silent (each also listed in the design notes):
+ * Readings where the pages are silent:
  *   - RMSNorm in the compressor has unit gain and eps (default 1e-6); the
  *     caller may switch it off (plain mean-pool).
  *   - the indexer score carries a per-(query, head) weight w; w = 1 gives the

@@ -1,0 +1,162 @@
+"""GPU vs oracle parity at the benchmarked workloads, on sampled rows.
+
+Every result of a row depends on that row alone (its scores against the earlier
+compressed keys, its own top-k, its own attention), so the fp64 oracle is run
+on a sample of rows of the full-size problem: the first 64 rows, the last 64,
+256 seeded random rows and the first and last row of each random row's
+micro-block.  The GPU side runs exactly as the benchmark does (the same inputs,
+16 384-row chunks, the same launches).  Per sampled row:
+
+  scores     GPU indexer scores within the score tolerance of the oracle's
+  selection  the GPU's top-k against the oracle's under the near-threshold rule
+  attention  the GPU's output against the oracle's attention on the GPU's selection
+
+Workloads: prefill of one 262 144-token sequence (N(0,1) inputs), prefill of two
+65 536-token sequences with peaked indexer keys, and decode steps at batch 64
+with every cache at 131 072 tokens and with lengths U{32 768 .. 262 144}.
+"""
+import os
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_long_09_b200 import inputs
+from parity_common import (SCALE, bits, check_attn, check_scores, check_selection_invariants,
+                           check_selection_near_threshold, sampled_rows)
+
+pytestmark = pytest.mark.gpu
+
+K = 512
+CHUNK = 16384
+
+
+@pytest.fixture(scope="module")
+def qsa():
+    from block_sparse_long_09_b200 import build
+    build.build()
+    from block_sparse_long_09_b200 import qsa as q
+    assert torch.cuda.is_available()
+    q.device_status(clear=True)
+    return q
+
+
+def row_runs(rows):
+    """Contiguous runs [a, b) covering the sorted rows."""
+    runs, a, prev = [], int(rows[0]), int(rows[0])
+    for x in rows[1:]:
+        x = int(x)
+        if x != prev + 1:
+            runs.append((a, prev + 1))
+            a = x
+        prev = x
+    runs.append((a, prev + 1))
+    return runs
+
+
+def prefill_case(qsa, lengths, peaked, seed):
+    """Run the prefill of the benchmark and check sampled rows of every sequence."""
+    dev = torch.device("cuda")
+    x = inputs.make_prefill(lengths, seed=seed, peaked=peaked, device=dev)
+    cfg = qsa.default_config(budget_blocks=K)
+    pre = qsa.Prefill(lengths, chunk_rows=CHUNK, cfg=cfg, device=dev)
+    o = pre(x.q, x.k, x.v, x.q_idx, x.w, x.k_idx)
+    torch.cuda.synchronize()
+    assert qsa.device_status(clear=True) == 0
+    start = 0
+    for s, L in enumerate(lengths):
+        rows = sampled_rows(L, seed=1000 + s)
+        g_rows = start + rows
+        # GPU scores of the sampled rows: the indexer on each contiguous run of them
+        gs = np.full((rows.size, pre.ld), np.nan, dtype=np.float32)
+        pos = {int(r): n for n, r in enumerate(g_rows)}
+        for a, b in row_runs(g_rows):
+            sc = qsa.index_scores(x.q_idx, x.w, pre.kc[: pre.n_blocks], pre.cu, pre.cu, pre.cu_blocks, pre.max_len,
+                                  pre.ld, a, b, cfg=cfg)
+            sc = sc.cpu().numpy()
+            for i in range(a, b):
+                gs[pos[i]] = sc[i - a]
+        sel_g = pre.sel[torch.as_tensor(g_rows, device=dev)].cpu().numpy()
+        o_g = o[torch.as_tensor(g_rows, device=dev)].float().cpu().numpy()
+        # the oracle: scores of the sampled rows (query t of the sequence sees keys 0 .. t),
+        # then attention row by row on host threads (each call releases the GIL)
+        k_b = bits(x.k[start:start + L])
+        v_b = bits(x.v[start:start + L])
+        kc_o = oracle.compress(bits(x.k_idx[start:start + L]), 4)
+        q_b = bits(x.q[torch.as_tensor(g_rows, device=dev)])
+        bt = rows // 4
+        sc_o = oracle.index_scores(bits(x.q_idx[start:start + L]), x.w[start:start + L].cpu(), kc_o, L, L, 4, rows,
+                                   ld=pre.ld)
+        check_scores(gs, sc_o, bt, K)
+        check_selection_invariants(sel_g, bt, K)
+        sel_o = oracle.select(sc_o, bt, K)
+        agree = check_selection_near_threshold(sel_g, sel_o, sc_o, bt, K)
+        assert agree.mean() > 0.9, agree.mean()
+
+        def attend_row(n):
+            t = int(rows[n])
+            return oracle.attend(q_b[n:n + 1], k_b[:t + 1], v_b[:t + 1], sel_g[n:n + 1], 1, t + 1, 4, SCALE, [0])[0][0]
+
+        with ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
+            ref_o = np.stack(list(ex.map(attend_row, range(rows.size))))
+        check_attn(o_g, ref_o)
+        start += L
+    assert qsa.device_status(clear=True) == 0
+
+
+def test_prefill_262144_sampled_rows(qsa):
+    """Batch 1, n = 262 144, N(0,1) inputs, budget 512 blocks (the benchmark's prefill)."""
+    prefill_case(qsa, [262144], peaked=False, seed=0)
+
+
+def test_prefill_2x65536_peaked_sampled_rows(qsa):
+    """Batch 2, n = 65 536 each, indexer keys with one N(0, 0.5^2) offset per block."""
+    prefill_case(qsa, [65536, 65536], peaked=True, seed=0)
+
+
+def decode_case(qsa, lo, hi, seed):
+    """One decode step at batch 64 exactly as the benchmark runs it (CUDA graph of
+    compress refresh, indexer, select, attention, merge); every sequence checked."""
+    from block_sparse_long_09_b200 import ranks
+    dev = torch.device("cuda")
+    batch = 64
+    d = inputs.make_decode(batch, lo, hi, seed=seed, device=dev)
+    cfg = qsa.default_config(budget_blocks=K)
+    kc = qsa.compress_keys(d.k_idx, d.cu_seqlens_k, d.cu_blocks, n_blocks=int(d.cu_blocks[-1]), cfg=cfg)
+    last = torch.tensor([L // 4 - 1 for L in d.seqlens], dtype=torch.int32, device=dev)
+    step = qsa.DecodeStep(d.q, d.q_idx, d.w, d.k_cache, d.v_cache, d.k_idx, kc, d.cu_seqlens_k, d.cu_blocks,
+                          max(d.seqlens), refresh_blocks=last, cfg=cfg, graph=True)
+    o = step().float().cpu().numpy()
+    torch.cuda.synchronize()
+    assert qsa.device_status(clear=True) == 0
+    sel_g = step.sel.cpu().numpy()
+    gs = step.scores.cpu().numpy()
+    cu = d.cu_seqlens_k.cpu().numpy()
+    agree = 0
+    for s, L in enumerate(d.seqlens):
+        a, b = int(cu[s]), int(cu[s + 1])
+        bt = (L - 1) // 4
+        kc_o = oracle.compress(bits(d.k_idx[a:b]), 4)
+        sc_o = oracle.index_scores(bits(d.q_idx[s:s + 1]), d.w[s:s + 1].cpu(), kc_o, 1, L, 4, [0], ld=step.ld)
+        check_scores(gs[s:s + 1], sc_o, [bt], K)
+        check_selection_invariants(sel_g[s:s + 1], [bt], K)
+        sel_o = oracle.select(sc_o, [bt], K)
+        agree += int(check_selection_near_threshold(sel_g[s:s + 1], sel_o, sc_o, [bt], K)[0])
+        ref_o, _ = oracle.attend(bits(d.q[s:s + 1]), bits(d.k_cache[a:b]), bits(d.v_cache[a:b]), sel_g[s:s + 1], 1, L,
+                                 4, SCALE, [0])
+        check_attn(o[s:s + 1], ref_o)
+    assert agree >= 0.9 * batch, agree
+    del step
+    assert ranks.rank_seeds(0)["decode"] == 100  # the benchmark's decode seed
+
+
+def test_decode_b64_ctx131072(qsa):
+    """Every cache at 131 072 tokens (the decode metric's context), the benchmark's seed."""
+    decode_case(qsa, 131072, None, seed=100)
+
+
+def test_decode_b64_mixed_lengths(qsa):
+    """Cache lengths U{32 768 .. 262 144}."""
+    decode_case(qsa, 32768, 262144, seed=0)

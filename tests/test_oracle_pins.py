@@ -122,6 +122,49 @@ def test_scores_w_one_is_unweighted_relu_sum():
         assert np.all(np.isneginf(s[i, bt:]))
 
 
+def _read_scores_fixture():
+    kc, q, w, s = {}, {}, {}, {}
+    with open(os.path.join(GOLDEN, "scores_hand.txt")) as f:
+        for line in f:
+            if line.startswith("#") or ":" not in line:
+                continue
+            head, vals = line.split(":")
+            key = head.split()
+            v = [float(x) for x in vals.split()]
+            if key[0] == "kc":
+                kc[int(key[1])] = v
+            elif key[0] == "q":
+                q[(int(key[1]), int(key[2]))] = v
+            elif key[0] == "w":
+                w[int(key[1])] = v
+            elif key[0] == "s":
+                s[(int(key[1]), int(key[2]))] = v[0]
+    return kc, q, w, s
+
+
+def test_scores_hand_fixture():
+    """Hand-worked scores (tests/golden/scores_hand.txt): a negative dot that the
+    ReLU must zero, unequal head weights, the own block and earlier rows at -inf."""
+    kc_d, q_d, w_d, s_d = _read_scores_fixture()
+    L, H, d = 12, 4, 4
+    kc = np.array([kc_d[b] for b in range(3)], dtype=np.float64)
+    q = np.zeros((L, H, d), dtype=np.float32)
+    w = np.zeros((L, H), dtype=np.float32)
+    for (t, h), v in q_d.items():
+        q[t, h] = v
+    for t, v in w_d.items():
+        w[t] = v
+    rows = sorted({t for t, _ in s_d})
+    s = oracle.index_scores(bf16(q), torch.from_numpy(w), kc, L, L, 4, rows, ld=3)
+    for n, t in enumerate(rows):
+        for b in range(3):
+            want = s_d[(t, b)]
+            if math.isinf(want):
+                assert np.isneginf(s[n, b]), (t, b, s[n, b])
+            else:
+                assert s[n, b] == want, (t, b, s[n, b], want)
+
+
 def test_scores_decode_position():
     """Lq < Lk: query row i sits at t = Lk - Lq + i."""
     Lk, Lq = 41, 3
