@@ -55,10 +55,11 @@ def _load():
             lib.qsa_oracle_compress.argtypes = [P, I64, I, I, I, D, P]
             lib.qsa_oracle_index_scores.argtypes = [P, P, P, I64, I64, I, I, I, P, I64, P, I64]
             lib.qsa_oracle_select.argtypes = [P, I64, P, I64, I, P]
+            lib.qsa_oracle_select_shared.argtypes = [P, I64, P, I64, I, I, I, P]
             lib.qsa_oracle_attend.argtypes = [P, P, P, P, I, I64, I64, I, I, I, I, D, P, I64, P, P]
             lib.qsa_oracle_dense.argtypes = [P, P, P, I64, I64, I, I, I, D, P, I64, P, P]
             lib.qsa_oracle_threads.restype = I
-            for f in ("qsa_oracle_compress", "qsa_oracle_index_scores", "qsa_oracle_select",
+            for f in ("qsa_oracle_compress", "qsa_oracle_index_scores", "qsa_oracle_select", "qsa_oracle_select_shared",
                       "qsa_oracle_attend", "qsa_oracle_dense"):
                 getattr(lib, f).restype = None
             _lib = lib
@@ -143,6 +144,20 @@ def select(scores, bt, k: int) -> np.ndarray:
     assert bt.size == 0 or bt.max() <= s.shape[1]
     out = np.empty((s.shape[0], k), dtype=np.int32)
     _load().qsa_oracle_select(_ptr(s), s.shape[1], _ptr(bt), s.shape[0], int(k), _ptr(out))
+    return out
+
+
+def select_shared(scores, lengths, next_n: int, k: int, r: int = 4) -> np.ndarray:
+    """One selection per sequence for its next_n queries t = L - next_n .. L - 1, from the
+    scores of its last query (row n of scores): the own blocks of all of them forced,
+    the rest the best earlier blocks (score desc, index asc); int32 [nrows, k]."""
+    s = _f64(scores)
+    L = np.ascontiguousarray(np.asarray(lengths, dtype=np.int64))
+    assert s.ndim == 2 and L.shape == (s.shape[0],) and next_n >= 1
+    assert L.size == 0 or ((L - 1) // r).max() <= s.shape[1]
+    out = np.empty((s.shape[0], k), dtype=np.int32)
+    _load().qsa_oracle_select_shared(_ptr(s), s.shape[1], _ptr(L), s.shape[0], int(next_n), int(r), int(k),
+                                     _ptr(out))
     return out
 
 

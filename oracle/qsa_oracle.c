@@ -158,6 +158,46 @@ void qsa_oracle_select(const double *scores, int64_t ld, const int64_t *bt,
     }
 }
 
+/* Decode with multi-token prediction ("结果 2": decode at next_n = 4 with three MTP
+ * steps; section 5, step 5: the MTP steps reuse the QSA top-k indices).  Reading
+ * taken: ONE selection per sequence serves its next_n queries t = L - next_n ..
+ * L - 1, made from the indexer scores of the last query (row n of `scores`, blocks
+ * b < floor((L - 1) / r)).  Every query keeps its own trailing causal block (the
+ * budget sentence), so the own blocks floor((L - next_n) / r) .. floor((L - 1) / r)
+ * are all forced; the other slots, at most k minus their number, go to the best
+ * blocks below the first of them (score descending, lower index first on ties).
+ * Output ascending, padded with -1.  next_n = 1 is qsa_oracle_select. */
+void qsa_oracle_select_shared(const double *scores, int64_t ld, const int64_t *L, int64_t nrows,
+                              int next_n, int r, int k, int32_t *sel)
+{
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t n = 0; n < nrows; ++n) {
+        int32_t *out = sel + n * k;
+        int64_t t_last = L[n] - 1, t_first = L[n] - next_n;
+        if (t_first < 0) t_first = 0;
+        int64_t b_first = t_first / r, b_last = t_last / r;
+        int64_t nf = b_last - b_first + 1;
+        struct cand *c = (struct cand *)malloc((size_t)(b_first > 0 ? b_first : 1) * sizeof *c);
+        for (int64_t b = 0; b < b_first; ++b) {
+            c[b].s = scores[n * ld + b];
+            c[b].b = b;
+        }
+        qsort(c, (size_t)b_first, sizeof *c, cand_cmp);
+        int64_t room = (int64_t)k - nf;
+        if (room < 0) room = 0;
+        int64_t take = b_first < room ? b_first : room;
+        int64_t m = 0;
+        for (int64_t j = 0; j < take; ++j)
+            out[m++] = (int32_t)c[j].b;
+        for (int64_t b = b_first; b <= b_last && m < k; ++b)
+            out[m++] = (int32_t)b;
+        qsort(out, (size_t)m, sizeof *out, i32_cmp);
+        for (int64_t j = m; j < k; ++j)
+            out[j] = -1;
+        free(c);
+    }
+}
+
 /* one query row, one head: softmax attention over an explicit token list */
 static void attend_tokens(const double *qh, const uint16_t *k, const uint16_t *v,
                           int Hkv, int D, int g, double scale,

@@ -363,3 +363,53 @@ def test_duplicate_and_padding_entries_are_ignored():
     ob, lb = oracle.attend(x.q, x.k, x.v, b, n, n, 4, 1 / 16, rows)
     np.testing.assert_array_equal(oa, ob)
     np.testing.assert_array_equal(la, lb)
+
+
+# --------------------------------------------------------------------------
+# Shared selection of a multi-token decode step
+# --------------------------------------------------------------------------
+
+def test_select_shared_hand_fixture():
+    with open(os.path.join(GOLDEN, "select_shared_hand.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            head, scores, expect = line.split("|")
+            k, next_n, L = (int(x) for x in head.split())
+            sc = [float(x) for x in scores.split()]
+            row = np.full((1, max(1, (L - 1) // 4)), -np.inf)
+            row[0, :len(sc)] = sc
+            got = oracle.select_shared(row, [L], next_n, k)
+            assert got[0].tolist() == [int(x) for x in expect.split()], (line, got)
+
+
+@pytest.mark.parametrize("L", [1, 4, 5, 17, 40, 203])
+def test_select_shared_next_n_1_is_select(L):
+    rng = np.random.default_rng(L)
+    bt = (L - 1) // 4
+    sc = rng.integers(0, 4, (1, max(1, bt))).astype(np.float64)
+    for k in (1, 2, 5, 16):
+        np.testing.assert_array_equal(oracle.select_shared(sc, [L], 1, k), oracle.select(sc, [bt], k))
+
+
+@pytest.mark.parametrize("next_n", [2, 3, 4])
+def test_select_shared_brute_force(next_n):
+    """Every subset of the candidates below the first forced block: the max-sum subset,
+    lexicographically smallest among equal sums, plus the forced own blocks."""
+    rng = np.random.default_rng(next_n)
+    for trial in range(40):
+        L = int(rng.integers(1, 36))
+        k = int(rng.integers(2, 6))
+        b_first, b_last = max(L - next_n, 0) // 4, (L - 1) // 4
+        nf = b_last - b_first + 1
+        sc = rng.integers(0, 3, (1, max(1, (L - 1) // 4))).astype(np.float64)
+        m = min(b_first, k - nf)
+        best = None
+        for sub in itertools.combinations(range(b_first), m):
+            key = (-sum(sc[0, b] for b in sub), sub)
+            if best is None or key < best:
+                best = key
+        want = sorted(list(best[1]) + list(range(b_first, b_last + 1)))
+        want += [-1] * (k - len(want))
+        got = oracle.select_shared(sc, [L], next_n, k)[0].tolist()
+        assert got == want, (L, k, next_n, sc, got, want)
