@@ -166,7 +166,7 @@ def run_qsa(args, rank, world, device):
     stream = torch.cuda.current_stream()
     n_chunks = (N_PREFILL + CHUNK - 1) // CHUNK
 
-    ev = {k: [] for k in ("p0", "p1", "a0", "a1", "d0", "d1", "ix", "sl")}
+    ev = {k: [] for k in ("p0", "p1", "a0", "a1", "d0", "d1", "ix")}
 
     def mk():
         return torch.cuda.Event(enable_timing=True)
@@ -175,22 +175,17 @@ def run_qsa(args, rank, world, device):
         e = {k: mk() for k in ("p0", "p1", "a0", "a1", "d0", "d1")} if record else None
         if record:
             e["p0"].record(stream)
-        # compress, then index and select per chunk (qsa.Prefill.index_select, with events)
+        # compress, then the fused index -> select per chunk (qsa.Prefill.index_select, with events)
         qsa.compress_keys(x.k_idx, pre.cu, pre.cu_blocks, kc=pre.kc, cfg=cfg)
         for r0 in range(0, N_PREFILL, CHUNK):
             r1 = min(N_PREFILL, r0 + CHUNK)
-            e0, e1, e2 = (mk(), mk(), mk()) if record else (None, None, None)
+            e0, e1 = (mk(), mk()) if record else (None, None)
             if record:
                 e0.record(stream)
-            qsa.index_scores(x.q_idx, x.w, pre.kc[: pre.n_blocks], pre.cu, pre.cu, pre.cu_blocks, pre.max_len,
-                             pre.ld, r0, r1, scores=pre.scores, cfg=cfg)
+            pre.select_chunk(x.q_idx, x.w, r0, r1)
             if record:
                 e1.record(stream)
-            qsa.select_blocks(pre.scores, pre.cu, pre.cu, pre.total, r0, r1, sel=pre.sel, cfg=cfg)
-            if record:
-                e2.record(stream)
                 ev["ix"].append((e0, e1))
-                ev["sl"].append((e1, e2))
         if record:
             e["a0"].record(stream)
         pre.attend(x.q, x.k, x.v, o=o)  # one pass per query
@@ -226,15 +221,14 @@ def run_qsa(args, rank, world, device):
     prefill_ms = ev_ms(list(zip(ev["p0"], ev["p1"])))
     attn_ms = ev_ms(list(zip(ev["a0"], ev["a1"])))
     dec_ms = ev_ms(list(zip(ev["d0"], ev["d1"])))
-    index_ms = ev_ms(ev["ix"]) * n_chunks  # per step: all chunks
-    select_ms = ev_ms(ev["sl"]) * n_chunks
+    index_ms = ev_ms(ev["ix"]) * n_chunks  # per step: all chunks of the fused index -> select
     assert qsa.device_status() == 0, "a kernel flagged a device-side error in the timed region"
 
     def allmax(v):
         return ranks.max_over_ranks([v], world, device)[0]
 
-    total_ms, prefill_ms, attn_ms, dec_ms, index_ms, select_ms = ranks.max_over_ranks(
-        [total_ms, prefill_ms, attn_ms, dec_ms, index_ms, select_ms], world, device)
+    total_ms, prefill_ms, attn_ms, dec_ms, index_ms = ranks.max_over_ranks(
+        [total_ms, prefill_ms, attn_ms, dec_ms, index_ms], world, device)
 
     def timed(fn, reps=5):
         fn()
@@ -248,13 +242,13 @@ def run_qsa(args, rank, world, device):
         return allmax(a.elapsed_time(b) / reps)
 
     # decode kernels one by one at 131072 (eager launches of the step's calls)
-    dec_index_us = timed(lambda: qsa.index_scores(dec.q_idx, dec.w, dec.kc, dec.cu_q, dec.cu_k, dec.cu_b, 1, dec.ld,
-                                                  scores=dec.scores, cfg=cfg)) * 1e3
-    dec_select_us = timed(lambda: qsa.select_blocks(dec.scores, dec.cu_q, dec.cu_k, DEC_BATCH, sel=dec.sel,
-                                                    cfg=cfg)) * 1e3
+    # the decode selection reads the hi plane of kc (half of each compressed key), then
+    # rescores each row's near-threshold window exactly
+    dec_select_us = timed(lambda: qsa.index_select(dec.q_idx, dec.w, dec.kc, dec.cu_q, dec.cu_k, dec.cu_b, 1,
+                                                   DEC_LEN, sel=dec.sel, ws=dec.ws_sel, cfg=cfg)) * 1e3
     dec_attn_us = timed(lambda: qsa.sparse_attn_decode(d.q, d.k_cache, d.v_cache, cu_k, dec.sel, o=dec_o, ws=dec.ws,
                                                        cfg=cfg)) * 1e3
-    step_bytes, kc_scan, dec_gather = decode_bytes(d.seqlens, kc_bpb)
+    step_bytes, kc_scan, dec_gather = decode_bytes(d.seqlens, kc_bpb // 2)
 
     # decode at 262144 tokens per sequence: the step, and the attention kernel alone
     del d, dec
@@ -267,9 +261,9 @@ def run_qsa(args, rank, world, device):
     step262_us = timed(dec2, reps=10) * 1e3
     attn262_us = timed(lambda: qsa.sparse_attn_decode(d2.q, d2.k_cache, d2.v_cache, d2.cu_seqlens_k, dec2.sel,
                                                       o=dec2.o, ws=dec2.ws, cfg=cfg), reps=10) * 1e3
-    index262_us = timed(lambda: qsa.index_scores(dec2.q_idx, dec2.w, dec2.kc, dec2.cu_q, dec2.cu_k, dec2.cu_b, 1,
-                                                 dec2.ld, scores=dec2.scores, cfg=cfg), reps=10) * 1e3
-    step262_bytes, kc262, gather262 = decode_bytes(d2.seqlens, kc_bpb)
+    index262_us = timed(lambda: qsa.index_select(dec2.q_idx, dec2.w, dec2.kc, dec2.cu_q, dec2.cu_k, dec2.cu_b, 1,
+                                                 262144, sel=dec2.sel, ws=dec2.ws_sel, cfg=cfg), reps=10) * 1e3
+    step262_bytes, kc262, gather262 = decode_bytes(d2.seqlens, kc_bpb // 2)
     assert qsa.device_status() == 0
     del d2, kc2, dec2
     torch.cuda.empty_cache()
@@ -342,8 +336,8 @@ def run_qsa(args, rank, world, device):
     if attn_src_hash() == ATTN_SMALL_TRAFFIC["src_sha256_16"] and world == 1:
         traffic = ATTN_SMALL_TRAFFIC["bytes"] * gather / ATTN_SMALL_TRAFFIC["gather_bytes"]
     attn_tflops = attn_flops / (attn_ms / 1e3) / 1e12
-    launches_prefill = 1 + 2 * n_chunks + 1  # compress; index + select per chunk; attention over all rows
-    launches_decode = 1 + 1 + 1 + 2           # refresh, indexer, select, attention + merge
+    launches_prefill = 1 + 5 * n_chunks + 1  # compress; 5 launches of the fused index -> select per chunk; attention
+    launches_decode = 1 + 4 + 2               # refresh; hi-plane scan, count reset, refine, fallback; attention + merge
     kern = {
         "sparse_attn_prefill": {
             "ms": attn_ms, "bound": "tensor", "flop": attn_flops, "achieved_tflops": attn_tflops,
@@ -351,28 +345,23 @@ def run_qsa(args, rank, world, device):
             "gather_bytes": gather, "effective_gather_TBps": gather / (attn_ms / 1e3) / 1e12,
             "dram_traffic_est": traffic,
             "dram_frac": (traffic / (attn_ms / 1e3) / 1e9 / hbm) if traffic else None},
-        "index_tc": {
+        "index_select": {
             "ms_per_step": index_ms, "bound": "tensor", "method_flop": 1024.0 * pairs,
             "achieved_tflops": 1024.0 * pairs / (index_ms / 1e3) / 1e12, "peak_tflops": tflops_sus,
             "frac": 1024.0 * pairs / (index_ms / 1e3) / 1e12 / tflops_sus,
-            "score_bytes_written": 4.0 * pairs},
-        "select": {
-            "ms_per_step": select_ms, "bound": "hbm", "bytes": 4.0 * pairs,
-            "achieved_gbs": 4.0 * pairs / (select_ms / 1e3) / 1e9, "peak_gbs": hbm,
-            "frac": 4.0 * pairs / (select_ms / 1e3) / 1e9 / hbm},
+            "note": "fused: sampled thresholds, candidate lists, exact top-k; no score rows in memory"},
         "decode_131k": {
             "step_us": dec_ms * 1e3, "step_bytes": step_bytes,
             "step_frac": step_bytes / (dec_ms / 1e3) / 1e9 / hbm,
-            "index_us": dec_index_us, "kc_scan_bytes": kc_scan,
-            "index_frac": kc_scan / (dec_index_us / 1e6) / 1e9 / hbm,
-            "select_us": dec_select_us,
+            "index_select_us": dec_select_us, "kc_scan_bytes": kc_scan,
+            "index_select_frac": kc_scan / (dec_select_us / 1e6) / 1e9 / hbm,
             "attn_us": dec_attn_us, "attn_bytes": dec_gather,
             "attn_frac": dec_gather / (dec_attn_us / 1e6) / 1e9 / hbm},
         "decode_262k": {
             "step_us": step262_us, "step_bytes": step262_bytes,
             "step_frac": step262_bytes / (step262_us / 1e6) / 1e9 / hbm,
-            "index_us": index262_us, "kc_scan_bytes": kc262,
-            "index_frac": kc262 / (index262_us / 1e6) / 1e9 / hbm,
+            "index_select_us": index262_us, "kc_scan_bytes": kc262,
+            "index_select_frac": kc262 / (index262_us / 1e6) / 1e9 / hbm,
             "attn_us": attn262_us, "attn_bytes": gather262,
             "attn_frac": gather262 / (attn262_us / 1e6) / 1e9 / hbm},
     }
@@ -508,28 +497,26 @@ def run_profile_case(case: str, reps: int = 3):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     cfg = qsa.default_config(budget_blocks=BUDGET)
-    if case in ("attn", "index", "select"):
+    if case in ("attn", "index", "select", "index_select"):
         n, rows = 131072, 8192
         x = inputs.make_prefill([n], seed=0, device=dev)
-        pre = qsa.Prefill([n], chunk_rows=rows, cfg=cfg, device=dev)
+        pre = qsa.Prefill([n], chunk_rows=rows, cfg=cfg, device=dev, fused=case in ("attn", "index_select"))
         qsa.compress_keys(x.k_idx, pre.cu, pre.cu_blocks, kc=pre.kc, cfg=cfg)
         r0 = n - rows
         for _ in range(reps):
-            if case in ("index", "select", "attn"):
-                qsa.index_scores(x.q_idx, x.w, pre.kc[: pre.n_blocks], pre.cu, pre.cu, pre.cu_blocks, n, pre.ld,
-                                 r0, n, scores=pre.scores, cfg=cfg)
-                qsa.select_blocks(pre.scores, pre.cu, pre.cu, n, r0, n, sel=pre.sel, cfg=cfg)
+            pre.select_chunk(x.q_idx, x.w, r0, n)
             if case == "attn":
                 qsa.sparse_attn_prefill(x.q, x.k, x.v, pre.sel, pre.cu, pre.cu, r0, n, cfg=cfg, max_len_k=n)
-    elif case == "decode":
-        d = inputs.make_decode(DEC_BATCH, 16384, None, seed=1, device=dev)
+    elif case in ("decode", "decode131k"):
+        # decode steps of batch 64 (16384-token caches: small; 131072: the benchmark's, 17 GB)
+        L = 16384 if case == "decode" else DEC_LEN
+        d = inputs.make_decode(DEC_BATCH, L, None, seed=1, device=dev)
         cu_q = torch.arange(DEC_BATCH + 1, dtype=torch.int32, device=dev)
         kc = qsa.compress_keys(d.k_idx, d.cu_seqlens_k, d.cu_blocks, n_blocks=int(d.cu_blocks[-1]), cfg=cfg)
-        ld = (16384 - 1) // 4
-        sc = torch.empty((DEC_BATCH, ld), dtype=torch.float32, device=dev)
+        ws = torch.empty((qsa.workspace_size(qsa.OP_INDEX_SELECT, DEC_BATCH, DEC_BATCH, L, cfg),), dtype=torch.uint8,
+                         device=dev)
         for _ in range(reps):
-            qsa.index_scores(d.q_idx, d.w, kc, cu_q, d.cu_seqlens_k, d.cu_blocks, 1, ld, scores=sc, cfg=cfg)
-            sel = qsa.select_blocks(sc, cu_q, d.cu_seqlens_k, DEC_BATCH, cfg=cfg)
+            sel = qsa.index_select(d.q_idx, d.w, kc, cu_q, d.cu_seqlens_k, d.cu_blocks, 1, L, ws=ws, cfg=cfg)
             qsa.sparse_attn_decode(d.q, d.k_cache, d.v_cache, d.cu_seqlens_k, sel, cfg=cfg)
     torch.cuda.synchronize()
     assert qsa.device_status() == 0
@@ -549,7 +536,8 @@ def main():
     ap.add_argument("--extra-configs", action="store_true",
                     help="also time the other workloads (peaked 2 x 65536 prefill, decode at 262144 and mixed "
                          "lengths) and print them on stderr")
-    ap.add_argument("--profile-case", choices=["attn", "index", "select", "decode"], default=None,
+    ap.add_argument("--profile-case", choices=["attn", "index", "select", "index_select", "decode", "decode131k"],
+                    default=None,
                     help="run one small case for an ncu capture and exit")
     args = ap.parse_args()
     if args.profile_case:

@@ -4,11 +4,16 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "kernels.cuh"
 
 namespace qsa {
 
 __device__ int g_device_status = 0;
+#ifdef QSA_DEBUG_CHECKS
+__device__ int g_debug_fault_site = 0;
+#endif
 
 namespace {
 
@@ -32,6 +37,14 @@ EncodeTiledFn encode_fn()
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// one NVTX range per entry point, named after it (a no-op unless a profiler is attached)
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 }  // namespace
 
@@ -185,12 +198,34 @@ size_t qsa_workspace_size(const qsa_config *cfg, int32_t op, int32_t batch, int6
     if (op == QSA_OP_DECODE)  // the even schedule runs below two rows per CTA
         return batch < 2 * kMaxEvenCtas ? even_workspace_bytes(batch, kMaxEvenCtas) : 0;
     if (op == QSA_OP_DECODE_PAGED) return even_workspace_bytes(batch, kMaxEvenCtas);
+    if (op == QSA_OP_DECODE_MTP) return mtp_workspace_bytes(batch, cfg->budget_blocks);
+    if (op == QSA_OP_INDEX_SELECT_PAGED)  // one score row per sequence
+        return (size_t)batch * (max_len_k > 0 ? ((max_len_k - 1) / cfg->r + 3) / 4 * 4 + 4 : 4) * sizeof(float);
     if (op == QSA_OP_PREFILL) {
         const int nc = nchunks_of(cfg, max_len_k);
         return nc > 1 ? chunked_workspace_bytes(rows, nc) : 0;
     }
     if (op == QSA_OP_DENSE) return split_workspace_bytes(rows, dense_decode_nsplit(max_len_k, cfg->r));
+    if (op == QSA_OP_INDEX_SELECT) {
+        // prefill: samples, thresholds, candidate lists, fallback scratch; decode: one score row per row
+        const size_t fused = index_select_workspace_bytes(rows, max_len_k, cfg->budget_blocks, cfg->r, num_sms());
+        const int64_t ld = max_len_k > 0 ? ((max_len_k - 1) / cfg->r + 3) / 4 * 4 + 4 : 4;
+        const size_t dec = decode_select_workspace_bytes(rows, ld, num_sms());
+        return fused > dec ? fused : dec;
+    }
     return 0;
+}
+
+qsa_status qsa_debug_inject(int32_t site)
+{
+#ifdef QSA_DEBUG_CHECKS
+    if (site < 0 || site > 1) return QSA_ERR_INVALID_ARG;
+    int v = site;
+    return cudaMemcpyToSymbol(g_debug_fault_site, &v, sizeof(int)) == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
+#else
+    (void)site;
+    return QSA_ERR_UNSUPPORTED;
+#endif
 }
 
 qsa_status qsa_get_device_status(void *stream, int32_t *status, int32_t clear)
@@ -212,6 +247,7 @@ qsa_status qsa_compress_keys(const qsa_config *cfg, const qsa_bf16 *k_idx, const
                              const int32_t *cu_blocks, int32_t batch, int64_t total_k, const int32_t *blk_begin,
                              int32_t max_new_blocks, qsa_bf16 *kc, void *stream)
 {
+    const qsa::NvtxRange nvtx_range("qsa_compress_keys");
     qsa_status st = check_config(cfg);
     if (st != QSA_OK) return st;
     if (batch <= 0 || total_k < 0 || cu_seqlens_k == nullptr || cu_blocks == nullptr) return QSA_ERR_INVALID_ARG;
@@ -229,6 +265,7 @@ qsa_status qsa_index_scores(const qsa_config *cfg, const qsa_bf16 *q_idx, const 
                             int64_t row_begin, int64_t row_end, float *scores, int64_t ld, void *ws,
                             size_t ws_bytes, void *stream)
 {
+    const qsa::NvtxRange nvtx_range("qsa_index_scores");
     (void)ws;
     (void)ws_bytes;
     qsa_status st = check_config(cfg);
@@ -246,10 +283,95 @@ qsa_status qsa_index_scores(const qsa_config *cfg, const qsa_bf16 *q_idx, const 
     return cuda_status(launch_index_tc(a, s));
 }
 
+qsa_status qsa_index_select(const qsa_config *cfg, const qsa_bf16 *q_idx, const float *w, const qsa_bf16 *kc,
+                            int64_t kc_rows, const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                            const int32_t *cu_blocks, int32_t batch, int64_t total_q, int32_t max_len_q,
+                            int64_t max_len_k, int64_t row_begin, int64_t row_end, int32_t *sel, void *ws,
+                            size_t ws_bytes, void *stream)
+{
+    const qsa::NvtxRange nvtx_range("qsa_index_select");
+    qsa_status st = check_config(cfg);
+    if (st != QSA_OK) return st;
+    if (batch <= 0 || total_q < 0 || kc_rows < 0 || max_len_q < 0 || max_len_k < 0) return QSA_ERR_INVALID_ARG;
+    if (row_begin < 0 || row_end < row_begin || row_end > total_q) return QSA_ERR_INVALID_ARG;
+    if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr || cu_blocks == nullptr) return QSA_ERR_INVALID_ARG;
+    if (row_end == row_begin) return QSA_OK;
+    if (q_idx == nullptr || w == nullptr || kc == nullptr || sel == nullptr || !al16(q_idx) || !al16(kc))
+        return QSA_ERR_INVALID_ARG;
+    const int64_t rows = row_end - row_begin;
+    if (ws == nullptr || !al16(ws)) return QSA_ERR_WORKSPACE_TOO_SMALL;
+    if (ws_bytes < qsa_workspace_size(cfg, QSA_OP_INDEX_SELECT, batch, rows, max_len_k))
+        return QSA_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t ld = max_len_k > 0 ? ((max_len_k - 1) / cfg->r + 3) / 4 * 4 + 4 : 4;
+    IndexArgs a{bf(q_idx), w, bf(kc), kc_rows, cu_seqlens_q, cu_seqlens_k, cu_blocks, batch, total_q,
+                row_begin, row_end, static_cast<float *>(ws), ld, cfg->r};
+    if (kc_rows == 0) {  // no complete block anywhere: every row keeps only its own block
+        SelectArgs sa{static_cast<const float *>(ws), ld, cu_seqlens_q, cu_seqlens_k, batch, row_begin, row_end, sel,
+                      cfg->budget_blocks, cfg->r};
+        return cuda_status(launch_select(sa, s));
+    }
+    if (max_len_q == 1) {
+        // decode rows: the hi-plane scan and the exact rescoring of each row's window
+        // (the error bound needs RMSNorm'ed keys; without the norm, the exact scan)
+        const bool refine = (cfg->flags & QSA_COMPRESS_NO_NORM) == 0;
+        return cuda_status(launch_decode_index_select(a, cfg->budget_blocks, ws, num_sms(), refine, sel, s));
+    }
+    return cuda_status(launch_index_select(a, cfg->budget_blocks, ws, num_sms(), max_len_k, sel, s));
+}
+
+qsa_status qsa_compress_keys_paged(const qsa_config *cfg, const qsa_bf16 *k_idx_pages, qsa_bf16 *kc_pages,
+                                   int64_t num_pages, int32_t page_size, const int32_t *block_table,
+                                   int32_t max_pages, const int32_t *cu_seqlens_k, int32_t batch, int64_t max_len_k,
+                                   const int32_t *blk_begin, int32_t max_new_blocks, void *stream)
+{
+    const qsa::NvtxRange nvtx_range("qsa_compress_keys_paged");
+    qsa_status st = check_config(cfg);
+    if (st != QSA_OK) return st;
+    if (batch <= 0 || num_pages <= 0 || page_size <= 0 || max_pages <= 0 || max_len_k < 0 ||
+        cu_seqlens_k == nullptr || block_table == nullptr)
+        return QSA_ERR_INVALID_ARG;
+    if (page_size % cfg->r != 0 || (blk_begin != nullptr && max_new_blocks <= 0)) return QSA_ERR_INVALID_ARG;
+    if (num_pages * (int64_t)page_size >= ((int64_t)1 << 40)) return QSA_ERR_UNSUPPORTED;
+    if (k_idx_pages == nullptr || kc_pages == nullptr || !al16(k_idx_pages) || !al16(kc_pages))
+        return QSA_ERR_INVALID_ARG;
+    PagedArgs p{num_pages, page_size, block_table, max_pages, cu_seqlens_k, batch, cfg->r};
+    return cuda_status(launch_compress_paged(p, bf(k_idx_pages), bf(kc_pages), blk_begin, max_new_blocks, max_len_k,
+                                             (cfg->flags & QSA_COMPRESS_NO_NORM) == 0, cfg->rms_eps,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+qsa_status qsa_index_select_paged(const qsa_config *cfg, const qsa_bf16 *q_idx, const float *w,
+                                  const qsa_bf16 *kc_pages, int64_t num_pages, int32_t page_size,
+                                  const int32_t *block_table, int32_t max_pages, const int32_t *cu_seqlens_k,
+                                  int32_t batch, int64_t max_len_k, int32_t *sel, void *ws, size_t ws_bytes,
+                                  void *stream)
+{
+    const qsa::NvtxRange nvtx_range("qsa_index_select_paged");
+    qsa_status st = check_config(cfg);
+    if (st != QSA_OK) return st;
+    if (batch <= 0 || batch > 65535 || num_pages <= 0 || page_size <= 0 || max_pages <= 0 || max_len_k <= 0 ||
+        cu_seqlens_k == nullptr || block_table == nullptr)
+        return QSA_ERR_INVALID_ARG;
+    if (page_size % cfg->r != 0) return QSA_ERR_INVALID_ARG;
+    if (q_idx == nullptr || w == nullptr || kc_pages == nullptr || sel == nullptr || !al16(q_idx) || !al16(kc_pages))
+        return QSA_ERR_INVALID_ARG;
+    const int64_t ld = ((max_len_k - 1) / cfg->r + 3) / 4 * 4 + 4;
+    if (ws == nullptr || !al16(ws) || ws_bytes < (size_t)batch * ld * sizeof(float)) return QSA_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    PagedArgs p{num_pages, page_size, block_table, max_pages, cu_seqlens_k, batch, cfg->r};
+    float *scores = static_cast<float *>(ws);
+    cudaError_t e = launch_index_paged(p, bf(q_idx), w, bf(kc_pages), scores, ld, s);
+    if (e != cudaSuccess) return QSA_ERR_CUDA;
+    SelectArgs sa{scores, ld, nullptr, cu_seqlens_k, batch, 0, batch, sel, cfg->budget_blocks, cfg->r};
+    return cuda_status(launch_select(sa, s));
+}
+
 qsa_status qsa_select_blocks(const qsa_config *cfg, const float *scores, int64_t ld, const int32_t *cu_seqlens_q,
                              const int32_t *cu_seqlens_k, int32_t batch, int64_t row_begin, int64_t row_end,
                              int32_t *sel, void *ws, size_t ws_bytes, void *stream)
 {
+    const qsa::NvtxRange nvtx_range("qsa_select_blocks");
     (void)ws;
     (void)ws_bytes;
     qsa_status st = check_config(cfg);
@@ -268,6 +390,7 @@ qsa_status qsa_sparse_attn_prefill(const qsa_config *cfg, const qsa_bf16 *q, con
                                    int64_t row_begin, int64_t row_end, qsa_bf16 *o, float *lse, void *ws,
                                    size_t ws_bytes, void *stream)
 {
+    const qsa::NvtxRange nvtx_range("qsa_sparse_attn_prefill");
     qsa_status st = check_config(cfg);
     if (st != QSA_OK) return st;
     if (batch <= 0 || total_q < 0 || total_k < 0 || max_len_k < 0 || row_begin < 0 || row_end < row_begin ||
@@ -295,6 +418,7 @@ qsa_status qsa_sparse_attn_decode(const qsa_config *cfg, const qsa_bf16 *q, cons
                                   int64_t total_k, const int32_t *sel, qsa_bf16 *o, float *lse, void *ws,
                                   size_t ws_bytes, void *stream)
 {
+    const qsa::NvtxRange nvtx_range("qsa_sparse_attn_decode");
     qsa_status st = check_config(cfg);
     if (st != QSA_OK) return st;
     if (batch <= 0 || total_k <= 0 || cu_seqlens_k == nullptr) return QSA_ERR_INVALID_ARG;
@@ -323,6 +447,7 @@ qsa_status qsa_sparse_attn_decode_paged(const qsa_config *cfg, const qsa_bf16 *q
                                         const int32_t *cu_seqlens_k, int32_t batch, const int32_t *sel,
                                         qsa_bf16 *o, float *lse, void *ws, size_t ws_bytes, void *stream)
 {
+    const qsa::NvtxRange nvtx_range("qsa_sparse_attn_decode_paged");
     qsa_status st = check_config(cfg);
     if (st != QSA_OK) return st;
     if (batch <= 0 || num_pages <= 0 || page_size <= 0 || max_pages <= 0 || cu_seqlens_k == nullptr ||
@@ -345,11 +470,66 @@ qsa_status qsa_sparse_attn_decode_paged(const qsa_config *cfg, const qsa_bf16 *q
     return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
 }
 
+qsa_status qsa_index_select_mtp(const qsa_config *cfg, const qsa_bf16 *q_idx, const float *w, const qsa_bf16 *kc,
+                                int64_t kc_rows, const int32_t *cu_seqlens_k, const int32_t *cu_blocks,
+                                int32_t batch, int32_t next_n, int64_t max_len_k, int32_t *sel, void *ws,
+                                size_t ws_bytes, void *stream)
+{
+    const qsa::NvtxRange nvtx_range("qsa_index_select_mtp");
+    qsa_status st = check_config(cfg);
+    if (st != QSA_OK) return st;
+    if (batch <= 0 || kc_rows < 0 || max_len_k <= 0 || next_n < 1 || next_n > 4 || cu_seqlens_k == nullptr ||
+        cu_blocks == nullptr)
+        return QSA_ERR_INVALID_ARG;
+    if (cfg->budget_blocks < 2) return QSA_ERR_UNSUPPORTED;  // two own blocks may be forced
+    if (q_idx == nullptr || w == nullptr || sel == nullptr || (kc_rows > 0 && kc == nullptr) || !al16(q_idx) ||
+        (kc != nullptr && !al16(kc)))
+        return QSA_ERR_INVALID_ARG;
+    if (ws == nullptr || !al16(ws) ||
+        ws_bytes < qsa_workspace_size(cfg, QSA_OP_INDEX_SELECT, batch, batch, max_len_k))
+        return QSA_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t ld = ((max_len_k - 1) / cfg->r + 3) / 4 * 4 + 4;
+    // the one query row of each sequence whose scores serve the step: its last (t = L - 1)
+    const int32_t *cu_q = nullptr;
+    IndexArgs a{bf(q_idx), w, bf(kc), kc_rows, cu_q, cu_seqlens_k, cu_blocks, batch, batch, 0, batch,
+                static_cast<float *>(ws), ld, cfg->r};
+    if (kc_rows == 0) {
+        SelectArgs sa{static_cast<const float *>(ws), ld, nullptr, cu_seqlens_k, batch, 0, batch, sel,
+                      cfg->budget_blocks, cfg->r};
+        sa.next_n = next_n;
+        return cuda_status(launch_select(sa, s));
+    }
+    const bool refine = (cfg->flags & QSA_COMPRESS_NO_NORM) == 0;
+    return cuda_status(launch_decode_index_select(a, cfg->budget_blocks, ws, num_sms(), refine, sel, s, next_n));
+}
+
+qsa_status qsa_sparse_attn_decode_mtp(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k_cache,
+                                      const qsa_bf16 *v_cache, const int32_t *cu_seqlens_k, int32_t batch,
+                                      int64_t total_k, int32_t next_n, const int32_t *sel, qsa_bf16 *o, float *lse,
+                                      void *ws, size_t ws_bytes, void *stream)
+{
+    const qsa::NvtxRange nvtx_range("qsa_sparse_attn_decode_mtp");
+    qsa_status st = check_config(cfg);
+    if (st != QSA_OK) return st;
+    if (batch <= 0 || total_k <= 0 || next_n < 1 || next_n > 4 || cu_seqlens_k == nullptr) return QSA_ERR_INVALID_ARG;
+    if (q == nullptr || k_cache == nullptr || v_cache == nullptr || sel == nullptr || o == nullptr || !al16(q) ||
+        !al16(k_cache) || !al16(v_cache) || !al16(o))
+        return QSA_ERR_INVALID_ARG;
+    const size_t need = mtp_workspace_bytes(batch, cfg->budget_blocks);
+    if (need > 0 && (ws == nullptr || ws_bytes < need)) return QSA_ERR_WORKSPACE_TOO_SMALL;
+    if (need > 0 && !al16(ws)) return QSA_ERR_INVALID_ARG;
+    AttnArgs a{bf(q), bf(k_cache), bf(v_cache), sel, nullptr, cu_seqlens_k, batch, batch, total_k, 0, batch,
+               bf(o), lse, static_cast<float *>(ws), 1, cfg->budget_blocks, cfg->r, cfg->softmax_scale};
+    return cuda_status(launch_sparse_mtp(a, next_n, static_cast<cudaStream_t>(stream)));
+}
+
 qsa_status qsa_dense_attn_prefill(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k, const qsa_bf16 *v,
                                   const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int32_t batch,
                                   int64_t total_q, int64_t total_k, int32_t max_len_q, int64_t max_len_k,
                                   qsa_bf16 *o, float *lse, void *ws, size_t ws_bytes, void *stream)
 {
+    const qsa::NvtxRange nvtx_range("qsa_dense_attn_prefill");
     qsa_status st = check_config(cfg);
     if (st != QSA_OK) return st;
     if (batch <= 0 || total_q < 0 || total_k < 0 || max_len_q < 0 || max_len_k < 0 || cu_seqlens_q == nullptr ||
@@ -423,6 +603,7 @@ qsa_status qsa_sparse_attn_decode_static_scratch(const qsa_config *cfg, const qs
                                                  int64_t total_k, const int32_t *sel, qsa_bf16 *o, float *lse,
                                                  void *stream)
 {
+    const qsa::NvtxRange nvtx_range("qsa_sparse_attn_decode_static_scratch");
     qsa_status st = check_config(cfg);
     if (st != QSA_OK) return st;
     if (batch <= 0 || total_k <= 0 || cu_seqlens_k == nullptr) return QSA_ERR_INVALID_ARG;

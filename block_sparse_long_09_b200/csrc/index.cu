@@ -7,29 +7,28 @@
 // cost is O(n^2 / r) (the section's complexity equation).
 //
 // Prefill path (index_tc_kernel): a causal GEMM on the 5th-generation tensor
-// cores.  A CTA owns 64 consecutive query rows = 2 x 128 A-rows (token-major,
-// head-minor, exactly the q_idx memory order), loaded once by TMA.  It walks
-// the kc blocks below its causal bound in N-tiles of 128 blocks; kc holds a
-// compensated bf16 pair (hi, lo) per value, and both planes are multiplied
-// into the same fp32 accumulator:
-//   warp 0      TMA producer (kc hi+lo tiles, 2-stage ring, 128-byte swizzle)
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer: two M128 N128
-//               accumulators (one per 32-row sub-tile) share each kc tile, so the
-//               L2 traffic of kc is halved against 32-row tiles
-//   warps 2..9  epilogue: tcgen05.ld of the fp32 accumulators (double-buffered in
-//               TMEM -- all 512 columns -- so the next tile's MMAs overlap), ReLU
-//               * w, a 4-lane butterfly that sums the heads while scattering
-//               columns, 128-byte-swizzled staging in shared memory and 32 x 32
-//               TMA bulk stores of the scores (scattered per-thread stores would
-//               saturate the L1 store path).  Tiles that straddle two sequences
-//               fall back to masked per-thread stores.
+// cores, "swap AB": the compressed keys are the MMA's M side and the CTA's 64
+// query rows x 4 heads (256 rows, the q_idx memory order) its N side, so one
+// M128 N256 accumulator holds, in TMEM lane b, all 4 heads of all 64 rows
+// against kc block b.  The head sum is then local to a thread and the scores
+// of a row leave as coalesced 128-byte runs of consecutive blocks.
+//   warp 0       TMA producer: the q tile once (64 rows x 4 heads x 128), then
+//                kc tiles of 128 blocks (hi and lo planes) through a 2-stage ring
+//                (128-byte swizzle)
+//   warp 1       TMEM allocator + single-thread tcgen05.mma issue (kind::f16, bf16
+//                operands, fp32 accumulation): kc is a compensated bf16 pair, so
+//                every k-step multiplies q by the hi plane and then by the lo plane
+//                into the same accumulator; two 256-column accumulators in TMEM so
+//                the next tile's MMAs overlap the epilogue
+//   warps 2..17  the epilogue: tcgen05.ld of the thread's 16 rows x 4 heads,
+//                ReLU * w, the head sum, and what the mode asks for (below)
 // Tiles above the diagonal are never issued; heavy (late) row tiles launch first.
 //
 // Decode path (index_rowwise_kernel): one query row per sequence is a GEMV over
 // the kc cache -- HBM-bound, so it runs on CUDA cores: each warp streams 8 kc
 // rows with coalesced 8-byte loads, keeps its 4 heads' query slice in
-// registers, adds the hi and lo planes of kc in fp32, and reduces the 32
-// (block, head) partial dots with a 5-step butterfly reduce-scatter.
+// registers, and reduces the 32 (block, head) partial dots with a 5-step
+// butterfly reduce-scatter.
 #include "kernels.cuh"
 
 namespace qsa {
@@ -38,46 +37,51 @@ namespace {
 
 // ------------------------------------------------------------------ tcgen05 path
 constexpr int kTokTile = 64;                  // query rows per CTA
-constexpr int kSubTok = 32;                   // query rows per A sub-tile
-constexpr int kBM = kSubTok * 4;              // A rows of a sub-tile (token x head) = MMA M
-constexpr int kBN = 128;                      // kc blocks per N tile
+constexpr int kQRowsT = kTokTile * 4;         // N: rows x heads = 256
+constexpr int kBM = 128;                      // M: kc blocks per tile
 constexpr int kIdxDim = 128;
 constexpr int kStages = 2;
-constexpr int kChunkA = kBM * 128;            // 16 KB: one 64-column swizzled chunk of a sub-tile
-constexpr int kChunkB = kBN * 128;            // 16 KB
-constexpr int kABytes = 2 * 2 * kChunkA;      // 64 KB: two sub-tiles
-constexpr int kBBytes = 4 * kChunkB;          // 64 KB per stage: hi and lo planes
-constexpr int kStgChunk = kSubTok * 128;      // 4 KB: 32 rows x 32 fp32 scores, swizzled
-constexpr int kStgBytes = 2 * 4 * kStgChunk;  // 32 KB: 2 sub-tiles x 4 column groups
-constexpr int kIdxThreads = 320;              // producer, MMA, 8 epilogue warps
-constexpr uint32_t kAccCols = 512;            // 2 buffers x 2 sub-tiles x 128 columns
+constexpr int kChunkQ = kQRowsT * 128;        // 32 KB: one 64-dim swizzled chunk of the q tile
+constexpr int kQBytes = 2 * kChunkQ;          // 64 KB
+constexpr int kChunkKc = kBM * 128;           // 16 KB: one 64-dim chunk of one plane
+constexpr int kKcBytes = 4 * kChunkKc;        // 64 KB per stage: hi and lo planes
+constexpr int kEpiWarps = 16;                 // 4 per TMEM lane quadrant
+constexpr int kIdxThreads = 64 + kEpiWarps * 32;
+constexpr uint32_t kAccCols = 512;            // 2 buffers x 256 columns
 
 struct IdxShared {
     uint64_t full[kStages];
     uint64_t empty[kStages];
-    uint64_t a_full;
+    uint64_t q_full;      // the q tile landed
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint32_t tmem_base;
     int abort_flag;
+    alignas(16) float wq[kQRowsT];  // w[row, head]; read as float4
+    float theta[kTokTile];  // emit mode: the rows' thresholds
+    int seg_len[kEpiWarps][16];  // emit mode: each epilogue warp's list-segment lengths
 };
 
-constexpr int kIdxSmem = kABytes + kStages * kBBytes + kStgBytes + (int)sizeof(IdxShared) + 1024;
+static_assert(offsetof(IdxShared, wq) % 16 == 0, "the weight table is read as float4");
+constexpr int kIdxSmem = kQBytes + kStages * kKcBytes + (int)sizeof(IdxShared) + 1024;
+static_assert(kIdxSmem <= 232448, "shared memory of one CTA");
 
 struct Segment {
     int s;
     int64_t seg_begin, seg_end;  // packed rows of this tile that belong to sequence s
     int64_t pos_offset;          // t = pos_offset + (i - cu_q[s])
+    int64_t q0;                  // cu_q[s]
     int64_t kc_base;
     int n_tiles;
 };
 
-// Iterates the (sequence, N-tile) work of a row tile identically in every role.
+// Iterates the (sequence, kc-tile) work of a row tile identically in every role.
 struct SegIter {
     const int32_t *cu_q, *cu_k, *cu_blocks;
     int batch, r;
     int64_t m0, m1;
     int s;
+    int64_t min_bt;  // segments whose last row has b_t <= min_bt are skipped (sample mode)
     __device__ bool next(Segment &seg)
     {
         while (s < batch && (int64_t)cu_q[s] < m1) {
@@ -91,41 +95,45 @@ struct SegIter {
             seg.seg_begin = b;
             seg.seg_end = e;
             seg.pos_offset = Lk - Lq;
+            seg.q0 = q0;
             seg.kc_base = cu_blocks[cs];
             const int64_t t_last = (Lk - Lq) + (e - 1 - q0);
             const int64_t bt_max = t_last >= 0 ? t_last / r : 0;
-            seg.n_tiles = (int)((bt_max + kBN - 1) / kBN);
-            if (seg.n_tiles == 0) continue;
+            seg.n_tiles = (int)((bt_max + kBM - 1) / kBM);
+            if (seg.n_tiles == 0 || bt_max <= min_bt) continue;
             return true;
         }
         return false;
     }
 };
 
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int32_t x, int32_t y)
-{
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
-                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(x), "r"(y)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void sub_bar(int sub) { asm volatile("bar.sync %0, 128;" ::"r"(2 + sub) : "memory"); }
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); }
 
+// What the epilogue does with the scores (IdxMode):
+//   kScores  S[t, b] into the score rows (b < b_t)
+//   kSample  only every stride-th kc tile is computed; its scores go to a compact
+//            sample row (tile n lands at (n / stride) * 128), rows whose b_t is at
+//            most min_bt are skipped
+//   kEmit    every tile; (S, b) is appended to the row's candidate list when
+//            S >= theta of the row (a lower bound on the row's (k-1)-th best score)
+enum IdxMode { kScores = 0, kSample = 1, kEmit = 2 };
+
+template <int kMode>
 __global__ void __launch_bounds__(kIdxThreads, 1)
 index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kc,
-                const __grid_constant__ CUtensorMap map_s, int use_tma_store,
                 const float *__restrict__ w, const int32_t *__restrict__ cu_q,
                 const int32_t *__restrict__ cu_k, const int32_t *__restrict__ cu_blocks, int batch,
-                int64_t row_begin, int64_t row_end, float *__restrict__ scores, int64_t ld, int r)
+                int64_t row_begin, int64_t row_end, const __grid_constant__ IdxOut out, int r)
 {
+    const int step = kMode == kSample ? out.stride : 1;           // kc tiles advanced per iteration
+    const int64_t min_bt = kMode == kSample ? out.min_bt : -1;
+    float *const scores = kMode == kScores ? out.scores : out.sample;
+    const int64_t ld = kMode == kScores ? out.ld : out.sample_ld;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = smem;
-    uint8_t *sB = smem + kABytes;
-    uint8_t *sStg = sB + kStages * kBBytes;
-    IdxShared *sh = reinterpret_cast<IdxShared *>(sStg + kStgBytes);
+    uint8_t *sQ = smem;
+    uint8_t *sK = smem + kQBytes;
+    IdxShared *sh = reinterpret_cast<IdxShared *>(sK + kStages * kKcBytes);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t ntile_rows = (row_end - row_begin + kTokTile - 1) / kTokTile;
@@ -138,10 +146,10 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             mbar_init(&sh->full[i], 1);
             mbar_init(&sh->empty[i], 1);
         }
-        mbar_init(&sh->a_full, 1);
+        mbar_init(&sh->q_full, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sh->acc_full[i], 1);
-            mbar_init(&sh->acc_empty[i], 8);
+            mbar_init(&sh->acc_empty[i], kEpiWarps);
         }
         sh->abort_flag = 0;
         fence_barrier_init();
@@ -155,35 +163,31 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     tc_fence_after();
     const uint32_t tmem = sh->tmem_base;
     volatile int *abort_flag = &sh->abort_flag;
-
     const int s0 = find_seq(cu_q, batch, m0);
-    // one sequence covers the whole tile: whole 32 x 32 score boxes can be stored by TMA
-    const bool single = use_tma_store && (int64_t)cu_q[s0 + 1] >= m1;
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (elect_one()) {
             tma_prefetch_desc(&map_q);
             tma_prefetch_desc(&map_kc);
-            mbar_arrive_expect_tx(&sh->a_full, kABytes);
-            for (int sub = 0; sub < 2; ++sub)
-                for (int c = 0; c < 2; ++c)
-                    tma_load_2d(sA + (sub * 2 + c) * kChunkA, &map_q, &sh->a_full, c * 64,
-                                (int32_t)((m0 + sub * kSubTok) * 4));
-            SegIter it{cu_q, cu_k, cu_blocks, batch, r, m0, m1, s0};
+            mbar_arrive_expect_tx(&sh->q_full, kQBytes);
+            for (int c = 0; c < 2; ++c) tma_load_2d(sQ + c * kChunkQ, &map_q, &sh->q_full, c * 64, (int32_t)(m0 * 4));
+            SegIter it{cu_q, cu_k, cu_blocks, batch, r, m0, m1, s0, min_bt};
             Segment seg;
             uint32_t k = 0;
             bool ok = true;
             while (ok && it.next(seg)) {
-                for (int n = 0; n < seg.n_tiles; ++n, ++k) {
+                for (int n = 0; n < seg.n_tiles; n += step, ++k) {
                     const uint32_t st = k % kStages, round = k / kStages;
                     if (!mbar_wait(&sh->empty[st], (round & 1) ^ 1, abort_flag)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&sh->full[st], kBBytes);
-                    const int32_t y = (int32_t)(seg.kc_base + (int64_t)n * kBN);
-                    for (int c = 0; c < 4; ++c)
-                        tma_load_2d(sB + st * kBBytes + c * kChunkB, &map_kc, &sh->full[st], c * 64, y);
+                    mbar_arrive_expect_tx(&sh->full[st], kKcBytes);
+                    const int32_t y = (int32_t)(seg.kc_base + (int64_t)n * kBM);
+                    for (int c = 0; c < 4; ++c)  // hi dims 0..63, 64..127, then lo
+                        tma_load_2d(sK + st * kKcBytes + c * kChunkKc, &map_kc, &sh->full[st], c * 64, y);
                 }
             }
+            // drain: every copy issued must land before the CTA exits
+            mbar_wait(&sh->q_full, 0, nullptr);
             if (!ok) {
                 for (uint32_t j = (k > kStages ? k - kStages : 0); j < k; ++j)
                     mbar_wait(&sh->full[j % kStages], (j / kStages) & 1, nullptr);
@@ -192,30 +196,27 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (elect_one()) {
-            constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, 0, 0);
-            const uint32_t a_addr = smem_u32(sA), b_addr = smem_u32(sB);
-            bool ok = mbar_wait(&sh->a_full, 0, abort_flag);
-            SegIter it{cu_q, cu_k, cu_blocks, batch, r, m0, m1, s0};
+            constexpr uint32_t idesc = idesc_bf16_f32(kBM, kQRowsT, 0, 0);
+            const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK);
+            bool ok = mbar_wait(&sh->q_full, 0, abort_flag);
+            SegIter it{cu_q, cu_k, cu_blocks, batch, r, m0, m1, s0, min_bt};
             Segment seg;
             uint32_t k = 0;
             while (ok && it.next(seg)) {
-                for (int n = 0; n < seg.n_tiles; ++n, ++k) {
+                for (int n = 0; n < seg.n_tiles; n += step, ++k) {
                     const uint32_t st = k % kStages, round = k / kStages;
                     const uint32_t acc = k & 1, use = k >> 1;
                     if (!mbar_wait(&sh->acc_empty[acc], (use & 1) ^ 1, abort_flag)) { ok = false; break; }
                     if (!mbar_wait(&sh->full[st], round & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
+                    const uint32_t d = tmem + acc * kQRowsT;
 #pragma unroll
-                    for (int sub = 0; sub < 2; ++sub) {
-                        const uint32_t d = tmem + (acc * 2 + sub) * kBN;
-#pragma unroll
-                        for (int ks = 0; ks < 2 * kIdxDim / 16; ++ks) {  // hi plane, then lo plane
-                            const int ka = ks & 7;                    // k-step within the 128 dims
-                            const uint32_t koff = (ka & 3) * 32;
-                            const uint64_t ad = sdesc_sw128(a_addr + (sub * 2 + (ka >> 2)) * kChunkA + koff, 16, 1024);
-                            const uint64_t bd = sdesc_sw128(b_addr + st * kBBytes + (ks >> 2) * kChunkB + koff, 16, 1024);
-                            mma_bf16_ss(d, ad, bd, idesc, ks > 0 ? 1u : 0u);
-                        }
+                    for (int ks = 0; ks < 2 * kIdxDim / 16; ++ks) {  // hi plane, then lo plane
+                        const int kk = ks & 7;                       // k-step within the 128 dims
+                        const uint32_t koff = (kk & 3) * 32;
+                        const uint64_t ad = sdesc_sw128(k_addr + st * kKcBytes + (ks >> 2) * kChunkKc + koff, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(q_addr + (kk >> 2) * kChunkQ + koff, 16, 1024);
+                        mma_bf16_ss(d, ad, bd, idesc, ks > 0 ? 1u : 0u);
                     }
                     mma_commit(&sh->empty[st]);
                     mma_commit(&sh->acc_full[acc]);
@@ -223,100 +224,102 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             }
         }
     } else {
-        // ---------------- epilogue (warps 2..9) ----------------
-        const int ew = warp - 2;
-        const int sub = ew >> 2;                   // A sub-tile
-        const int quad = warp & 3;                 // TMEM lane quadrant this warp may read
-        const int row_in_sub = quad * 8 + (lane >> 2);
-        const int head = lane & 3;
-        const int64_t i = m0 + sub * kSubTok + row_in_sub;  // packed query row of this lane
-        const float wv = (i < m1) ? __ldg(w + i * 4 + head) : 0.f;
-        const bool b0 = lane & 1, b1 = (lane >> 1) & 1;
-        const int col_sub = (b0 ? 16 : 0) + (b1 ? 8 : 0);
-        const bool vec_ok = (ld & 3) == 0;
-        const bool store_thread = (ew & 3) == 0 && lane == 0;  // issues this sub-tile's TMA stores
-        uint8_t *stg = sStg + sub * 4 * kStgChunk;
-        const uint32_t stg_row = (uint32_t)row_in_sub * 128;
-        const int unit0 = col_sub >> 2;            // first 16-byte unit of the 8 values
+        // ---------------- the epilogue (warps 2..17) ----------------
+        const int et = threadIdx.x - 64;            // 0 .. 511
+        if (et < kQRowsT) {  // the tile's weights, (row, head) in q_idx order
+            const int64_t i = m0 + (et >> 2);
+            sh->wq[et] = i < m1 ? __ldg(w + i * 4 + (et & 3)) : 0.f;
+        }
+        if (kMode == kEmit && et < kTokTile) {
+            const int64_t i = m0 + et;
+            sh->theta[et] = i < m1 ? __ldg(out.theta + (i - row_begin)) : INFINITY;
+        }
+        epi_bar();  // the weight table is complete
+        // emit mode: list segment (row, quad) belongs to exactly one warp, which keeps its
+        // 16 rows' lengths in its own shared-memory slots (read by every lane, advanced
+        // by lane 0, ordered by the warp barrier at the end of each tile): no atomics
+        int *seg_len = sh->seg_len[warp - 2];
+        if (kMode == kEmit && lane < 16) seg_len[lane] = 0;
+        __syncwarp();
+        const int cap_q = out.list_cap / 4;
 
-        SegIter it{cu_q, cu_k, cu_blocks, batch, r, m0, m1, s0};
+        const int ew = warp - 2;
+        const int quad = warp & 3;                 // TMEM lane quadrant this warp may read
+        const int part = ew >> 2;                  // rows [16 part, 16 part + 16) of the tile
+        const int b_local = quad * 32 + lane;      // kc block within the tile (TMEM lane)
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        const float4 *wq4 = reinterpret_cast<const float4 *>(sh->wq);
+
+        SegIter it{cu_q, cu_k, cu_blocks, batch, r, m0, m1, s0, min_bt};
         Segment seg;
         uint32_t k = 0;
         bool ok = true;
+        const uint32_t lt_mask = (1u << lane) - 1u;
         while (ok && it.next(seg)) {
-            const bool row_in_seg = (i >= seg.seg_begin && i < seg.seg_end);
-            const int64_t t = seg.pos_offset + (i - cu_q[seg.s]);
-            int64_t bt = row_in_seg ? t / r : 0;
-            if (bt > ld) {
-                if (lane == 0) set_device_status(QSA_ERR_DEVICE_CHECK);
-                bt = ld;
-            }
-            float *srow = scores + (i - row_begin) * ld;
-            for (int n = 0; n < seg.n_tiles; ++n, ++k) {
+            // this thread's rows j (bit j of vmask) belong to the segment; row j sits at
+            // t = t0 + j, b_t = t >> rs (r a power of two); blocks b < b_t are scored
+            const int64_t i0 = m0 + part * 16;
+            const int j_lo = (int)(seg.seg_begin > i0 ? (seg.seg_begin - i0 < 16 ? seg.seg_begin - i0 : 16) : 0);
+            const int j_hi = (int)(seg.seg_end > i0 ? (seg.seg_end - i0 < 16 ? seg.seg_end - i0 : 16) : 0);
+            const uint32_t vmask = j_hi > j_lo ? (((1u << j_hi) - 1u) & ~((1u << j_lo) - 1u)) : 0u;
+            const int32_t t0 = (int32_t)(seg.pos_offset + (i0 - seg.q0));
+            const int rs = 31 - __clz(r);
+            if (kMode == kScores && j_hi > j_lo && ((t0 + j_hi - 1) >> rs) > ld) set_device_status(QSA_ERR_DEVICE_CHECK);
+            const int32_t cap = ld < 0x7FFFFFFF ? (int32_t)ld : 0x7FFFFFFF;  // score / sample columns
+            float *row0 = kMode == kEmit ? nullptr : scores + (i0 - row_begin) * ld;
+            // emit mode: segment (row i0 + j, quad) starts at lbase + j * 4 cap_q
+            uint2 *const lbase = kMode == kEmit ? out.lists + ((i0 - row_begin) * 4 + quad) * cap_q : nullptr;
+            for (int n = 0; n < seg.n_tiles; n += step, ++k) {
                 const uint32_t acc = k & 1, use = k >> 1;
                 if (!mbar_wait(&sh->acc_full[acc], use & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                if (single) {
-                    if (store_thread) bulk_wait_read0();  // staging free again
-                    sub_bar(sub);
-                }
-#pragma unroll 1
-                for (int c = 0; c < kBN / 32; ++c) {
-                    float v[32];
-                    tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (acc * 2 + sub) * kBN + c * 32, v);
+                const int32_t b = n * kBM + b_local;
+                const int32_t col = kMode == kSample ? (n / step) * kBM + b_local : b;  // where the score goes
+                const bool col_ok = kMode == kEmit || col < cap;
+                float *p = row0 + col;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float v[16];  // rows 16 part + 4 c .. + 3, heads 0..3
+                    tmem_ld16(tmem + lane_addr + acc * kQRowsT + part * 64 + c * 16, v);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = wv * fmaxf(v[j], 0.f);
-                    // butterfly over the 4 head lanes: sum heads, scatter columns
-                    float h16[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float send = b0 ? v[j] : v[j + 16];
-                        const float keep = b0 ? v[j + 16] : v[j];
-                        h16[j] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-                    }
-                    float h8[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float send = b1 ? h16[j] : h16[j + 8];
-                        const float keep = b1 ? h16[j + 8] : h16[j];
-                        h8[j] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-                    }
-                    if (single) {
-                        // 128-byte swizzled staging row: 16-byte unit u lands at u ^ (row & 7)
-                        uint8_t *base = stg + c * kStgChunk + stg_row;
-                        const int sw = row_in_sub & 7;
-                        *reinterpret_cast<float4 *>(base + (((unit0) ^ sw) << 4)) = make_float4(h8[0], h8[1], h8[2], h8[3]);
-                        *reinterpret_cast<float4 *>(base + (((unit0 + 1) ^ sw) << 4)) = make_float4(h8[4], h8[5], h8[6], h8[7]);
-                    } else if (row_in_seg) {
-                        const int64_t bcol = (int64_t)n * kBN + c * 32 + col_sub;
-                        if (vec_ok && bcol + 8 <= bt) {
-                            float4 *dst = reinterpret_cast<float4 *>(srow + bcol);
-                            dst[0] = make_float4(h8[0], h8[1], h8[2], h8[3]);
-                            dst[1] = make_float4(h8[4], h8[5], h8[6], h8[7]);
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int j = c * 4 + jj;
+                        const float4 wv = wq4[part * 16 + j];
+                        float s = wv.x * fmaxf(v[4 * jj], 0.f);
+                        s = fmaf(wv.y, fmaxf(v[4 * jj + 1], 0.f), s);
+                        s = fmaf(wv.z, fmaxf(v[4 * jj + 2], 0.f), s);
+                        s = fmaf(wv.w, fmaxf(v[4 * jj + 3], 0.f), s);
+                        const bool in = ((vmask >> j) & 1u) && b < ((t0 + j) >> rs) && col_ok;
+                        if (kMode != kEmit) {
+                            if (in) __stcs(p, s);
+                            p += ld;
                         } else {
-#pragma unroll
-                            for (int j = 0; j < 8; ++j)
-                                if (bcol + j < bt) srow[bcol + j] = h8[j];
+                            // append (S, b) to this warp's segment of row j's list when S >= theta:
+                            // the warp's hits take consecutive slots in ballot order
+                            const bool hit = in && s >= sh->theta[part * 16 + j];
+                            const uint32_t m = __ballot_sync(0xffffffffu, hit);
+                            if (m != 0u) {  // warp-uniform; most (row, tile) pairs have no hit
+                                const int len = seg_len[j];
+                                const int pos = len + __popc(m & lt_mask);
+                                if (hit && pos < cap_q)
+                                    lbase[j * 4 * cap_q + pos] = make_uint2(__float_as_uint(s), (uint32_t)b);
+                                if (lane == 0) seg_len[j] = len + __popc(m);  // read again only after
+                            }                                                  // the tile's warp barrier
                         }
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh->acc_empty[acc]);
-                if (single) {
-                    fence_proxy_async_smem();
-                    sub_bar(sub);
-                    if (store_thread) {
-                        const int32_t y = (int32_t)(m0 + sub * kSubTok - row_begin);
-                        for (int c = 0; c < 4; ++c)
-                            tma_store_2d(&map_s, stg + c * kStgChunk, n * kBN + c * 32, y);
-                        bulk_commit();
-                    }
-                }
             }
         }
-        if (store_thread) bulk_wait0();
+        if (kMode == kEmit) {  // the lengths of this warp's 16 list segments (lane j: row j)
+            __syncwarp();
+            const int mine = lane < 16 ? seg_len[lane] : 0;
+            const int64_t i = m0 + part * 16 + lane;
+            if (lane < 16 && i < m1) out.counts[(i - row_begin) * 4 + quad] = mine;
+        }
     }
 
     tc_fence_before();
@@ -331,6 +334,9 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
 constexpr int kRowWarps = 8;
 constexpr int kRowChunk = 1024;  // kc blocks per CTA
 
+// kPlanes = 2: the exact scores (hi + lo planes); 1: the hi plane only (the decode
+// selector then refines the near-threshold blocks exactly)
+template <int kPlanes>
 __global__ void __launch_bounds__(kRowWarps * 32)
 index_rowwise_kernel(const __nv_bfloat16 *__restrict__ q_idx, const float *__restrict__ w,
                      const __nv_bfloat16 *__restrict__ kc, const int32_t *__restrict__ cu_q,
@@ -339,10 +345,11 @@ index_rowwise_kernel(const __nv_bfloat16 *__restrict__ q_idx, const float *__res
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t i = row_begin + blockIdx.y;
-    const int s = find_seq(cu_q, batch, i);
-    const int64_t Lq = (int64_t)cu_q[s + 1] - cu_q[s];
+    // cu_q == nullptr: decode rows, row i is sequence i at t = L - 1
+    const int s = cu_q != nullptr ? find_seq(cu_q, batch, i) : (int)i;
     const int64_t Lk = (int64_t)cu_k[s + 1] - cu_k[s];
-    const int64_t t = (Lk - Lq) + (i - cu_q[s]);
+    const int64_t Lq = cu_q != nullptr ? (int64_t)cu_q[s + 1] - cu_q[s] : 1;
+    const int64_t t = cu_q != nullptr ? (Lk - Lq) + (i - cu_q[s]) : Lk - 1;
     int64_t bt = t >= 0 ? t / r : 0;
     if (bt > ld || (int64_t)cu_blocks[s + 1] - cu_blocks[s] != Lk / r) {
         if (threadIdx.x == 0) set_device_status(QSA_ERR_DEVICE_CHECK);
@@ -353,84 +360,199 @@ index_rowwise_kernel(const __nv_bfloat16 *__restrict__ q_idx, const float *__res
     const int64_t c1 = (c0 + kRowChunk < bt) ? c0 + kRowChunk : bt;
     if (c0 >= c1) return;
 
-    // this lane's slice of the 4 query heads: dims 4 lane .. 4 lane + 3
-    float q[4][4];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-        uint2 raw = *reinterpret_cast<const uint2 *>(q_idx + (i * 4 + h) * 128 + lane * 4);
-        float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw.x));
-        float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw.y));
-        q[h][0] = a.x; q[h][1] = a.y; q[h][2] = b.x; q[h][3] = b.y;
-    }
-    const float wv = __ldg(w + i * 4 + (lane & 3));
-    const __nv_bfloat16 *kbase = kc + (int64_t)cu_blocks[s] * 256 + lane * 4;
-    float *srow = scores + (int64_t)blockIdx.y * ld;
+    index_row_cuda<kPlanes>(q_idx + i * 512, w + i * 4, kc + (int64_t)cu_blocks[s] * 256, c0, c1,
+                   scores + (int64_t)blockIdx.y * ld, warp, kRowWarps, lane);
+}
 
-    for (int64_t b0 = c0 + warp * 8; b0 < c1; b0 += kRowWarps * 8) {
-        uint2 raw[8], rlo[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int64_t b = b0 + j;
-            const bool in = b < c1;
-            raw[j] = in ? __ldg(reinterpret_cast<const uint2 *>(kbase + b * 256)) : make_uint2(0u, 0u);
-            rlo[j] = in ? __ldg(reinterpret_cast<const uint2 *>(kbase + b * 256 + 128)) : make_uint2(0u, 0u);
+// ------------------------------------------------------------------ decode GEMV on the tensor cores
+// The decode scan of the hi planes as a stream of TMA tiles: per 128-block kc tile,
+// D[b, h] = <hi_b, q_h> with the kc tile as the M = 128 side and the row's 4 heads
+// (plus 12 zero rows) as the N = 16 side, 8 MMAs of K = 16; an epilogue thread per
+// block (TMEM lane) sums w_h ReLU(D[b, h]) and stores a coalesced score row.  The
+// tensor cores take the arithmetic off the CUDA cores, so the kernel streams the
+// hi planes at the HBM rate.
+constexpr int kGvBN = 16;                       // N: 4 heads + 12 zero rows
+constexpr int kGvChunkQ = kGvBN * 128;          // 2 KB: one 64-dim chunk of the q tile
+constexpr int kGvTile = 128 * 128 * 2;          // 32 KB: a 128-block tile of hi planes
+constexpr int kGvStages = 3;
+constexpr int kGvChunk = 1024;                  // kc blocks per CTA (8 tiles)
+constexpr int kGvThreads = 192;
+constexpr int kGvSmem = 2 * kGvChunkQ + kGvStages * kGvTile + 256 + 1024;
+
+__global__ void __launch_bounds__(kGvThreads, 2)
+index_gemv_hi_kernel(const __grid_constant__ CUtensorMap map_kc, const __nv_bfloat16 *__restrict__ q_idx,
+                     const float *__restrict__ w, const int32_t *__restrict__ cu_q,
+                     const int32_t *__restrict__ cu_k, const int32_t *__restrict__ cu_blocks, int batch,
+                     int64_t row_begin, float *__restrict__ scores, int64_t ld, int r)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sK = smem;                               // stages of kc tiles (1 KB aligned)
+    uint8_t *sQ = smem + kGvStages * kGvTile;         // the q tile
+    uint64_t *full = reinterpret_cast<uint64_t *>(sQ + 2 * kGvChunkQ);
+    uint64_t *empty = full + kGvStages;
+    uint64_t *acc_full = empty + kGvStages;           // [2]
+    uint64_t *acc_empty = acc_full + 2;               // [2]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    int *abort_slot = reinterpret_cast<int *>(tmem_slot + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const int64_t i = row_begin + blockIdx.y;
+    const int s = cu_q != nullptr ? find_seq(cu_q, batch, i) : (int)i;
+    const int64_t Lk = (int64_t)cu_k[s + 1] - cu_k[s];
+    const int64_t Lq = cu_q != nullptr ? (int64_t)cu_q[s + 1] - cu_q[s] : 1;
+    const int64_t t = cu_q != nullptr ? (Lk - Lq) + (i - cu_q[s]) : Lk - 1;
+    int64_t bt = t >= 0 ? t / r : 0;
+    if (bt > ld) {
+        if (threadIdx.x == 0) set_device_status(QSA_ERR_DEVICE_CHECK);
+        bt = ld;
+    }
+    const int64_t c0 = (int64_t)blockIdx.x * kGvChunk;
+    const int64_t c1 = (c0 + kGvChunk < bt) ? c0 + kGvChunk : bt;
+    if (c0 >= c1) return;  // uniform: the whole CTA leaves before any set-up
+    const int n_tiles = (int)((c1 - c0 + 127) / 128);
+    const int64_t kc0 = (int64_t)cu_blocks[s] + c0;
+
+    // the q tile: rows 0..3 the row's 4 heads, rows 4..15 zero (128-byte swizzle, K-major)
+    for (int x = threadIdx.x; x < 2 * kGvChunkQ / 16; x += kGvThreads) {
+        const int ch = x / (kGvChunkQ / 16), row = (x % (kGvChunkQ / 16)) / 8, u = x % 8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (row < 4) v = *reinterpret_cast<const uint4 *>(q_idx + (i * 4 + row) * 128 + ch * 64 + u * 8);
+        *reinterpret_cast<uint4 *>(sQ + ch * kGvChunkQ + row * 128 + ((u ^ (row & 7)) << 4)) = v;
+    }
+    fence_proxy_async_smem();
+    if (threadIdx.x == 0) {
+        for (int x = 0; x < kGvStages; ++x) {
+            mbar_init(&full[x], 1);
+            mbar_init(&empty[x], 1);
         }
-        float v[32];  // v[j * 4 + h] = partial dot of block b0 + j with head h
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw[j].x));
-            float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw[j].y));
-            const float2 al = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&rlo[j].x));
-            const float2 bl = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&rlo[j].y));
-            a.x += al.x; a.y += al.y; b.x += bl.x; b.y += bl.y;
-#pragma unroll
-            for (int h = 0; h < 4; ++h)
-                v[j * 4 + h] = q[h][0] * a.x + q[h][1] * a.y + q[h][2] * b.x + q[h][3] * b.y;
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&acc_full[x], 1);
+            mbar_init(&acc_empty[x], 4);
         }
-        // reduce-scatter over the 32 lanes: lane l ends with the full dot of index l
+        *abort_slot = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 32);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    volatile int *abort_flag = abort_slot;
+
+    if (warp == 0) {
+        if (elect_one()) {
+            tma_prefetch_desc(&map_kc);
+            int n = 0;
+#ifdef QSA_DEBUG_CHECKS
+            const bool skip_tile1 = g_debug_fault_site == 1;
+#endif
+            for (; n < n_tiles; ++n) {
+                const uint32_t st = n % kGvStages, round = n / kGvStages;
+                if (!mbar_wait(&empty[st], (round & 1) ^ 1, abort_flag)) break;
+#ifdef QSA_DEBUG_CHECKS
+                if (skip_tile1 && n == 1) continue;  // injected fault: tile 1's full barrier never completes
+#endif
+                mbar_arrive_expect_tx(&full[st], kGvTile);
+                for (int c = 0; c < 2; ++c)  // the hi plane: dims 0..63, 64..127
+                    tma_load_2d(sK + st * kGvTile + c * (kGvTile / 2), &map_kc, &full[st], c * 64,
+                                (int32_t)(kc0 + (int64_t)n * 128));
+            }
+            if (n < n_tiles)  // gave up: the copies in flight land before the CTA exits
+                for (int j = (n > kGvStages ? n - kGvStages : 0); j < n; ++j)
+                    mbar_wait(&full[j % kGvStages], (j / kGvStages) & 1, nullptr);
+        }
+    } else if (warp == 1) {
+        if (elect_one()) {
+            constexpr uint32_t idesc = idesc_bf16_f32(128, kGvBN, 0, 0);
+            const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK);
+            for (int n = 0; n < n_tiles; ++n) {
+                const uint32_t st = n % kGvStages, round = n / kGvStages;
+                const uint32_t acc = n & 1, use = n >> 1;
+                if (!mbar_wait(&acc_empty[acc], (use & 1) ^ 1, abort_flag)) break;
+                if (!mbar_wait(&full[st], round & 1, abort_flag)) break;
+                tc_fence_after();
 #pragma unroll
-        for (int step = 16; step >= 1; step >>= 1) {
-            const bool hi = lane & step;
-#pragma unroll
-            for (int j = 0; j < step; ++j) {
-                const float send = hi ? v[j] : v[j + step];
-                const float keep = hi ? v[j + step] : v[j];
-                v[j] = keep + __shfl_xor_sync(0xffffffffu, send, step);
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t koff = (ks & 3) * 32;
+                    const uint64_t ad = sdesc_sw128(k_addr + st * kGvTile + (ks >> 2) * (kGvTile / 2) + koff, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(q_addr + (ks >> 2) * kGvChunkQ + koff, 16, 1024);
+                    mma_bf16_ss(tmem + acc * kGvBN, ad, bd, idesc, ks > 0 ? 1u : 0u);
+                }
+                mma_commit(&empty[st]);
+                mma_commit(&acc_full[acc]);
             }
         }
-        float sc = wv * fmaxf(v[0], 0.f);  // lane l: block b0 + l/4, head l%4
-        sc += __shfl_xor_sync(0xffffffffu, sc, 1);
-        sc += __shfl_xor_sync(0xffffffffu, sc, 2);
-        const int64_t b = b0 + (lane >> 2);
-        if ((lane & 3) == 0 && b < c1) srow[b] = sc;
+    } else {
+        const int quad = warp & 3;
+        const int b_local = quad * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        const float4 wv = *reinterpret_cast<const float4 *>(w + i * 4);
+        float *srow = scores + (int64_t)blockIdx.y * ld;
+        for (int n = 0; n < n_tiles; ++n) {
+            const uint32_t acc = n & 1, use = n >> 1;
+            if (!mbar_wait(&acc_full[acc], use & 1, abort_flag)) break;
+            tc_fence_after();
+            float v[8];
+            tmem_ld8(tmem + lane_addr + acc * kGvBN, v);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            float sc = wv.x * fmaxf(v[0], 0.f);
+            sc = fmaf(wv.y, fmaxf(v[1], 0.f), sc);
+            sc = fmaf(wv.z, fmaxf(v[2], 0.f), sc);
+            sc = fmaf(wv.w, fmaxf(v[3], 0.f), sc);
+            const int64_t b = c0 + (int64_t)n * 128 + b_local;
+            if (b < c1) srow[b] = sc;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 32);
     }
 }
 
 }  // namespace
 
-cudaError_t launch_index_tc(const IndexArgs &a, cudaStream_t stream)
+cudaError_t launch_index_tc_mode(const IndexArgs &a, const IdxOut &out, cudaStream_t stream)
 {
     const int64_t rows = a.row_end - a.row_begin;
     if (rows <= 0 || a.kc_rows <= 0) return cudaSuccess;
-    CUtensorMap mq, mk, ms;
-    if (!make_tmap_2d(&mq, a.q_idx, 128, (uint64_t)a.total_q * 4, 256, 64, kBM)) return cudaErrorInvalidValue;
-    if (!make_tmap_2d(&mk, a.kc, 256, (uint64_t)a.kc_rows, 512, 64, kBN)) return cudaErrorInvalidValue;
-    // the scores of this call as an fp32 [rows, ld] tensor for 32 x 32 TMA stores (needs ld % 4 == 0)
-    int use_tma = ((a.ld & 3) == 0) && make_tmap_2d_f32(&ms, a.scores, (uint64_t)a.ld, (uint64_t)rows,
-                                                       (uint64_t)a.ld * 4, 32, 32);
-    if (!use_tma) ms = mq;  // unused
+    CUtensorMap mq, mk;
+    // q_idx as [total_q * 4, 128] bf16, 256-row boxes; kc as [kc_rows, 128] 16-bit, 128-row boxes
+    if (!make_tmap_2d(&mq, a.q_idx, 128, (uint64_t)a.total_q * 4, 256, 64, kQRowsT)) return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&mk, a.kc, 256, (uint64_t)a.kc_rows, 512, 64, kBM)) return cudaErrorInvalidValue;
+    if (out.mode == kSample && out.stride <= 0) return cudaErrorInvalidValue;
+    auto kern = out.mode == kSample ? index_tc_kernel<kSample>
+                                    : (out.mode == kEmit ? index_tc_kernel<kEmit> : index_tc_kernel<kScores>);
     {
-        const cudaError_t e = set_smem_attr_once(reinterpret_cast<const void *>(index_tc_kernel), kIdxSmem);
+        const cudaError_t e = set_smem_attr_once(reinterpret_cast<const void *>(kern), kIdxSmem);
         if (e != cudaSuccess) return e;
     }
     const int64_t tiles = (rows + kTokTile - 1) / kTokTile;
-    index_tc_kernel<<<(unsigned)tiles, kIdxThreads, kIdxSmem, stream>>>(
-        mq, mk, ms, use_tma, a.w, a.cu_q, a.cu_k, a.cu_blocks, a.batch, a.row_begin, a.row_end, a.scores, a.ld,
-        a.r);
+    kern<<<(unsigned)tiles, kIdxThreads, kIdxSmem, stream>>>(mq, mk, a.w, a.cu_q, a.cu_k, a.cu_blocks, a.batch,
+                                                             a.row_begin, a.row_end, out, a.r);
     return cudaGetLastError();
 }
 
-cudaError_t launch_index_rowwise(const IndexArgs &a, cudaStream_t stream)
+cudaError_t launch_index_tc(const IndexArgs &a, cudaStream_t stream)
+{
+    IdxOut out{};
+    out.mode = kScores;
+    out.scores = a.scores;
+    out.ld = a.ld;
+    return launch_index_tc_mode(a, out, stream);
+}
+
+template <int kPlanes>
+static cudaError_t launch_rowwise(const IndexArgs &a, cudaStream_t stream)
 {
     const int64_t rows = a.row_end - a.row_begin;
     if (rows <= 0 || a.kc_rows <= 0) return cudaSuccess;
@@ -438,9 +560,35 @@ cudaError_t launch_index_rowwise(const IndexArgs &a, cudaStream_t stream)
     for (int64_t done = 0; done < rows; done += 65535) {
         const int64_t n = rows - done < 65535 ? rows - done : 65535;
         dim3 grid((unsigned)chunks, (unsigned)n);
-        index_rowwise_kernel<<<grid, kRowWarps * 32, 0, stream>>>(
+        index_rowwise_kernel<kPlanes><<<grid, kRowWarps * 32, 0, stream>>>(
             a.q_idx, a.w, a.kc, a.cu_q, a.cu_k, a.cu_blocks, a.batch, a.row_begin + done,
             a.scores + done * a.ld, a.ld, a.r);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_index_rowwise(const IndexArgs &a, cudaStream_t stream) { return launch_rowwise<2>(a, stream); }
+
+cudaError_t launch_index_rowwise_hi(const IndexArgs &a, cudaStream_t stream)
+{
+    const int64_t rows = a.row_end - a.row_begin;
+    if (rows <= 0 || a.kc_rows <= 0) return cudaSuccess;
+    // w rows are read as float4: 16-byte aligned (the caller's fp32 [rows, 4] array)
+    // (and kc tile rows are int32 TMA coordinates)
+    if ((reinterpret_cast<uintptr_t>(a.w) & 15u) != 0 || a.kc_rows > (int64_t)INT32_MAX - 2 * kGvChunk)
+        return launch_rowwise<1>(a, stream);
+    CUtensorMap mk;
+    if (!make_tmap_2d(&mk, a.kc, 256, (uint64_t)a.kc_rows, 512, 64, 128)) return cudaErrorInvalidValue;
+    {
+        const cudaError_t e = set_smem_attr_once(reinterpret_cast<const void *>(index_gemv_hi_kernel), kGvSmem);
+        if (e != cudaSuccess) return e;
+    }
+    const int64_t chunks = (a.ld + kGvChunk - 1) / kGvChunk;
+    for (int64_t done = 0; done < rows; done += 65535) {
+        const int64_t n = rows - done < 65535 ? rows - done : 65535;
+        index_gemv_hi_kernel<<<dim3((unsigned)chunks, (unsigned)n), kGvThreads, kGvSmem, stream>>>(
+            mk, a.q_idx, a.w, a.cu_q, a.cu_k, a.cu_blocks, a.batch, a.row_begin + done, a.scores + done * a.ld, a.ld,
+            a.r);
     }
     return cudaGetLastError();
 }

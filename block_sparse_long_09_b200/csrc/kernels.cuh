@@ -17,6 +17,83 @@ __device__ __forceinline__ int find_seq(const int32_t *cu, int batch, int64_t x)
     return lo;
 }
 
+// Indexer scores of one query row against kc blocks [c0, c1) on CUDA cores (the
+// decode GEMV, and the fused selector's fallback and rescoring): warp `warp` of
+// `nwarps` streams 8 kc rows at a time with 8-byte loads, keeps its 4 heads' slice
+// of q in fp32 registers and reduces the 32 (block, head) partial dots with a
+// 5-step butterfly reduce-scatter; srow[b] = sum_h w[h] * ReLU(<q[h], kc[b]>).
+// kc_at(b) is the address of block b's compressed key (packed or through a page
+// table): its hi plane, and 128 values further its lo plane.  kPlanes = 2 adds the
+// planes in fp32 before the products (the exact scores); kPlanes = 1 reads the hi
+// plane only (half the bytes; each dot then moves by at most |q| |lo|).
+template <int kPlanes, typename KcAt>
+__device__ __forceinline__ void index_row_cuda_at(const __nv_bfloat16 *__restrict__ q_row,
+                                                  const float *__restrict__ w_row, KcAt kc_at, int64_t c0,
+                                                  int64_t c1, float *__restrict__ srow, int warp, int nwarps,
+                                                  int lane)
+{
+    float q[4][4];  // this lane's slice of the 4 query heads: dims 4 lane .. 4 lane + 3
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        uint2 raw = *reinterpret_cast<const uint2 *>(q_row + h * 128 + lane * 4);
+        float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw.x));
+        float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw.y));
+        q[h][0] = a.x; q[h][1] = a.y; q[h][2] = b.x; q[h][3] = b.y;
+    }
+    const float wv = __ldg(w_row + (lane & 3));
+    for (int64_t b0 = c0 + warp * 8; b0 < c1; b0 += (int64_t)nwarps * 8) {
+        uint2 raw[8], rlo[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int64_t b = b0 + j;
+            const __nv_bfloat16 *p = b < c1 ? kc_at(b) + lane * 4 : nullptr;
+            raw[j] = p != nullptr ? __ldg(reinterpret_cast<const uint2 *>(p)) : make_uint2(0u, 0u);
+            if (kPlanes == 2) rlo[j] = p != nullptr ? __ldg(reinterpret_cast<const uint2 *>(p + 128)) : make_uint2(0u, 0u);
+        }
+        float v[32];  // v[j * 4 + h] = partial dot of block b0 + j with head h
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw[j].x));
+            float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw[j].y));
+            if (kPlanes == 2) {
+                const float2 al = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&rlo[j].x));
+                const float2 bl = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&rlo[j].y));
+                a.x += al.x; a.y += al.y; b.x += bl.x; b.y += bl.y;
+            }
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+                v[j * 4 + h] = q[h][0] * a.x + q[h][1] * a.y + q[h][2] * b.x + q[h][3] * b.y;
+        }
+        // reduce-scatter over the 32 lanes: lane l ends with the full dot of index l
+#pragma unroll
+        for (int step = 16; step >= 1; step >>= 1) {
+            const bool hi = lane & step;
+#pragma unroll
+            for (int j = 0; j < step; ++j) {
+                const float send = hi ? v[j] : v[j + step];
+                const float keep = hi ? v[j + step] : v[j];
+                v[j] = keep + __shfl_xor_sync(0xffffffffu, send, step);
+            }
+        }
+        float sc = wv * fmaxf(v[0], 0.f);  // lane l: block b0 + l/4, head l%4
+        sc += __shfl_xor_sync(0xffffffffu, sc, 1);
+        sc += __shfl_xor_sync(0xffffffffu, sc, 2);
+        const int64_t b = b0 + (lane >> 2);
+        if ((lane & 3) == 0 && b < c1) srow[b] = sc;
+    }
+}
+
+// the packed layout: block b of the sequence at kc_seq + 256 b (hi, then lo)
+template <int kPlanes = 2>
+__device__ __forceinline__ void index_row_cuda(const __nv_bfloat16 *__restrict__ q_row,
+                                               const float *__restrict__ w_row, const __nv_bfloat16 *__restrict__ kc_seq,
+                                               int64_t c0, int64_t c1, float *__restrict__ srow, int warp,
+                                               int nwarps, int lane)
+{
+    index_row_cuda_at<kPlanes>(q_row, w_row, [=](int64_t b) { return kc_seq + b * 256; }, c0, c1, srow, warp,
+                               nwarps, lane);
+}
+
 cudaError_t launch_compress(const __nv_bfloat16 *k_idx, const int32_t *cu_k, const int32_t *cu_blocks,
                             int batch, int64_t total_k, const int32_t *blk_begin, int max_new, int r,
                             bool normalise, float eps, __nv_bfloat16 *kc, cudaStream_t stream);
@@ -35,7 +112,30 @@ struct IndexArgs {
     int r;
 };
 cudaError_t launch_index_tc(const IndexArgs &a, cudaStream_t stream);      // tcgen05 GEMM path
+
+// Output of the tcgen05 indexer (index.cu describes the modes): 0 = scores rows,
+// 1 = compact sample rows of every stride-th kc tile, 2 = candidate lists.
+struct IdxOut {
+    int mode;
+    float *scores;
+    int64_t ld;
+    float *sample;
+    int64_t sample_ld;
+    int stride;
+    int64_t min_bt;
+    const float *theta;
+    uint2 *lists;
+    int list_cap;
+    int32_t *counts;
+};
+cudaError_t launch_index_tc_mode(const IndexArgs &a, const IdxOut &out, cudaStream_t stream);
 cudaError_t launch_index_rowwise(const IndexArgs &a, cudaStream_t stream); // one-row-per-sequence path
+cudaError_t launch_index_rowwise_hi(const IndexArgs &a, cudaStream_t stream);  // the same, hi plane only
+// decode rows: the scores into ws, then the selector; refine = hi-plane scan plus the
+// exact rescoring of each row's near-threshold window (select.cu)
+size_t decode_select_workspace_bytes(int64_t rows, int64_t ld, int grid);
+cudaError_t launch_decode_index_select(const IndexArgs &a, int k, void *ws, int grid, bool refine, int32_t *sel,
+                                       cudaStream_t stream, int next_n = 1);
 
 struct SelectArgs {
     const float *scores;
@@ -45,8 +145,38 @@ struct SelectArgs {
     int64_t row_begin, row_end;
     int32_t *sel;
     int k, r;
+    int next_n = 1;  // > 1: decode rows serving next_n queries share one selection (select.cu)
 };
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t stream);
+
+// A paged decode cache (paged.cu): block_table [batch, max_pages] maps page j of
+// sequence s to a page of the pool; a page holds page_size tokens (k_idx rows) and
+// page_size / r compressed keys.
+struct PagedArgs {
+    int64_t num_pages;
+    int page_size;
+    const int32_t *table;
+    int max_pages;
+    const int32_t *cu_k;
+    int batch, r;
+};
+cudaError_t launch_compress_paged(const PagedArgs &p, const __nv_bfloat16 *k_pages, __nv_bfloat16 *kc_pages,
+                                  const int32_t *blk_begin, int max_new, int64_t max_len_k, bool normalise,
+                                  float eps, cudaStream_t stream);
+cudaError_t launch_index_paged(const PagedArgs &p, const __nv_bfloat16 *q_idx, const float *w,
+                               const __nv_bfloat16 *kc_pages, float *scores, int64_t ld, cudaStream_t stream);
+
+// Fused prefill index -> select (select.cu): workspace layout and launch.
+struct IndexSelectLayout {
+    int list_cap, stride;
+    int64_t sample_ld, scratch_ld;
+    int grid;
+    size_t off_sample, off_theta, off_counts, off_lists, off_fb, off_scratch, total;
+};
+IndexSelectLayout index_select_layout(int64_t rows, int64_t max_len_k, int k, int r, int grid);
+size_t index_select_workspace_bytes(int64_t rows, int64_t max_len_k, int k, int r, int grid);
+cudaError_t launch_index_select(const IndexArgs &a, int k, void *ws, int grid, int64_t max_len_k, int32_t *sel,
+                                cudaStream_t stream);
 
 struct AttnArgs {
     const __nv_bfloat16 *q, *k, *v;  // q [rows_total, 24, 256]; k, v [total_k, 2, 256]
@@ -72,6 +202,10 @@ struct AttnArgs {
 };
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream);
 cudaError_t launch_sparse_decode(const AttnArgs &a, cudaStream_t stream);  // a.even: the decode kernel
+// multi-token decode (attn_mtp.cu): next_n <= 4 queries per sequence, one shared selection
+int mtp_nsplit(int batch, int kb);
+size_t mtp_workspace_bytes(int batch, int kb);
+cudaError_t launch_sparse_mtp(const AttnArgs &a, int next_n, cudaStream_t stream);
 int dense_decode_nsplit(int64_t max_len_k, int r);  // splits of the dense flash-decoding path
 constexpr int kMaxEvenCtas = 256;               // CTAs of the even decode schedule, at most
 int even_grid();                                // CTAs of the even decode schedule on this device

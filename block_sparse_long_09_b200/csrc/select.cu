@@ -283,48 +283,41 @@ __device__ __forceinline__ void emit_segment(const uint32_t *gtw, const uint32_t
     *out_base += stot;
 }
 
+// Query row i: its sequence *s_out and position t (decode rows, cu_q == nullptr,
+// are sequence i at t = L - 1).
+__device__ __forceinline__ int64_t row_position(const int32_t *cu_q, const int32_t *cu_k, int batch, int64_t i,
+                                                int *s_out)
+{
+    if (cu_q != nullptr) {
+        const int s = find_seq(cu_q, batch, i);
+        *s_out = s;
+        const int64_t Lq = (int64_t)cu_q[s + 1] - cu_q[s];
+        const int64_t Lk = (int64_t)cu_k[s + 1] - cu_k[s];
+        return (Lk - Lq) + (i - cu_q[s]);
+    }
+    *s_out = (int)i;
+    return (int64_t)cu_k[i + 1] - cu_k[i] - 1;
+}
+
+// The selection of one row from its materialised scores srow[0 .. b_t): the own
+// block b_t plus the k - 1 best, ascending, into out[0 .. k).  The whole CTA runs it.
+// With nf > 1 (a multi-token decode step) the blocks bt .. bt + nf - 1 are all
+// forced and the best k - nf of the candidates 0 .. bt - 1 fill the other slots.
 template <int kSelThreads>
-__global__ void __launch_bounds__(kSelThreads, kSelThreads == 128 ? 8 : 2)
-select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ cu_q,
-              const int32_t *__restrict__ cu_k, int batch, int64_t row_begin, int k, int r,
-              int32_t *__restrict__ sel)
+__device__ __forceinline__ void select_row(const float *__restrict__ srow, int64_t bt, int k,
+                                           int32_t *__restrict__ out, uint32_t *smem_sel, SelScratch &sc,
+                                           int nf = 1)
 {
     constexpr int kSelWarps = kSelThreads / 32;
     constexpr int kCapW = kCandCap / kSelWarps;         // candidate list of one warp
-    extern __shared__ uint32_t smem_sel[];
     uint32_t *regA = smem_sel;                          // kSegWords words
     uint2 *cand = reinterpret_cast<uint2 *>(regA + kSegWords);  // kCandCap (score bits, index)
     uint32_t *regB = reinterpret_cast<uint32_t *>(cand);         // the same bytes, as words
-    __shared__ SelScratch sc;
-
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int64_t i = row_begin + blockIdx.x;
-    int s;
-    int64_t t;
-    if (cu_q != nullptr) {
-        s = find_seq(cu_q, batch, i);
-        const int64_t Lq = (int64_t)cu_q[s + 1] - cu_q[s];
-        const int64_t Lk = (int64_t)cu_k[s + 1] - cu_k[s];
-        t = (Lk - Lq) + (i - cu_q[s]);
-    } else {
-        s = (int)i;
-        t = (int64_t)cu_k[s + 1] - cu_k[s] - 1;
-    }
-    if (t < 0) {
-        if (tid == 0) set_device_status(QSA_ERR_DEVICE_CHECK);
-        return;
-    }
-    const int64_t bt = t / r;
-    if (bt > ld || bt > 0x7FFFFFFF) {  // scores row too short for this query
-        if (tid == 0) set_device_status(QSA_ERR_DEVICE_CHECK);
-        return;
-    }
-    const float *srow = scores + (int64_t)blockIdx.x * ld;
-    int32_t *out = sel + i * k;
-    const int need_total = k - 1;
+    const int need_total = k - nf;
 
-    if (bt <= need_total) {  // every candidate fits: 0 .. b_t, then padding
-        for (int j = tid; j < k; j += kSelThreads) out[j] = (j <= bt) ? j : -1;
+    if (bt <= need_total) {  // every candidate fits: 0 .. b_t + nf - 1, then padding
+        for (int j = tid; j < k; j += kSelThreads) out[j] = (j < bt + nf) ? j : -1;
         return;
     }
     const int n = (int)bt;
@@ -539,9 +532,426 @@ select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__res
     }
     if (tid == 0) {
         if (out_base != need_total) set_device_status(QSA_ERR_DEVICE_CHECK);
-        out[need_total] = (int32_t)bt;
+        for (int f = 0; f < nf; ++f) out[need_total + f] = (int32_t)(bt + f);
     }
 }
+
+// the candidates and forced blocks of decode row s (t = L - 1) serving next_n queries
+// t = L - next_n .. L - 1: candidates 0 .. b_first - 1, forced b_first .. b_last
+__device__ __forceinline__ void mtp_blocks(int64_t L, int next_n, int r, int64_t *b_first, int *nf)
+{
+    const int64_t t_first = L - next_n > 0 ? L - next_n : 0;
+    *b_first = t_first / r;
+    *nf = (int)((L - 1) / r - *b_first + 1);
+}
+
+template <int kSelThreads>
+__global__ void __launch_bounds__(kSelThreads, kSelThreads == 128 ? 8 : 2)
+select_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ cu_q,
+              const int32_t *__restrict__ cu_k, int batch, int64_t row_begin, int k, int r,
+              int32_t *__restrict__ sel, int next_n)
+{
+    extern __shared__ uint32_t smem_sel[];
+    __shared__ SelScratch sc;
+    const int64_t i = row_begin + blockIdx.x;
+    int s;
+    const int64_t t = row_position(cu_q, cu_k, batch, i, &s);
+    if (t < 0) {
+        if (threadIdx.x == 0) set_device_status(QSA_ERR_DEVICE_CHECK);
+        return;
+    }
+    int64_t bt = t / r;
+    int nf = 1;
+    if (next_n > 1) mtp_blocks(t + 1, next_n, r, &bt, &nf);
+    if (bt > ld || bt > 0x7FFFFFFF || nf > k) {  // scores row too short for this query
+        if (threadIdx.x == 0) set_device_status(QSA_ERR_DEVICE_CHECK);
+        return;
+    }
+    select_row<kSelThreads>(scores + (int64_t)blockIdx.x * ld, bt, k, sel + i * k, smem_sel, sc, nf);
+}
+
+
+// ============================ fused index -> select ============================
+// The prefill selection without materialised score rows (the launch order is in
+// launch_index_select):
+//   1. the indexer scores every stride-th kc tile of each row into a compact sample;
+//   2. threshold_kernel: theta = the r_lo-th largest sample score of the row, r_lo =
+//      mu + 4 sqrt(mu) + 8 with mu the expected number of the row's k - 1 winners in
+//      the sample (theta = -inf where every candidate fits the candidate list);
+//   3. the indexer scores every tile and appends (S, b) with S >= theta to the row's
+//      candidate list (capacity cap);
+//   4. select_list_kernel: the exact top k - 1 of the list.  The list holds every
+//      block scoring >= theta; when it holds at least k - 1 entries and did not
+//      overflow, the (k - 1)-th best is >= theta, so every block that can win, ties
+//      included, is in the list and the selection equals the one over the full row.
+//      Otherwise the row goes to a fallback list;
+//   5. fallback_kernel: for those rows, the full score row on CUDA cores into
+//      scratch, then the materialised selector.
+constexpr int kThrThreads = 128;
+
+// the compact sample row of b_t candidates: sampled tiles n = 0, stride, 2 stride, ...;
+// every sample entry is valid except the tail of the last sampled tile
+__device__ __forceinline__ int sample_count(int64_t bt, int stride)
+{
+    const int64_t tiles = (bt + 127) / 128;
+    const int64_t ns_tiles = (tiles + stride - 1) / stride;
+    if (ns_tiles == 0) return 0;
+    const int64_t last = (ns_tiles - 1) * stride * 128;
+    const int64_t tail = bt - last < 128 ? bt - last : 128;
+    return (int)((ns_tiles - 1) * 128 + tail);
+}
+
+__global__ void __launch_bounds__(kThrThreads)
+threshold_kernel(const float *__restrict__ sample, int64_t sample_ld, int stride, const int32_t *__restrict__ cu_q,
+                 const int32_t *__restrict__ cu_k, int batch, int64_t row_begin, int k, int r, int list_cap,
+                 float *__restrict__ theta, int32_t *__restrict__ fb_count)
+{
+    extern __shared__ uint32_t smem_sel[];
+    uint32_t *hist = smem_sel;            // kSegWords words
+    uint32_t *keys = smem_sel + kSegWords;  // sample_ld words
+    __shared__ SelScratch sc;
+    const int tid = threadIdx.x;
+    if (blockIdx.x == 0 && tid == 0) *fb_count = 0;  // the fallback list of this call starts empty
+    const int64_t rl = blockIdx.x, i = row_begin + rl;
+    int s;
+    const int64_t t = row_position(cu_q, cu_k, batch, i, &s);
+    const int64_t bt = t >= 0 ? t / r : 0;
+    if (bt <= list_cap) {  // every candidate fits the list
+        if (tid == 0) theta[rl] = -INFINITY;
+        return;
+    }
+    const int ns = sample_count(bt, stride);
+    const float mu = (float)(k - 1) * (float)ns / (float)bt;
+    const int r_lo = (int)ceilf(mu + 4.f * sqrtf(mu) + 8.f);
+    if (ns > sample_ld || r_lo > ns) {  // no usable sample: collect everything (the fallback takes it)
+        if (tid == 0) theta[rl] = -INFINITY;
+        return;
+    }
+    const float *srow = sample + rl * sample_ld;
+    for (int p = tid; p < ns; p += kThrThreads) keys[p] = order_key(__ldg(srow + p));
+    __syncthreads();
+    uint32_t prefix, mask;
+    int need, in_bin;
+    radix_select<kThrThreads, 8>(
+        [&](auto f) {
+            for (int p = tid; p < ns; p += kThrThreads) f(keys[p]);
+        },
+        ns, r_lo, 31, hist, &sc, &prefix, &mask, &need, &in_bin);
+    // prefix is the r_lo-th largest key, or (bin taken whole) a lower bound of it
+    if (tid == 0) theta[rl] = key_value(prefix);
+}
+
+// The exact top k - 1 of a candidate list (order key, block index) in shared
+// memory that holds every block able to win, ascending into out[0 .. k), with
+// out[k - 1] = b_t.  Ties at the threshold value go to the lowest block indices.
+template <int kT>
+__device__ __forceinline__ void select_from_list(const uint2 *cand, int cnt, int64_t bt, int k,
+                                                 int32_t *__restrict__ out, uint32_t *regA, SelScratch &sc,
+                                                 int nf = 1)
+{
+    const int tid = threadIdx.x;
+    const int need_total = k - nf;
+    uint32_t prefix, mask;
+    int need, in_bin;
+    radix_select<kT, 8>(
+        [&](auto f) {
+            for (int c = tid; c < cnt; c += kT) f(cand[c].x);
+        },
+        cnt, need_total, 31, regA, &sc, &prefix, &mask, &need, &in_bin);
+    // winners: keys above the threshold bin, and of the bin either all (need == in_bin) or,
+    // when the exact threshold value has more entries than slots left, its lowest indices
+    uint32_t iprefix = 0u, imask = 0u;
+    const bool partial = need < in_bin;
+    if (partial) {
+        int n2, b2;
+        radix_select<kT, 8>(
+            [&](auto f) {
+                for (int c = tid; c < cnt; c += kT)
+                    if ((cand[c].x & mask) == prefix) f(~cand[c].y);
+            },
+            in_bin, need, 31, regA, &sc, &iprefix, &imask, &n2, &b2);
+    }
+    auto wins = [&](const uint2 e) -> bool {
+        const uint32_t u = e.x & mask;
+        if (u != prefix) return u > prefix;
+        return !partial || ((~e.y) & imask) >= iprefix;
+    };
+    // ordered emission, one 65536-block segment of the bitmap at a time
+    int out_base = 0, eq_base = 0;
+    for (int64_t seg0 = 0; seg0 < bt; seg0 += kSegElems) {
+        const int seg_n = (int)(bt - seg0 < kSegElems ? bt - seg0 : kSegElems);
+        const int words = (seg_n + 31) >> 5;
+        for (int wd = tid; wd < words; wd += kT) regA[wd] = 0u;
+        __syncthreads();
+        for (int c = tid; c < cnt; c += kT) {
+            const uint2 e = cand[c];
+            const int64_t b = (int64_t)e.y - seg0;
+            if (b >= 0 && b < seg_n && wins(e)) atomicOr(&regA[b >> 5], 1u << (b & 31));
+        }
+        __syncthreads();
+        emit_segment<kT>(regA, regA, words, (int)seg0, false, need_total, need_total, &out_base, &eq_base,
+                                  out, &sc);
+        __syncthreads();
+    }
+    if (tid == 0) {
+        if (out_base != need_total) set_device_status(QSA_ERR_DEVICE_CHECK);
+        for (int f = 0; f < nf; ++f) out[need_total + f] = (int32_t)(bt + f);
+    }
+}
+
+__global__ void __launch_bounds__(kThrThreads, 8)
+select_list_kernel(const uint2 *__restrict__ lists, const int32_t *__restrict__ counts, int list_cap,
+                   const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k, int batch, int64_t row_begin,
+                   int k, int r, int32_t *__restrict__ sel, int32_t *__restrict__ fb_count,
+                   int32_t *__restrict__ fb_rows)
+{
+    extern __shared__ uint32_t smem_sel[];
+    uint32_t *regA = smem_sel;                                   // kSegWords words
+    uint2 *cand = reinterpret_cast<uint2 *>(smem_sel + kSegWords);  // list_cap (key, index)
+    __shared__ SelScratch sc;
+    const int tid = threadIdx.x;
+    const int64_t rl = blockIdx.x, i = row_begin + rl;
+    int s;
+    const int64_t t = row_position(cu_q, cu_k, batch, i, &s);
+    if (t < 0) {
+        if (tid == 0) set_device_status(QSA_ERR_DEVICE_CHECK);
+        return;
+    }
+    const int64_t bt = t / r;
+    int32_t *out = sel + i * k;
+    const int need_total = k - 1;
+    if (bt <= need_total) {
+        for (int j = tid; j < k; j += kThrThreads) out[j] = (j <= bt) ? j : -1;
+        return;
+    }
+    // the row's list is 4 segments of list_cap / 4 entries (one per TMEM lane quadrant
+    // of the indexer), each with its own length
+    const int cap_q = list_cap / 4;
+    const int4 c4 = *reinterpret_cast<const int4 *>(counts + rl * 4);
+    const int cq[4] = {c4.x, c4.y, c4.z, c4.w};
+    const int cnt = cq[0] + cq[1] + cq[2] + cq[3];
+    if (cnt < need_total || cq[0] > cap_q || cq[1] > cap_q || cq[2] > cap_q || cq[3] > cap_q) {
+        // the bound was too high, or a segment overflowed
+        if (tid == 0) fb_rows[atomicAdd(fb_count, 1)] = (int32_t)rl;
+        return;
+    }
+    const uint2 *lrow = lists + rl * list_cap;
+    int off = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        for (int c = tid; c < cq[q]; c += kThrThreads) {
+            const uint2 e = lrow[q * cap_q + c];
+            cand[off + c] = make_uint2(order_key(__uint_as_float(e.x)), e.y);
+        }
+        off += cq[q];
+    }
+    __syncthreads();
+    select_from_list<kThrThreads>(cand, cnt, bt, k, out, regA, sc);
+}
+
+constexpr int kFbThreads = 512;
+
+__global__ void __launch_bounds__(kFbThreads, 1)
+fallback_kernel(const __nv_bfloat16 *__restrict__ q_idx, const float *__restrict__ w, const __nv_bfloat16 *__restrict__ kc,
+                const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
+                const int32_t *__restrict__ cu_blocks, int batch, int64_t row_begin, int k, int r,
+                const int32_t *__restrict__ fb_count, const int32_t *__restrict__ fb_rows, float *__restrict__ scratch,
+                int64_t scratch_ld, int32_t *__restrict__ sel, int next_n)
+{
+    extern __shared__ uint32_t smem_sel[];
+    __shared__ SelScratch sc;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n = *fb_count;
+    float *srow = scratch + (int64_t)blockIdx.x * scratch_ld;
+    for (int f = blockIdx.x; f < n; f += gridDim.x) {
+        const int64_t i = row_begin + fb_rows[f];
+        int s;
+        const int64_t t = row_position(cu_q, cu_k, batch, i, &s);
+        int64_t bt = t / r;
+        int nf = 1;
+        if (next_n > 1) mtp_blocks(t + 1, next_n, r, &bt, &nf);
+        if (bt > scratch_ld || nf > k) {
+            if (threadIdx.x == 0) set_device_status(QSA_ERR_DEVICE_CHECK);
+            continue;
+        }
+        index_row_cuda<2>(q_idx + i * 512, w + i * 4, kc + (int64_t)cu_blocks[s] * 256, 0, bt, srow, warp,
+                       kFbThreads / 32, lane);
+        __syncthreads();
+        select_row<kFbThreads>(srow, bt, k, sel + i * k, smem_sel, sc, nf);
+        __syncthreads();
+    }
+}
+
+// ============================ decode: hi-plane scan, then refine ============================
+// The decode indexer reads only the hi plane of the compressed keys (half the
+// bytes of the exact hi + lo scan).  With the RMSNorm, ||kc_b|| <= sqrt(d), and
+// the lo plane is the rounding residue of the hi plane, ||lo_b|| <= 2^-8 ||kc_b||;
+// a head's dot moves by at most ||q_h|| ||lo_b||, ReLU is 1-Lipschitz, so every
+// approximate score is within E = sum_h |w_h| ||q_h|| sqrt(d) (2^-8 1.01 + 1e-4) of
+// the exact one (the last term covers fp32 accumulation).  Per row:
+//   1. tau = the (k-1)-th largest approximate score (radix select over the row);
+//   2. the window W = {b : approx_b >= tau - 2E} holds every block that can win:
+//      at least k - 1 blocks have approx >= tau, so exact >= tau - E for them,
+//      while a block outside W has exact < tau - E;
+//   3. the blocks of W are rescored exactly (hi + lo planes, the same arithmetic
+//      as the exact decode indexer) and their exact top k - 1 is the selection.
+// A window larger than kRefCap goes to the fallback (exact scores of the whole row).
+constexpr int kRefThreads = 512;
+constexpr int kRefCap = 4096;
+constexpr int kRefSmem = kSegWords * 4 + kRefCap * (8 + 4 + 4);
+
+__global__ void __launch_bounds__(kRefThreads, 1)
+refine_select_kernel(const float *__restrict__ approx, int64_t ld, const __nv_bfloat16 *__restrict__ q_idx,
+                     const float *__restrict__ w, const __nv_bfloat16 *__restrict__ kc,
+                     const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
+                     const int32_t *__restrict__ cu_blocks, int batch, int64_t row_begin, int k, int r,
+                     int32_t *__restrict__ sel, int32_t *__restrict__ fb_count, int32_t *__restrict__ fb_rows,
+                     int next_n)
+{
+    extern __shared__ uint32_t smem_sel[];
+    uint32_t *regA = smem_sel;                                        // kSegWords words
+    uint2 *cand = reinterpret_cast<uint2 *>(smem_sel + kSegWords);    // kRefCap (key, index)
+    float *exact = reinterpret_cast<float *>(cand + kRefCap);         // kRefCap exact scores
+    int32_t *widx = reinterpret_cast<int32_t *>(exact + kRefCap);     // kRefCap window block ids
+    __shared__ SelScratch sc;
+    __shared__ int wcount;
+    __shared__ float e_row;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t rl = blockIdx.x, i = row_begin + rl;
+    int s;
+    const int64_t t = row_position(cu_q, cu_k, batch, i, &s);
+    if (t < 0) {
+        if (tid == 0) set_device_status(QSA_ERR_DEVICE_CHECK);
+        return;
+    }
+    int64_t bt = t / r;
+    int nf = 1;
+    if (next_n > 1) mtp_blocks(t + 1, next_n, r, &bt, &nf);
+    if (bt > ld || bt > 0x7FFFFFFF || nf > k) {
+        if (tid == 0) set_device_status(QSA_ERR_DEVICE_CHECK);
+        return;
+    }
+    int32_t *out = sel + i * k;
+    const int need_total = k - nf;
+    if (bt <= need_total) {
+        for (int j = tid; j < k; j += kRefThreads) out[j] = (j < bt + nf) ? j : -1;
+        return;
+    }
+    const int n = (int)bt;
+    const float *srow = approx + rl * ld;
+    // the error bound E of the row
+    if (warp == 0) {
+        const __nv_bfloat16 *qr = q_idx + i * 512;
+        float e = 0.f;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const uint2 raw = *reinterpret_cast<const uint2 *>(qr + h * 128 + lane * 4);
+            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+            const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+            float ss = a.x * a.x + a.y * a.y + b.x * b.x + b.y * b.y;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            e += fabsf(__ldg(w + i * 4 + h)) * sqrtf(ss);
+        }
+        if (lane == 0) {
+            e_row = e * 11.3137085f * (1.01f * 0.00390625f + 1e-4f) * 1.01f;  // sqrt(128) (2^-8 1.01 + 1e-4)
+            wcount = 0;
+        }
+    }
+    // 1. a lower bound theta_s of tau, the (k-1)-th largest approximate score: the
+    //    r_lo-th largest of a sample of the row (runs of 8 keys spread over it), r_lo =
+    //    mu + 4 sqrt(mu) + 8 for mu expected winners in the sample; every block when the
+    //    row fits the list
+    float theta_s = -INFINITY;
+    if (n > kRefCap) {
+        const int runs = kCandCap / 8;
+        const int ns = runs * 8;
+        uint32_t *skeys = reinterpret_cast<uint32_t *>(cand);  // the list area, free until step 2
+        for (int g = tid; g < runs; g += kRefThreads) {
+            const int at = (int)(((int64_t)g * n) / runs) & ~3;
+            const float4 x0 = __ldg(reinterpret_cast<const float4 *>(srow + at));
+            const float4 x1 = __ldg(reinterpret_cast<const float4 *>(srow + at + 4));
+            const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) skeys[g * 8 + e] = order_key(xs[e]);
+        }
+        __syncthreads();
+        const float mu = (float)need_total * (float)ns / (float)n;
+        int r_lo = (int)ceilf(mu + 4.f * sqrtf(mu) + 8.f);
+        if (r_lo > ns) r_lo = ns;
+        uint32_t sp, sm;
+        int sn, sb;
+        radix_select<kRefThreads, 8>(
+            [&](auto f) {
+                for (int q = tid; q < ns; q += kRefThreads) f(skeys[q]);
+            },
+            ns, r_lo, 31, regA, &sc, &sp, &sm, &sn, &sb);
+        theta_s = key_value(sp);
+    }
+    __syncthreads();
+    // 2. the candidates W' = {b : approx_b >= theta_s - 2E} (with their approximate keys)
+    const float lo_bound = theta_s - 2.f * e_row;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (int j0 = 0; j0 < n; j0 += kRefThreads) {
+        const int j = j0 + tid;
+        const float x = j < n ? __ldg(srow + j) : -INFINITY;
+        const bool hit = j < n && x >= lo_bound;
+        const uint32_t m = __ballot_sync(0xffffffffu, hit);
+        int base = 0;
+        if (lane == 0 && m != 0u) base = atomicAdd(&wcount, __popc(m));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        const int pos = base + __popc(m & lt_mask);
+        if (hit && pos < kRefCap) cand[pos] = make_uint2(order_key(x), (uint32_t)j);
+    }
+    __syncthreads();
+    int nw = wcount;
+    if (nw > kRefCap || nw < need_total) {  // the list does not fit, or the bound was too high
+        if (tid == 0) fb_rows[atomicAdd(fb_count, 1)] = (int32_t)rl;
+        return;
+    }
+    //    tau among them (every key >= tau is listed when at least k - 1 keys are >= theta_s)
+    const uint32_t ks = order_key(theta_s);
+    int above = 0;
+    for (int c = tid; c < nw; c += kRefThreads) above += cand[c].x >= ks ? 1 : 0;
+    above = (int)block_reduce<kRefThreads, false>((uint32_t)above, &sc);
+    if (above < need_total) {
+        if (tid == 0) fb_rows[atomicAdd(fb_count, 1)] = (int32_t)rl;
+        return;
+    }
+    uint32_t prefix, mask;
+    int need, in_bin;
+    radix_select<kRefThreads, 8>(
+        [&](auto f) {
+            for (int c = tid; c < nw; c += kRefThreads) f(cand[c].x);
+        },
+        nw, need_total, 31, regA, &sc, &prefix, &mask, &need, &in_bin);
+    //    the window W = {b : approx_b >= tau - 2E}: its block ids, compacted
+    const uint32_t kw = order_key(key_value(prefix) - 2.f * e_row);
+    if (tid == 0) wcount = 0;
+    __syncthreads();
+    for (int c0 = 0; c0 < nw; c0 += kRefThreads) {
+        const int c = c0 + tid;
+        const bool hit = c < nw && cand[c].x >= kw;
+        const uint32_t m = __ballot_sync(0xffffffffu, hit);
+        int base = 0;
+        if (lane == 0 && m != 0u) base = atomicAdd(&wcount, __popc(m));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (hit) widx[base + __popc(m & lt_mask)] = (int32_t)cand[c].y;
+    }
+    __syncthreads();
+    nw = wcount;
+    // 3. exact scores of the window, then its exact top k - 1
+    const __nv_bfloat16 *kc_seq = kc + (int64_t)cu_blocks[s] * 256;
+    index_row_cuda_at<2>(q_idx + i * 512, w + i * 4,
+                         [=](int64_t p) { return kc_seq + (int64_t)widx[p] * 256; }, 0, nw, exact, warp,
+                         kRefThreads / 32, lane);
+    __syncthreads();
+    for (int c = tid; c < nw; c += kRefThreads) cand[c] = make_uint2(order_key(exact[c]), (uint32_t)widx[c]);
+    __syncthreads();
+    select_from_list<kRefThreads>(cand, nw, bt, k, out, regA, sc, nf);
+}
+
+__global__ void clear_count_kernel(int32_t *c) { *c = 0; }
 
 }  // namespace
 
@@ -555,11 +965,133 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t stream)
         const int64_t chunk = rows - done < 0x7FFFFFFF ? rows - done : 0x7FFFFFFF;
         if (wide)
             select_kernel<512><<<(unsigned)chunk, 512, sel_smem_bytes<512>(), stream>>>(
-                a.scores + done * a.ld, a.ld, a.cu_q, a.cu_k, a.batch, a.row_begin + done, a.k, a.r, a.sel);
+                a.scores + done * a.ld, a.ld, a.cu_q, a.cu_k, a.batch, a.row_begin + done, a.k, a.r, a.sel, a.next_n);
         else
             select_kernel<128><<<(unsigned)chunk, 128, sel_smem_bytes<128>(), stream>>>(
-                a.scores + done * a.ld, a.ld, a.cu_q, a.cu_k, a.batch, a.row_begin + done, a.k, a.r, a.sel);
+                a.scores + done * a.ld, a.ld, a.cu_q, a.cu_k, a.batch, a.row_begin + done, a.k, a.r, a.sel, a.next_n);
     }
+    return cudaGetLastError();
+}
+
+
+size_t index_select_workspace_bytes(int64_t rows, int64_t max_len_k, int k, int r, int grid)
+{
+    const IndexSelectLayout L = index_select_layout(rows, max_len_k, k, r, grid);
+    return L.total;
+}
+
+IndexSelectLayout index_select_layout(int64_t rows, int64_t max_len_k, int k, int r, int grid)
+{
+    IndexSelectLayout L{};
+    const int64_t max_bt = max_len_k > 0 ? (max_len_k - 1) / r : 0;
+    const int64_t tiles = (max_bt + 127) / 128;
+    L.list_cap = 4 * k;
+    L.stride = 16;
+    // at most 8192 sample entries per row (32 KB of keys for the threshold kernel)
+    while ((tiles + L.stride - 1) / L.stride > 64) L.stride *= 2;
+    L.sample_ld = ((tiles + L.stride - 1) / L.stride) * 128;
+    if (L.sample_ld == 0) L.sample_ld = 128;
+    L.scratch_ld = (max_bt + 3) / 4 * 4 + 4;
+    L.grid = grid;
+    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    size_t off = 0;
+    L.off_sample = off; off = al(off + (size_t)rows * L.sample_ld * 4);
+    L.off_theta = off; off = al(off + (size_t)rows * 4);
+    L.off_counts = off; off = al(off + (size_t)rows * 4 * 4);  // 4 list segments per row
+    L.off_lists = off; off = al(off + (size_t)rows * L.list_cap * 8);
+    L.off_fb = off; off = al(off + (size_t)(rows + 1) * 4);
+    L.off_scratch = off; off = al(off + (size_t)grid * L.scratch_ld * 4);
+    L.total = off;
+    return L;
+}
+
+cudaError_t launch_index_select(const IndexArgs &a, int k, void *ws, int grid, int64_t max_len_k, int32_t *sel,
+                                cudaStream_t stream)
+{
+    const int64_t rows = a.row_end - a.row_begin;
+    if (rows <= 0) return cudaSuccess;
+    if (rows > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    const IndexSelectLayout L = index_select_layout(rows, max_len_k, k, a.r, grid);
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    float *sample = reinterpret_cast<float *>(base + L.off_sample);
+    float *theta = reinterpret_cast<float *>(base + L.off_theta);
+    int32_t *counts = reinterpret_cast<int32_t *>(base + L.off_counts);
+    uint2 *lists = reinterpret_cast<uint2 *>(base + L.off_lists);
+    int32_t *fb_count = reinterpret_cast<int32_t *>(base + L.off_fb);
+    int32_t *fb_rows = fb_count + 1;
+    float *scratch = reinterpret_cast<float *>(base + L.off_scratch);
+    cudaError_t e;
+    // 1. sample scores (rows whose candidates all fit the list are skipped)
+    IdxOut o1{};
+    o1.mode = 1;
+    o1.sample = sample;
+    o1.sample_ld = L.sample_ld;
+    o1.stride = L.stride;
+    o1.min_bt = L.list_cap;
+    if ((e = launch_index_tc_mode(a, o1, stream)) != cudaSuccess) return e;
+    // 2. thresholds (also clears the fallback count)
+    threshold_kernel<<<(unsigned)rows, kThrThreads, (kSegWords + (int)L.sample_ld) * 4, stream>>>(
+        sample, L.sample_ld, L.stride, a.cu_q, a.cu_k, a.batch, a.row_begin, k, a.r, L.list_cap, theta, fb_count);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // 3. candidate lists
+    IdxOut o3{};
+    o3.mode = 2;
+    o3.theta = theta;
+    o3.lists = lists;
+    o3.list_cap = L.list_cap;
+    o3.counts = counts;
+    if ((e = launch_index_tc_mode(a, o3, stream)) != cudaSuccess) return e;
+    // 4. exact selection over each list
+    const int smem4 = (kSegWords + 2 * L.list_cap) * 4;
+    if ((e = set_smem_attr_once(reinterpret_cast<const void *>(select_list_kernel), smem4)) != cudaSuccess) return e;
+    select_list_kernel<<<(unsigned)rows, kThrThreads, smem4, stream>>>(
+        lists, counts, L.list_cap, a.cu_q, a.cu_k, a.batch, a.row_begin, k, a.r, sel, fb_count, fb_rows);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // 5. fallback rows
+    fallback_kernel<<<(unsigned)L.grid, kFbThreads, sel_smem_bytes<kFbThreads>(), stream>>>(
+        a.q_idx, a.w, a.kc, a.cu_q, a.cu_k, a.cu_blocks, a.batch, a.row_begin, k, a.r, fb_count, fb_rows, scratch,
+        L.scratch_ld, sel, 1);
+    return cudaGetLastError();
+}
+
+size_t decode_select_workspace_bytes(int64_t rows, int64_t ld, int grid)
+{
+    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    return al((size_t)rows * ld * 4) + al((size_t)(rows + 1) * 4) + al((size_t)grid * ld * 4);
+}
+
+cudaError_t launch_decode_index_select(const IndexArgs &a, int k, void *ws, int grid, bool refine, int32_t *sel,
+                                       cudaStream_t stream, int next_n)
+{
+    const int64_t rows = a.row_end - a.row_begin;
+    if (rows <= 0) return cudaSuccess;
+    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    float *scores = reinterpret_cast<float *>(base);
+    int32_t *fb_count = reinterpret_cast<int32_t *>(base + al((size_t)rows * a.ld * 4));
+    int32_t *fb_rows = fb_count + 1;
+    float *scratch = reinterpret_cast<float *>(base + al((size_t)rows * a.ld * 4) + al((size_t)(rows + 1) * 4));
+    IndexArgs a2 = a;
+    a2.scores = scores;
+    cudaError_t e;
+    if (!refine) {  // exact scores (hi + lo), then the selector
+        if ((e = launch_index_rowwise(a2, stream)) != cudaSuccess) return e;
+        SelectArgs sa{scores, a.ld, a.cu_q, a.cu_k, a.batch, a.row_begin, a.row_end, sel, k, a.r};
+        sa.next_n = next_n;
+        return launch_select(sa, stream);
+    }
+    if ((e = launch_index_rowwise_hi(a2, stream)) != cudaSuccess) return e;
+    clear_count_kernel<<<1, 1, 0, stream>>>(fb_count);
+    if ((e = set_smem_attr_once(reinterpret_cast<const void *>(refine_select_kernel), kRefSmem)) != cudaSuccess)
+        return e;
+    if (rows > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    refine_select_kernel<<<(unsigned)rows, kRefThreads, kRefSmem, stream>>>(
+        scores, a.ld, a.q_idx, a.w, a.kc, a.cu_q, a.cu_k, a.cu_blocks, a.batch, a.row_begin, k, a.r, sel, fb_count,
+        fb_rows, next_n);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    fallback_kernel<<<(unsigned)grid, kFbThreads, sel_smem_bytes<kFbThreads>(), stream>>>(
+        a.q_idx, a.w, a.kc, a.cu_q, a.cu_k, a.cu_blocks, a.batch, a.row_begin, k, a.r, fb_count, fb_rows, scratch,
+        a.ld, sel, next_n);
     return cudaGetLastError();
 }
 

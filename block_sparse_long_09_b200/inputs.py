@@ -54,7 +54,7 @@ class PrefillInputs:
 
 @dataclasses.dataclass
 class DecodeInputs:
-    q: torch.Tensor          # [B, 24, 256] bf16 (one new token per sequence)
+    q: torch.Tensor          # [B, 24, 256] bf16 (one new token per sequence), [B, next_n, 24, 256] for next_n > 1
     k_cache: torch.Tensor    # [sum L_s, 2, 256] bf16, the new token's row included
     v_cache: torch.Tensor    # [sum L_s, 2, 256] bf16
     q_idx: torch.Tensor      # [B, 4, 128] bf16
@@ -112,8 +112,10 @@ def draw_decode_lengths(batch: int, len_lo: int, len_hi: int, seed: int) -> list
 
 
 def make_decode(batch: int, len_lo: int, len_hi: Optional[int] = None, seed: int = 0,
-                device: str = "cpu", r: int = R) -> DecodeInputs:
-    """Decode inputs: one new query per sequence against packed bf16 caches.
+                device: str = "cpu", r: int = R, next_n: int = 1) -> DecodeInputs:
+    """Decode inputs: one new query per sequence against packed bf16 caches (next_n > 1:
+    q holds next_n new queries per sequence, [batch, next_n, 24, 256], the last of them
+    the one whose indexer query q_idx and weights w are drawn).
 
     Lengths are U{len_lo..len_hi} (fixed length when len_hi is None or equal)."""
     if len_hi is None or len_hi == len_lo:
@@ -124,7 +126,8 @@ def make_decode(batch: int, len_lo: int, len_hi: Optional[int] = None, seed: int
     g = torch.Generator(device=device)
     g.manual_seed(seed + 1)
     total = int(sum(seqlens))
-    q = _randn_bf16(g, (batch, N_HEADS_Q, HEAD_DIM), device)
+    q = _randn_bf16(g, (batch, N_HEADS_Q, HEAD_DIM) if next_n == 1 else (batch, next_n, N_HEADS_Q, HEAD_DIM),
+                    device)
     k = _randn_bf16(g, (total, N_HEADS_KV, HEAD_DIM), device)
     v = _randn_bf16(g, (total, N_HEADS_KV, HEAD_DIM), device)
     q_idx = _randn_bf16(g, (batch, N_HEADS_IDX, IDX_DIM), device)

@@ -14,7 +14,8 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libqsa.so")
+# QSA_DEBUG_BUILD=1 loads the QSA_DEBUG_CHECKS build (short waits, fault injection)
+LIB_PATH = os.path.join(_HERE, "libqsa_debug.so" if os.environ.get("QSA_DEBUG_BUILD") == "1" else "libqsa.so")
 
 QSA_OK = 0
 QSA_ERR_INVALID_ARG = 1
@@ -26,14 +27,16 @@ QSA_ERR_DEVICE_CHECK = 6
 QSA_ERR_SCRATCH_LIMIT = 7
 STATIC_SCRATCH_BYTES = 16 * 1024 * 1024  # QSA_STATIC_SCRATCH_BYTES
 QSA_COMPRESS_NO_NORM = 0x1
-OP_COMPRESS, OP_INDEX, OP_SELECT, OP_PREFILL, OP_DECODE, OP_DENSE, OP_DECODE_PAGED = range(7)
+(OP_COMPRESS, OP_INDEX, OP_SELECT, OP_PREFILL, OP_DECODE, OP_DENSE, OP_DECODE_PAGED, OP_INDEX_SELECT,
+ OP_INDEX_SELECT_PAGED, OP_DECODE_MTP) = range(10)
 
 EXPORTED = (
-    "qsa_config_init", "qsa_compress_keys", "qsa_index_scores", "qsa_select_blocks",
+    "qsa_config_init", "qsa_compress_keys", "qsa_index_scores", "qsa_select_blocks", "qsa_index_select",
     "qsa_sparse_attn_prefill", "qsa_sparse_attn_decode", "qsa_sparse_attn_decode_paged",
-    "qsa_sparse_attn_decode_static_scratch",
+    "qsa_sparse_attn_decode_static_scratch", "qsa_compress_keys_paged", "qsa_index_select_paged",
+    "qsa_index_select_mtp", "qsa_sparse_attn_decode_mtp",
     "qsa_dense_attn_prefill",
-    "qsa_workspace_size", "qsa_status_string", "qsa_get_device_status", "qsa_version",
+    "qsa_workspace_size", "qsa_status_string", "qsa_get_device_status", "qsa_version", "qsa_debug_inject",
 )
 
 
@@ -61,7 +64,8 @@ class QSAError(RuntimeError):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError("libqsa.so is not built (python -m block_sparse_long_09_b200.build)")
+        raise ImportError("%s is not built (python -m block_sparse_long_09_b200.build --all)"
+                          % os.path.basename(LIB_PATH))
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     CP = ctypes.POINTER(Config)
@@ -70,6 +74,11 @@ def _load():
         "qsa_compress_keys": (I32, [CP, P, P, P, I32, I64, P, I32, P, P]),
         "qsa_index_scores": (I32, [CP, P, P, P, I64, P, P, P, I32, I64, I32, I64, I64, P, I64, P, SZ, P]),
         "qsa_select_blocks": (I32, [CP, P, I64, P, P, I32, I64, I64, P, P, SZ, P]),
+        "qsa_index_select": (I32, [CP, P, P, P, I64, P, P, P, I32, I64, I32, I64, I64, I64, P, P, SZ, P]),
+        "qsa_compress_keys_paged": (I32, [CP, P, P, I64, I32, P, I32, P, I32, I64, P, I32, P]),
+        "qsa_index_select_paged": (I32, [CP, P, P, P, I64, I32, P, I32, P, I32, I64, P, P, SZ, P]),
+        "qsa_index_select_mtp": (I32, [CP, P, P, P, I64, P, P, I32, I32, I64, P, P, SZ, P]),
+        "qsa_sparse_attn_decode_mtp": (I32, [CP, P, P, P, P, I32, I64, I32, P, P, P, P, SZ, P]),
         "qsa_sparse_attn_prefill": (I32, [CP, P, P, P, P, P, P, I32, I64, I64, I64, I64, I64, P, P, P, SZ, P]),
         "qsa_sparse_attn_decode": (I32, [CP, P, P, P, P, I32, I64, P, P, P, P, SZ, P]),
         "qsa_sparse_attn_decode_static_scratch": (I32, [CP, P, P, P, P, I32, I64, P, P, P, P]),
@@ -79,6 +88,7 @@ def _load():
         "qsa_status_string": (ctypes.c_char_p, [I32]),
         "qsa_get_device_status": (I32, [P, ctypes.POINTER(I32), I32]),
         "qsa_version": (I32, []),
+        "qsa_debug_inject": (I32, [I32]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -163,6 +173,98 @@ def index_scores(q_idx, w, kc, cu_seqlens_q, cu_seqlens_k, cu_blocks, max_len_q:
                                  row_begin, row_end, _p(scores), ld, None, 0, _stream()),
            "qsa_index_scores")
     return scores
+
+
+def index_select(q_idx, w, kc, cu_seqlens_q, cu_seqlens_k, cu_blocks, max_len_q: int, max_len_k: int,
+                 row_begin: int = 0, row_end: Optional[int] = None, sel=None, ws=None, cfg: Optional[Config] = None):
+    """Indexer + top-k selection for packed rows [row_begin, row_end) without writing the
+    rows' full score rows (qsa_index_select); sel[i] for those rows."""
+    cfg = _cfg(cfg)
+    total_q = q_idx.shape[0]
+    if row_end is None:
+        row_end = total_q
+    if sel is None:
+        sel = torch.empty((total_q, cfg.budget_blocks), dtype=torch.int32, device=q_idx.device)
+    batch = cu_seqlens_q.numel() - 1
+    need = workspace_size(OP_INDEX_SELECT, batch, row_end - row_begin, max_len_k, cfg)
+    if ws is None:
+        ws = torch.empty((max(need, 16),), dtype=torch.uint8, device=q_idx.device)
+    _check(_lib.qsa_index_select(ctypes.byref(cfg), _p(q_idx), _p(w), _p(kc), kc.shape[0], _p(cu_seqlens_q),
+                                 _p(cu_seqlens_k), _p(cu_blocks), batch, total_q, max_len_q, max_len_k, row_begin,
+                                 row_end, _p(sel), _p(ws), ws.numel(), _stream()),
+           "qsa_index_select")
+    return sel
+
+
+def compress_keys_paged(k_idx_pages, kc_pages, block_table, cu_seqlens_k, max_len_k: int, blk_begin=None,
+                        max_new_blocks: int = 0, cfg: Optional[Config] = None):
+    """Compressed keys of a paged cache: k_idx_pages [num_pages, page_size, 128] bf16 ->
+    kc_pages [num_pages, page_size / r, 2, 128] bf16 (hi, lo), through block_table
+    [batch, max_pages]."""
+    cfg = _cfg(cfg)
+    num_pages, page_size = k_idx_pages.shape[0], k_idx_pages.shape[1]
+    _check(_lib.qsa_compress_keys_paged(ctypes.byref(cfg), _p(k_idx_pages), _p(kc_pages), num_pages, page_size,
+                                        _p(block_table), block_table.shape[1], _p(cu_seqlens_k),
+                                        cu_seqlens_k.numel() - 1, max_len_k, _p(blk_begin), max_new_blocks,
+                                        _stream()),
+           "qsa_compress_keys_paged")
+    return kc_pages
+
+
+def index_select_paged(q_idx, w, kc_pages, page_size: int, block_table, cu_seqlens_k, max_len_k: int, sel=None,
+                       ws=None, cfg: Optional[Config] = None):
+    """Decode indexer + top-k over a paged kc cache (one query per sequence)."""
+    cfg = _cfg(cfg)
+    batch = q_idx.shape[0]
+    if sel is None:
+        sel = torch.empty((batch, cfg.budget_blocks), dtype=torch.int32, device=q_idx.device)
+    if ws is None:
+        ws = torch.empty((max(workspace_size(OP_INDEX_SELECT_PAGED, batch, batch, max_len_k, cfg), 16),),
+                         dtype=torch.uint8, device=q_idx.device)
+    _check(_lib.qsa_index_select_paged(ctypes.byref(cfg), _p(q_idx), _p(w), _p(kc_pages), kc_pages.shape[0],
+                                       page_size, _p(block_table), block_table.shape[1], _p(cu_seqlens_k), batch,
+                                       max_len_k, _p(sel), _p(ws), ws.numel(), _stream()),
+           "qsa_index_select_paged")
+    return sel
+
+
+def index_select_mtp(q_idx, w, kc, cu_seqlens_k, cu_blocks, next_n: int, max_len_k: int, sel=None, ws=None,
+                     cfg: Optional[Config] = None):
+    """The shared selection of a multi-token decode step: one per sequence, from the
+    scores of its last query (q_idx [batch, 4, 128], w [batch, 4]), every query's own
+    block kept; sel [batch, k]."""
+    cfg = _cfg(cfg)
+    batch = cu_seqlens_k.numel() - 1
+    if sel is None:
+        sel = torch.empty((batch, cfg.budget_blocks), dtype=torch.int32, device=q_idx.device)
+    if ws is None:
+        ws = torch.empty((max(workspace_size(OP_INDEX_SELECT, batch, batch, max_len_k, cfg), 16),),
+                         dtype=torch.uint8, device=q_idx.device)
+    _check(_lib.qsa_index_select_mtp(ctypes.byref(cfg), _p(q_idx), _p(w), _p(kc), kc.shape[0], _p(cu_seqlens_k),
+                                     _p(cu_blocks), batch, next_n, max_len_k, _p(sel), _p(ws), ws.numel(),
+                                     _stream()),
+           "qsa_index_select_mtp")
+    return sel
+
+
+def sparse_attn_decode_mtp(q, k_cache, v_cache, cu_seqlens_k, sel, o=None, lse=None, ws=None,
+                           want_lse: bool = False, cfg: Optional[Config] = None):
+    """Attention of next_n queries per sequence (q [batch, next_n, 24, 256]) over one
+    shared selection per sequence, each query cut to its own tokens."""
+    cfg = _cfg(cfg)
+    batch, next_n = q.shape[0], q.shape[1]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((batch, next_n, cfg.n_heads_q), dtype=torch.float32, device=q.device)
+    need = workspace_size(OP_DECODE_MTP, batch, batch, 0, cfg)
+    if ws is None and need > 0:
+        ws = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    _check(_lib.qsa_sparse_attn_decode_mtp(ctypes.byref(cfg), _p(q), _p(k_cache), _p(v_cache), _p(cu_seqlens_k),
+                                           batch, k_cache.shape[0], next_n, _p(sel), _p(o), _p(lse), _p(ws),
+                                           ws.numel() if ws is not None else 0, _stream()),
+           "qsa_sparse_attn_decode_mtp")
+    return (o, lse) if want_lse or lse is not None else o
 
 
 def select_blocks(scores, cu_seqlens_q, cu_seqlens_k, total_q: int, row_begin: int = 0,
@@ -282,17 +384,21 @@ def dense_attn_prefill(q, k, v, cu_seqlens_q, cu_seqlens_k, max_len_q: int, o=No
 class Prefill:
     """One QSA layer's prefill through the C ABI, with query rows processed in
     chunks (the pages measure with 16K-token chunks).  Buffers are allocated
-    once and reused across calls of the same shape."""
+    once and reused across calls of the same shape.  fused=True (default) selects
+    with qsa_index_select (no score rows in memory); fused=False materialises each
+    chunk's scores (qsa_index_scores) and selects on them (qsa_select_blocks)."""
 
-    def __init__(self, seqlens, chunk_rows: int = 16384, cfg: Optional[Config] = None, device="cuda"):
+    def __init__(self, seqlens, chunk_rows: int = 16384, cfg: Optional[Config] = None, device="cuda",
+                 fused: bool = True):
         self.cfg = _cfg(cfg)
         r = self.cfg.r
         self.seqlens = [int(x) for x in seqlens]
         self.total = sum(self.seqlens)
         self.max_len = max(self.seqlens)
         self.n_blocks = sum(L // r for L in self.seqlens)
-        self.ld = max(4, ((self.max_len - 1) // r + 3) // 4 * 4)  # a multiple of 4: whole-tile score stores
+        self.ld = max(4, ((self.max_len - 1) // r + 3) // 4 * 4)  # a multiple of 4
         self.chunk = int(chunk_rows)
+        self.fused = bool(fused)
         self.device = torch.device(device)
         cu = [0]
         for L in self.seqlens:
@@ -303,9 +409,15 @@ class Prefill:
         self.cu = torch.tensor(cu, dtype=torch.int32, device=self.device)
         self.cu_blocks = torch.tensor(cb, dtype=torch.int32, device=self.device)
         self.kc = torch.empty((max(self.n_blocks, 1), 2, self.cfg.idx_dim), dtype=torch.bfloat16, device=self.device)
-        self.scores = torch.empty((min(self.chunk, self.total), self.ld), dtype=torch.float32, device=self.device)
-        self.sel = torch.empty((self.total, self.cfg.budget_blocks), dtype=torch.int32, device=self.device)
         rows = min(self.chunk, self.total)
+        if self.fused:
+            self.scores = None
+            need = workspace_size(OP_INDEX_SELECT, len(self.seqlens), rows, self.max_len, self.cfg)
+            self.ws_sel = torch.empty((max(need, 16),), dtype=torch.uint8, device=self.device)
+        else:
+            self.scores = torch.empty((rows, self.ld), dtype=torch.float32, device=self.device)
+            self.ws_sel = None
+        self.sel = torch.empty((self.total, self.cfg.budget_blocks), dtype=torch.int32, device=self.device)
         need = workspace_size(OP_PREFILL, len(self.seqlens), rows, self.max_len, self.cfg)
         self.ws = torch.empty((need,), dtype=torch.uint8, device=self.device) if need > 0 else None
 
@@ -325,10 +437,19 @@ class Prefill:
         compress_keys(k_idx, self.cu, self.cu_blocks, kc=self.kc, cfg=self.cfg)
         for r0 in range(0, self.total, self.chunk):
             r1 = min(self.total, r0 + self.chunk)
-            index_scores(q_idx, w, self.kc[: self.n_blocks], self.cu, self.cu, self.cu_blocks, self.max_len,
-                         self.ld, r0, r1, scores=self.scores, cfg=self.cfg)
-            select_blocks(self.scores, self.cu, self.cu, self.total, r0, r1, sel=self.sel, cfg=self.cfg)
+            self.select_chunk(q_idx, w, r0, r1)
         return self.sel
+
+    def select_chunk(self, q_idx, w, r0: int, r1: int):
+        """Selection of rows [r0, r1) from the compressed keys already in self.kc."""
+        kc = self.kc[: self.n_blocks]
+        if self.fused:
+            index_select(q_idx, w, kc, self.cu, self.cu, self.cu_blocks, self.max_len, self.max_len, r0, r1,
+                         sel=self.sel, ws=self.ws_sel, cfg=self.cfg)
+        else:
+            index_scores(q_idx, w, kc, self.cu, self.cu, self.cu_blocks, self.max_len, self.ld, r0, r1,
+                         scores=self.scores, cfg=self.cfg)
+            select_blocks(self.scores, self.cu, self.cu, self.total, r0, r1, sel=self.sel, cfg=self.cfg)
 
     def __call__(self, q, k, v, q_idx, w, k_idx, o=None, lse=None):
         self.index_select(q_idx, w, k_idx)
@@ -337,14 +458,16 @@ class Prefill:
 
 class DecodeStep:
     """One QSA decode step for a fixed batch, one new query per sequence: refresh
-    the compressed block each sequence just completed, score every earlier block,
-    select the top k, and run the decode attention (the batch's tiles spread evenly
-    over the CTAs) and the merge of the row pieces.  The five launches can be
+    the compressed block each sequence just completed, select the top k
+    (qsa_index_select: the hi-plane scan of every earlier block and the exact
+    rescoring of each row's near-threshold window; fused=False: the exact scores,
+    then the selector), and run the decode attention (the batch's tiles spread
+    evenly over the CTAs) and the merge of the row pieces.  The launches can be
     captured once in a CUDA graph and replayed (graph=True): the tensors passed
     here are the graph's fixed inputs, so a caller refreshes them in place."""
 
     def __init__(self, q, q_idx, w, k_cache, v_cache, k_idx, kc, cu_seqlens_k, cu_blocks, max_len_k: int,
-                 refresh_blocks=None, cfg: Optional[Config] = None, graph: bool = True):
+                 refresh_blocks=None, cfg: Optional[Config] = None, graph: bool = True, fused: bool = True):
         self.cfg = _cfg(cfg)
         r = self.cfg.r
         self.q, self.q_idx, self.w = q, q_idx, w
@@ -355,7 +478,11 @@ class DecodeStep:
         self.cu_q = torch.arange(self.batch + 1, dtype=torch.int32, device=dev)
         self.refresh = refresh_blocks  # [batch] int32 block ids to recompute, or None
         self.ld = max(4, ((max_len_k - 1) // r + 3) // 4 * 4)
-        self.scores = torch.empty((self.batch, self.ld), dtype=torch.float32, device=dev)
+        self.max_len_k = int(max_len_k)
+        self.fused = bool(fused)
+        self.scores = None if self.fused else torch.empty((self.batch, self.ld), dtype=torch.float32, device=dev)
+        self.ws_sel = torch.empty((max(workspace_size(OP_INDEX_SELECT, self.batch, self.batch, max_len_k, self.cfg),
+                                       16),), dtype=torch.uint8, device=dev) if self.fused else None
         self.sel = torch.empty((self.batch, self.cfg.budget_blocks), dtype=torch.int32, device=dev)
         self.o = torch.empty_like(q)
         self.ws = torch.empty((max(workspace_size(OP_DECODE, self.batch, self.batch, max_len_k, self.cfg), 16),),
@@ -373,9 +500,13 @@ class DecodeStep:
         if self.refresh is not None:
             compress_keys(self.k_idx, self.cu_k, self.cu_b, kc=self.kc, blk_begin=self.refresh, max_new_blocks=1,
                           cfg=self.cfg)
-        index_scores(self.q_idx, self.w, self.kc, self.cu_q, self.cu_k, self.cu_b, 1, self.ld, scores=self.scores,
-                     cfg=self.cfg)
-        select_blocks(self.scores, self.cu_q, self.cu_k, self.batch, sel=self.sel, cfg=self.cfg)
+        if self.fused:
+            index_select(self.q_idx, self.w, self.kc, self.cu_q, self.cu_k, self.cu_b, 1, self.max_len_k,
+                         sel=self.sel, ws=self.ws_sel, cfg=self.cfg)
+        else:
+            index_scores(self.q_idx, self.w, self.kc, self.cu_q, self.cu_k, self.cu_b, 1, self.ld,
+                         scores=self.scores, cfg=self.cfg)
+            select_blocks(self.scores, self.cu_q, self.cu_k, self.batch, sel=self.sel, cfg=self.cfg)
         sparse_attn_decode(self.q, self.k_cache, self.v_cache, self.cu_k, self.sel, o=self.o, ws=self.ws,
                            cfg=self.cfg)
         return self.o

@@ -65,7 +65,7 @@ typedef int32_t qsa_status;
 #define QSA_ERR_DEVICE_CHECK 6
 #define QSA_ERR_SCRATCH_LIMIT 7 /* the call needs more than QSA_STATIC_SCRATCH_BYTES */
 
-typedef uint16_t qsa_bf16;
+typedef uint16_t qsa_bf16; /* bfloat16 bit pattern */
 
 /* flags */
 #define QSA_COMPRESS_NO_NORM 0x1u /* plain mean-pool, no RMSNorm in the compressor */
@@ -93,6 +93,9 @@ typedef struct qsa_config {
 #define QSA_OP_DECODE 4
 #define QSA_OP_DENSE 5
 #define QSA_OP_DECODE_PAGED 6 /* qsa_sparse_attn_decode_paged */
+#define QSA_OP_INDEX_SELECT 7 /* qsa_index_select */
+#define QSA_OP_INDEX_SELECT_PAGED 8 /* qsa_index_select_paged */
+#define QSA_OP_DECODE_MTP 9 /* qsa_sparse_attn_decode_mtp */
 
 /* Fill *cfg with the model's values (r 4, k 512, 24/2/256, 4/128, scale 1/16,
  * eps 1e-6, flags 0, kv_chunk_blocks 0).  Host only. */
@@ -104,8 +107,9 @@ void qsa_config_init(qsa_config *cfg);
  * for every complete block b < floor(L_k,s / r) of every sequence (the mean
  * alone with QSA_COMPRESS_NO_NORM).  fp32 arithmetic.  Each value x is stored as
  * a compensated bf16 pair, hi = bf16(x) and lo = bf16(x - hi) (round to nearest
- * even), so kc = hi + lo carries about 16 significant bits: bf16 alone shifts
- * small indexer scores by percents and flips top-k choices.
+ * even), so kc = hi + lo carries about 16 significant bits: a single 16-bit
+ * value (bf16, and in rows of small scores fp16 too) shifts indexer scores by
+ * more than the selection tolerance.
  *   k_idx      [total_k, idx_dim] bf16   raw indexer keys (one shared key head)
  *   cu_seqlens_k, cu_blocks  [batch+1] int32
  *   total_k    host: rows of k_idx (bounds the launch)
@@ -130,8 +134,8 @@ qsa_status qsa_compress_keys(const qsa_config *cfg, const qsa_bf16 *k_idx,
  *           cu_blocks[batch]); both planes enter the products
  *   rows    packed query rows [row_begin, row_end) are scored (a chunk of a prefill)
  *   scores  fp32, row i at scores + (i - row_begin) * ld; entries b < b_t(i) hold
- *           the scores, entries b_t(i) <= b < ld are unspecified (whole tiles are
- *           stored when ld % 4 == 0).  ld >= every b_t(i).
+ *           the scores, entries b_t(i) <= b < ld are left as they were.
+ *           ld >= every b_t(i).
  *   total_q host: rows of q_idx; max_len_q host: max over s of L_q,s (a launch hint:
  *           1 selects the one-row-per-sequence decode kernel)
  * Workspace: none (ws may be NULL).
@@ -157,6 +161,89 @@ qsa_status qsa_select_blocks(const qsa_config *cfg, const float *scores, int64_t
                              const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
                              int32_t batch, int64_t row_begin, int64_t row_end, int32_t *sel,
                              void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Fused indexer + top-k selection -- the indexer equation, the budget sentence
+ * and the O(n^2 / r) complexity equation of section 6: for packed rows
+ * [row_begin, row_end), the same selection qsa_select_blocks makes on the scores
+ * of qsa_index_scores (same arguments as those two calls), without writing the
+ * rows' full score rows to memory.  Prefill rows (max_len_q > 1), per row:
+ *   - the tensor-core indexer scores every stride-th 128-block kc tile into a
+ *     compact sample, and a lower bound theta of the row's (k-1)-th best score is
+ *     the sample's r_lo-th best, r_lo = mu + 4 sqrt(mu) + 8 (mu = the expected
+ *     number of the row's winners in the sample);
+ *   - the indexer scores every tile and appends (score, block) with score >= theta
+ *     to the row's candidate list (4 k entries);
+ *   - the exact top k - 1 of the list is the row's selection whenever the list
+ *     holds at least k - 1 entries and did not overflow (every block that can win,
+ *     ties included, is then in the list); otherwise the row's full score row is
+ *     recomputed on CUDA cores into workspace scratch and selected from there.
+ * The tensor-core scores are the same fp32 values qsa_index_scores stores, so
+ * the selection equals the materialised path's bit for bit, except for rows that
+ * take the fallback, whose scores carry CUDA-core fp32 rounding.
+ * Decode rows (max_len_q == 1): the one-row indexer reads only the hi plane of kc
+ * (half the bytes of the exact scan) into the workspace.  With the RMSNorm every
+ * ||kc_b|| <= sqrt(idx_dim) and the lo plane is hi's rounding residue, so each such
+ * score is within E = sum_h |w_h| ||q_h|| sqrt(idx_dim) (2^-8 1.01 + 1e-4) of the
+ * exact one; the blocks within 2E of the row's (k-1)-th best are rescored exactly
+ * (hi + lo) and the row's exact top k - 1 is taken among them -- the same selection
+ * as qsa_index_scores + qsa_select_blocks.  A window of more than 4096 blocks, or
+ * QSA_COMPRESS_NO_NORM, takes the exact scan of the whole row instead.
+ *   max_len_k  host: an upper bound of every L_k,s (sizes the samples and scratch)
+ *   sel        [total_q, k] int32 as qsa_select_blocks writes it
+ * Workspace: qsa_workspace_size(cfg, QSA_OP_INDEX_SELECT, batch, row_end - row_begin,
+ * max_len_k) bytes, 16-byte aligned (about 576 MB for 16384 rows at 262144 tokens,
+ * against 4.3 GB of materialised scores).
+ */
+qsa_status qsa_index_select(const qsa_config *cfg, const qsa_bf16 *q_idx, const float *w, const qsa_bf16 *kc,
+                            int64_t kc_rows, const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                            const int32_t *cu_blocks, int32_t batch, int64_t total_q, int32_t max_len_q,
+                            int64_t max_len_k, int64_t row_begin, int64_t row_end, int32_t *sel, void *ws,
+                            size_t ws_bytes, void *stream);
+
+/*
+ * The compressed-key side of a paged decode cache.  The reading notes' decode
+ * measurement ("结果 2") compares against a paged GQA cache; here every per-token
+ * tensor of a sequence lives in fixed-size pages found through ONE block table:
+ *   block_table  [batch, max_pages] int32 (device): page j of sequence s holds its
+ *                tokens [j page_size, (j + 1) page_size); ids in 0 .. num_pages - 1
+ *   page_size    a multiple of r (a micro-block never straddles a page)
+ *   k_idx_pages  [num_pages, page_size, idx_dim] bf16: raw indexer keys
+ *   kc_pages     [num_pages, page_size / r, 2, idx_dim] bf16 hi/lo pairs; block b
+ *                of sequence s is row (b r mod page_size) / r of page
+ *                block_table[s][b r / page_size]
+ * K/V pages for qsa_sparse_attn_decode_paged use the same table.  Lengths come from
+ * cu_seqlens_k [batch + 1] (only L_s = cu[s+1] - cu[s] is used).  A page id out of
+ * range is skipped (compress) or read as page row 0 (index) and flags
+ * QSA_ERR_DEVICE_CHECK.
+ *
+ * qsa_compress_keys_paged: the pooled-key equation of section 6 (the same
+ * arithmetic and hi/lo store as qsa_compress_keys) for every complete block of
+ * every sequence (blk_begin == NULL; max_len_k bounds every L_s), or, with
+ * blk_begin [batch], for blocks [blk_begin[s], blk_begin[s] + max_new_blocks) that
+ * are complete (a decode step refreshes the block it completed).
+ */
+qsa_status qsa_compress_keys_paged(const qsa_config *cfg, const qsa_bf16 *k_idx_pages, qsa_bf16 *kc_pages,
+                                   int64_t num_pages, int32_t page_size, const int32_t *block_table,
+                                   int32_t max_pages, const int32_t *cu_seqlens_k, int32_t batch, int64_t max_len_k,
+                                   const int32_t *blk_begin, int32_t max_new_blocks, void *stream);
+
+/*
+ * qsa_index_select_paged: decode indexer + top-k selection over a paged kc cache,
+ * one new query per sequence at t = L_s - 1 (indexer equation and budget sentence
+ * of section 6): the same scores (CUDA-core fp32 GEMV) and the same selection as
+ * qsa_index_scores (max_len_q = 1) + qsa_select_blocks on the packed cache.
+ *   q_idx [batch, n_heads_idx, idx_dim] bf16; w [batch, n_heads_idx] fp32
+ *   sel   [batch, k] int32 (ascending, -1 padded)
+ *   max_len_k  host: an upper bound of every L_s
+ * Workspace: qsa_workspace_size(cfg, QSA_OP_INDEX_SELECT_PAGED, batch, batch,
+ * max_len_k) bytes (one fp32 score row per sequence), 16-byte aligned.
+ */
+qsa_status qsa_index_select_paged(const qsa_config *cfg, const qsa_bf16 *q_idx, const float *w,
+                                  const qsa_bf16 *kc_pages, int64_t num_pages, int32_t page_size,
+                                  const int32_t *block_table, int32_t max_pages, const int32_t *cu_seqlens_k,
+                                  int32_t batch, int64_t max_len_k, int32_t *sel, void *ws, size_t ws_bytes,
+                                  void *stream);
 
 /*
  * Sparse GQA attention, prefill -- expansion + core attention of section 6:
@@ -260,6 +347,43 @@ qsa_status qsa_sparse_attn_decode_static_scratch(const qsa_config *cfg, const qs
                                                  float *lse, void *stream);
 
 /*
+ * Decode with multi-token prediction.  The reading notes' decode measurement
+ * ("结果 2") verifies next_n = 4 tokens per sequence per step (three MTP
+ * prediction steps), and their section 5, step 5 says the MTP steps reuse the
+ * QSA top-k indices.  Reading taken here: ONE selection per sequence serves its
+ * next_n queries t = L - next_n .. L - 1 (L = cu_seqlens_k[s+1] - cu_seqlens_k[s],
+ * the cache holding all next_n new tokens):
+ *
+ * qsa_index_select_mtp: the selection, from the indexer scores of the LAST query
+ * (q_idx, w: [batch, n_heads_idx, idx_dim] / [batch, n_heads_idx], that query's).
+ * Every query keeps its own trailing block (the budget sentence of section 6), so
+ * the blocks floor((L - next_n) / r) .. floor((L - 1) / r) are all kept and the
+ * other slots, at most k minus their number, go to the best blocks below the
+ * first of them (ties to the lower index).  sel [batch, k] int32, ascending, -1
+ * padded.  The scan and the exact rescoring are those of qsa_index_select's decode
+ * rows.  1 <= next_n <= 4, k >= 2.  Workspace: qsa_workspace_size(cfg,
+ * QSA_OP_INDEX_SELECT, batch, batch, max_len_k) bytes.
+ *
+ * qsa_sparse_attn_decode_mtp: the sparse attention of the next_n queries over the
+ * shared selection, each cut to its own tokens j <= t (section 6).  One gathered
+ * K/V tile serves every query of the sequence: the kernel puts the next_n x 24
+ * (query, head) rows on the tensor cores' M side.
+ *   q [batch, next_n, n_heads_q, head_dim] bf16; o the same shape;
+ *   lse [batch, next_n, n_heads_q] fp32 or NULL; k_cache, v_cache packed as for
+ *   qsa_sparse_attn_decode.
+ * Workspace: qsa_workspace_size(cfg, QSA_OP_DECODE_MTP, batch, batch, 0) bytes
+ * (partial softmax states when a sequence's tiles are split over several CTAs).
+ */
+qsa_status qsa_index_select_mtp(const qsa_config *cfg, const qsa_bf16 *q_idx, const float *w, const qsa_bf16 *kc,
+                                int64_t kc_rows, const int32_t *cu_seqlens_k, const int32_t *cu_blocks,
+                                int32_t batch, int32_t next_n, int64_t max_len_k, int32_t *sel, void *ws,
+                                size_t ws_bytes, void *stream);
+qsa_status qsa_sparse_attn_decode_mtp(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k_cache,
+                                      const qsa_bf16 *v_cache, const int32_t *cu_seqlens_k, int32_t batch,
+                                      int64_t total_k, int32_t next_n, const int32_t *sel, qsa_bf16 *o, float *lse,
+                                      void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Dense causal GQA attention (the baseline the pages measure QSA against):
  * query t attends to every key j <= t of its sequence.  Same layouts as the
  * sparse prefill.  max_len_q and max_len_k are host bounds of L_q,s and L_k,s.
@@ -287,6 +411,17 @@ qsa_status qsa_get_device_status(void *stream, int32_t *status, int32_t clear);
 
 /* ABI version (major * 100 + minor). */
 int32_t qsa_version(void);
+
+/* Fault injection for the failure-path tests.  Only a library built with
+ * QSA_DEBUG_CHECKS (libqsa_debug.so: mbarrier waits limited to 20 ms) acts on
+ * it; the release library returns QSA_ERR_UNSUPPORTED and changes nothing.
+ *   site 0  no fault (the default)
+ *   site 1  the decode scan's producer (qsa_index_select, decode rows) issues no
+ *           copies for the second kc tile of each CTA, so the consumer's bounded
+ *           wait runs out: the call's kernels return, the status word reads
+ *           QSA_ERR_TIMEOUT and the next call without the fault runs normally.
+ * Host only (one device-symbol copy); not thread-safe with calls in flight. */
+qsa_status qsa_debug_inject(int32_t site);
 
 #ifdef __cplusplus
 }

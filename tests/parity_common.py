@@ -78,3 +78,9 @@ def bits(t):
     """bf16 tensor -> numpy uint16 bit patterns (on the host)."""
     import torch
     return np.ascontiguousarray(t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def mean_blocks_differing(sel_g, sel_o):
+    """Mean over rows of the number of selected blocks that differ between two selections."""
+    d = [len(set(a.tolist()) ^ set(b.tolist())) / 2.0 for a, b in zip(sel_g, sel_o)]
+    return float(np.mean(d)) if d else 0.0

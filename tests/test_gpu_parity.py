@@ -47,6 +47,7 @@ def seq_slices(lengths):
 
 def kc_value(kc):
     """hi + lo planes of the compressed keys, in fp64: [n_blocks, 128]."""
+    assert kc.dtype == torch.bfloat16 and kc.dim() == 3
     return kc.double().sum(dim=1).cpu().numpy()
 
 
@@ -481,12 +482,70 @@ def test_decode_step_cuda_graph(qsa):
     graphed = qsa.DecodeStep(*args, kc, cu_k, cu_b, max(d.seqlens), refresh_blocks=last, graph=True)
     for _ in range(3):
         o_graph = graphed()
+    exact = qsa.DecodeStep(*args, kc, cu_k, cu_b, max(d.seqlens), refresh_blocks=last, graph=False, fused=False)
+    o_exact = exact()
     torch.cuda.synchronize()
     assert torch.equal(graphed.sel, sel_eager)
     assert torch.equal(o_graph, o_eager)
+    # the fused selection (hi-plane scan + exact window) equals the exact scan's
+    assert torch.equal(exact.sel, sel_eager)
+    assert torch.equal(o_exact, o_eager)
     sel_g = sel_eager.cpu().numpy()
     for s in (0, 7):
         a, b = int(cu_k[s]), int(cu_k[s + 1])
         ref_o, _ = oracle.attend(d.q[s:s + 1], d.k_cache[a:b], d.v_cache[a:b], sel_g[s:s + 1], 1, b - a, 4, SCALE, [0])
         check_attn(o_eager.float().cpu().numpy()[s:s + 1], ref_o)
+    status_ok(qsa)
+
+
+@pytest.mark.parametrize("batch,lo,hi,k,page", [(5, 1, 3000, 512, 16), (64, 2000, 9000, 512, 64),
+                                                (9, 4100, 20000, 512, 256), (300, 1, 600, 64, 4)])
+def test_paged_kc_decode_chain(qsa, batch, lo, hi, k, page):
+    """The compressed keys and the decode indexer through the same block table as the
+    paged K/V: compressed keys, selection and attention equal the packed path bit for bit."""
+    d = inputs.make_decode(batch, lo, hi, seed=33)
+    cfg = qsa.default_config(budget_blocks=k)
+    cu_k, cu_b = cu(d.seqlens)
+    cu_q = torch.arange(batch + 1, dtype=torch.int32, device="cuda")
+    max_len = max(d.seqlens)
+    # the packed chain
+    kc = qsa.compress_keys(d.k_idx.cuda(), cu_k, cu_b, n_blocks=max(int(cu_b[-1]), 1), cfg=cfg)
+    ld = max(4, ((max_len - 1) // 4 + 3) // 4 * 4)
+    scores = torch.empty((batch, ld), dtype=torch.float32, device="cuda")
+    qsa.index_scores(d.q_idx.cuda(), d.w.cuda(), kc[: max(int(cu_b[-1]), 1)], cu_q, cu_k, cu_b, 1, ld, scores=scores,
+                     cfg=cfg)
+    sel_p = qsa.select_blocks(scores, cu_q, cu_k, batch, cfg=cfg)
+    o_p = qsa.sparse_attn_decode(d.q.cuda(), d.k_cache.cuda(), d.v_cache.cuda(), cu_k, sel_p, cfg=cfg)
+    # the paged chain: one table for k_idx, kc, K and V
+    kip, table = paged_cache(d.k_idx, d.seqlens, page, seed=34)
+    kp, _ = paged_cache(d.k_cache, d.seqlens, page, seed=34)
+    vp, _ = paged_cache(d.v_cache, d.seqlens, page, seed=34)
+    kip, table, kp, vp = kip.cuda(), table.cuda(), kp.cuda(), vp.cuda()
+    kcp = torch.zeros((kip.shape[0], page // 4, 2, 128), dtype=torch.bfloat16, device="cuda")
+    qsa.compress_keys_paged(kip, kcp, table, cu_k, max_len, cfg=cfg)
+    sel_g = qsa.index_select_paged(d.q_idx.cuda(), d.w.cuda(), kcp, page, table, cu_k, max_len, cfg=cfg)
+    o_g = qsa.sparse_attn_decode_paged(d.q.cuda(), kp, vp, table, cu_k, sel_g, cfg=cfg)
+    torch.cuda.synchronize()
+    # the compressed keys, row by row through the table
+    tab = table.cpu().numpy()
+    kcp_h, kc_h = kcp.cpu(), kc.cpu()
+    for s, L in enumerate(d.seqlens):
+        for b in range(L // 4):
+            assert torch.equal(kcp_h[tab[s, (4 * b) // page], (4 * b % page) // 4], kc_h[int(cu_b[s]) + b]), (s, b)
+    assert torch.equal(sel_g, sel_p)
+    if batch < 296:  # both ran the even-schedule decode kernel on the same values
+        assert torch.equal(o_g, o_p)
+    else:
+        check_attn(o_g.float().cpu().numpy(), o_p.float().cpu().numpy().astype(np.float64))
+    # a decode step's refresh of the block just completed, into cleared pages
+    last = torch.tensor([max(L // 4 - 1, 0) for L in d.seqlens], dtype=torch.int32, device="cuda")
+    kcp2 = torch.zeros_like(kcp)
+    qsa.compress_keys_paged(kip, kcp2, table, cu_k, max_len, blk_begin=last, max_new_blocks=1, cfg=cfg)
+    torch.cuda.synchronize()
+    kcp2_h = kcp2.cpu()
+    for s, L in enumerate(d.seqlens):
+        b = L // 4 - 1
+        if b >= 0:
+            pg, rw = tab[s, (4 * b) // page], (4 * b % page) // 4
+            assert torch.equal(kcp2_h[pg, rw], kcp_h[pg, rw])
     status_ok(qsa)
