@@ -132,6 +132,16 @@ def _cfg(cfg: Optional[Config]) -> Config:
     return cfg if cfg is not None else default_config()
 
 
+def _check_sel(sel, rows: int, cfg: Config):
+    """A selection buffer must be int32 [>= rows, budget_blocks], contiguous: the kernels
+    address row i at sel + i * budget_blocks and cannot see the tensor's extent."""
+    if sel.dtype != torch.int32 or sel.dim() != 2 or not sel.is_contiguous():
+        raise ValueError("sel must be a contiguous int32 [rows, budget_blocks] tensor")
+    if sel.shape[1] != cfg.budget_blocks or sel.shape[0] < rows:
+        raise ValueError("sel is %s; the call needs [>= %d, %d] (cfg.budget_blocks)"
+                         % (tuple(sel.shape), rows, cfg.budget_blocks))
+
+
 def workspace_size(op: int, batch: int, rows: int = 0, max_len_k: int = 0, cfg: Optional[Config] = None) -> int:
     return int(_lib.qsa_workspace_size(ctypes.byref(_cfg(cfg)), op, batch, rows, max_len_k))
 
@@ -189,6 +199,7 @@ def index_select(q_idx, w, kc, cu_seqlens_q, cu_seqlens_k, cu_blocks, max_len_q:
     need = workspace_size(OP_INDEX_SELECT, batch, row_end - row_begin, max_len_k, cfg)
     if ws is None:
         ws = torch.empty((max(need, 16),), dtype=torch.uint8, device=q_idx.device)
+    _check_sel(sel, row_end, cfg)
     _check(_lib.qsa_index_select(ctypes.byref(cfg), _p(q_idx), _p(w), _p(kc), kc.shape[0], _p(cu_seqlens_q),
                                  _p(cu_seqlens_k), _p(cu_blocks), batch, total_q, max_len_q, max_len_k, row_begin,
                                  row_end, _p(sel), _p(ws), ws.numel(), _stream()),
@@ -221,6 +232,7 @@ def index_select_paged(q_idx, w, kc_pages, page_size: int, block_table, cu_seqle
     if ws is None:
         ws = torch.empty((max(workspace_size(OP_INDEX_SELECT_PAGED, batch, batch, max_len_k, cfg), 16),),
                          dtype=torch.uint8, device=q_idx.device)
+    _check_sel(sel, batch, cfg)
     _check(_lib.qsa_index_select_paged(ctypes.byref(cfg), _p(q_idx), _p(w), _p(kc_pages), kc_pages.shape[0],
                                        page_size, _p(block_table), block_table.shape[1], _p(cu_seqlens_k), batch,
                                        max_len_k, _p(sel), _p(ws), ws.numel(), _stream()),
@@ -240,6 +252,7 @@ def index_select_mtp(q_idx, w, kc, cu_seqlens_k, cu_blocks, next_n: int, max_len
     if ws is None:
         ws = torch.empty((max(workspace_size(OP_INDEX_SELECT, batch, batch, max_len_k, cfg), 16),),
                          dtype=torch.uint8, device=q_idx.device)
+    _check_sel(sel, batch, cfg)
     _check(_lib.qsa_index_select_mtp(ctypes.byref(cfg), _p(q_idx), _p(w), _p(kc), kc.shape[0], _p(cu_seqlens_k),
                                      _p(cu_blocks), batch, next_n, max_len_k, _p(sel), _p(ws), ws.numel(),
                                      _stream()),
@@ -260,6 +273,7 @@ def sparse_attn_decode_mtp(q, k_cache, v_cache, cu_seqlens_k, sel, o=None, lse=N
     need = workspace_size(OP_DECODE_MTP, batch, batch, 0, cfg)
     if ws is None and need > 0:
         ws = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    _check_sel(sel, batch, cfg)
     _check(_lib.qsa_sparse_attn_decode_mtp(ctypes.byref(cfg), _p(q), _p(k_cache), _p(v_cache), _p(cu_seqlens_k),
                                            batch, k_cache.shape[0], next_n, _p(sel), _p(o), _p(lse), _p(ws),
                                            ws.numel() if ws is not None else 0, _stream()),
@@ -275,6 +289,7 @@ def select_blocks(scores, cu_seqlens_q, cu_seqlens_k, total_q: int, row_begin: i
         row_end = total_q
     if sel is None:
         sel = torch.empty((total_q, cfg.budget_blocks), dtype=torch.int32, device=scores.device)
+    _check_sel(sel, row_end, cfg)
     _check(_lib.qsa_select_blocks(ctypes.byref(cfg), _p(scores), scores.shape[1], _p(cu_seqlens_q),
                                   _p(cu_seqlens_k), cu_seqlens_q.numel() - 1, row_begin, row_end, _p(sel),
                                   None, 0, _stream()),
@@ -301,6 +316,7 @@ def sparse_attn_prefill(q, k, v, sel, cu_seqlens_q, cu_seqlens_k, row_begin: int
     need = workspace_size(OP_PREFILL, batch, row_end - row_begin, max_len_k, cfg)
     if ws is None and need > 0:
         ws = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    _check_sel(sel, row_end, cfg)
     _check(_lib.qsa_sparse_attn_prefill(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(sel), _p(cu_seqlens_q),
                                         _p(cu_seqlens_k), batch, total_q, k.shape[0], max_len_k, row_begin, row_end,
                                         _p(o), _p(lse), _p(ws), ws.numel() if ws is not None else 0, _stream()),
@@ -319,6 +335,7 @@ def sparse_attn_decode(q, k_cache, v_cache, cu_seqlens_k, sel, o=None, lse=None,
     need = workspace_size(OP_DECODE, batch, batch, 0, cfg)
     if ws is None and need > 0:
         ws = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    _check_sel(sel, batch, cfg)
     _check(_lib.qsa_sparse_attn_decode(ctypes.byref(cfg), _p(q), _p(k_cache), _p(v_cache), _p(cu_seqlens_k),
                                        batch, k_cache.shape[0], _p(sel), _p(o), _p(lse), _p(ws),
                                        ws.numel() if ws is not None else 0, _stream()),
@@ -339,6 +356,7 @@ def sparse_attn_decode_paged(q, k_pages, v_pages, block_table, cu_seqlens_k, sel
         lse = torch.empty((batch, cfg.n_heads_q), dtype=torch.float32, device=q.device)
     if ws is None:
         ws = torch.empty((workspace_size(OP_DECODE_PAGED, batch, batch, 0, cfg),), dtype=torch.uint8, device=q.device)
+    _check_sel(sel, batch, cfg)
     _check(_lib.qsa_sparse_attn_decode_paged(ctypes.byref(cfg), _p(q), _p(k_pages), _p(v_pages), num_pages, page_size,
                                              _p(block_table), block_table.shape[1], _p(cu_seqlens_k), batch, _p(sel),
                                              _p(o), _p(lse), _p(ws), ws.numel(), _stream()),
@@ -352,6 +370,7 @@ def sparse_attn_decode_static_scratch(q, k_cache, v_cache, cu_seqlens_k, sel, o,
     device scratch: neither this wrapper nor the call allocates device memory.
     Calls that overlap on the GPU share that scratch and race."""
     cfg = _cfg(cfg)
+    _check_sel(sel, q.shape[0], cfg)
     _check(_lib.qsa_sparse_attn_decode_static_scratch(ctypes.byref(cfg), _p(q), _p(k_cache), _p(v_cache),
                                                       _p(cu_seqlens_k), q.shape[0], k_cache.shape[0], _p(sel),
                                                       _p(o), _p(lse), _stream()),

@@ -114,3 +114,24 @@ def test_workspace_sizes(qsa):
     assert small >= 1000 * 32 * 24 * 257 * 4
     ws = qsa.workspace_size(qsa.OP_DECODE, 64, 64, 262144)
     assert ws >= 64 * 24 * 257 * 4
+
+
+def test_fault_injection_is_inert_in_the_release_library(qsa):
+    # the release build compiles no injection site: the call is refused before any CUDA call
+    assert qsa.LIB_PATH.endswith("libqsa.so")
+    assert qsa.library().qsa_debug_inject(1) == qsa.QSA_ERR_UNSUPPORTED
+    assert qsa.library().qsa_debug_inject(0) == qsa.QSA_ERR_UNSUPPORTED
+
+
+def test_binding_refuses_a_selection_that_does_not_match_the_budget(qsa):
+    # checked on the host before the library is called (CPU tensors never reach it)
+    import torch
+    q = torch.zeros((8, 24, 256), dtype=torch.bfloat16)
+    kv = torch.zeros((8, 2, 256), dtype=torch.bfloat16)
+    cu_ = torch.tensor([0, 8], dtype=torch.int32)
+    for bad in (torch.zeros((8, 64), dtype=torch.int32), torch.zeros((4, 512), dtype=torch.int32),
+                torch.zeros((8, 512), dtype=torch.int64), torch.zeros((8, 1024), dtype=torch.int32)[:, :512]):
+        with pytest.raises(ValueError):
+            qsa.sparse_attn_prefill(q, kv, kv, bad, cu_, cu_)
+    with pytest.raises(ValueError):
+        qsa.sparse_attn_decode(q[:1], kv, kv, cu_, torch.zeros((1, 16), dtype=torch.int32))
