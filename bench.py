@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 N_PREFILL = 262144
 DEC_BATCH = 64
 DEC_LEN = 131072
+MTP_NEXT_N = 4       # queries per sequence of the multi-token-prediction decode step
 CHUNK = 16384
 BUDGET = 512
 METRIC = "QSA prefill tokens/s at 262K ctx; decode µs/token at 128K; % of roofline"
@@ -250,6 +251,35 @@ def run_qsa(args, rank, world, device):
                                                        cfg=cfg)) * 1e3
     step_bytes, kc_scan, dec_gather = decode_bytes(d.seqlens, kc_bpb // 2)
 
+    # multi-token-prediction decode at 131072: next_n = 4 new queries per sequence share one
+    # selection (made from the last query's indexer scores) and one gather of its K/V
+    g4 = torch.Generator(device=device)
+    g4.manual_seed(seeds["decode"] + 7)
+    q4 = torch.randn((DEC_BATCH, MTP_NEXT_N, 24, 256), generator=g4, device=device).to(torch.bfloat16)
+    sel4 = torch.empty((DEC_BATCH, BUDGET), dtype=torch.int32, device=device)
+    o4 = torch.empty_like(q4)
+    ws4s = torch.empty((qsa.workspace_size(qsa.OP_INDEX_SELECT, DEC_BATCH, DEC_BATCH, DEC_LEN, cfg),),
+                       dtype=torch.uint8, device=device)
+    ws4a = torch.empty((max(qsa.workspace_size(qsa.OP_DECODE_MTP, DEC_BATCH, DEC_BATCH, 0, cfg), 16),),
+                       dtype=torch.uint8, device=device)
+
+    def mtp_select():
+        qsa.index_select_mtp(dec.q_idx, dec.w, dec.kc, dec.cu_k, dec.cu_b, MTP_NEXT_N, DEC_LEN, sel=sel4, ws=ws4s,
+                             cfg=cfg)
+
+    def mtp_attend():
+        qsa.sparse_attn_decode_mtp(q4, d.k_cache, d.v_cache, cu_k, sel4, o=o4, ws=ws4a, cfg=cfg)
+
+    def mtp_step():
+        mtp_select()
+        mtp_attend()
+
+    mtp_step_us = timed(mtp_step, reps=10) * 1e3
+    mtp_select_us = timed(mtp_select, reps=10) * 1e3
+    mtp_attn_us = timed(mtp_attend, reps=10) * 1e3
+    assert qsa.device_status() == 0
+    del q4, sel4, o4, ws4s, ws4a
+
     # decode at 262144 tokens per sequence: the step, and the attention kernel alone
     del d, dec
     torch.cuda.empty_cache()
@@ -357,6 +387,12 @@ def run_qsa(args, rank, world, device):
             "index_select_frac": kc_scan / (dec_select_us / 1e6) / 1e9 / hbm,
             "attn_us": dec_attn_us, "attn_bytes": dec_gather,
             "attn_frac": dec_gather / (dec_attn_us / 1e6) / 1e9 / hbm},
+        "decode_mtp_131k": {
+            "next_n": MTP_NEXT_N, "batch": DEC_BATCH, "step_us": mtp_step_us,
+            "us_per_token": mtp_step_us / MTP_NEXT_N,
+            "index_select_us": mtp_select_us, "attn_us": mtp_attn_us, "attn_bytes": dec_gather,
+            "attn_frac": dec_gather / (mtp_attn_us / 1e6) / 1e9 / hbm,
+            "note": "eager launches: one shared selection and one K/V gather for the 4 queries of a sequence"},
         "decode_262k": {
             "step_us": step262_us, "step_bytes": step262_bytes,
             "step_frac": step262_bytes / (step262_us / 1e6) / 1e9 / hbm,

@@ -453,13 +453,18 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
 // merge the pieces of each row under the even schedule: the piece at the row's first
 // tile (slot grid + row) and one per share that starts inside the row and holds tiles
 // (slot = share).  The rows' first tiles come from the attention kernel (CTA 0).
-__global__ void __launch_bounds__(256)
+static_assert(kMaxEvenCtas <= kD, "one thread per share of the even schedule");
+
+__global__ void __launch_bounds__(kD)
 even_combine_kernel(const float *__restrict__ ws, int grid, int64_t row_begin, int64_t rows,
                     __nv_bfloat16 *__restrict__ out, float *__restrict__ lse_out)
 {
+    __shared__ int s_slot[kMaxEvenCtas + 1];
+    __shared__ float s_l[kMaxEvenCtas + 1];
+    __shared__ int s_cnt[kD / 32];
     const int64_t rl = blockIdx.x;
     const int h = blockIdx.y;
-    const int d = threadIdx.x;
+    const int d = threadIdx.x, lane = d & 31, warp = d >> 5;
     const int64_t n_slots = (int64_t)grid + rows;
     const float *lbase = ws + (size_t)n_slots * kHQ * kD;
     const int64_t *tile_prefix = reinterpret_cast<const int64_t *>(ws + (size_t)n_slots * kHQ * (kD + 1));
@@ -470,22 +475,45 @@ even_combine_kernel(const float *__restrict__ ws, int grid, int64_t row_begin, i
         if (lse_out != nullptr && d == 0) lse_out[(row_begin + rl) * kHQ + h] = -INFINITY;
         return;
     }
+    // the row's pieces: its first-tile slot (grid + rl), then every share c >= c0 that
+    // starts inside the row and is not empty; share starts grow with c, so thread t tests
+    // share c0 + t (a row meets at most `grid` shares)
     auto share_start = [&](int64_t c) { return c * total / grid; };
-    auto piece = [&](int64_t c) { return share_start(c) > rs && share_start(c + 1) > share_start(c); };
     const int64_t c0 = rs * grid / total;
-    float mx = lbase[((int64_t)grid + rl) * kHQ + h];
-    for (int64_t c = c0; c < grid && share_start(c) < re; ++c)
-        if (piece(c)) mx = fmaxf(mx, lbase[c * kHQ + h]);
+    const int64_t c = c0 + d;
+    bool mine = false;
+    if (c < grid) {
+        const int64_t sc = share_start(c);
+        mine = sc < re && sc > rs && share_start(c + 1) > sc;
+    }
+    const uint32_t m = __ballot_sync(0xffffffffu, mine);
+    if (lane == 0) s_cnt[warp] = __popc(m);
+    if (d == 0) {
+        s_slot[0] = grid + (int)rl;
+        s_l[0] = lbase[((int64_t)grid + rl) * kHQ + h];
+    }
+    __syncthreads();
+    int before = 1, npieces = 1;
+#pragma unroll
+    for (int x = 0; x < kD / 32; ++x) {
+        before += x < warp ? s_cnt[x] : 0;
+        npieces += s_cnt[x];
+    }
+    if (mine) {
+        const int pos = before + __popc(m & ((1u << lane) - 1u));
+        s_slot[pos] = (int)c;
+        s_l[pos] = lbase[c * kHQ + h];
+    }
+    __syncthreads();
+    float mx = -INFINITY;
+    for (int p = 0; p < npieces; ++p) mx = fmaxf(mx, s_l[p]);
     float tot = 0.f, acc = 0.f;
-    auto add = [&](int64_t slot) {
-        const float l = lbase[slot * kHQ + h];
+    for (int p = 0; p < npieces; ++p) {
+        const float l = s_l[p];
         const float wgt = (l == -INFINITY) ? 0.f : __expf(l - mx);
         tot += wgt;
-        acc += wgt * __ldcs(ws + (slot * kHQ + h) * kD + d);
-    };
-    add((int64_t)grid + rl);
-    for (int64_t c = c0; c < grid && share_start(c) < re; ++c)
-        if (piece(c)) add(c);
+        acc += wgt * __ldcs(ws + ((int64_t)s_slot[p] * kHQ + h) * kD + d);
+    }
     *dst = __float2bfloat16_rn(tot > 0.f ? acc / tot : 0.f);
     if (lse_out != nullptr && d == 0) lse_out[(row_begin + rl) * kHQ + h] = mx + logf(tot);
 }

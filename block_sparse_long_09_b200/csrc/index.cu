@@ -58,11 +58,12 @@ struct IdxShared {
     uint32_t tmem_base;
     int abort_flag;
     alignas(16) float wq[kQRowsT];  // w[row, head]; read as float4
-    float theta[kTokTile];  // emit mode: the rows' thresholds
+    alignas(16) float theta[kTokTile];  // emit mode: the rows' thresholds; read as float4
     int seg_len[kEpiWarps][16];  // emit mode: each epilogue warp's list-segment lengths
 };
 
 static_assert(offsetof(IdxShared, wq) % 16 == 0, "the weight table is read as float4");
+static_assert(offsetof(IdxShared, theta) % 16 == 0, "the thresholds are read as float4");
 constexpr int kIdxSmem = kQBytes + kStages * kKcBytes + (int)sizeof(IdxShared) + 1024;
 static_assert(kIdxSmem <= 232448, "shared memory of one CTA");
 
@@ -276,36 +277,57 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 const int32_t b = n * kBM + b_local;
                 const int32_t col = kMode == kSample ? (n / step) * kBM + b_local : b;  // where the score goes
                 const bool col_ok = kMode == kEmit || col < cap;
+                // warp-uniform: all 16 rows belong to the segment and see every block of the tile
+                const bool full = vmask == 0xFFFFu && n * kBM + kBM <= (t0 >> rs);
                 float *p = row0 + col;
+                const uint32_t tbase = tmem + lane_addr + acc * kQRowsT + part * 64;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     float v[16];  // rows 16 part + 4 c .. + 3, heads 0..3
-                    tmem_ld16(tmem + lane_addr + acc * kQRowsT + part * 64 + c * 16, v);
+                    tmem_ld16(tbase + c * 16, v);
                     tmem_wait_ld();
+                    // the 4 rows' scores first (independent chains), then their use
+                    float sc[4];
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
-                        const int j = c * 4 + jj;
-                        const float4 wv = wq4[part * 16 + j];
-                        float s = wv.x * fmaxf(v[4 * jj], 0.f);
-                        s = fmaf(wv.y, fmaxf(v[4 * jj + 1], 0.f), s);
-                        s = fmaf(wv.z, fmaxf(v[4 * jj + 2], 0.f), s);
-                        s = fmaf(wv.w, fmaxf(v[4 * jj + 3], 0.f), s);
-                        const bool in = ((vmask >> j) & 1u) && b < ((t0 + j) >> rs) && col_ok;
-                        if (kMode != kEmit) {
-                            if (in) __stcs(p, s);
+                        const float4 wv = wq4[part * 16 + c * 4 + jj];
+                        float x = wv.x * fmaxf(v[4 * jj], 0.f);
+                        x = fmaf(wv.y, fmaxf(v[4 * jj + 1], 0.f), x);
+                        x = fmaf(wv.z, fmaxf(v[4 * jj + 2], 0.f), x);
+                        sc[jj] = fmaf(wv.w, fmaxf(v[4 * jj + 3], 0.f), x);
+                    }
+                    if (kMode != kEmit) {
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            const int j = c * 4 + jj;
+                            const bool in = full ? col_ok : (((vmask >> j) & 1u) && b < ((t0 + j) >> rs) && col_ok);
+                            if (in) __stcs(p, sc[jj]);
                             p += ld;
-                        } else {
-                            // append (S, b) to this warp's segment of row j's list when S >= theta:
-                            // the warp's hits take consecutive slots in ballot order
-                            const bool hit = in && s >= sh->theta[part * 16 + j];
-                            const uint32_t m = __ballot_sync(0xffffffffu, hit);
-                            if (m != 0u) {  // warp-uniform; most (row, tile) pairs have no hit
+                        }
+                    } else {
+                        // append (S, b) to this warp's segment of row j's list when S >= theta:
+                        // the warp's hits take consecutive slots in ballot order
+                        const float4 th4 = reinterpret_cast<const float4 *>(sh->theta)[part * 4 + c];
+                        const float th[4] = {th4.x, th4.y, th4.z, th4.w};
+                        uint32_t m[4], any = 0u;
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            const int j = c * 4 + jj;
+                            const bool in = full || (((vmask >> j) & 1u) && b < ((t0 + j) >> rs));
+                            m[jj] = __ballot_sync(0xffffffffu, in && sc[jj] >= th[jj]);
+                            any |= m[jj];
+                        }
+                        if (any != 0u) {  // warp-uniform
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj) {
+                                if (m[jj] == 0u) continue;  // warp-uniform
+                                const int j = c * 4 + jj;
                                 const int len = seg_len[j];
-                                const int pos = len + __popc(m & lt_mask);
-                                if (hit && pos < cap_q)
-                                    lbase[j * 4 * cap_q + pos] = make_uint2(__float_as_uint(s), (uint32_t)b);
-                                if (lane == 0) seg_len[j] = len + __popc(m);  // read again only after
-                            }                                                  // the tile's warp barrier
+                                const int pos = len + __popc(m[jj] & lt_mask);
+                                if (((m[jj] >> lane) & 1u) && pos < cap_q)
+                                    lbase[j * 4 * cap_q + pos] = make_uint2(__float_as_uint(sc[jj]), (uint32_t)b);
+                                if (lane == 0) seg_len[j] = len + __popc(m[jj]);  // read again only after
+                            }                                                      // the tile's warp barrier
                         }
                     }
                 }

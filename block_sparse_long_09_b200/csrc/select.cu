@@ -892,16 +892,37 @@ refine_select_kernel(const float *__restrict__ approx, int64_t ld, const __nv_bf
     // 2. the candidates W' = {b : approx_b >= theta_s - 2E} (with their approximate keys)
     const float lo_bound = theta_s - 2.f * e_row;
     const uint32_t lt_mask = (1u << lane) - 1u;
-    for (int j0 = 0; j0 < n; j0 += kRefThreads) {
-        const int j = j0 + tid;
-        const float x = j < n ? __ldg(srow + j) : -INFINITY;
-        const bool hit = j < n && x >= lo_bound;
-        const uint32_t m = __ballot_sync(0xffffffffu, hit);
-        int base = 0;
-        if (lane == 0 && m != 0u) base = atomicAdd(&wcount, __popc(m));
-        base = __shfl_sync(0xffffffffu, base, 0);
-        const int pos = base + __popc(m & lt_mask);
-        if (hit && pos < kRefCap) cand[pos] = make_uint2(order_key(x), (uint32_t)j);
+    {
+        // rows are 16-byte aligned with ld a multiple of 4: float4 groups, kRefUnroll of
+        // them in flight per thread; keys past n (inside the last group) are masked
+        constexpr int kRefUnroll = 4;
+        const int n4 = (n + 3) / 4;
+        const float4 *srow4 = reinterpret_cast<const float4 *>(srow);
+        for (int g0 = 0; g0 < n4; g0 += kRefThreads * kRefUnroll) {
+            float4 x4[kRefUnroll];
+#pragma unroll
+            for (int u = 0; u < kRefUnroll; ++u) {
+                const int g = g0 + u * kRefThreads + tid;
+                x4[u] = g < n4 ? __ldg(srow4 + g) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+            }
+#pragma unroll
+            for (int u = 0; u < kRefUnroll; ++u) {
+                const int g = g0 + u * kRefThreads + tid;
+                const float xs[4] = {x4[u].x, x4[u].y, x4[u].z, x4[u].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 4 * g + e;
+                    const bool hit = j < n && xs[e] >= lo_bound;
+                    const uint32_t m = __ballot_sync(0xffffffffu, hit);
+                    if (m == 0u) continue;  // warp-uniform
+                    int base = 0;
+                    if (lane == 0) base = atomicAdd(&wcount, __popc(m));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    const int pos = base + __popc(m & lt_mask);
+                    if (hit && pos < kRefCap) cand[pos] = make_uint2(order_key(xs[e]), (uint32_t)j);
+                }
+            }
+        }
     }
     __syncthreads();
     int nw = wcount;
