@@ -56,10 +56,12 @@ def _load():
             lib.qsa_oracle_index_scores.argtypes = [P, P, P, I64, I64, I, I, I, P, I64, P, I64]
             lib.qsa_oracle_select.argtypes = [P, I64, P, I64, I, P]
             lib.qsa_oracle_select_shared.argtypes = [P, I64, P, I64, I, I, I, P]
+            lib.qsa_oracle_rope.argtypes = [P, I64, I, P, I, D]
             lib.qsa_oracle_attend.argtypes = [P, P, P, P, I, I64, I64, I, I, I, I, D, P, I64, P, P]
             lib.qsa_oracle_dense.argtypes = [P, P, P, I64, I64, I, I, I, D, P, I64, P, P]
             lib.qsa_oracle_threads.restype = I
             for f in ("qsa_oracle_compress", "qsa_oracle_index_scores", "qsa_oracle_select", "qsa_oracle_select_shared",
+                      "qsa_oracle_rope",
                       "qsa_oracle_attend", "qsa_oracle_dense"):
                 getattr(lib, f).restype = None
             _lib = lib
@@ -104,12 +106,30 @@ def _rows(rows, Lq) -> np.ndarray:
     return rows
 
 
-def compress(k_idx, r: int = 4, normalise: bool = True, eps: float = 1e-6) -> np.ndarray:
-    """kc[b] = RMSNorm(mean of k_idx[b r .. b r + r - 1]) for complete blocks; fp64 [Lk // r, d]."""
+def rope(x, pos, rope_dims: int, base: float) -> np.ndarray:
+    """Partial RoPE of the last axis of x (fp64 copy): the first rope_dims dims rotate in
+    pairs (i, i + rope_dims / 2) by pos * base^(-2i / rope_dims); pos has one entry per
+    vector (x reshaped to [n, d])."""
+    xv = np.array(x, dtype=np.float64, copy=True)
+    d = xv.shape[-1]
+    flat = np.ascontiguousarray(xv.reshape(-1, d))
+    p = np.ascontiguousarray(np.asarray(pos, dtype=np.int64).reshape(-1))
+    assert p.size == flat.shape[0]
+    assert rope_dims % 2 == 0 and 0 <= rope_dims <= d
+    _load().qsa_oracle_rope(_ptr(flat), flat.shape[0], d, _ptr(p), int(rope_dims), float(base))
+    return flat.reshape(xv.shape)
+
+
+def compress(k_idx, r: int = 4, normalise: bool = True, eps: float = 1e-6, rope_dims: int = 0,
+             rope_base: float = 10000.0) -> np.ndarray:
+    """kc[b] = RMSNorm(mean of k_idx[b r .. b r + r - 1]) for complete blocks; fp64 [Lk // r, d].
+    rope_dims > 0: then the partial RoPE of the pooled key at its block's first position b r."""
     kb = _bits(k_idx)
     Lk, d = kb.shape
     out = np.zeros((Lk // r, d), dtype=np.float64)
     _load().qsa_oracle_compress(_ptr(kb), Lk, r, d, int(normalise), float(eps), _ptr(out))
+    if rope_dims > 0:
+        out = rope(out, np.arange(out.shape[0], dtype=np.int64) * r, rope_dims, rope_base)
     return out
 
 

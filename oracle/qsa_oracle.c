@@ -27,6 +27,9 @@
  *     (descending) then block index (ascending).  |Sel_t| = min(k, b_t + 1).
  *   - inside the own block only tokens j <= t are attended.
  *   - plain softmax with scale s (1/sqrt(256) for the model), no sink or cap.
+ *   - the partial RoPE of the pooled key (optional): after the pool and the
+ *     norm, the first rope_dims dims rotate in pairs (i, i + rope_dims/2) by
+ *     (b r) base^(-2i / rope_dims); queries arrive already rotated at t.
  *
  * All inputs that are bf16 on the device are passed here as raw 16-bit
  * patterns and widened exactly to double.  Every accumulation is fp64.
@@ -70,6 +73,33 @@ void qsa_oracle_compress(const uint16_t *k_idx, int64_t Lk, int r, int d,
             double inv = 1.0 / sqrt(ms + eps);
             for (int c = 0; c < d; ++c)
                 out[c] *= inv;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* [notes] section 6, the sentence before the pooled-key equation: the keys   */
+/* are average-pooled first and the partial RoPE is applied afterwards, so     */
+/* token representations of different rotation phases are never averaged.     */
+/* Readings (the pages give no dims, base or position): the first rope_dims   */
+/* dims rotate, in pairs (i, i + rope_dims/2), by the angle pos * base^(-2i /  */
+/* rope_dims); a pooled key sits at the position of its block's first token   */
+/* (b * r), a query at its own position t.  x is rotated in place:            */
+/*   x[i]     <- x[i] cos a - x[i + h] sin a                                   */
+/*   x[i + h] <- x[i] sin a + x[i + h] cos a                                   */
+/* ------------------------------------------------------------------------ */
+void qsa_oracle_rope(double *x, int64_t n, int d, const int64_t *pos, int rope_dims, double base)
+{
+    int h = rope_dims / 2;
+#pragma omp parallel for schedule(static)
+    for (int64_t v = 0; v < n; ++v) {
+        double *xv = x + v * d;
+        for (int i = 0; i < h; ++i) {
+            double a = (double)pos[v] * pow(base, -2.0 * (double)i / (double)rope_dims);
+            double c = cos(a), s = sin(a);
+            double x0 = xv[i], x1 = xv[i + h];
+            xv[i] = x0 * c - x1 * s;
+            xv[i + h] = x0 * s + x1 * c;
         }
     }
 }

@@ -413,3 +413,67 @@ def test_select_shared_brute_force(next_n):
         want += [-1] * (k - len(want))
         got = oracle.select_shared(sc, [L], next_n, k)[0].tolist()
         assert got == want, (L, k, next_n, sc, got, want)
+
+
+# ---------------------------------------------------------------- partial RoPE of the pooled key
+
+def _rope_cases():
+    out = []
+    for line in open(os.path.join(GOLDEN, "rope_hand.txt")):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        head, x, want = (part.split() for part in line.split("|"))
+        out.append((int(head[0]), int(head[1]), float(head[2]), np.array(x, float), np.array(want, float)))
+    return out
+
+
+def test_rope_hand_fixture():
+    cases = _rope_cases()
+    assert len(cases) == 2
+    for pos, rd, base, x, want in cases:
+        np.testing.assert_allclose(oracle.rope(x[None], [pos], rd, base)[0], want, rtol=0, atol=1e-12)
+
+
+def test_rope_identity_cases_and_norm():
+    g = np.random.default_rng(11)
+    x = g.standard_normal((9, 128))
+    np.testing.assert_array_equal(oracle.rope(x, np.zeros(9, np.int64), 64, 1e4), x)  # position 0
+    np.testing.assert_array_equal(oracle.rope(x, np.arange(9) * 4, 0, 1e4), x)       # no rotated dims
+    y = oracle.rope(x, np.arange(9) * 1000 + 7, 64, 1e4)
+    np.testing.assert_array_equal(y[:, 64:], x[:, 64:])                              # only the first 64 dims
+    np.testing.assert_allclose(np.linalg.norm(y[:, :64], axis=1), np.linalg.norm(x[:, :64], axis=1), rtol=1e-12)
+
+
+def test_rope_dot_depends_on_relative_position_only():
+    # <R(p) a, R(s) b> = <R(p + D) a, R(s + D) b>: a wrong pairing, sign or frequency index
+    # breaks either this or the hand fixture
+    g = np.random.default_rng(12)
+    a, b = g.standard_normal((2, 64))
+    for p, s, D in [(3, 0, 5), (1000, 17, 12345), (40, 40, 262140)]:
+        d0 = oracle.rope(a[None], [p], 64, 1e4)[0] @ oracle.rope(b[None], [s], 64, 1e4)[0]
+        d1 = oracle.rope(a[None], [p + D], 64, 1e4)[0] @ oracle.rope(b[None], [s + D], 64, 1e4)[0]
+        assert abs(d0 - d1) <= 1e-9 * (np.abs(a) @ np.abs(b))
+    # and it does depend on the offset p - s
+    d0 = oracle.rope(a[None], [5], 64, 1e4)[0] @ oracle.rope(b[None], [0], 64, 1e4)[0]
+    d1 = oracle.rope(a[None], [6], 64, 1e4)[0] @ oracle.rope(b[None], [0], 64, 1e4)[0]
+    assert abs(d0 - d1) > 1e-6
+
+
+def test_compress_rope_pools_before_rotating():
+    # the page's order: average-pool the r keys, then rotate the pooled key at b r; it differs
+    # from pooling keys that were each rotated at their own position
+    g = torch.Generator().manual_seed(13)
+    k = torch.randn((64, 128), generator=g).to(torch.bfloat16)
+    kc = oracle.compress(k, 4, rope_dims=64, rope_base=1e4)
+    plain = oracle.compress(k, 4)
+    np.testing.assert_allclose(kc, oracle.rope(plain, np.arange(16) * 4, 64, 1e4), rtol=0, atol=1e-12)
+    kk = k.double().numpy()
+    per_token = oracle.rope(kk, np.arange(64), 64, 1e4).reshape(16, 4, 128).mean(axis=1)
+    per_token /= np.sqrt((per_token ** 2).mean(axis=1, keepdims=True) + 1e-6)
+    assert np.abs(per_token - kc).max() > 1e-3
+    # RMSNorm (unit gain) commutes with the rotation: rotating before or after the norm agrees
+    mean = kk.reshape(16, 4, 128).mean(axis=1)
+    rot_then_norm = oracle.rope(mean, np.arange(16) * 4, 64, 1e4)
+    rot_then_norm /= np.sqrt((rot_then_norm ** 2).mean(axis=1, keepdims=True) + 1e-6)
+    np.testing.assert_allclose(kc, rot_then_norm, rtol=0, atol=1e-12)
