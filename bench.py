@@ -1,7 +1,7 @@
 """QSA benchmark: prefill tokens/s at 262,144 context and decode latency at 131,072.
 
 One step = one pass of the whole QSA hot path on synthetic inputs resident in HBM:
-  prefill  batch 1, n = 262,144: compress -> (index -> select) per 16,384-row chunk
+  prefill  batch 1, n = 262,144: compress -> (index -> select) per chunk of query rows (--chunk-rows)
            -> sparse GQA attention                            (value = tokens/s of this part)
   decode   batch 64, every cache 131,072 tokens: refresh of the last compressed block,
            one-row indexer, top-512 select, split-K sparse attention (the "decode" object)
@@ -152,7 +152,8 @@ def run_qsa(args, rank, world, device):
     seeds = ranks.rank_seeds(rank)
     x = inputs.make_prefill([N_PREFILL], seed=seeds["prefill"], device=device)
     cfg = qsa.default_config(budget_blocks=BUDGET)
-    pre = qsa.Prefill([N_PREFILL], chunk_rows=CHUNK, cfg=cfg, device=device)
+    chunk = args.chunk_rows
+    pre = qsa.Prefill([N_PREFILL], chunk_rows=chunk, cfg=cfg, device=device)
     o = torch.empty_like(x.q)
 
     d = inputs.make_decode(DEC_BATCH, DEC_LEN, None, seed=seeds["decode"], device=device)
@@ -165,7 +166,7 @@ def run_qsa(args, rank, world, device):
                          refresh_blocks=last_blk, cfg=cfg, graph=True)
     dec_o = dec.o
     stream = torch.cuda.current_stream()
-    n_chunks = (N_PREFILL + CHUNK - 1) // CHUNK
+    n_chunks = (N_PREFILL + chunk - 1) // chunk
 
     ev = {k: [] for k in ("p0", "p1", "a0", "a1", "d0", "d1", "ix")}
 
@@ -178,8 +179,8 @@ def run_qsa(args, rank, world, device):
             e["p0"].record(stream)
         # compress, then the fused index -> select per chunk (qsa.Prefill.index_select, with events)
         qsa.compress_keys(x.k_idx, pre.cu, pre.cu_blocks, kc=pre.kc, cfg=cfg)
-        for r0 in range(0, N_PREFILL, CHUNK):
-            r1 = min(N_PREFILL, r0 + CHUNK)
+        for r0 in range(0, N_PREFILL, chunk):
+            r1 = min(N_PREFILL, r0 + chunk)
             e0, e1 = (mk(), mk()) if record else (None, None)
             if record:
                 e0.record(stream)
@@ -414,7 +415,8 @@ def run_qsa(args, rank, world, device):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) activations, U(0,1) indexer weights)",
-        "config": {"workload": "QSA layer: prefill batch 1 n=262144 (16384-row chunks) + decode batch 64 ctx 131072",
+        "config": {"workload": "QSA layer: prefill batch 1 n=262144 (%d-row chunks) + decode batch 64 ctx 131072"
+                                % chunk,
                    "budget_blocks": BUDGET, "r": 4, "heads": "24q/2kv/256, indexer 4/128",
                    "prefill_ms": prefill_ms, "attn_prefill_ms": attn_ms, "l2": "inputs > L2, no flush",
                    "parallelism": "independent layer per rank" if world > 1 else "1 GPU"},
@@ -543,9 +545,18 @@ def run_profile_case(case: str, reps: int = 3):
             pre.select_chunk(x.q_idx, x.w, r0, n)
             if case == "attn":
                 qsa.sparse_attn_prefill(x.q, x.k, x.v, pre.sel, pre.cu, pre.cu, r0, n, cfg=cfg, max_len_k=n)
-    elif case in ("decode", "decode131k"):
-        # decode steps of batch 64 (16384-token caches: small; 131072: the benchmark's, 17 GB)
-        L = 16384 if case == "decode" else DEC_LEN
+    elif case == "mtp":
+        # multi-token decode (next_n = 4) at batch 64 with 65536-token caches
+        L = 65536
+        d = inputs.make_decode(DEC_BATCH, L, None, seed=2, device=dev, next_n=MTP_NEXT_N)
+        kc = qsa.compress_keys(d.k_idx, d.cu_seqlens_k, d.cu_blocks, n_blocks=int(d.cu_blocks[-1]), cfg=cfg)
+        for _ in range(reps):
+            sel = qsa.index_select_mtp(d.q_idx, d.w, kc, d.cu_seqlens_k, d.cu_blocks, MTP_NEXT_N, L, cfg=cfg)
+            qsa.sparse_attn_decode_mtp(d.q, d.k_cache, d.v_cache, d.cu_seqlens_k, sel, cfg=cfg)
+    elif case in ("decode", "decode64k", "decode131k"):
+        # decode steps of batch 64 (16384-token caches: small; 65536: kc hi planes of 268 MB,
+        # above L2, 5.5 GB on the device; 131072: the benchmark's, 11 GB)
+        L = {"decode": 16384, "decode64k": 65536, "decode131k": DEC_LEN}[case]
         d = inputs.make_decode(DEC_BATCH, L, None, seed=1, device=dev)
         cu_q = torch.arange(DEC_BATCH + 1, dtype=torch.int32, device=dev)
         kc = qsa.compress_keys(d.k_idx, d.cu_seqlens_k, d.cu_blocks, n_blocks=int(d.cu_blocks[-1]), cfg=cfg)
@@ -566,13 +577,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="qsa", choices=["qsa", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--chunk-rows", type=int, default=CHUNK,
+                    help="query rows per fused index -> select launch of the prefill")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", dest="dense", action="store_false",
                     help="skip the dense causal-attention comparison")
     ap.add_argument("--extra-configs", action="store_true",
                     help="also time the other workloads (peaked 2 x 65536 prefill, decode at 262144 and mixed "
                          "lengths) and print them on stderr")
-    ap.add_argument("--profile-case", choices=["attn", "index", "select", "index_select", "decode", "decode131k"],
+    ap.add_argument("--profile-case", choices=["attn", "index", "select", "index_select", "decode", "decode64k", "decode131k", "mtp"],
                     default=None,
                     help="run one small case for an ncu capture and exit")
     args = ap.parse_args()

@@ -28,6 +28,44 @@ constexpr uint32_t kDecOCol = 2 * kDecSBuf;             // O^T after two chunk b
 constexpr uint32_t kDecTmemCols = 512;
 static_assert(kDecOCol + 64 <= kDecTmemCols, "two chunks of S and O^T fit in TMEM");
 
+// The producer's TMA issue of one ring slot: lane 0 waits for the slot and arms its
+// barrier, lanes 0..15 each load one block (its first token row in the packed cache,
+// or through the block table; -8 reads zeros).  Called by the whole warp.
+static __device__ __noinline__ bool dec_issue(const CUtensorMap *map, AttShared *sh, uint8_t *sSlot,
+                                              uint32_t *slot_it, volatile int *abort_flag, int lane,
+                                              int64_t tok_base, int64_t row, int32_t blk, int r,
+                                              const int32_t *block_table, int page_size, int max_pages,
+                                              int64_t num_pages)
+{
+    const uint32_t st = *slot_it % kNSlot, round = *slot_it / kNSlot;
+    bool good = true;
+    if (lane == 0) {
+        good = mbar_wait(&sh->slot_empty[st], (round & 1) ^ 1, abort_flag);
+        if (good) mbar_arrive_expect_tx(&sh->slot_full[st], kSlotBytes);
+    }
+    good = __shfl_sync(0xffffffffu, good, 0);
+    if (!good) return false;
+    if (lane < kBlkTile) {
+        int32_t y = -8;
+        if (blk >= 0) {
+            const int64_t tok = (int64_t)blk * r;  // position in the sequence
+            if (block_table == nullptr) {
+                y = (int32_t)((tok_base + tok) * kHKV);
+            } else {
+                const int64_t j = tok / page_size;
+                const int32_t page = j < max_pages ? __ldg(block_table + row * max_pages + j) : -1;
+                if (page >= 0 && page < num_pages)
+                    y = (int32_t)(((int64_t)page * page_size + tok % page_size) * kHKV);
+                else
+                    set_device_status(QSA_ERR_DEVICE_CHECK);
+            }
+        }
+        tma_load_3d(sSlot + st * kSlotBytes + lane * kBlockBytes, map, &sh->slot_full[st], 0, y, 0);
+    }
+    ++*slot_it;
+    return true;
+}
+
 __global__ void __launch_bounds__(kAttThreads, 1)
 sparse_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                      const __grid_constant__ CUtensorMap map_v, const int32_t *__restrict__ sel,
@@ -91,35 +129,11 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
         }
         uint32_t slot_it = 0, q_it = 0;
         bool ok = true;
+        // one call site per ring slot use, 21 per chunk pair: a real call keeps the
+        // producer's code small (the kernel's warps share the instruction cache)
         auto issue = [&](const CUtensorMap *map, const RowInfo &ri, int32_t blk) -> bool {
-            const uint32_t st = slot_it % kNSlot, round = slot_it / kNSlot;
-            bool good = true;
-            if (lane == 0) {
-                good = mbar_wait(&sh->slot_empty[st], (round & 1) ^ 1, abort_flag);
-                if (good) mbar_arrive_expect_tx(&sh->slot_full[st], kSlotBytes);
-            }
-            good = __shfl_sync(0xffffffffu, good, 0);
-            if (!good) return false;
-            if (lane < kBlkTile) {
-                // the block's first token row (token, group) in the cache; -8 reads zeros
-                int32_t y = -8;
-                if (blk >= 0) {
-                    const int64_t tok = (int64_t)blk * r;  // position in the sequence
-                    if (block_table == nullptr) {
-                        y = (int32_t)((ri.tok_base + tok) * kHKV);
-                    } else {
-                        const int64_t j = tok / page_size;
-                        const int32_t page = j < max_pages ? __ldg(block_table + ri.row * max_pages + j) : -1;
-                        if (page >= 0 && page < num_pages)
-                            y = (int32_t)(((int64_t)page * page_size + tok % page_size) * kHKV);
-                        else
-                            set_device_status(QSA_ERR_DEVICE_CHECK);
-                    }
-                }
-                tma_load_3d(sSlot + st * kSlotBytes + lane * kBlockBytes, map, &sh->slot_full[st], 0, y, 0);
-            }
-            ++slot_it;
-            return true;
+            return dec_issue(map, sh, sSlot, &slot_it, abort_flag, lane, ri.tok_base, ri.row, blk, r, block_table,
+                             page_size, max_pages, num_pages);
         };
         for (int64_t item = 0; ok && item < n_items; ++item) {
             const RowInfo ri = row_info_even(item, sh, cu_k, row_begin, kb, r);
@@ -290,7 +304,7 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
                 float tm[kGrp];
 #pragma unroll
                 for (int h = 0; h < kGrp; ++h) tm[h] = -INFINITY;
-#pragma unroll
+#pragma unroll 1
                 for (int u = 0; u < kCT; ++u) {
                     if (u < len) {
                         float s[kHQ];
@@ -366,7 +380,7 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
 #pragma unroll
                 for (int h = 0; h < kGrp; ++h) mc[h] = (g ? m[kGrp + h] : m[h]) * c2;
                 // phase B: P = exp(S - m) tile by tile, for the PVs as their V lands
-#pragma unroll
+#pragma unroll 1
                 for (int u = 0; u < kCT; ++u) {
                     if (!ok || u >= len) continue;
                     const uint32_t pb = p_it % kNP, pround = p_it / kNP;

@@ -447,18 +447,35 @@ __global__ void __launch_bounds__(kD)
 mtp_combine_kernel(const float *__restrict__ ws, int64_t n_items, int nsplit, int next_n,
                    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse_out)
 {
+    constexpr int kU = 8;  // splits whose loads are in flight together
     const int64_t s = blockIdx.x;
     const int R = blockIdx.y;  // < next_n * 24
     const int d = threadIdx.x;
     const float *lp = ws + (size_t)n_items * kMRows * kD + (s * nsplit) * kMRows + R;
+    const float *pp = ws + ((s * nsplit) * kMRows + R) * kD + d;
     float mx = -INFINITY;
-    for (int sp = 0; sp < nsplit; ++sp) mx = fmaxf(mx, lp[sp * kMRows]);
+    for (int sp0 = 0; sp0 < nsplit; sp0 += kU) {
+        float l[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) l[u] = sp0 + u < nsplit ? lp[(sp0 + u) * kMRows] : -INFINITY;
+#pragma unroll
+        for (int u = 0; u < kU; ++u) mx = fmaxf(mx, l[u]);
+    }
     float tot = 0.f, acc = 0.f;
-    for (int sp = 0; sp < nsplit; ++sp) {
-        const float l = lp[sp * kMRows];
-        const float wgt = (l == -INFINITY) ? 0.f : __expf(l - mx);
-        tot += wgt;
-        acc += wgt * __ldcs(ws + ((s * nsplit + sp) * kMRows + R) * kD + d);
+    for (int sp0 = 0; sp0 < nsplit; sp0 += kU) {
+        float l[kU], o[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const bool in = sp0 + u < nsplit;
+            l[u] = in ? lp[(sp0 + u) * kMRows] : -INFINITY;
+            o[u] = in ? __ldcs(pp + (size_t)(sp0 + u) * kMRows * kD) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {  // the splits in order, as one sequential sum
+            const float wgt = (l[u] == -INFINITY) ? 0.f : __expf(l[u] - mx);
+            tot += wgt;
+            acc += wgt * o[u];
+        }
     }
     const int qi = R / kHQ, h = R % kHQ;
     out[((s * next_n + qi) * kHQ + h) * kD + d] = __float2bfloat16_rn(tot > 0.f ? acc / tot : 0.f);
