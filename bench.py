@@ -33,7 +33,7 @@ N_PREFILL = 262144
 DEC_BATCH = 64
 DEC_LEN = 131072
 MTP_NEXT_N = 4       # queries per sequence of the multi-token-prediction decode step
-CHUNK = 16384
+CHUNK = 65536          # query rows per fused index -> select launch (1024 row tiles: 7 waves on 148 SMs)
 BUDGET = 512
 METRIC = "QSA prefill tokens/s at 262K ctx; decode µs/token at 128K; % of roofline"
 

@@ -132,9 +132,19 @@ qsa_status check_config(const qsa_config *c)
         c->kv_chunk_blocks < 0)
         return QSA_ERR_INVALID_ARG;
     if (c->r != 4 || c->budget_blocks > 2048 || c->n_heads_q != 24 || c->n_heads_kv != 2 || c->head_dim != 256 ||
-        c->n_heads_idx != 4 || c->idx_dim != 128 || (c->flags & ~QSA_COMPRESS_NO_NORM) != 0)
+        c->n_heads_idx != 4 || c->idx_dim != 128 || (c->flags & ~(QSA_COMPRESS_NO_NORM | QSA_INDEX_ROPE)) != 0)
         return QSA_ERR_UNSUPPORTED;
+    if ((c->flags & QSA_INDEX_ROPE) != 0 &&
+        (c->rope_dims < 8 || c->rope_dims > c->idx_dim || c->rope_dims % 8 != 0 || !(c->rope_base > 1.f) ||
+         !(c->rope_base < 3.0e38f)))
+        return QSA_ERR_INVALID_ARG;
     return QSA_OK;
+}
+
+// the pooled keys' partial RoPE of a config (dims 0: none)
+qsa::RopeSpec rope_of(const qsa_config *c)
+{
+    return (c->flags & QSA_INDEX_ROPE) != 0 ? qsa::RopeSpec{c->rope_dims, c->rope_base} : qsa::RopeSpec{0, 0.f};
 }
 
 qsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA; }
@@ -171,6 +181,8 @@ void qsa_config_init(qsa_config *cfg)
     cfg->rms_eps = 1e-6f;
     cfg->flags = 0u;
     cfg->kv_chunk_blocks = 0;
+    cfg->rope_dims = 64;
+    cfg->rope_base = 10000.f;
 }
 
 int32_t qsa_version(void) { return 100; }
@@ -256,7 +268,22 @@ qsa_status qsa_compress_keys(const qsa_config *cfg, const qsa_bf16 *k_idx, const
     if (blk_begin != nullptr && max_new_blocks <= 0) return QSA_ERR_INVALID_ARG;
     return cuda_status(launch_compress(bf(k_idx), cu_seqlens_k, cu_blocks, batch, total_k, blk_begin,
                                        max_new_blocks, cfg->r, (cfg->flags & QSA_COMPRESS_NO_NORM) == 0,
-                                       cfg->rms_eps, bf(kc), static_cast<cudaStream_t>(stream)));
+                                       cfg->rms_eps, bf(kc), static_cast<cudaStream_t>(stream), rope_of(cfg)));
+}
+
+qsa_status qsa_rope_queries(const qsa_config *cfg, qsa_bf16 *q_idx, const int32_t *cu_seqlens_q,
+                            const int32_t *cu_seqlens_k, int32_t batch, int64_t total_q, void *stream)
+{
+    const qsa::NvtxRange nvtx_range("qsa_rope_queries");
+    qsa_status st = check_config(cfg);
+    if (st != QSA_OK) return st;
+    if ((cfg->flags & QSA_INDEX_ROPE) == 0) return QSA_ERR_INVALID_ARG;
+    if (batch <= 0 || total_q < 0 || cu_seqlens_q == nullptr || cu_seqlens_k == nullptr) return QSA_ERR_INVALID_ARG;
+    if (total_q == 0) return QSA_OK;
+    if (q_idx == nullptr || !al16(q_idx)) return QSA_ERR_INVALID_ARG;
+    __nv_bfloat16 *q = reinterpret_cast<__nv_bfloat16 *>(q_idx);
+    return cuda_status(launch_rope_queries(q, q, cu_seqlens_q, cu_seqlens_k, batch, total_q, cfg->n_heads_idx,
+                                           rope_of(cfg), static_cast<cudaStream_t>(stream)));
 }
 
 qsa_status qsa_index_scores(const qsa_config *cfg, const qsa_bf16 *q_idx, const float *w, const qsa_bf16 *kc,
@@ -338,7 +365,7 @@ qsa_status qsa_compress_keys_paged(const qsa_config *cfg, const qsa_bf16 *k_idx_
     PagedArgs p{num_pages, page_size, block_table, max_pages, cu_seqlens_k, batch, cfg->r};
     return cuda_status(launch_compress_paged(p, bf(k_idx_pages), bf(kc_pages), blk_begin, max_new_blocks, max_len_k,
                                              (cfg->flags & QSA_COMPRESS_NO_NORM) == 0, cfg->rms_eps,
-                                             static_cast<cudaStream_t>(stream)));
+                                             static_cast<cudaStream_t>(stream), rope_of(cfg)));
 }
 
 qsa_status qsa_index_select_paged(const qsa_config *cfg, const qsa_bf16 *q_idx, const float *w,

@@ -447,39 +447,45 @@ __global__ void __launch_bounds__(kD)
 mtp_combine_kernel(const float *__restrict__ ws, int64_t n_items, int nsplit, int next_n,
                    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse_out)
 {
-    constexpr int kU = 8;  // splits whose loads are in flight together
+    __shared__ float s_wgt[kD];  // the splits' weights exp(lse_sp - max), one per split (nsplit <= kD)
+    __shared__ float s_mx, s_tot;
     const int64_t s = blockIdx.x;
     const int R = blockIdx.y;  // < next_n * 24
     const int d = threadIdx.x;
     const float *lp = ws + (size_t)n_items * kMRows * kD + (s * nsplit) * kMRows + R;
     const float *pp = ws + ((s * nsplit) * kMRows + R) * kD + d;
-    float mx = -INFINITY;
-    for (int sp0 = 0; sp0 < nsplit; sp0 += kU) {
-        float l[kU];
+    if (d < 32) {  // warp 0: the max and the weights of the splits, in split order
+        float mx = -INFINITY;
+        for (int sp = d; sp < nsplit; sp += 32) mx = fmaxf(mx, lp[sp * kMRows]);
 #pragma unroll
-        for (int u = 0; u < kU; ++u) l[u] = sp0 + u < nsplit ? lp[(sp0 + u) * kMRows] : -INFINITY;
-#pragma unroll
-        for (int u = 0; u < kU; ++u) mx = fmaxf(mx, l[u]);
-    }
-    float tot = 0.f, acc = 0.f;
-    for (int sp0 = 0; sp0 < nsplit; sp0 += kU) {
-        float l[kU], o[kU];
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            const bool in = sp0 + u < nsplit;
-            l[u] = in ? lp[(sp0 + u) * kMRows] : -INFINITY;
-            o[u] = in ? __ldcs(pp + (size_t)(sp0 + u) * kMRows * kD) : 0.f;
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        for (int sp = d; sp < nsplit; sp += 32) {
+            const float l = lp[sp * kMRows];
+            s_wgt[sp] = (l == -INFINITY) ? 0.f : __expf(l - mx);
         }
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {  // the splits in order, as one sequential sum
-            const float wgt = (l[u] == -INFINITY) ? 0.f : __expf(l[u] - mx);
-            tot += wgt;
-            acc += wgt * o[u];
+        __syncwarp();
+        if (d == 0) {
+            float tot = 0.f;
+            for (int sp = 0; sp < nsplit; ++sp) tot += s_wgt[sp];
+            s_mx = mx;
+            s_tot = tot;
         }
     }
+    __syncthreads();
+    constexpr int kU = 8;  // partial outputs in flight per thread
+    float acc = 0.f;
+    for (int sp0 = 0; sp0 < nsplit; sp0 += kU) {
+        float o[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) o[u] = sp0 + u < nsplit ? __ldcs(pp + (size_t)(sp0 + u) * kMRows * kD) : 0.f;
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+            if (sp0 + u < nsplit) acc += s_wgt[sp0 + u] * o[u];
+    }
+    const float tot = s_tot;
     const int qi = R / kHQ, h = R % kHQ;
     out[((s * next_n + qi) * kHQ + h) * kD + d] = __float2bfloat16_rn(tot > 0.f ? acc / tot : 0.f);
-    if (lse_out != nullptr && d == 0) lse_out[(s * next_n + qi) * kHQ + h] = tot > 0.f ? mx + logf(tot) : -INFINITY;
+    if (lse_out != nullptr && d == 0) lse_out[(s * next_n + qi) * kHQ + h] = tot > 0.f ? s_mx + logf(tot) : -INFINITY;
 }
 
 }  // namespace
@@ -489,6 +495,7 @@ int mtp_nsplit(int batch, int kb)
     const int tiles = (kb + kBlkTile - 1) / kBlkTile;
     int ns = (2 * num_sms() + batch - 1) / (batch > 0 ? batch : 1);
     if (ns > tiles) ns = tiles;
+    if (ns > kD) ns = kD;  // the merge keeps one weight per split in shared memory
     return ns > 0 ? ns : 1;
 }
 

@@ -26,7 +26,7 @@ __global__ void __launch_bounds__(kCompressWarps * 32)
 compress_kernel(const __nv_bfloat16 *__restrict__ k_idx, const int32_t *__restrict__ cu_k,
                 const int32_t *__restrict__ cu_blocks, int batch, int64_t n_items,
                 const int32_t *__restrict__ blk_begin, int max_new, int r, int normalise,
-                float eps, __nv_bfloat16 *__restrict__ kc)
+                float eps, __nv_bfloat16 *__restrict__ kc, const RopeSpec rope)
 {
     const int lane = threadIdx.x & 31;
     const int64_t warp_global = (int64_t)blockIdx.x * kCompressWarps + (threadIdx.x >> 5);
@@ -78,6 +78,7 @@ compress_kernel(const __nv_bfloat16 *__restrict__ k_idx, const int32_t *__restri
 #pragma unroll
             for (int c = 0; c < 4; ++c) m[c] *= inv;
         }
+        rope_rotate4(m, lane, b * r, rope);  // the pooled key at its block's first position
         __nv_bfloat162 h0 = __floats2bfloat162_rn(m[0], m[1]);
         __nv_bfloat162 h1 = __floats2bfloat162_rn(m[2], m[3]);
         const float2 fh0 = __bfloat1622float2(h0), fh1 = __bfloat1622float2(h1);
@@ -94,11 +95,55 @@ compress_kernel(const __nv_bfloat16 *__restrict__ k_idx, const int32_t *__restri
     }
 }
 
+// partial RoPE of indexer query rows: one warp per (row, head), 4 dims per lane
+constexpr int kRopeWarps = 8;
+
+__global__ void __launch_bounds__(kRopeWarps * 32)
+rope_queries_kernel(const __nv_bfloat16 *__restrict__ q_in, __nv_bfloat16 *__restrict__ q_out,
+                    const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k, int batch,
+                    int64_t total_q, int heads, const RopeSpec rope)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t n_items = total_q * heads;
+    for (int64_t item = (int64_t)blockIdx.x * kRopeWarps + (threadIdx.x >> 5); item < n_items;
+         item += (int64_t)gridDim.x * kRopeWarps) {
+        const int64_t i = item / heads;
+        const int s = find_seq(cu_q, batch, i);
+        const int64_t Lq = (int64_t)cu_q[s + 1] - cu_q[s], Lk = (int64_t)cu_k[s + 1] - cu_k[s];
+        const int64_t t = (Lk - Lq) + (i - cu_q[s]);
+        const int64_t off = item * 128 + lane * 4;
+        const uint2 raw = *reinterpret_cast<const uint2 *>(q_in + off);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+        const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+        float m[4] = {a.x, a.y, c.x, c.y};
+        rope_rotate4(m, lane, t, rope);
+        __nv_bfloat162 o0 = __floats2bfloat162_rn(m[0], m[1]), o1 = __floats2bfloat162_rn(m[2], m[3]);
+        uint2 w;
+        w.x = *reinterpret_cast<uint32_t *>(&o0);
+        w.y = *reinterpret_cast<uint32_t *>(&o1);
+        *reinterpret_cast<uint2 *>(q_out + off) = w;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_rope_queries(const __nv_bfloat16 *q_idx_in, __nv_bfloat16 *q_idx, const int32_t *cu_q,
+                                const int32_t *cu_k, int batch, int64_t total_q, int heads, const RopeSpec &rope,
+                                cudaStream_t stream)
+{
+    const int64_t n_items = total_q * heads;
+    if (n_items <= 0) return cudaSuccess;
+    int64_t grid = (n_items + kRopeWarps - 1) / kRopeWarps;
+    if (grid > 148 * 16) grid = 148 * 16;
+    rope_queries_kernel<<<(unsigned)grid, kRopeWarps * 32, 0, stream>>>(q_idx_in, q_idx, cu_q, cu_k, batch,
+                                                                        total_q, heads, rope);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_compress(const __nv_bfloat16 *k_idx, const int32_t *cu_k, const int32_t *cu_blocks,
                             int batch, int64_t total_k, const int32_t *blk_begin, int max_new, int r,
-                            bool normalise, float eps, __nv_bfloat16 *kc, cudaStream_t stream)
+                            bool normalise, float eps, __nv_bfloat16 *kc, cudaStream_t stream,
+                            const RopeSpec &rope)
 {
     int64_t n_items = blk_begin ? (int64_t)batch * max_new : total_k / r;
     if (n_items <= 0) return cudaSuccess;
@@ -106,7 +151,7 @@ cudaError_t launch_compress(const __nv_bfloat16 *k_idx, const int32_t *cu_k, con
     const int64_t cap = 148 * 16;
     if (grid > cap) grid = cap;
     compress_kernel<<<(unsigned)grid, kCompressWarps * 32, 0, stream>>>(
-        k_idx, cu_k, cu_blocks, batch, n_items, blk_begin, max_new, r, normalise ? 1 : 0, eps, kc);
+        k_idx, cu_k, cu_blocks, batch, n_items, blk_begin, max_new, r, normalise ? 1 : 0, eps, kc, rope);
     return cudaGetLastError();
 }
 

@@ -29,6 +29,8 @@
 // rows with coalesced 8-byte loads, keeps its 4 heads' query slice in
 // registers, and reduces the 32 (block, head) partial dots with a 5-step
 // butterfly reduce-scatter.
+#include <type_traits>
+
 #include "kernels.cuh"
 
 namespace qsa {
@@ -281,56 +283,70 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 const bool full = vmask == 0xFFFFu && n * kBM + kBM <= (t0 >> rs);
                 float *p = row0 + col;
                 const uint32_t tbase = tmem + lane_addr + acc * kQRowsT + part * 64;
+                // one tile of this thread (kc block b, 16 rows): the whole-tile case is compiled
+                // apart, without the per-row causal test
+                auto tile = [&](auto full_tag) {
+                    constexpr bool kFull = decltype(full_tag)::value;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    float v[16];  // rows 16 part + 4 c .. + 3, heads 0..3
-                    tmem_ld16(tbase + c * 16, v);
-                    tmem_wait_ld();
-                    // the 4 rows' scores first (independent chains), then their use
-                    float sc[4];
+                    for (int c = 0; c < 4; ++c) {
+                        float v[16];  // rows 16 part + 4 c .. + 3, heads 0..3
+                        tmem_ld16(tbase + c * 16, v);
+                        tmem_wait_ld();
+                        // the 4 rows' scores, two rows per packed fp32x2 operation (each lane of
+                        // an fp32x2 op rounds as the scalar op does: the same bits)
+                        float sc[4];
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const float4 wv = wq4[part * 16 + c * 4 + jj];
-                        float x = wv.x * fmaxf(v[4 * jj], 0.f);
-                        x = fmaf(wv.y, fmaxf(v[4 * jj + 1], 0.f), x);
-                        x = fmaf(wv.z, fmaxf(v[4 * jj + 2], 0.f), x);
-                        sc[jj] = fmaf(wv.w, fmaxf(v[4 * jj + 3], 0.f), x);
-                    }
-                    if (kMode != kEmit) {
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) {
-                            const int j = c * 4 + jj;
-                            const bool in = full ? col_ok : (((vmask >> j) & 1u) && b < ((t0 + j) >> rs) && col_ok);
-                            if (in) __stcs(p, sc[jj]);
-                            p += ld;
+                        for (int jp = 0; jp < 4; jp += 2) {
+                            const float4 wa = wq4[part * 16 + c * 4 + jp], wb = wq4[part * 16 + c * 4 + jp + 1];
+                            const float *va = v + 4 * jp, *vb = v + 4 * jp + 4;
+                            float2 x = __fmul2_rn(make_float2(wa.x, wb.x),
+                                                  make_float2(fmaxf(va[0], 0.f), fmaxf(vb[0], 0.f)));
+                            x = __ffma2_rn(make_float2(wa.y, wb.y), make_float2(fmaxf(va[1], 0.f), fmaxf(vb[1], 0.f)), x);
+                            x = __ffma2_rn(make_float2(wa.z, wb.z), make_float2(fmaxf(va[2], 0.f), fmaxf(vb[2], 0.f)), x);
+                            x = __ffma2_rn(make_float2(wa.w, wb.w), make_float2(fmaxf(va[3], 0.f), fmaxf(vb[3], 0.f)), x);
+                            sc[jp] = x.x;
+                            sc[jp + 1] = x.y;
                         }
-                    } else {
-                        // append (S, b) to this warp's segment of row j's list when S >= theta:
-                        // the warp's hits take consecutive slots in ballot order
-                        const float4 th4 = reinterpret_cast<const float4 *>(sh->theta)[part * 4 + c];
-                        const float th[4] = {th4.x, th4.y, th4.z, th4.w};
-                        uint32_t m[4], any = 0u;
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) {
-                            const int j = c * 4 + jj;
-                            const bool in = full || (((vmask >> j) & 1u) && b < ((t0 + j) >> rs));
-                            m[jj] = __ballot_sync(0xffffffffu, in && sc[jj] >= th[jj]);
-                            any |= m[jj];
-                        }
-                        if (any != 0u) {  // warp-uniform
+                        if (kMode != kEmit) {
 #pragma unroll
                             for (int jj = 0; jj < 4; ++jj) {
-                                if (m[jj] == 0u) continue;  // warp-uniform
                                 const int j = c * 4 + jj;
-                                const int len = seg_len[j];
-                                const int pos = len + __popc(m[jj] & lt_mask);
-                                if (((m[jj] >> lane) & 1u) && pos < cap_q)
-                                    lbase[j * 4 * cap_q + pos] = make_uint2(__float_as_uint(sc[jj]), (uint32_t)b);
-                                if (lane == 0) seg_len[j] = len + __popc(m[jj]);  // read again only after
-                            }                                                      // the tile's warp barrier
+                                const bool in = kFull ? col_ok : (((vmask >> j) & 1u) && b < ((t0 + j) >> rs) && col_ok);
+                                if (in) __stcs(p, sc[jj]);
+                                p += ld;
+                            }
+                        } else {
+                            // append (S, b) to this warp's segment of row j's list when S >= theta:
+                            // the warp's hits take consecutive slots in ballot order
+                            const float4 th4 = reinterpret_cast<const float4 *>(sh->theta)[part * 4 + c];
+                            const float th[4] = {th4.x, th4.y, th4.z, th4.w};
+                            uint32_t m[4], any = 0u;
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj) {
+                                const int j = c * 4 + jj;
+                                const bool in = kFull || (((vmask >> j) & 1u) && b < ((t0 + j) >> rs));
+                                m[jj] = __ballot_sync(0xffffffffu, in && sc[jj] >= th[jj]);
+                                any |= m[jj];
+                            }
+                            if (any != 0u) {  // warp-uniform
+#pragma unroll
+                                for (int jj = 0; jj < 4; ++jj) {
+                                    if (m[jj] == 0u) continue;  // warp-uniform
+                                    const int j = c * 4 + jj;
+                                    const int len = seg_len[j];
+                                    const int pos = len + __popc(m[jj] & lt_mask);
+                                    if (((m[jj] >> lane) & 1u) && pos < cap_q)
+                                        lbase[j * 4 * cap_q + pos] = make_uint2(__float_as_uint(sc[jj]), (uint32_t)b);
+                                    if (lane == 0) seg_len[j] = len + __popc(m[jj]);  // read again only after
+                                }                                                      // the tile's warp barrier
+                            }
                         }
                     }
-                }
+                };
+                if (full)
+                    tile(std::true_type{});
+                else
+                    tile(std::false_type{});
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh->acc_empty[acc]);

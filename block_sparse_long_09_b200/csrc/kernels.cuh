@@ -94,9 +94,46 @@ __device__ __forceinline__ void index_row_cuda(const __nv_bfloat16 *__restrict__
                                nwarps, lane);
 }
 
+// Partial RoPE of a 128-dim vector held as 4 consecutive dims per lane (lane l: dims
+// 4l .. 4l + 3), called by the whole warp: the first rope_dims dims (a multiple of 8)
+// rotate in pairs (i, i + rope_dims/2) by pos * base^(-2i / rope_dims), the partner of a
+// dim living rope_dims/8 lanes away.  Angle and its sine and cosine in fp64 (positions
+// reach 2^18, where an fp32 angle is off by ~1e-2 rad).
+struct RopeSpec {
+    int dims;    // 0: no rotation
+    float base;
+};
+
+__device__ __forceinline__ void rope_rotate4(float (&m)[4], int lane, int64_t pos, const RopeSpec &rope)
+{
+    if (rope.dims <= 0) return;
+    const int h = rope.dims / 2;
+    const int lo_lanes = h / 4;  // lanes holding dims < h
+    const int in_lo = 4 * lane < h, in_hi = !in_lo && 4 * lane < rope.dims;
+    const int partner = in_lo ? lane + lo_lanes : (in_hi ? lane - lo_lanes : lane);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const float other = __shfl_sync(0xffffffffu, m[c], partner);
+        if (in_lo || in_hi) {
+            const int i = 4 * lane + c - (in_hi ? h : 0);  // frequency index
+            const double a = (double)pos * pow((double)rope.base, -2.0 * (double)i / (double)rope.dims);
+            double sn, cs;
+            sincos(a, &sn, &cs);
+            const float cf = (float)cs, sf = (float)sn;
+            // low half: x_i cos - x_{i+h} sin; high half: x_{i} sin + x_{i+h} cos
+            m[c] = in_lo ? fmaf(m[c], cf, -other * sf) : fmaf(other, sf, m[c] * cf);
+        }
+    }
+}
+
+cudaError_t launch_rope_queries(const __nv_bfloat16 *q_idx_in, __nv_bfloat16 *q_idx, const int32_t *cu_q,
+                                const int32_t *cu_k, int batch, int64_t total_q, int heads, const RopeSpec &rope,
+                                cudaStream_t stream);
+
 cudaError_t launch_compress(const __nv_bfloat16 *k_idx, const int32_t *cu_k, const int32_t *cu_blocks,
                             int batch, int64_t total_k, const int32_t *blk_begin, int max_new, int r,
-                            bool normalise, float eps, __nv_bfloat16 *kc, cudaStream_t stream);
+                            bool normalise, float eps, __nv_bfloat16 *kc, cudaStream_t stream,
+                            const RopeSpec &rope = RopeSpec{0, 0.f});
 
 struct IndexArgs {
     const __nv_bfloat16 *q_idx;  // [total_q, 4, 128]
@@ -162,7 +199,7 @@ struct PagedArgs {
 };
 cudaError_t launch_compress_paged(const PagedArgs &p, const __nv_bfloat16 *k_pages, __nv_bfloat16 *kc_pages,
                                   const int32_t *blk_begin, int max_new, int64_t max_len_k, bool normalise,
-                                  float eps, cudaStream_t stream);
+                                  float eps, cudaStream_t stream, const RopeSpec &rope = RopeSpec{0, 0.f});
 cudaError_t launch_index_paged(const PagedArgs &p, const __nv_bfloat16 *q_idx, const float *w,
                                const __nv_bfloat16 *kc_pages, float *scores, int64_t ld, cudaStream_t stream);
 

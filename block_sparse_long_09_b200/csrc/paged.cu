@@ -37,7 +37,7 @@ __global__ void __launch_bounds__(kPagedWarps * 32)
 compress_paged_kernel(const __nv_bfloat16 *__restrict__ k_pages, __nv_bfloat16 *__restrict__ kc_pages, int64_t num_pages,
                       int page_size, const int32_t *__restrict__ table, int max_pages,
                       const int32_t *__restrict__ cu_k, int batch, const int32_t *__restrict__ blk_begin,
-                      int max_new, int64_t blocks_per_seq, int r, int normalise, float eps)
+                      int max_new, int64_t blocks_per_seq, int r, int normalise, float eps, const RopeSpec rope)
 {
     const int lane = threadIdx.x & 31;
     const int64_t n_items = (int64_t)batch * (blk_begin != nullptr ? max_new : blocks_per_seq);
@@ -81,6 +81,7 @@ compress_paged_kernel(const __nv_bfloat16 *__restrict__ k_pages, __nv_bfloat16 *
 #pragma unroll
             for (int c = 0; c < 4; ++c) m[c] *= inv;
         }
+        rope_rotate4(m, lane, b * r, rope);  // the pooled key at its block's first position
         // the compensated pair: hi = bf16(x), lo = bf16(x - hi)
         const __nv_bfloat162 h0 = __floats2bfloat162_rn(m[0], m[1]);
         const __nv_bfloat162 h1 = __floats2bfloat162_rn(m[2], m[3]);
@@ -133,7 +134,7 @@ index_paged_kernel(const __nv_bfloat16 *__restrict__ q_idx, const float *__restr
 
 cudaError_t launch_compress_paged(const PagedArgs &p, const __nv_bfloat16 *k_pages, __nv_bfloat16 *kc_pages,
                                   const int32_t *blk_begin, int max_new, int64_t max_len_k, bool normalise,
-                                  float eps, cudaStream_t stream)
+                                  float eps, cudaStream_t stream, const RopeSpec &rope)
 {
     const int64_t per = blk_begin != nullptr ? max_new : max_len_k / p.r;
     const int64_t n_items = (int64_t)p.batch * per;
@@ -142,7 +143,7 @@ cudaError_t launch_compress_paged(const PagedArgs &p, const __nv_bfloat16 *k_pag
     if (grid > 148 * 16) grid = 148 * 16;
     compress_paged_kernel<<<(unsigned)grid, kPagedWarps * 32, 0, stream>>>(
         k_pages, kc_pages, p.num_pages, p.page_size, p.table, p.max_pages, p.cu_k, p.batch, blk_begin, max_new,
-        max_len_k / p.r, p.r, normalise ? 1 : 0, eps);
+        max_len_k / p.r, p.r, normalise ? 1 : 0, eps, rope);
     return cudaGetLastError();
 }
 

@@ -27,6 +27,7 @@ QSA_ERR_DEVICE_CHECK = 6
 QSA_ERR_SCRATCH_LIMIT = 7
 STATIC_SCRATCH_BYTES = 16 * 1024 * 1024  # QSA_STATIC_SCRATCH_BYTES
 QSA_COMPRESS_NO_NORM = 0x1
+QSA_INDEX_ROPE = 0x2
 (OP_COMPRESS, OP_INDEX, OP_SELECT, OP_PREFILL, OP_DECODE, OP_DENSE, OP_DECODE_PAGED, OP_INDEX_SELECT,
  OP_INDEX_SELECT_PAGED, OP_DECODE_MTP) = range(10)
 
@@ -37,6 +38,7 @@ EXPORTED = (
     "qsa_index_select_mtp", "qsa_sparse_attn_decode_mtp",
     "qsa_dense_attn_prefill",
     "qsa_workspace_size", "qsa_status_string", "qsa_get_device_status", "qsa_version", "qsa_debug_inject",
+    "qsa_rope_queries",
 )
 
 
@@ -53,6 +55,8 @@ class Config(ctypes.Structure):
         ("rms_eps", ctypes.c_float),
         ("flags", ctypes.c_uint32),
         ("kv_chunk_blocks", ctypes.c_int32),
+        ("rope_dims", ctypes.c_int32),
+        ("rope_base", ctypes.c_float),
     ]
 
 
@@ -89,6 +93,7 @@ def _load():
         "qsa_get_device_status": (I32, [P, ctypes.POINTER(I32), I32]),
         "qsa_version": (I32, []),
         "qsa_debug_inject": (I32, [I32]),
+        "qsa_rope_queries": (I32, [CP, P, P, P, I32, I64, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -166,6 +171,16 @@ def compress_keys(k_idx, cu_seqlens_k, cu_blocks, kc=None, blk_begin=None, max_n
                                   k_idx.shape[0], _p(blk_begin), max_new_blocks, _p(kc), _stream()),
            "qsa_compress_keys")
     return kc
+
+
+def rope_queries(q_idx, cu_seqlens_q, cu_seqlens_k, cfg: Optional[Config] = None):
+    """Partial RoPE of the indexer queries in place (q_idx [total_q, 4, 128] bf16), each row
+    at its position t; cfg must carry QSA_INDEX_ROPE (the pooled keys rotate the same way)."""
+    cfg = _cfg(cfg)
+    _check(_lib.qsa_rope_queries(ctypes.byref(cfg), _p(q_idx), _p(cu_seqlens_q), _p(cu_seqlens_k),
+                                 cu_seqlens_q.numel() - 1, q_idx.shape[0], _stream()),
+           "qsa_rope_queries")
+    return q_idx
 
 
 def index_scores(q_idx, w, kc, cu_seqlens_q, cu_seqlens_k, cu_blocks, max_len_q: int, ld: int,

@@ -69,6 +69,7 @@ typedef uint16_t qsa_bf16; /* bfloat16 bit pattern */
 
 /* flags */
 #define QSA_COMPRESS_NO_NORM 0x1u /* plain mean-pool, no RMSNorm in the compressor */
+#define QSA_INDEX_ROPE 0x2u       /* partial RoPE of the pooled indexer key (rope_dims, rope_base) */
 
 typedef struct qsa_config {
     int32_t r;             /* micro-block size (4) */
@@ -80,9 +81,12 @@ typedef struct qsa_config {
     int32_t idx_dim;       /* indexer head dim (128) */
     float softmax_scale;   /* 1/sqrt(256) */
     float rms_eps;         /* compressor RMSNorm eps (1e-6) */
-    uint32_t flags;        /* QSA_COMPRESS_NO_NORM */
+    uint32_t flags;        /* QSA_COMPRESS_NO_NORM | QSA_INDEX_ROPE */
     int32_t kv_chunk_blocks; /* > 0: key-chunk size (micro-blocks) of the L2-blocked prefill
                                 schedule; 0 (default): one pass per query */
+    int32_t rope_dims;     /* with QSA_INDEX_ROPE: rotated leading dims of the indexer head
+                              (a multiple of 8, at most idx_dim; default 64) */
+    float rope_base;       /* with QSA_INDEX_ROPE: frequency base (default 10000) */
 } qsa_config;
 
 /* op ids for qsa_workspace_size */
@@ -98,7 +102,7 @@ typedef struct qsa_config {
 #define QSA_OP_DECODE_MTP 9 /* qsa_sparse_attn_decode_mtp */
 
 /* Fill *cfg with the model's values (r 4, k 512, 24/2/256, 4/128, scale 1/16,
- * eps 1e-6, flags 0, kv_chunk_blocks 0).  Host only. */
+ * eps 1e-6, flags 0, kv_chunk_blocks 0, rope_dims 64, rope_base 10000).  Host only. */
 void qsa_config_init(qsa_config *cfg);
 
 /*
@@ -118,11 +122,31 @@ void qsa_config_init(qsa_config *cfg);
  *              that are complete (a decode step refreshes the blocks it completed).
  *   kc         [cu_blocks[batch], 2, idx_dim] bf16, written: per block the hi
  *              plane, then the lo plane.
+ * QSA_INDEX_ROPE (the sentence before the pooled-key equation: pool first, then a
+ * partial RoPE, so keys of different rotation phases are never averaged; the
+ * pages fix no dims, base or position): after the pool and the norm, the first
+ * cfg->rope_dims dims rotate in pairs (i, i + rope_dims/2) by the angle
+ * (b r) * rope_base^(-2i / rope_dims), b r the block's first position; angles and
+ * their sines in fp64.  The indexer queries must then be rotated at their own
+ * positions t (qsa_rope_queries), as the attention's q and k arrive rotated.
  */
 qsa_status qsa_compress_keys(const qsa_config *cfg, const qsa_bf16 *k_idx,
                              const int32_t *cu_seqlens_k, const int32_t *cu_blocks,
                              int32_t batch, int64_t total_k, const int32_t *blk_begin,
                              int32_t max_new_blocks, qsa_bf16 *kc, void *stream);
+
+/*
+ * Partial RoPE of the indexer queries, in place: row i of sequence s sits at
+ * t = (L_k,s - L_q,s) + (i - cu_seqlens_q[s]) and every head of it rotates as the
+ * pooled keys do under QSA_INDEX_ROPE (same dims, pairs and base; angle t * f_i).
+ * fp32 arithmetic on the bf16 values, fp64 angles, bf16 round-to-nearest-even
+ * stores.  Requires QSA_INDEX_ROPE in cfg->flags (QSA_ERR_INVALID_ARG otherwise).
+ *   q_idx      [total_q, n_heads_idx, idx_dim] bf16, read and written
+ *   cu_seqlens_q, cu_seqlens_k  [batch+1] int32
+ *   total_q    host: rows of q_idx
+ */
+qsa_status qsa_rope_queries(const qsa_config *cfg, qsa_bf16 *q_idx, const int32_t *cu_seqlens_q,
+                            const int32_t *cu_seqlens_k, int32_t batch, int64_t total_q, void *stream);
 
 /*
  * Indexer scores -- indexer equation of section 6, with one weight per

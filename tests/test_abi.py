@@ -135,3 +135,18 @@ def test_binding_refuses_a_selection_that_does_not_match_the_budget(qsa):
             qsa.sparse_attn_prefill(q, kv, kv, bad, cu_, cu_)
     with pytest.raises(ValueError):
         qsa.sparse_attn_decode(q[:1], kv, kv, cu_, torch.zeros((1, 16), dtype=torch.int32))
+
+
+def test_rope_config_checked_on_the_host(qsa):
+    import ctypes
+    lib = qsa.library()
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: each call returns before any device work
+    c = qsa.default_config()
+    assert (c.rope_dims, c.rope_base) == (64, 10000.0)
+    # qsa_rope_queries needs QSA_INDEX_ROPE
+    assert lib.qsa_rope_queries(ctypes.byref(c), fake, fake, fake, 1, 8, None) == qsa.QSA_ERR_INVALID_ARG
+    for dims, base in ((0, 1e4), (12, 1e4), (136, 1e4), (64, 1.0), (64, float("nan"))):
+        bad = qsa.default_config(flags=qsa.QSA_INDEX_ROPE, rope_dims=dims, rope_base=base)
+        assert lib.qsa_rope_queries(ctypes.byref(bad), fake, fake, fake, 1, 8, None) == qsa.QSA_ERR_INVALID_ARG
+        assert lib.qsa_compress_keys(ctypes.byref(bad), fake, fake, fake, 1, 8, None, 0, fake, None) == \
+            qsa.QSA_ERR_INVALID_ARG
