@@ -35,25 +35,27 @@ constexpr int kMaxNQ = 4;
 constexpr int kMRows = kMaxNQ * kHQ;              // 96 (query, head) rows
 constexpr int kQChunkM = 128 * 128;               // 16 KB: 64 d-columns x 128 rows
 constexpr int kQBytesM = 4 * kQChunkM;            // 64 KB
-constexpr int kPChunkM = 128 * 128;               // 16 KB: 64 key columns x 128 rows
-constexpr int kPBytesM = 2 * kPChunkM;            // 32 KB
+constexpr int kMtpBlk = 8;                        // micro-blocks per tile
+constexpr int kMtpKeys = kMtpBlk * 8;             // 64 K/V rows per tile: 8 blocks x 4 tokens x 2 groups
+constexpr int kMtpSlot = kMtpBlk * kBlockBytes;   // 32 KB: one tile of K (or V)
+constexpr int kPBufM = 128 * 128;                 // 16 KB: P of one tile, 64 key columns x 128 rows
 constexpr int kMtpThreads = 192;
 constexpr uint32_t kMtpSCol = 0, kMtpOCol = 256, kMtpTmemCols = 512;
 
 struct MtpShared {
-    uint64_t k_full, k_empty, v_full, v_empty;
+    uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
     uint64_t q_full, q_empty;
     uint64_t s_full[2], s_empty[2];
-    uint64_t p_full, p_empty;
+    uint64_t p_full[2], p_empty[2];
     uint64_t o_full, o_empty;
     uint32_t tmem_base;
     int abort_flag;
 };
 
 constexpr int kOffKM = kQBytesM;
-constexpr int kOffVM = kOffKM + kSlotBytes;
-constexpr int kOffPM = kOffVM + kSlotBytes;
-constexpr int kOffShM = kOffPM + kPBytesM;
+constexpr int kOffVM = kOffKM + 2 * kMtpSlot;
+constexpr int kOffPM = kOffVM + 2 * kMtpSlot;
+constexpr int kOffShM = kOffPM + 2 * kPBufM;
 constexpr int kMtpSmem = kOffShM + (int)sizeof(MtpShared) + 1024;
 static_assert(kMtpSmem <= 232448, "shared memory of one CTA");
 
@@ -86,10 +88,10 @@ __device__ __forceinline__ MtpItem mtp_item(int64_t item, int nsplit, const int3
     const int64_t room = kb - nf > 0 ? kb - nf : 0;
     it.nsel = (int)((b_first < room ? b_first : room) + nf);
     if (it.nsel > kb) it.nsel = kb;
-    const int tiles = (it.nsel + kBlkTile - 1) / kBlkTile;
+    const int tiles = (it.nsel + kMtpBlk - 1) / kMtpBlk;
     const int tps = (tiles + nsplit - 1) / nsplit;
     const int a = it.sp * tps, b = (it.sp + 1) * tps < tiles ? (it.sp + 1) * tps : tiles;
-    it.p0 = a * kBlkTile;
+    it.p0 = a * kMtpBlk;
     it.nt = b > a ? b - a : 0;
     return it;
 }
@@ -112,30 +114,26 @@ sparse_mtp_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        mbar_init(&sh->k_full, 1);
-        mbar_init(&sh->k_empty, 1);
-        mbar_init(&sh->v_full, 1);
-        mbar_init(&sh->v_empty, 1);
-        mbar_init(&sh->q_full, 1);
-        mbar_init(&sh->q_empty, 1);
         for (int i = 0; i < 2; ++i) {
+            mbar_init(&sh->k_full[i], 1);
+            mbar_init(&sh->k_empty[i], 1);
+            mbar_init(&sh->v_full[i], 1);
+            mbar_init(&sh->v_empty[i], 1);
             mbar_init(&sh->s_full[i], 1);
             mbar_init(&sh->s_empty[i], 128);
+            mbar_init(&sh->p_full[i], 128);
+            mbar_init(&sh->p_empty[i], 1);
         }
-        mbar_init(&sh->p_full, 128);
-        mbar_init(&sh->p_empty, 1);
+        mbar_init(&sh->q_full, 1);
+        mbar_init(&sh->q_empty, 1);
         mbar_init(&sh->o_full, 1);
         mbar_init(&sh->o_empty, 128);
         sh->abort_flag = 0;
         fence_barrier_init();
     }
-    // the rows the TMA never writes (Q rows 96..127, and all of P) start at zero
-    for (int i = threadIdx.x; i < (kQBytesM + kPBytesM) / 16; i += kMtpThreads) {
-        const int byte = i * 16;
-        const bool q_pad = byte < kQBytesM && (byte % kQChunkM) >= kMRows * 128;
-        if (q_pad) reinterpret_cast<uint4 *>(sQ)[i] = make_uint4(0u, 0u, 0u, 0u);
-        if (byte >= kQBytesM) reinterpret_cast<uint4 *>(sP)[i - kQBytesM / 16] = make_uint4(0u, 0u, 0u, 0u);
-    }
+    // the Q rows the TMA never writes (96..127) start at zero; P is written whole per tile
+    for (int i = threadIdx.x; i < kQBytesM / 16; i += kMtpThreads)
+        if ((i * 16) % kQChunkM >= kMRows * 128) reinterpret_cast<uint4 *>(sQ)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
     if (warp == 1) {
         tmem_alloc(&sh->tmem_base, kMtpTmemCols);
@@ -158,16 +156,18 @@ sparse_mtp_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         }
         uint32_t ku = 0, vu = 0, qu = 0;
         bool ok = true;
-        auto issue = [&](const CUtensorMap *map, uint8_t *slot, uint64_t *full, uint64_t *empty, uint32_t use,
+        // one ring use: lane 0 waits for the slot and arms its barrier, lanes 0..7 load a block each
+        auto issue = [&](const CUtensorMap *map, uint8_t *ring, uint64_t *full, uint64_t *empty, uint32_t use,
                          const MtpItem &it, int32_t raw) -> bool {
+            const uint32_t st = use & 1;
             bool good = true;
             if (lane == 0) {
-                good = mbar_wait(empty, (use & 1) ^ 1, abort_flag);
-                if (good) mbar_arrive_expect_tx(full, kSlotBytes);
+                good = mbar_wait(&empty[st], ((use >> 1) & 1) ^ 1, abort_flag);
+                if (good) mbar_arrive_expect_tx(&full[st], kMtpSlot);
             }
             good = __shfl_sync(0xffffffffu, good, 0);
             if (!good) return false;
-            if (lane < kBlkTile) {
+            if (lane < kMtpBlk) {
                 int32_t y = -8;  // reads zeros
                 if (raw != kNoBlock) {
                     if (raw < 0 || raw > it.b_last) {
@@ -186,7 +186,7 @@ sparse_mtp_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                         }
                     }
                 }
-                tma_load_3d(slot + lane * kBlockBytes, map, full, 0, y, 0);
+                tma_load_3d(ring + st * kMtpSlot + lane * kBlockBytes, map, &full[st], 0, y, 0);
             }
             return true;
         };
@@ -205,55 +205,58 @@ sparse_mtp_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             ok = __shfl_sync(0xffffffffu, ok, 0);
             ++qu;
             for (int j = 0; ok && j < it.nt; ++j) {
-                const int pos = it.p0 + j * kBlkTile + lane;
-                const int32_t raw = (lane < kBlkTile && pos < it.nsel) ? __ldg(sel + it.s * kb + pos) : kNoBlock;
-                ok = issue(&map_k, sK, &sh->k_full, &sh->k_empty, ku++, it, raw);
-                if (ok) ok = issue(&map_v, sV, &sh->v_full, &sh->v_empty, vu++, it, raw);
+                const int pos = it.p0 + j * kMtpBlk + lane;
+                const int32_t raw = (lane < kMtpBlk && pos < it.nsel) ? __ldg(sel + it.s * kb + pos) : kNoBlock;
+                ok = issue(&map_k, sK, sh->k_full, sh->k_empty, ku++, it, raw);
+                if (ok) ok = issue(&map_v, sV, sh->v_full, sh->v_empty, vu++, it, raw);
             }
         }
         if (!ok && lane == 0) {  // let every copy in flight land before the CTA exits
-            if (ku > 0) mbar_wait(&sh->k_full, (ku - 1) & 1, nullptr);
-            if (vu > 0) mbar_wait(&sh->v_full, (vu - 1) & 1, nullptr);
+            for (uint32_t u = (ku > 2 ? ku - 2 : 0); u < ku; ++u) mbar_wait(&sh->k_full[u & 1], (u >> 1) & 1, nullptr);
+            for (uint32_t u = (vu > 2 ? vu - 2 : 0); u < vu; ++u) mbar_wait(&sh->v_full[u & 1], (u >> 1) & 1, nullptr);
         }
     } else if (warp == 1) {
         // ======================= MMA issuer (one thread) =======================
         if (elect_one()) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(128, kRowsTile, 0, 0);
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, kMtpKeys, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kD, 0, 1);
             const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV),
                            p_addr = smem_u32(sP);
             uint32_t ku = 0, vu = 0, qu = 0, su = 0, pu = 0, ou = 0;
             bool ok = true;
-            auto do_s = [&]() -> bool {
-                const uint32_t sb = su & 1, sround = su >> 1;
-                if (!mbar_wait(&sh->k_full, ku & 1, abort_flag)) return false;
-                if (!mbar_wait(&sh->s_empty[sb], (sround & 1) ^ 1, abort_flag)) return false;
+            auto do_s = [&]() -> bool {  // S = Q K^T of the next K tile into S buffer su & 1
+                const uint32_t sb = su & 1, kb_ = ku & 1;
+                if (!mbar_wait(&sh->k_full[kb_], (ku >> 1) & 1, abort_flag)) return false;
+                if (!mbar_wait(&sh->s_empty[sb], ((su >> 1) & 1) ^ 1, abort_flag)) return false;
                 tc_fence_after();
+                const uint32_t k0 = k_addr + kb_ * kMtpSlot;
 #pragma unroll
                 for (int ks = 0; ks < kD / 16; ++ks) {
                     const uint32_t off = (ks & 3) * 32;
                     const uint64_t ad = sdesc_sw128(q_addr + (ks >> 2) * kQChunkM + off, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(k_addr + (ks >> 2) * 1024 + off, 16, kBlockBytes);
-                    mma_bf16_ss(tmem + kMtpSCol + sb * 128, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+                    const uint64_t bd = sdesc_sw128(k0 + (ks >> 2) * 1024 + off, 16, kBlockBytes);
+                    mma_bf16_ss(tmem + kMtpSCol + sb * kMtpKeys, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
                 }
-                mma_commit(&sh->k_empty);
+                mma_commit(&sh->k_empty[kb_]);
                 mma_commit(&sh->s_full[sb]);
                 ++ku;
                 ++su;
                 return true;
             };
-            auto do_pv = [&](bool first) -> bool {
-                if (!mbar_wait(&sh->v_full, vu & 1, abort_flag)) return false;
-                if (!mbar_wait(&sh->p_full, pu & 1, abort_flag)) return false;
+            auto do_pv = [&](bool first) -> bool {  // O += P V of the next V tile
+                const uint32_t vb = vu & 1, pb = pu & 1;
+                if (!mbar_wait(&sh->v_full[vb], (vu >> 1) & 1, abort_flag)) return false;
+                if (!mbar_wait(&sh->p_full[pb], (pu >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
+                const uint32_t v0 = v_addr + vb * kMtpSlot, p0 = p_addr + pb * kPBufM;
 #pragma unroll
-                for (int ks = 0; ks < kRowsTile / 16; ++ks) {
-                    const uint64_t ad = sdesc_sw128(p_addr + (ks >> 2) * kPChunkM + (ks & 3) * 32, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(v_addr + (2 * ks) * kBlockBytes, 1024, kBlockBytes);
+                for (int ks = 0; ks < kMtpKeys / 16; ++ks) {
+                    const uint64_t ad = sdesc_sw128(p0 + ks * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(v0 + (2 * ks) * kBlockBytes, 1024, kBlockBytes);
                     mma_bf16_ss(tmem + kMtpOCol, ad, bd, idesc_pv, (first && ks == 0) ? 0u : 1u);
                 }
-                mma_commit(&sh->v_empty);
-                mma_commit(&sh->p_empty);
+                mma_commit(&sh->v_empty[vb]);
+                mma_commit(&sh->p_empty[pb]);
                 ++vu;
                 ++pu;
                 return true;
@@ -308,22 +311,23 @@ sparse_mtp_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             const int64_t t = it.L - next_n + qi;  // this row's position
             float m = -INFINITY, l = 0.f;
             for (int j = 0; ok && j < it.nt; ++j) {
-                const uint32_t sb = su & 1, sround = su >> 1;
-                if (!(ok = mbar_wait(&sh->s_full[sb], sround & 1, abort_flag))) break;
+                const uint32_t sb = su & 1;
+                if (!(ok = mbar_wait(&sh->s_full[sb], (su >> 1) & 1, abort_flag))) break;
                 tc_fence_after();
-                float s[kRowsTile];
+                float s[kMtpKeys];
                 __syncwarp();
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_addr + kMtpSCol + sb * 128 + c * 32, s + c * 32);
+                for (int c = 0; c < kMtpKeys / 32; ++c)
+                    tmem_ld32(tmem + lane_addr + kMtpSCol + sb * kMtpKeys + c * 32, s + c * 32);
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&sh->s_empty[sb]);
                 ++su;
                 // which key columns this row sees: its KV group, a selected block, token <= t
-                const int pbase = it.p0 + j * kBlkTile;
+                const int pbase = it.p0 + j * kMtpBlk;
                 float mt = -INFINITY;
 #pragma unroll
-                for (int bs = 0; bs < kBlkTile; ++bs) {
+                for (int bs = 0; bs < kMtpBlk; ++bs) {
                     const int pos = pbase + bs;
                     const int32_t blk = pos < it.nsel ? __ldg(sel + it.s * kb + pos) : -1;
                     const bool bok = live && blk >= 0 && blk <= it.b_last;
@@ -335,15 +339,17 @@ sparse_mtp_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                         mt = fmaxf(mt, s[c]);
                     }
                 }
-                // P(j) replaces P(j - 1): PV(j - 1), and every PV before it, has completed
-                if (!(ok = mbar_wait(&sh->p_empty, (pu & 1) ^ 1, abort_flag))) break;
-                tc_fence_after();
                 // the running maxima move when some row of the warp grows by more than the margin
-                // (and on the first tile); the TMEM rescale is then done by the whole warp, rows
-                // whose maximum stayed put scaling by 1
+                // (and on the first tile); O is then rescaled by the whole warp once every earlier
+                // PV has landed (rows whose maximum stayed put scale by 1)
                 if (__any_sync(0xffffffffu, mt > m + margin || j == 0)) {
                     const float mn = fmaxf(m, mt);
                     if (j > 0) {
+                        {  // PV(j - 1) used P buffer (pu - 1) & 1: its completion covers every PV before it
+                            const uint32_t x = pu - 1;
+                            if (!(ok = mbar_wait(&sh->p_empty[x & 1], (x >> 1) & 1, abort_flag))) break;
+                        }
+                        tc_fence_after();
                         const float f = mn == -INFINITY ? 1.f : exp2f((m - mn) * c2);
                         l *= f;
 #pragma unroll 1
@@ -360,32 +366,35 @@ sparse_mtp_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     }
                     m = mn;
                 }
-                const float mc = (m == -INFINITY ? 0.f : m) * c2;
-                // P row: own-group columns exp(S - m), the rest 0; 128-byte swizzled K-major layout
-#pragma unroll
-                for (int ch = 0; ch < 2; ++ch) {
+                // P(j) goes to buffer pu & 1, free once PV(j - 2) has completed
+                {
+                    const uint32_t pb = pu & 1;
+                    if (!(ok = mbar_wait(&sh->p_empty[pb], ((pu >> 1) & 1) ^ 1, abort_flag))) break;
+                    tc_fence_after();
+                    const float mc = (m == -INFINITY ? 0.f : m) * c2;
+                    // P row: own-group columns exp(S - m), the rest 0; 128-byte swizzled K-major layout
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         uint32_t pk[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const int c = ch * 64 + u * 8 + e * 2;
+                            const int c = u * 8 + e * 2;
                             const float p0 = exp2f(fmaf(s[c], c2, -mc));      // -inf gives 0
                             const float p1 = exp2f(fmaf(s[c + 1], c2, -mc));
                             l += p0 + p1;
                             const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
                             pk[e] = *reinterpret_cast<const uint32_t *>(&b2);
                         }
-                        const uint32_t addr = p_row + ch * kPChunkM + ((u ^ (R & 7)) << 4);
+                        const uint32_t addr = p_row + pb * kPBufM + ((u ^ (R & 7)) << 4);
                         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[0]),
                                      "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
                                      : "memory");
                     }
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    mbar_arrive(&sh->p_full[pb]);
+                    ++pu;
                 }
-                fence_proxy_async_smem();
-                tc_fence_before();
-                mbar_arrive(&sh->p_full);
-                ++pu;
             }
             if (!ok) break;
             // epilogue: O / l of this row
@@ -442,61 +451,68 @@ sparse_mtp_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
 }
 
 // merge the splits of each (sequence, query row): lse = logsumexp of the parts,
-// o = sum exp(lse_part - lse) o_part
-__global__ void __launch_bounds__(kD)
+// o = sum exp(lse_part - lse) o_part / sum exp(lse_part - lse).  A warp per row: lane sp
+// holds split sp's weight (nsplit <= 32), each lane 8 of the 256 dims.
+constexpr int kCombRows = 8;  // rows (warps) per CTA
+
+__global__ void __launch_bounds__(kCombRows * 32)
 mtp_combine_kernel(const float *__restrict__ ws, int64_t n_items, int nsplit, int next_n,
                    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse_out)
 {
-    __shared__ float s_wgt[kD];  // the splits' weights exp(lse_sp - max), one per split (nsplit <= kD)
-    __shared__ float s_mx, s_tot;
     const int64_t s = blockIdx.x;
-    const int R = blockIdx.y;  // < next_n * 24
-    const int d = threadIdx.x;
+    const int lane = threadIdx.x & 31;
+    const int R = blockIdx.y * kCombRows + (threadIdx.x >> 5);  // (query, head) row
+    if (R >= next_n * kHQ) return;  // warp-uniform
     const float *lp = ws + (size_t)n_items * kMRows * kD + (s * nsplit) * kMRows + R;
-    const float *pp = ws + ((s * nsplit) * kMRows + R) * kD + d;
-    if (d < 32) {  // warp 0: the max and the weights of the splits, in split order
-        float mx = -INFINITY;
-        for (int sp = d; sp < nsplit; sp += 32) mx = fmaxf(mx, lp[sp * kMRows]);
+    const float *pp = ws + ((s * nsplit) * kMRows + R) * kD + lane;
+    const float l = lane < nsplit ? lp[lane * kMRows] : -INFINITY;
+    float mx = l;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        for (int sp = d; sp < nsplit; sp += 32) {
-            const float l = lp[sp * kMRows];
-            s_wgt[sp] = (l == -INFINITY) ? 0.f : __expf(l - mx);
-        }
-        __syncwarp();
-        if (d == 0) {
-            float tot = 0.f;
-            for (int sp = 0; sp < nsplit; ++sp) tot += s_wgt[sp];
-            s_mx = mx;
-            s_tot = tot;
-        }
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    const float wgt = (l == -INFINITY) ? 0.f : __expf(l - mx);
+    float tot = 0.f, acc[kD / 32];
+#pragma unroll
+    for (int i = 0; i < kD / 32; ++i) acc[i] = 0.f;
+    for (int sp = 0; sp < nsplit; ++sp) {  // the splits in order
+        const float w = __shfl_sync(0xffffffffu, wgt, sp);
+        tot += w;
+        float o[kD / 32];
+#pragma unroll
+        for (int i = 0; i < kD / 32; ++i) o[i] = __ldcs(pp + (size_t)sp * kMRows * kD + i * 32);
+#pragma unroll
+        for (int i = 0; i < kD / 32; ++i) acc[i] += w * o[i];
     }
-    __syncthreads();
-    constexpr int kU = 8;  // partial outputs in flight per thread
-    float acc = 0.f;
-    for (int sp0 = 0; sp0 < nsplit; sp0 += kU) {
-        float o[kU];
-#pragma unroll
-        for (int u = 0; u < kU; ++u) o[u] = sp0 + u < nsplit ? __ldcs(pp + (size_t)(sp0 + u) * kMRows * kD) : 0.f;
-#pragma unroll
-        for (int u = 0; u < kU; ++u)
-            if (sp0 + u < nsplit) acc += s_wgt[sp0 + u] * o[u];
-    }
-    const float tot = s_tot;
     const int qi = R / kHQ, h = R % kHQ;
-    out[((s * next_n + qi) * kHQ + h) * kD + d] = __float2bfloat16_rn(tot > 0.f ? acc / tot : 0.f);
-    if (lse_out != nullptr && d == 0) lse_out[(s * next_n + qi) * kHQ + h] = tot > 0.f ? s_mx + logf(tot) : -INFINITY;
+    __nv_bfloat16 *dst = out + ((s * next_n + qi) * kHQ + h) * kD + lane;
+    const float inv = tot > 0.f ? 1.f / tot : 0.f;
+#pragma unroll
+    for (int i = 0; i < kD / 32; ++i) dst[i * 32] = __float2bfloat16_rn(tot > 0.f ? acc[i] * inv : 0.f);
+    if (lse_out != nullptr && lane == 0) lse_out[(s * next_n + qi) * kHQ + h] = tot > 0.f ? mx + logf(tot) : -INFINITY;
 }
 
 }  // namespace
 
 int mtp_nsplit(int batch, int kb)
 {
-    const int tiles = (kb + kBlkTile - 1) / kBlkTile;
-    int ns = (2 * num_sms() + batch - 1) / (batch > 0 ? batch : 1);
-    if (ns > tiles) ns = tiles;
-    if (ns > kD) ns = kD;  // the merge keeps one weight per split in shared memory
-    return ns > 0 ? ns : 1;
+    // splits per sequence: the fewest that minimise the busiest CTA's work in tile units,
+    // ceil(batch * ns / G) items of tiles / ns tiles each, plus the partial states that
+    // splits write and the merge reads back (96 x 257 fp32 twice: about 3 tiles of K/V
+    // bytes each), spread over the G CTAs
+    const int tiles = (kb + kMtpBlk - 1) / kMtpBlk;
+    const int64_t G = num_sms();
+    if (batch <= 0) return 1;
+    int best = 1;
+    double best_cost = -1.0;
+    for (int ns = 1; ns <= tiles && ns <= 32; ++ns) {  // the merge keeps a split's weight per lane
+        const int64_t items_per_cta = ((int64_t)batch * ns + G - 1) / G;
+        const double cost = (double)(items_per_cta * ((tiles + ns - 1) / ns)) +
+                            (ns > 1 ? 3.0 * (double)batch * ns / (double)G : 0.0);
+        if (best_cost < 0.0 || cost < best_cost) {
+            best = ns;
+            best_cost = cost;
+        }
+    }
+    return best;
 }
 
 size_t mtp_workspace_bytes(int batch, int kb)
@@ -532,8 +548,8 @@ cudaError_t launch_sparse_mtp(const AttnArgs &a, int next_n, cudaStream_t stream
         a.page_size, a.max_pages, a.block_table != nullptr ? a.total_k / a.page_size : 0);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || nsplit == 1) return e;
-    mtp_combine_kernel<<<dim3((unsigned)batch, (unsigned)(next_n * kHQ)), kD, 0, stream>>>(a.ws, n_items, nsplit,
-                                                                                         next_n, a.o, a.lse);
+    mtp_combine_kernel<<<dim3((unsigned)batch, (unsigned)((next_n * kHQ + kCombRows - 1) / kCombRows)),
+                         kCombRows * 32, 0, stream>>>(a.ws, n_items, nsplit, next_n, a.o, a.lse);
     return cudaGetLastError();
 }
 

@@ -59,7 +59,9 @@ struct IdxShared {
     uint64_t acc_empty[2];
     uint32_t tmem_base;
     int abort_flag;
-    alignas(16) float wq[kQRowsT];  // w[row, head]; read as float4
+    // w of the tile's rows, by row pairs (2p, 2p + 1): {w[2p][0], w[2p+1][0], w[2p][1], w[2p+1][1]},
+    // then the same for heads 2, 3 -- each float2 an operand of the packed fp32x2 epilogue
+    alignas(16) float wq[kQRowsT];
     alignas(16) float theta[kTokTile];  // emit mode: the rows' thresholds; read as float4
     int seg_len[kEpiWarps][16];  // emit mode: each epilogue warp's list-segment lengths
 };
@@ -231,7 +233,8 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         const int et = threadIdx.x - 64;            // 0 .. 511
         if (et < kQRowsT) {  // the tile's weights, (row, head) in q_idx order
             const int64_t i = m0 + (et >> 2);
-            sh->wq[et] = i < m1 ? __ldg(w + i * 4 + (et & 3)) : 0.f;
+            const int row = et >> 2, h = et & 3;
+            sh->wq[(row >> 1) * 8 + (h >> 1) * 4 + (h & 1) * 2 + (row & 1)] = i < m1 ? __ldg(w + i * 4 + h) : 0.f;
         }
         if (kMode == kEmit && et < kTokTile) {
             const int64_t i = m0 + et;
@@ -297,13 +300,14 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                         float sc[4];
 #pragma unroll
                         for (int jp = 0; jp < 4; jp += 2) {
-                            const float4 wa = wq4[part * 16 + c * 4 + jp], wb = wq4[part * 16 + c * 4 + jp + 1];
+                            const int pr = part * 8 + c * 2 + jp / 2;  // row pair of the tile
+                            const float4 w01 = wq4[2 * pr], w23 = wq4[2 * pr + 1];
                             const float *va = v + 4 * jp, *vb = v + 4 * jp + 4;
-                            float2 x = __fmul2_rn(make_float2(wa.x, wb.x),
+                            float2 x = __fmul2_rn(make_float2(w01.x, w01.y),
                                                   make_float2(fmaxf(va[0], 0.f), fmaxf(vb[0], 0.f)));
-                            x = __ffma2_rn(make_float2(wa.y, wb.y), make_float2(fmaxf(va[1], 0.f), fmaxf(vb[1], 0.f)), x);
-                            x = __ffma2_rn(make_float2(wa.z, wb.z), make_float2(fmaxf(va[2], 0.f), fmaxf(vb[2], 0.f)), x);
-                            x = __ffma2_rn(make_float2(wa.w, wb.w), make_float2(fmaxf(va[3], 0.f), fmaxf(vb[3], 0.f)), x);
+                            x = __ffma2_rn(make_float2(w01.z, w01.w), make_float2(fmaxf(va[1], 0.f), fmaxf(vb[1], 0.f)), x);
+                            x = __ffma2_rn(make_float2(w23.x, w23.y), make_float2(fmaxf(va[2], 0.f), fmaxf(vb[2], 0.f)), x);
+                            x = __ffma2_rn(make_float2(w23.z, w23.w), make_float2(fmaxf(va[3], 0.f), fmaxf(vb[3], 0.f)), x);
                             sc[jp] = x.x;
                             sc[jp + 1] = x.y;
                         }
