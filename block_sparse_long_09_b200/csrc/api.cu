@@ -468,6 +468,49 @@ qsa_status qsa_sparse_attn_decode(const qsa_config *cfg, const qsa_bf16 *q, cons
     return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
 }
 
+qsa_status qsa_sparse_attn_decode_window(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k_local,
+                                         const qsa_bf16 *v_local, const int32_t *cu_seqlens_k, int32_t batch,
+                                         int64_t total_k_local, const int64_t *tok_local, const int32_t *blk_lo,
+                                         const int32_t *blk_hi, const int32_t *sel, qsa_bf16 *o, float *lse,
+                                         void *ws, size_t ws_bytes, void *stream)
+{
+    const qsa::NvtxRange nvtx_range("qsa_sparse_attn_decode_window");
+    qsa_status st = check_config(cfg);
+    if (st != QSA_OK) return st;
+    if (batch <= 0 || total_k_local <= 0 || cu_seqlens_k == nullptr || tok_local == nullptr || blk_lo == nullptr ||
+        blk_hi == nullptr)
+        return QSA_ERR_INVALID_ARG;
+    if (q == nullptr || k_local == nullptr || v_local == nullptr || sel == nullptr || o == nullptr || lse == nullptr ||
+        !al16(q) || !al16(k_local) || !al16(v_local))
+        return QSA_ERR_INVALID_ARG;
+    const int grid = even_grid();
+    if (batch >= 2 * grid) return QSA_ERR_UNSUPPORTED;  // the even schedule only
+    if (ws == nullptr) return QSA_ERR_WORKSPACE_TOO_SMALL;
+    if (ws_bytes < even_workspace_bytes(batch, grid)) return QSA_ERR_WORKSPACE_TOO_SMALL;
+    if (!al16(ws)) return QSA_ERR_INVALID_ARG;
+    AttnArgs a{bf(q), bf(k_local), bf(v_local), sel, nullptr, cu_seqlens_k, batch, batch, total_k_local, 0, batch,
+               bf(o), lse, static_cast<float *>(ws), 1, cfg->budget_blocks, cfg->r, cfg->softmax_scale};
+    a.even = 1;
+    a.tok_local = tok_local;
+    a.blk_lo = blk_lo;
+    a.blk_hi = blk_hi;
+    return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
+}
+
+qsa_status qsa_merge_attn_states(const qsa_config *cfg, const qsa_bf16 *o_parts, const float *lse_parts,
+                                 int32_t parts, int64_t rows, qsa_bf16 *o, float *lse, void *stream)
+{
+    const qsa::NvtxRange nvtx_range("qsa_merge_attn_states");
+    qsa_status st = check_config(cfg);
+    if (st != QSA_OK) return st;
+    if (parts <= 0 || rows < 0) return QSA_ERR_INVALID_ARG;
+    if (rows == 0) return QSA_OK;
+    if (o_parts == nullptr || lse_parts == nullptr || o == nullptr) return QSA_ERR_INVALID_ARG;
+    return cuda_status(launch_merge_states(bf(o_parts), lse_parts, parts, rows,
+                                           reinterpret_cast<__nv_bfloat16 *>(o), lse,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
 qsa_status qsa_sparse_attn_decode_paged(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k_pages,
                                         const qsa_bf16 *v_pages, int64_t num_pages, int32_t page_size,
                                         const int32_t *block_table, int32_t max_pages,

@@ -66,12 +66,25 @@ static __device__ __noinline__ bool dec_issue(const CUtensorMap *map, AttShared 
     return true;
 }
 
+// A selection entry as a block to attend: -1 when there is none, when it lies outside
+// 0 .. b_t (flagged), or, for a context-parallel shard (blk_lo != nullptr), when it lies
+// outside the shard's block window [blk_lo[row], blk_hi[row]) (not flagged: another
+// shard holds it).
+__device__ __forceinline__ int32_t dec_block(int32_t raw, const RowInfo &ri, const int32_t *blk_lo,
+                                             const int32_t *blk_hi)
+{
+    int32_t b = check_block(raw, ri);
+    if (b >= 0 && blk_lo != nullptr && (b < __ldg(blk_lo + ri.row) || b >= __ldg(blk_hi + ri.row))) b = -1;
+    return b;
+}
+
 __global__ void __launch_bounds__(kAttThreads, 1)
 sparse_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                      const __grid_constant__ CUtensorMap map_v, const int32_t *__restrict__ sel,
                      const int32_t *__restrict__ cu_k, int64_t rows, int kb, int r, float scale,
                      float *__restrict__ ws, const int32_t *__restrict__ block_table, int page_size,
-                     int max_pages, int64_t num_pages)
+                     int max_pages, int64_t num_pages, const int64_t *__restrict__ tok_local,
+                     const int32_t *__restrict__ blk_lo, const int32_t *__restrict__ blk_hi)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -132,7 +145,10 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
         // one call site per ring slot use, 21 per chunk pair: a real call keeps the
         // producer's code small (the kernel's warps share the instruction cache)
         auto issue = [&](const CUtensorMap *map, const RowInfo &ri, int32_t blk) -> bool {
-            return dec_issue(map, sh, sSlot, &slot_it, abort_flag, lane, ri.tok_base, ri.row, blk, r, block_table,
+            // a shard's cache holds the window's tokens from tok_local[row] on
+            const int64_t tok_base =
+                tok_local != nullptr ? __ldg(tok_local + ri.row) - (int64_t)__ldg(blk_lo + ri.row) * r : ri.tok_base;
+            return dec_issue(map, sh, sSlot, &slot_it, abort_flag, lane, tok_base, ri.row, blk, r, block_table,
                              page_size, max_pages, num_pages);
         };
         for (int64_t item = 0; ok && item < n_items; ++item) {
@@ -156,7 +172,7 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
             const int len0 = nt < kCT ? nt : kCT;
 #pragma unroll
             for (int u = 0; u < kCT; ++u)
-                if (ok && u < len0) ok = issue(&map_k, ri, check_block(cur[u], ri));
+                if (ok && u < len0) ok = issue(&map_k, ri, dec_block(cur[u], ri, blk_lo, blk_hi));
             for (int q = 0; ok && q < nch; ++q) {
                 const int len = nt - q * kCT < kCT ? nt - q * kCT : kCT;
                 const int rest = nt - (q + 1) * kCT;
@@ -168,8 +184,8 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
                                  : kNoBlock;
 #pragma unroll
                 for (int u = 0; u < kCT; ++u) {
-                    if (ok && u < len) ok = issue(&map_v, ri, check_block(cur[u], ri));
-                    if (ok && u < lenn) ok = issue(&map_k, ri, check_block(nxt[u], ri));
+                    if (ok && u < len) ok = issue(&map_v, ri, dec_block(cur[u], ri, blk_lo, blk_hi));
+                    if (ok && u < lenn) ok = issue(&map_k, ri, dec_block(nxt[u], ri, blk_lo, blk_hi));
                 }
 #pragma unroll
                 for (int u = 0; u < kCT; ++u) cur[u] = nxt[u];
@@ -294,7 +310,8 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
 #pragma unroll
                 for (int u = 0; u < kCT; ++u) {
                     if (u < len) {
-                        const int32_t blk = check_block(load_block(sel, ri, kb, ri.p0 + (q * kCT + u) * kBlkTile + blk_slot), ri);
+                        const int32_t blk = dec_block(load_block(sel, ri, kb, ri.p0 + (q * kCT + u) * kBlkTile + blk_slot),
+                                                      ri, blk_lo, blk_hi);
                         if (blk >= 0 && (int64_t)blk * r + tok_in_blk <= ri.t) vmask |= 1u << u;
                     }
                 }
@@ -467,69 +484,108 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
 // merge the pieces of each row under the even schedule: the piece at the row's first
 // tile (slot grid + row) and one per share that starts inside the row and holds tiles
 // (slot = share).  The rows' first tiles come from the attention kernel (CTA 0).
-static_assert(kMaxEvenCtas <= kD, "one thread per share of the even schedule");
+// A warp per (row, head): its lanes find the row's pieces (32 shares at a time),
+// reduce their log-sum-exps, then sum the partial outputs in piece order, 8 dims per lane.
+constexpr int kMergeWarps = 8;  // heads per CTA (24 = 3 x 8)
+static_assert(kHQ % kMergeWarps == 0, "whole heads per CTA");
 
-__global__ void __launch_bounds__(kD)
+__global__ void __launch_bounds__(kMergeWarps * 32)
 even_combine_kernel(const float *__restrict__ ws, int grid, int64_t row_begin, int64_t rows,
                     __nv_bfloat16 *__restrict__ out, float *__restrict__ lse_out)
 {
-    __shared__ int s_slot[kMaxEvenCtas + 1];
-    __shared__ float s_l[kMaxEvenCtas + 1];
-    __shared__ int s_cnt[kD / 32];
     const int64_t rl = blockIdx.x;
-    const int h = blockIdx.y;
-    const int d = threadIdx.x, lane = d & 31, warp = d >> 5;
+    const int lane = threadIdx.x & 31;
+    const int h = blockIdx.y * kMergeWarps + (threadIdx.x >> 5);
     const int64_t n_slots = (int64_t)grid + rows;
     const float *lbase = ws + (size_t)n_slots * kHQ * kD;
     const int64_t *tile_prefix = reinterpret_cast<const int64_t *>(ws + (size_t)n_slots * kHQ * (kD + 1));
     const int64_t total = tile_prefix[rows], rs = tile_prefix[rl], re = tile_prefix[rl + 1];
-    __nv_bfloat16 *dst = out + ((row_begin + rl) * kHQ + h) * kD + d;
+    __nv_bfloat16 *dst = out + ((row_begin + rl) * kHQ + h) * kD + lane;
     if (re <= rs) {  // an empty sequence: nothing attended
-        *dst = __float2bfloat16_rn(0.f);
-        if (lse_out != nullptr && d == 0) lse_out[(row_begin + rl) * kHQ + h] = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < kD / 32; ++i) dst[i * 32] = __float2bfloat16_rn(0.f);
+        if (lse_out != nullptr && lane == 0) lse_out[(row_begin + rl) * kHQ + h] = -INFINITY;
         return;
     }
     // the row's pieces: its first-tile slot (grid + rl), then every share c >= c0 that
-    // starts inside the row and is not empty; share starts grow with c, so thread t tests
-    // share c0 + t (a row meets at most `grid` shares)
+    // starts inside the row and is not empty (share starts grow with c)
     auto share_start = [&](int64_t c) { return c * total / grid; };
     const int64_t c0 = rs * grid / total;
-    const int64_t c = c0 + d;
-    bool mine = false;
-    if (c < grid) {
+    auto is_piece = [&](int64_t c) {
+        if (c >= grid) return false;
         const int64_t sc = share_start(c);
-        mine = sc < re && sc > rs && share_start(c + 1) > sc;
+        return sc < re && sc > rs && share_start(c + 1) > sc;
+    };
+    const float l_first = lbase[((int64_t)grid + rl) * kHQ + h];
+    float mx = l_first;
+    for (int64_t cb = c0; cb < grid && share_start(cb) < re; cb += 32) {
+        const int64_t c = cb + lane;
+        if (is_piece(c)) mx = fmaxf(mx, lbase[c * kHQ + h]);
     }
-    const uint32_t m = __ballot_sync(0xffffffffu, mine);
-    if (lane == 0) s_cnt[warp] = __popc(m);
-    if (d == 0) {
-        s_slot[0] = grid + (int)rl;
-        s_l[0] = lbase[((int64_t)grid + rl) * kHQ + h];
-    }
-    __syncthreads();
-    int before = 1, npieces = 1;
 #pragma unroll
-    for (int x = 0; x < kD / 32; ++x) {
-        before += x < warp ? s_cnt[x] : 0;
-        npieces += s_cnt[x];
-    }
-    if (mine) {
-        const int pos = before + __popc(m & ((1u << lane) - 1u));
-        s_slot[pos] = (int)c;
-        s_l[pos] = lbase[c * kHQ + h];
-    }
-    __syncthreads();
-    float mx = -INFINITY;
-    for (int p = 0; p < npieces; ++p) mx = fmaxf(mx, s_l[p]);
-    float tot = 0.f, acc = 0.f;
-    for (int p = 0; p < npieces; ++p) {
-        const float l = s_l[p];
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    float tot = 0.f, acc[kD / 32];
+#pragma unroll
+    for (int i = 0; i < kD / 32; ++i) acc[i] = 0.f;
+    auto add = [&](int64_t slot, float l) {
         const float wgt = (l == -INFINITY) ? 0.f : __expf(l - mx);
         tot += wgt;
-        acc += wgt * __ldcs(ws + ((int64_t)s_slot[p] * kHQ + h) * kD + d);
+        const float *p = ws + (slot * kHQ + h) * kD + lane;
+        float o[kD / 32];
+#pragma unroll
+        for (int i = 0; i < kD / 32; ++i) o[i] = __ldcs(p + i * 32);
+#pragma unroll
+        for (int i = 0; i < kD / 32; ++i) acc[i] += wgt * o[i];
+    };
+    add((int64_t)grid + rl, l_first);
+    for (int64_t cb = c0; cb < grid && share_start(cb) < re; cb += 32) {
+        const int64_t c = cb + lane;
+        const bool mine = is_piece(c);
+        const float lc = mine ? lbase[c * kHQ + h] : -INFINITY;
+        uint32_t m = __ballot_sync(0xffffffffu, mine);
+        while (m != 0u) {  // in share order
+            const int src = __ffs(m) - 1;
+            m &= m - 1u;
+            add(cb + src, __shfl_sync(0xffffffffu, lc, src));
+        }
     }
-    *dst = __float2bfloat16_rn(tot > 0.f ? acc / tot : 0.f);
-    if (lse_out != nullptr && d == 0) lse_out[(row_begin + rl) * kHQ + h] = mx + logf(tot);
+    const float inv = tot > 0.f ? 1.f / tot : 0.f;
+#pragma unroll
+    for (int i = 0; i < kD / 32; ++i) dst[i * 32] = __float2bfloat16_rn(tot > 0.f ? acc[i] * inv : 0.f);
+    if (lse_out != nullptr && lane == 0) lse_out[(row_begin + rl) * kHQ + h] = mx + logf(tot);
+}
+
+// Context-parallel merge: the shards' normalised outputs o_p and log-sum-exps lse_p of
+// the same (row, head) give o = sum_p exp(lse_p - lse) o_p, lse = log sum_p exp(lse_p).
+// A warp per (row, head), 8 dims per lane, shards in order.
+__global__ void __launch_bounds__(kMergeWarps * 32)
+merge_states_kernel(const __nv_bfloat16 *__restrict__ o_parts, const float *__restrict__ lse_parts, int parts,
+                    int64_t rows, __nv_bfloat16 *__restrict__ o, float *__restrict__ lse)
+{
+    const int64_t rl = blockIdx.x;
+    const int lane = threadIdx.x & 31;
+    const int h = blockIdx.y * kMergeWarps + (threadIdx.x >> 5);
+    const int64_t stride_o = rows * kHQ * kD, stride_l = rows * kHQ;
+    float mx = -INFINITY;
+    for (int p = lane; p < parts; p += 32) mx = fmaxf(mx, lse_parts[p * stride_l + rl * kHQ + h]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    float tot = 0.f, acc[kD / 32];
+#pragma unroll
+    for (int i = 0; i < kD / 32; ++i) acc[i] = 0.f;
+    for (int p = 0; p < parts; ++p) {
+        const float l = lse_parts[p * stride_l + rl * kHQ + h];
+        const float wgt = (l == -INFINITY) ? 0.f : __expf(l - mx);
+        tot += wgt;
+        const __nv_bfloat16 *src = o_parts + p * stride_o + (rl * kHQ + h) * kD + lane;
+#pragma unroll
+        for (int i = 0; i < kD / 32; ++i) acc[i] += wgt * __bfloat162float(src[i * 32]);
+    }
+    __nv_bfloat16 *dst = o + (rl * kHQ + h) * kD + lane;
+    const float inv = tot > 0.f ? 1.f / tot : 0.f;
+#pragma unroll
+    for (int i = 0; i < kD / 32; ++i) dst[i * 32] = __float2bfloat16_rn(acc[i] * inv);
+    if (lse != nullptr && lane == 0) lse[rl * kHQ + h] = tot > 0.f ? mx + logf(tot) : -INFINITY;
 }
 
 }  // namespace
@@ -555,10 +611,21 @@ cudaError_t launch_sparse_decode(const AttnArgs &a, cudaStream_t stream)
     const int grid = even_grid();
     sparse_decode_kernel<<<(unsigned)grid, kAttThreads, kAttSmem, stream>>>(
         mq, mk, mv, a.sel, a.cu_k, rows, a.kb, a.r, a.scale, a.ws, a.block_table, a.page_size, a.max_pages,
-        a.block_table != nullptr ? a.total_k / a.page_size : 0);
+        a.block_table != nullptr ? a.total_k / a.page_size : 0, a.tok_local, a.blk_lo, a.blk_hi);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    even_combine_kernel<<<dim3((unsigned)rows, kHQ), kD, 0, stream>>>(a.ws, grid, a.row_begin, rows, a.o, a.lse);
+    even_combine_kernel<<<dim3((unsigned)rows, kHQ / kMergeWarps), kMergeWarps * 32, 0, stream>>>(
+        a.ws, grid, a.row_begin, rows, a.o, a.lse);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_merge_states(const __nv_bfloat16 *o_parts, const float *lse_parts, int parts, int64_t rows,
+                                __nv_bfloat16 *o, float *lse, cudaStream_t stream)
+{
+    if (rows <= 0) return cudaSuccess;
+    if (parts <= 0 || rows > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    merge_states_kernel<<<dim3((unsigned)rows, kHQ / kMergeWarps), kMergeWarps * 32, 0, stream>>>(
+        o_parts, lse_parts, parts, rows, o, lse);
     return cudaGetLastError();
 }
 

@@ -236,9 +236,17 @@ struct AttnArgs {
     // block_table [batch, max_pages] maps page j of sequence s to a page of the pool
     const int32_t *block_table = nullptr;
     int page_size = 0, max_pages = 0;
+    // decode of a context-parallel shard: the rows attend only selected blocks in
+    // [blk_lo[s], blk_hi[s]), whose tokens sit in k, v from row tok_local[s] on (cu_k keeps
+    // the sequences' global lengths: positions and causality are global)
+    const int64_t *tok_local = nullptr;
+    const int32_t *blk_lo = nullptr, *blk_hi = nullptr;
 };
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream);
 cudaError_t launch_sparse_decode(const AttnArgs &a, cudaStream_t stream);  // a.even: the decode kernel
+// (o, lse) of the same rows from `parts` shards merged by their log-sum-exps
+cudaError_t launch_merge_states(const __nv_bfloat16 *o_parts, const float *lse_parts, int parts, int64_t rows,
+                                __nv_bfloat16 *o, float *lse, cudaStream_t stream);
 // multi-token decode (attn_mtp.cu): next_n <= 4 queries per sequence, one shared selection
 int mtp_nsplit(int batch, int kb);
 size_t mtp_workspace_bytes(int batch, int kb);

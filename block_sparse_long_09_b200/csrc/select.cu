@@ -628,17 +628,27 @@ threshold_kernel(const float *__restrict__ sample, int64_t sample_ld, int stride
         return;
     }
     const float *srow = sample + rl * sample_ld;
-    for (int p = tid; p < ns; p += kThrThreads) keys[p] = order_key(__ldg(srow + p));
-    __syncthreads();
+    // keys relative to the sample's smallest: the radix starts at their highest differing bit
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int p = tid; p < ns; p += kThrThreads) {
+        const uint32_t u = order_key(__ldg(srow + p));
+        keys[p] = u;
+        kmin = min(kmin, u);
+        kmax = max(kmax, u);
+    }
+    kmin = ~kmin;
+    block_max2<kThrThreads>(kmin, kmax, &sc);  // (its barrier also publishes keys[])
+    kmin = ~kmin;
+    const uint32_t span = kmax - kmin;
     uint32_t prefix, mask;
     int need, in_bin;
     radix_select<kThrThreads, 8>(
         [&](auto f) {
-            for (int p = tid; p < ns; p += kThrThreads) f(keys[p]);
+            for (int p = tid; p < ns; p += kThrThreads) f(keys[p] - kmin);
         },
-        ns, r_lo, 31, hist, &sc, &prefix, &mask, &need, &in_bin);
-    // prefix is the r_lo-th largest key, or (bin taken whole) a lower bound of it
-    if (tid == 0) theta[rl] = key_value(prefix);
+        ns, r_lo, span != 0u ? 31 - __clz(span) : 0, hist, &sc, &prefix, &mask, &need, &in_bin);
+    // prefix + kmin is the r_lo-th largest key, or (bin taken whole) a lower bound of it
+    if (tid == 0) theta[rl] = key_value(prefix + kmin);
 }
 
 // The exact top k - 1 of a candidate list (order key, block index) in shared
@@ -651,13 +661,23 @@ __device__ __forceinline__ void select_from_list(const uint2 *cand, int cnt, int
 {
     const int tid = threadIdx.x;
     const int need_total = k - nf;
+    // keys relative to the list's smallest, so the radix starts at their highest differing bit
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int c = tid; c < cnt; c += kT) {
+        kmin = min(kmin, cand[c].x);
+        kmax = max(kmax, cand[c].x);
+    }
+    kmin = ~kmin;
+    block_max2<kT>(kmin, kmax, &sc);
+    kmin = ~kmin;
+    const uint32_t span = cnt > 0 ? kmax - kmin : 0u;
     uint32_t prefix, mask;
     int need, in_bin;
     radix_select<kT, 8>(
         [&](auto f) {
-            for (int c = tid; c < cnt; c += kT) f(cand[c].x);
+            for (int c = tid; c < cnt; c += kT) f(cand[c].x - kmin);
         },
-        cnt, need_total, 31, regA, &sc, &prefix, &mask, &need, &in_bin);
+        cnt, need_total, span != 0u ? 31 - __clz(span) : 0, regA, &sc, &prefix, &mask, &need, &in_bin);
     // winners: keys above the threshold bin, and of the bin either all (need == in_bin) or,
     // when the exact threshold value has more entries than slots left, its lowest indices
     uint32_t iprefix = 0u, imask = 0u;
@@ -667,12 +687,12 @@ __device__ __forceinline__ void select_from_list(const uint2 *cand, int cnt, int
         radix_select<kT, 8>(
             [&](auto f) {
                 for (int c = tid; c < cnt; c += kT)
-                    if ((cand[c].x & mask) == prefix) f(~cand[c].y);
+                    if (((cand[c].x - kmin) & mask) == prefix) f(~cand[c].y);
             },
             in_bin, need, 31, regA, &sc, &iprefix, &imask, &n2, &b2);
     }
     auto wins = [&](const uint2 e) -> bool {
-        const uint32_t u = e.x & mask;
+        const uint32_t u = (e.x - kmin) & mask;
         if (u != prefix) return u > prefix;
         return !partial || ((~e.y) & imask) >= iprefix;
     };
@@ -879,14 +899,24 @@ refine_select_kernel(const float *__restrict__ approx, int64_t ld, const __nv_bf
         const float mu = (float)need_total * (float)ns / (float)n;
         int r_lo = (int)ceilf(mu + 4.f * sqrtf(mu) + 8.f);
         if (r_lo > ns) r_lo = ns;
+        // keys relative to the sample's smallest: the radix starts at their highest differing bit
+        uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+        for (int q = tid; q < ns; q += kRefThreads) {
+            kmin = min(kmin, skeys[q]);
+            kmax = max(kmax, skeys[q]);
+        }
+        kmin = ~kmin;
+        block_max2<kRefThreads>(kmin, kmax, &sc);
+        kmin = ~kmin;
+        const uint32_t span = kmax - kmin;
         uint32_t sp, sm;
         int sn, sb;
         radix_select<kRefThreads, 8>(
             [&](auto f) {
-                for (int q = tid; q < ns; q += kRefThreads) f(skeys[q]);
+                for (int q = tid; q < ns; q += kRefThreads) f(skeys[q] - kmin);
             },
-            ns, r_lo, 31, regA, &sc, &sp, &sm, &sn, &sb);
-        theta_s = key_value(sp);
+            ns, r_lo, span != 0u ? 31 - __clz(span) : 0, regA, &sc, &sp, &sm, &sn, &sb);
+        theta_s = key_value(sp + kmin);  // the sample's r_lo-th largest, or its bin's floor
     }
     __syncthreads();
     // 2. the candidates W' = {b : approx_b >= theta_s - 2E} (with their approximate keys)
@@ -941,11 +971,23 @@ refine_select_kernel(const float *__restrict__ approx, int64_t ld, const __nv_bf
     }
     uint32_t prefix, mask;
     int need, in_bin;
-    radix_select<kRefThreads, 8>(
-        [&](auto f) {
-            for (int c = tid; c < nw; c += kRefThreads) f(cand[c].x);
-        },
-        nw, need_total, 31, regA, &sc, &prefix, &mask, &need, &in_bin);
+    {
+        uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+        for (int c = tid; c < nw; c += kRefThreads) {
+            kmin = min(kmin, cand[c].x);
+            kmax = max(kmax, cand[c].x);
+        }
+        kmin = ~kmin;
+        block_max2<kRefThreads>(kmin, kmax, &sc);
+        kmin = ~kmin;
+        const uint32_t span = kmax - kmin;
+        radix_select<kRefThreads, 8>(
+            [&](auto f) {
+                for (int c = tid; c < nw; c += kRefThreads) f(cand[c].x - kmin);
+            },
+            nw, need_total, span != 0u ? 31 - __clz(span) : 0, regA, &sc, &prefix, &mask, &need, &in_bin);
+        prefix += kmin;  // tau (or its bin's floor, a lower bound) as an absolute key
+    }
     //    the window W = {b : approx_b >= tau - 2E}: its block ids, compacted
     const uint32_t kw = order_key(key_value(prefix) - 2.f * e_row);
     if (tid == 0) wcount = 0;

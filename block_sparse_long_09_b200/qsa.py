@@ -38,7 +38,7 @@ EXPORTED = (
     "qsa_index_select_mtp", "qsa_sparse_attn_decode_mtp",
     "qsa_dense_attn_prefill",
     "qsa_workspace_size", "qsa_status_string", "qsa_get_device_status", "qsa_version", "qsa_debug_inject",
-    "qsa_rope_queries",
+    "qsa_rope_queries", "qsa_sparse_attn_decode_window", "qsa_merge_attn_states",
 )
 
 
@@ -94,6 +94,8 @@ def _load():
         "qsa_version": (I32, []),
         "qsa_debug_inject": (I32, [I32]),
         "qsa_rope_queries": (I32, [CP, P, P, P, I32, I64, P]),
+        "qsa_sparse_attn_decode_window": (I32, [CP, P, P, P, P, I32, I64, P, P, P, P, P, P, P, SZ, P]),
+        "qsa_merge_attn_states": (I32, [CP, P, P, I32, I64, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -377,6 +379,44 @@ def sparse_attn_decode_paged(q, k_pages, v_pages, block_table, cu_seqlens_k, sel
                                              _p(o), _p(lse), _p(ws), ws.numel(), _stream()),
            "qsa_sparse_attn_decode_paged")
     return (o, lse) if want_lse or lse is not None else o
+
+
+def sparse_attn_decode_window(q, k_local, v_local, cu_seqlens_k, tok_local, blk_lo, blk_hi, sel, o=None, lse=None,
+                              ws=None, cfg: Optional[Config] = None):
+    """One context-parallel shard's decode attention: the selected blocks inside
+    [blk_lo[s], blk_hi[s]) of each sequence, whose tokens sit in k_local / v_local from
+    row tok_local[s] on; cu_seqlens_k holds the global lengths.  Returns the partial
+    (o, lse) for qsa_merge_attn_states."""
+    cfg = _cfg(cfg)
+    batch = q.shape[0]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((batch, cfg.n_heads_q), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = torch.empty((workspace_size(OP_DECODE_PAGED, batch, batch, 0, cfg),), dtype=torch.uint8,
+                         device=q.device)
+    _check_sel(sel, batch, cfg)
+    _check(_lib.qsa_sparse_attn_decode_window(ctypes.byref(cfg), _p(q), _p(k_local), _p(v_local), _p(cu_seqlens_k),
+                                              batch, k_local.shape[0], _p(tok_local), _p(blk_lo), _p(blk_hi),
+                                              _p(sel), _p(o), _p(lse), _p(ws), ws.numel(), _stream()),
+           "qsa_sparse_attn_decode_window")
+    return o, lse
+
+
+def merge_attn_states(o_parts, lse_parts, o=None, lse=None, cfg: Optional[Config] = None):
+    """o, lse of rows from the partial states of several shards: o_parts [P, rows, 24, 256]
+    bf16, lse_parts [P, rows, 24] fp32."""
+    cfg = _cfg(cfg)
+    parts, rows = o_parts.shape[0], o_parts.shape[1]
+    if o is None:
+        o = torch.empty(o_parts.shape[1:], dtype=o_parts.dtype, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty(lse_parts.shape[1:], dtype=torch.float32, device=o_parts.device)
+    _check(_lib.qsa_merge_attn_states(ctypes.byref(cfg), _p(o_parts), _p(lse_parts), parts, rows, _p(o), _p(lse),
+                                      _stream()),
+           "qsa_merge_attn_states")
+    return o, lse
 
 
 def sparse_attn_decode_static_scratch(q, k_cache, v_cache, cu_seqlens_k, sel, o, lse=None,

@@ -338,6 +338,48 @@ qsa_status qsa_sparse_attn_decode_paged(const qsa_config *cfg, const qsa_bf16 *q
                                         qsa_bf16 *o, float *lse, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Context-parallel decode, one shard: a long-context decode whose K/V cache is split
+ * by block ranges over GPUs, one process per GPU.  The shard holds, for every
+ * sequence s, the global micro-blocks [blk_lo[s], blk_hi[s]) of its cache, whose
+ * tokens sit in k_local / v_local from row tok_local[s] on (the shard that holds a
+ * sequence's last block also holds its partial tail, up to L_s).  Every shard gets
+ * the same selection (qsa_select_blocks over the shards' score rows, see below) and
+ * attends only its own selected blocks: an id outside its window is skipped without
+ * a flag (another shard holds it); ids outside 0 .. b_t are flagged as always.
+ * o and lse are the shard's partial state: softmax over its blocks only (a row with
+ * none gets o = 0, lse = -inf).  qsa_merge_attn_states then gives the result of
+ * qsa_sparse_attn_decode over the whole cache (up to rounding).
+ *   cu_seqlens_k  [batch+1] int32: the sequences' GLOBAL lengths (t = L_s - 1)
+ *   tok_local     [batch] int64; blk_lo, blk_hi [batch] int32 (device)
+ *   k_local, v_local [total_k_local, n_heads_kv, head_dim] bf16
+ *   lse           [batch, n_heads_q] fp32 (required)
+ * The even schedule only (batch < 2 x the CTAs of the GPU, else QSA_ERR_UNSUPPORTED).
+ * Workspace: qsa_workspace_size(cfg, QSA_OP_DECODE_PAGED, batch, batch, 0) bytes.
+ *
+ * The shards' indexer scores: each shard scores its own blocks (qsa_index_scores
+ * with its compressed keys and per-sequence lengths L' with floor((L' - 1) / r) = n,
+ * its candidate blocks, and floor(L' / r) = its complete blocks) into its columns of
+ * a [batch, ld] row buffer; a sum over the shards
+ * (NCCL all-reduce; disjoint columns) gives every shard the full rows, and
+ * qsa_select_blocks on them gives the one-GPU selection bit for bit.
+ */
+qsa_status qsa_sparse_attn_decode_window(const qsa_config *cfg, const qsa_bf16 *q, const qsa_bf16 *k_local,
+                                         const qsa_bf16 *v_local, const int32_t *cu_seqlens_k, int32_t batch,
+                                         int64_t total_k_local, const int64_t *tok_local, const int32_t *blk_lo,
+                                         const int32_t *blk_hi, const int32_t *sel, qsa_bf16 *o, float *lse,
+                                         void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Merge of partial attention states of the same rows (context-parallel shards):
+ *   lse = log sum_p exp(lse_p),  o = sum_p exp(lse_p - lse) o_p
+ * (a part with lse_p = -inf counts for nothing; all -inf gives o = 0, lse = -inf).
+ *   o_parts [parts, rows, n_heads_q, head_dim] bf16; lse_parts [parts, rows, n_heads_q] fp32
+ *   o [rows, n_heads_q, head_dim] bf16; lse [rows, n_heads_q] fp32 or NULL
+ */
+qsa_status qsa_merge_attn_states(const qsa_config *cfg, const qsa_bf16 *o_parts, const float *lse_parts,
+                                 int32_t parts, int64_t rows, qsa_bf16 *o, float *lse, void *stream);
+
+/*
  * Sparse GQA attention, decode, with library-held scratch instead of a caller
  * workspace.  Computes exactly what qsa_sparse_attn_decode computes, with the
  * same schedule, and takes the same arguments minus ws / ws_bytes.
