@@ -41,15 +41,23 @@ __device__ __forceinline__ void index_row_cuda_at(const __nv_bfloat16 *__restric
         q[h][0] = a.x; q[h][1] = a.y; q[h][2] = b.x; q[h][3] = b.y;
     }
     const float wv = __ldg(w_row + (lane & 3));
-    for (int64_t b0 = c0 + warp * 8; b0 < c1; b0 += (int64_t)nwarps * 8) {
-        uint2 raw[8], rlo[8];
+    const int64_t stride = (int64_t)nwarps * 8;
+    // the next group's loads are issued before this group's arithmetic: two groups of
+    // gathered rows in flight per warp
+    uint2 raw[8], rlo[8];
+    auto load = [&](int64_t g0, uint2 (&hi)[8], uint2 (&lo)[8]) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const int64_t b = b0 + j;
+            const int64_t b = g0 + j;
             const __nv_bfloat16 *p = b < c1 ? kc_at(b) + lane * 4 : nullptr;
-            raw[j] = p != nullptr ? __ldg(reinterpret_cast<const uint2 *>(p)) : make_uint2(0u, 0u);
-            if (kPlanes == 2) rlo[j] = p != nullptr ? __ldg(reinterpret_cast<const uint2 *>(p + 128)) : make_uint2(0u, 0u);
+            hi[j] = p != nullptr ? __ldg(reinterpret_cast<const uint2 *>(p)) : make_uint2(0u, 0u);
+            if (kPlanes == 2) lo[j] = p != nullptr ? __ldg(reinterpret_cast<const uint2 *>(p + 128)) : make_uint2(0u, 0u);
         }
+    };
+    if (c0 + warp * 8 < c1) load(c0 + warp * 8, raw, rlo);
+    for (int64_t b0 = c0 + warp * 8; b0 < c1; b0 += stride) {
+        uint2 nraw[8], nrlo[8];
+        if (b0 + stride < c1) load(b0 + stride, nraw, nrlo);
         float v[32];  // v[j * 4 + h] = partial dot of block b0 + j with head h
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -80,6 +88,11 @@ __device__ __forceinline__ void index_row_cuda_at(const __nv_bfloat16 *__restric
         sc += __shfl_xor_sync(0xffffffffu, sc, 2);
         const int64_t b = b0 + (lane >> 2);
         if ((lane & 3) == 0 && b < c1) srow[b] = sc;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            raw[j] = nraw[j];
+            if (kPlanes == 2) rlo[j] = nrlo[j];
+        }
     }
 }
 

@@ -935,21 +935,33 @@ refine_select_kernel(const float *__restrict__ approx, int64_t ld, const __nv_bf
                 const int g = g0 + u * kRefThreads + tid;
                 x4[u] = g < n4 ? __ldg(srow4 + g) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
             }
+            // the warp's hits of the whole batch take one reservation of list slots
+            uint32_t m[kRefUnroll * 4];
+            int total = 0;
 #pragma unroll
             for (int u = 0; u < kRefUnroll; ++u) {
                 const int g = g0 + u * kRefThreads + tid;
                 const float xs[4] = {x4[u].x, x4[u].y, x4[u].z, x4[u].w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int j = 4 * g + e;
-                    const bool hit = j < n && xs[e] >= lo_bound;
-                    const uint32_t m = __ballot_sync(0xffffffffu, hit);
-                    if (m == 0u) continue;  // warp-uniform
-                    int base = 0;
-                    if (lane == 0) base = atomicAdd(&wcount, __popc(m));
-                    base = __shfl_sync(0xffffffffu, base, 0);
-                    const int pos = base + __popc(m & lt_mask);
-                    if (hit && pos < kRefCap) cand[pos] = make_uint2(order_key(xs[e]), (uint32_t)j);
+                    m[u * 4 + e] = __ballot_sync(0xffffffffu, 4 * g + e < n && xs[e] >= lo_bound);
+                    total += __popc(m[u * 4 + e]);
+                }
+            }
+            if (total == 0) continue;  // warp-uniform
+            int base = 0;
+            if (lane == 0) base = atomicAdd(&wcount, total);
+            base = __shfl_sync(0xffffffffu, base, 0);
+#pragma unroll
+            for (int u = 0; u < kRefUnroll; ++u) {
+                const int g = g0 + u * kRefThreads + tid;
+                const float xs[4] = {x4[u].x, x4[u].y, x4[u].z, x4[u].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t mk = m[u * 4 + e];
+                    const int pos = base + __popc(mk & lt_mask);
+                    if (((mk >> lane) & 1u) && pos < kRefCap) cand[pos] = make_uint2(order_key(xs[e]), (uint32_t)(4 * g + e));
+                    base += __popc(mk);
                 }
             }
         }
