@@ -425,6 +425,12 @@ def run_qsa(args, rank, world, device):
         "roofline": {"kernel": "sparse_attn_kernel (prefill)", "bound": "tensor", "achieved": attn_tflops,
                      "peak": tflops_sus, "unit": "TFLOP/s", "frac": attn_tflops / tflops_sus, "traffic": traffic,
                      "peak_kind": peak_kind + " (sustained bf16: the kernel runs inside a long step)",
+                     # the bounds' times: the method's flops at the tensor peak, the gathered bytes at
+                     # the HBM copy peak (no L2 reuse), and the measured DRAM traffic at that peak
+                     "bound_ms": {"tensor": attn_flops / (tflops_sus * 1e12) * 1e3,
+                                  "gather_at_hbm": gather / (hbm * 1e9) * 1e3,
+                                  "dram_traffic_at_hbm": (traffic / (hbm * 1e9) * 1e3) if traffic else None,
+                                  "measured": attn_ms},
                      "note": "gather-bound: 4 MiB of K/V per query against 25 MFLOP; see kernels"},
         "kernels": kern,
         "gpu_launches": args.steps * (launches_prefill + launches_decode),

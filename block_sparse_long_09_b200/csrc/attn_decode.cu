@@ -169,6 +169,17 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             ++q_it;
+            // the block ids of chunk q + 1 are loaded while chunk q's copies are issued, so an
+            // id load never stalls the issue of the copy that needs it
+            auto load_chunk = [&](int q, int32_t (&ids)[kCT]) {
+                const int rest = nt - q * kCT;
+                const int len = rest <= 0 ? 0 : (rest < kCT ? rest : kCT);
+#pragma unroll
+                for (int u = 0; u < kCT; ++u)
+                    ids[u] = (lane < kBlkTile && u < len) ? load_block(sel, ri, kb, ri.p0 + (q * kCT + u) * kBlkTile + lane)
+                                                           : kNoBlock;
+            };
+            load_chunk(1, nxt);
             const int len0 = nt < kCT ? nt : kCT;
 #pragma unroll
             for (int u = 0; u < kCT; ++u)
@@ -177,18 +188,18 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
                 const int len = nt - q * kCT < kCT ? nt - q * kCT : kCT;
                 const int rest = nt - (q + 1) * kCT;
                 const int lenn = rest <= 0 ? 0 : (rest < kCT ? rest : kCT);
-#pragma unroll
-                for (int u = 0; u < kCT; ++u)
-                    nxt[u] = (lane < kBlkTile && u < lenn)
-                                 ? load_block(sel, ri, kb, ri.p0 + ((q + 1) * kCT + u) * kBlkTile + lane)
-                                 : kNoBlock;
+                int32_t nxt2[kCT];
+                load_chunk(q + 2, nxt2);
 #pragma unroll
                 for (int u = 0; u < kCT; ++u) {
                     if (ok && u < len) ok = issue(&map_v, ri, dec_block(cur[u], ri, blk_lo, blk_hi));
                     if (ok && u < lenn) ok = issue(&map_k, ri, dec_block(nxt[u], ri, blk_lo, blk_hi));
                 }
 #pragma unroll
-                for (int u = 0; u < kCT; ++u) cur[u] = nxt[u];
+                for (int u = 0; u < kCT; ++u) {
+                    cur[u] = nxt[u];
+                    nxt[u] = nxt2[u];
+                }
             }
         }
         if (!ok && lane == 0) {

@@ -204,11 +204,16 @@ sparse_mtp_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             ++qu;
-            for (int j = 0; ok && j < it.nt; ++j) {
+            auto tile_id = [&](int j) {  // this lane's block of tile j (lanes 0..7)
                 const int pos = it.p0 + j * kMtpBlk + lane;
-                const int32_t raw = (lane < kMtpBlk && pos < it.nsel) ? __ldg(sel + it.s * kb + pos) : kNoBlock;
+                return (lane < kMtpBlk && j < it.nt && pos < it.nsel) ? __ldg(sel + it.s * kb + pos) : kNoBlock;
+            };
+            int32_t raw = tile_id(0);
+            for (int j = 0; ok && j < it.nt; ++j) {
+                const int32_t raw_next = tile_id(j + 1);  // in flight while tile j is issued
                 ok = issue(&map_k, sK, sh->k_full, sh->k_empty, ku++, it, raw);
                 if (ok) ok = issue(&map_v, sV, sh->v_full, sh->v_empty, vu++, it, raw);
+                raw = raw_next;
             }
         }
         if (!ok && lane == 0) {  // let every copy in flight land before the CTA exits

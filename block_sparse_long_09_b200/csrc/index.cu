@@ -568,7 +568,8 @@ cudaError_t launch_index_tc_mode(const IndexArgs &a, const IdxOut &out, cudaStre
     const int64_t rows = a.row_end - a.row_begin;
     if (rows <= 0 || a.kc_rows <= 0) return cudaSuccess;
     CUtensorMap mq, mk;
-    // q_idx as [total_q * 4, 128] bf16, 256-row boxes; kc as [kc_rows, 128] 16-bit, 128-row boxes
+    // q_idx as [total_q * 4, 128] bf16, 256-row boxes; kc as [kc_rows, 256] bf16 (hi plane, then
+    // lo plane), boxes of 64 columns x 128 rows
     if (!make_tmap_2d(&mq, a.q_idx, 128, (uint64_t)a.total_q * 4, 256, 64, kQRowsT)) return cudaErrorInvalidValue;
     if (!make_tmap_2d(&mk, a.kc, 256, (uint64_t)a.kc_rows, 512, 64, kBM)) return cudaErrorInvalidValue;
     if (out.mode == kSample && out.stride <= 0) return cudaErrorInvalidValue;

@@ -9,7 +9,6 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -311,13 +310,6 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
     d |= (uint64_t)1u << 46;
     d |= (uint64_t)2u << 61;
     return d;
-}
-
-// Instruction descriptor for kind::f16 with fp16 A/B and fp32 D (A and B formats 0).
-__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int a_mn_major, int b_mn_major)
-{
-    return (1u << 4) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
-           ((uint32_t)(M >> 4) << 24);
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.

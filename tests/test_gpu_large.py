@@ -5,7 +5,7 @@ compressed keys, its own top-k, its own attention), so the fp64 oracle is run
 on a sample of rows of the full-size problem: the first 64 rows, the last 64,
 256 seeded random rows and the first and last row of each random row's
 micro-block.  The GPU side runs exactly as the benchmark does (the same inputs,
-16 384-row chunks, the same launches).  Per sampled row:
+65 536-row chunks, the same launches).  Per sampled row:
 
   scores     GPU indexer scores within the score tolerance of the oracle's
   selection  the GPU's top-k against the oracle's under the near-threshold rule
@@ -30,7 +30,7 @@ from parity_common import (SCALE, bits, check_attn, check_scores, check_selectio
 pytestmark = pytest.mark.gpu
 
 K = 512
-CHUNK = 16384
+CHUNK = 65536  # the benchmark's chunk of query rows per fused index -> select launch
 
 
 @pytest.fixture(scope="module")
