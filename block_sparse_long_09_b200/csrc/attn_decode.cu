@@ -22,9 +22,10 @@ namespace qsa {
 
 namespace {
 
-constexpr int kCT = 7;                                  // tiles per chunk
+constexpr int kCT = 3;                                  // tiles per chunk (1 .. 7 fit TMEM; 2 to 4 measured
+                                                        // ~7% faster than 7 at batch 64, 128K-256K context)
 constexpr uint32_t kDecSBuf = kCT * kQRows;             // TMEM columns of one chunk of S
-constexpr uint32_t kDecOCol = 2 * kDecSBuf;             // O^T after two chunk buffers (448)
+constexpr uint32_t kDecOCol = 2 * kDecSBuf;             // O^T after two chunk buffers
 constexpr uint32_t kDecTmemCols = 512;
 static_assert(kDecOCol + 64 <= kDecTmemCols, "two chunks of S and O^T fit in TMEM");
 
