@@ -529,6 +529,103 @@ class Prefill:
         self.index_select(q_idx, w, k_idx)
         return self.attend(q, k, v, o=o, lse=lse)
 
+    def from_host(self, q, k, v, q_idx, w, k_idx, o, lse=None, pipe_rows: int = 16384):
+        """The whole prefill from host memory, copies overlapped with the compute.
+
+        q, k, v, q_idx, w, k_idx are host tensors and o (and lse) host outputs, all
+        pinned so that the copies run asynchronously.  One copy stream brings in k_idx,
+        then q_idx and w per selection chunk, then k, v and q per attention chunk of
+        pipe_rows rows; the current stream compresses, selects and attends each chunk as
+        soon as its inputs have landed; a second copy stream returns each chunk's output
+        while the next one is computed.  The device buffers are allocated on the first
+        call and reused.  The current stream waits for the last copy back, so events
+        recorded on it around the call time the whole step; it returns o."""
+        dev = torch.device(self.device)
+        cur = torch.cuda.current_stream(dev)
+        if getattr(self, "_copy_streams", None) is None:
+            self._copy_streams = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+        h2d, d2h = self._copy_streams
+        host = {"q": q, "k": k, "v": v, "q_idx": q_idx, "w": w, "k_idx": k_idx}
+        stage = getattr(self, "_stage", None)
+        if stage is None or any(stage[n].shape != t.shape or stage[n].dtype != t.dtype for n, t in host.items()):
+            stage = {n: torch.empty(t.shape, dtype=t.dtype, device=dev) for n, t in host.items()}
+            stage["o"] = torch.empty(o.shape, dtype=o.dtype, device=dev)
+            self._stage = stage
+        d_lse = None
+        if lse is not None:
+            if getattr(self, "_stage_lse", None) is None or self._stage_lse.shape != lse.shape:
+                self._stage_lse = torch.empty(lse.shape, dtype=lse.dtype, device=dev)
+            d_lse = self._stage_lse
+        if self.ws is not None:  # the key-chunked schedule's workspace holds self.chunk rows
+            pipe_rows = min(int(pipe_rows), self.chunk)
+        plan = prefill_copy_plan(self.total, self.chunk, int(pipe_rows), self.cfg.r)
+        h2d.wait_stream(cur)  # the previous step's compute is done with the buffers
+        d2h.wait_stream(cur)
+
+        def put(name, a, b):
+            if b > a:
+                stage[name][a:b].copy_(host[name][a:b], non_blocking=True)
+
+        with torch.cuda.stream(h2d):
+            put("k_idx", 0, self.total)
+            ev_kidx = h2d.record_event()
+            ev_sel = []
+            for (_, _), (a, b) in plan["select"]:
+                put("q_idx", a, b)
+                put("w", a, b)
+                ev_sel.append(h2d.record_event())
+            ev_att = []
+            for (_, _), (ka, kb), (qa, qb) in plan["attend"]:
+                put("k", ka, kb)
+                put("v", ka, kb)
+                put("q", qa, qb)
+                ev_att.append(h2d.record_event())
+        cur.wait_event(ev_kidx)
+        compress_keys(stage["k_idx"], self.cu, self.cu_blocks, kc=self.kc, cfg=self.cfg)
+        for ((r0, r1), _), e in zip(plan["select"], ev_sel):
+            cur.wait_event(e)
+            self.select_chunk(stage["q_idx"], stage["w"], r0, r1)
+        ev_out = []
+        for ((r0, r1), _, _), e in zip(plan["attend"], ev_att):
+            cur.wait_event(e)
+            sparse_attn_prefill(stage["q"], stage["k"], stage["v"], self.sel, self.cu, self.cu, r0, r1, o=stage["o"],
+                                lse=d_lse, cfg=self.cfg, ws=self.ws, max_len_k=self.max_len)
+            ev_out.append(cur.record_event())
+        with torch.cuda.stream(d2h):
+            for ((r0, r1), _, _), e in zip(plan["attend"], ev_out):
+                d2h.wait_event(e)
+                o[r0:r1].copy_(stage["o"][r0:r1], non_blocking=True)
+                if lse is not None:
+                    lse[r0:r1].copy_(d_lse[r0:r1], non_blocking=True)
+            done = d2h.record_event()
+        cur.wait_event(done)
+        return o
+
+
+def prefill_copy_plan(total: int, select_rows: int, attend_rows: int, r: int = 4):
+    """The row ranges of Prefill.from_host: for each selection chunk (r0, r1) the rows of
+    q_idx and w copied before it, and for each attention chunk (r0, r1) the rows of k, v
+    and of q copied before it.  Every row is copied once, in order.  The indexer reads
+    whole 64-row tiles, so a selection chunk's copy reaches 63 rows past r1; the attention
+    loads whole micro-blocks, so its k and v copy reaches r - 1 rows past r1 (those keys
+    are masked, but must hold finite values)."""
+    if select_rows <= 0 or attend_rows <= 0:
+        raise ValueError("chunk sizes must be positive")
+    sel, att = [], []
+    done = 0
+    for r0 in range(0, total, select_rows):
+        r1 = min(total, r0 + select_rows)
+        hi = min(total, r1 + 63)
+        sel.append(((r0, r1), (done, max(done, hi))))
+        done = max(done, hi)
+    kv_done = q_done = 0
+    for r0 in range(0, total, attend_rows):
+        r1 = min(total, r0 + attend_rows)
+        kv_hi = max(kv_done, min(total, r1 + r - 1))
+        att.append(((r0, r1), (kv_done, kv_hi), (q_done, r1)))
+        kv_done, q_done = kv_hi, r1
+    return {"select": sel, "attend": att}
+
 
 class DecodeStep:
     """One QSA decode step for a fixed batch, one new query per sequence: refresh

@@ -150,3 +150,30 @@ def test_rope_config_checked_on_the_host(qsa):
         assert lib.qsa_rope_queries(ctypes.byref(bad), fake, fake, fake, 1, 8, None) == qsa.QSA_ERR_INVALID_ARG
         assert lib.qsa_compress_keys(ctypes.byref(bad), fake, fake, fake, 1, 8, None, 0, fake, None) == \
             qsa.QSA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("total,sel_rows,att_rows", [(1, 1, 1), (9001, 4096, 3000), (70000, 65536, 16384),
+                                                     (262144, 65536, 16384), (64, 1000, 7), (5, 2, 3)])
+def test_prefill_copy_plan_covers_every_row_once_and_in_time(qsa, total, sel_rows, att_rows):
+    """Prefill.from_host's copy plan: each tensor's rows are copied exactly once, in
+    order, and every chunk's reads (whole 64-row indexer tiles, whole 4-token blocks of
+    keys up to the chunk's last row) are covered by the copies issued before it."""
+    r = 4
+    plan = qsa.prefill_copy_plan(total, sel_rows, att_rows, r)
+    sel, att = plan["select"], plan["attend"]
+    # the chunks tile the rows
+    assert [c[0] for c in sel] == [(a, min(total, a + sel_rows)) for a in range(0, total, sel_rows)]
+    assert [c[0] for c in att] == [(a, min(total, a + att_rows)) for a in range(0, total, att_rows)]
+    for ranges in ([c[1] for c in sel], [c[1] for c in att], [c[2] for c in att]):
+        pos = 0
+        for a, b in ranges:  # contiguous, in order, never backwards
+            assert a == pos and b >= a
+            pos = b
+        assert pos == total   # every row copied, once
+    for (r0, r1), (_, hi) in sel:
+        assert hi >= min(total, (r1 + 63) // 64 * 64)  # the last indexer tile of the chunk
+    for (r0, r1), (_, kv_hi), (_, q_hi) in att:
+        assert q_hi >= r1
+        assert kv_hi >= min(total, r1 - 1 + r)          # the micro-block holding row r1 - 1, loaded whole
+    with pytest.raises(ValueError):
+        qsa.prefill_copy_plan(10, 0, 4)
