@@ -87,6 +87,7 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
                      int max_pages, int64_t num_pages, const int64_t *__restrict__ tok_local,
                      const int32_t *__restrict__ blk_lo, const int32_t *__restrict__ blk_hi)
 {
+    pdl_enter();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sSlot = smem;
@@ -505,6 +506,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
 even_combine_kernel(const float *__restrict__ ws, int grid, int64_t row_begin, int64_t rows,
                     __nv_bfloat16 *__restrict__ out, float *__restrict__ lse_out)
 {
+    pdl_enter();
     const int64_t rl = blockIdx.x;
     const int lane = threadIdx.x & 31;
     const int h = blockIdx.y * kMergeWarps + (threadIdx.x >> 5);
@@ -621,14 +623,13 @@ cudaError_t launch_sparse_decode(const AttnArgs &a, cudaStream_t stream)
         if (e != cudaSuccess) return e;
     }
     const int grid = even_grid();
-    sparse_decode_kernel<<<(unsigned)grid, kAttThreads, kAttSmem, stream>>>(
-        mq, mk, mv, a.sel, a.cu_k, rows, a.kb, a.r, a.scale, a.ws, a.block_table, a.page_size, a.max_pages,
-        a.block_table != nullptr ? a.total_k / a.page_size : 0, a.tok_local, a.blk_lo, a.blk_hi);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(sparse_decode_kernel, dim3((unsigned)grid), dim3(kAttThreads), kAttSmem, stream, mq, mk,
+                               mv, a.sel, a.cu_k, rows, a.kb, a.r, a.scale, a.ws, a.block_table, a.page_size,
+                               a.max_pages, a.block_table != nullptr ? a.total_k / a.page_size : (int64_t)0,
+                               a.tok_local, a.blk_lo, a.blk_hi);
     if (e != cudaSuccess) return e;
-    even_combine_kernel<<<dim3((unsigned)rows, kHQ / kMergeWarps), kMergeWarps * 32, 0, stream>>>(
-        a.ws, grid, a.row_begin, rows, a.o, a.lse);
-    return cudaGetLastError();
+    return launch_pdl(even_combine_kernel, dim3((unsigned)rows, kHQ / kMergeWarps), dim3(kMergeWarps * 32), 0, stream,
+                      (const float *)a.ws, grid, a.row_begin, rows, a.o, a.lse);
 }
 
 cudaError_t launch_merge_states(const __nv_bfloat16 *o_parts, const float *lse_parts, int parts, int64_t rows,

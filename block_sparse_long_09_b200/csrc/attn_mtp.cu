@@ -104,6 +104,7 @@ sparse_mtp_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                   float *__restrict__ ws, const int32_t *__restrict__ block_table, int page_size, int max_pages,
                   int64_t num_pages)
 {
+    pdl_enter();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem;
@@ -464,6 +465,7 @@ __global__ void __launch_bounds__(kCombRows * 32)
 mtp_combine_kernel(const float *__restrict__ ws, int64_t n_items, int nsplit, int next_n,
                    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse_out)
 {
+    pdl_enter();
     const int64_t s = blockIdx.x;
     const int lane = threadIdx.x & 31;
     const int R = blockIdx.y * kCombRows + (threadIdx.x >> 5);  // (query, head) row
@@ -548,14 +550,13 @@ cudaError_t launch_sparse_mtp(const AttnArgs &a, int next_n, cudaStream_t stream
     const int64_t n_items = batch * nsplit;
     int64_t grid = num_sms();
     if (grid > n_items) grid = n_items;
-    sparse_mtp_kernel<<<(unsigned)grid, kMtpThreads, kMtpSmem, stream>>>(
-        mq, mk, mv, a.sel, a.cu_k, (int)batch, next_n, nsplit, a.kb, a.r, a.scale, a.o, a.lse, a.ws, a.block_table,
-        a.page_size, a.max_pages, a.block_table != nullptr ? a.total_k / a.page_size : 0);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(sparse_mtp_kernel, dim3((unsigned)grid), dim3(kMtpThreads), kMtpSmem, stream, mq, mk, mv,
+                               a.sel, a.cu_k, (int)batch, next_n, nsplit, a.kb, a.r, a.scale, a.o, a.lse, a.ws,
+                               a.block_table, a.page_size, a.max_pages,
+                               a.block_table != nullptr ? a.total_k / a.page_size : (int64_t)0);
     if (e != cudaSuccess || nsplit == 1) return e;
-    mtp_combine_kernel<<<dim3((unsigned)batch, (unsigned)((next_n * kHQ + kCombRows - 1) / kCombRows)),
-                         kCombRows * 32, 0, stream>>>(a.ws, n_items, nsplit, next_n, a.o, a.lse);
-    return cudaGetLastError();
+    return launch_pdl(mtp_combine_kernel, dim3((unsigned)batch, (unsigned)((next_n * kHQ + kCombRows - 1) / kCombRows)),
+                      dim3(kCombRows * 32), 0, stream, (const float *)a.ws, n_items, nsplit, next_n, a.o, a.lse);
 }
 
 }  // namespace qsa

@@ -28,6 +28,7 @@ compress_kernel(const __nv_bfloat16 *__restrict__ k_idx, const int32_t *__restri
                 const int32_t *__restrict__ blk_begin, int max_new, int r, int normalise,
                 float eps, __nv_bfloat16 *__restrict__ kc, const RopeSpec rope)
 {
+    pdl_enter();
     const int lane = threadIdx.x & 31;
     const int64_t warp_global = (int64_t)blockIdx.x * kCompressWarps + (threadIdx.x >> 5);
     const int64_t nwarps = (int64_t)gridDim.x * kCompressWarps;
@@ -150,9 +151,8 @@ cudaError_t launch_compress(const __nv_bfloat16 *k_idx, const int32_t *cu_k, con
     int64_t grid = (n_items + kCompressWarps - 1) / kCompressWarps;
     const int64_t cap = 148 * 16;
     if (grid > cap) grid = cap;
-    compress_kernel<<<(unsigned)grid, kCompressWarps * 32, 0, stream>>>(
-        k_idx, cu_k, cu_blocks, batch, n_items, blk_begin, max_new, r, normalise ? 1 : 0, eps, kc, rope);
-    return cudaGetLastError();
+    return launch_pdl(compress_kernel, dim3((unsigned)grid), dim3(kCompressWarps * 32), 0, stream, k_idx, cu_k,
+                      cu_blocks, batch, n_items, blk_begin, max_new, r, normalise ? 1 : 0, eps, kc, rope);
 }
 
 }  // namespace qsa

@@ -427,6 +427,7 @@ index_gemv_hi_kernel(const __grid_constant__ CUtensorMap map_kc, const __nv_bflo
                      const int32_t *__restrict__ cu_k, const int32_t *__restrict__ cu_blocks, int batch,
                      int64_t row_begin, float *__restrict__ scores, int64_t ld, int r)
 {
+    pdl_enter();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sK = smem;                               // stages of kc tiles (1 KB aligned)
@@ -629,11 +630,12 @@ cudaError_t launch_index_rowwise_hi(const IndexArgs &a, cudaStream_t stream)
     const int64_t chunks = (a.ld + kGvChunk - 1) / kGvChunk;
     for (int64_t done = 0; done < rows; done += 65535) {
         const int64_t n = rows - done < 65535 ? rows - done : 65535;
-        index_gemv_hi_kernel<<<dim3((unsigned)chunks, (unsigned)n), kGvThreads, kGvSmem, stream>>>(
-            mk, a.q_idx, a.w, a.cu_q, a.cu_k, a.cu_blocks, a.batch, a.row_begin + done, a.scores + done * a.ld, a.ld,
-            a.r);
+        const cudaError_t e = launch_pdl(index_gemv_hi_kernel, dim3((unsigned)chunks, (unsigned)n), dim3(kGvThreads),
+                                         kGvSmem, stream, mk, a.q_idx, a.w, a.cu_q, a.cu_k, a.cu_blocks, a.batch,
+                                         a.row_begin + done, a.scores + done * a.ld, a.ld, a.r);
+        if (e != cudaSuccess) return e;
     }
-    return cudaGetLastError();
+    return cudaSuccess;
 }
 
 }  // namespace qsa

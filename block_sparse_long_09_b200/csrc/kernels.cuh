@@ -1,6 +1,8 @@
 // kernels.cuh -- internal launch interface between the C ABI (api.cu) and the kernels.
 #pragma once
 
+#include <utility>
+
 #include "sm100.cuh"
 
 namespace qsa {
@@ -291,6 +293,25 @@ bool make_tmap_2d_f32(CUtensorMap *map, const void *base, uint64_t inner, uint64
 bool make_tmap_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
 int num_sms();
+// Launch `kernel` with programmatic stream serialisation: it may be scheduled while the
+// previous kernel of the stream still runs, so it must begin with pdl_enter().
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args &&...args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Opt-in dynamic shared memory of `func` on the current device, set once per device
 // (thread-safe; later calls on that device only look it up).
 cudaError_t set_smem_attr_once(const void *func, int bytes);

@@ -778,6 +778,7 @@ fallback_kernel(const __nv_bfloat16 *__restrict__ q_idx, const float *__restrict
                 const int32_t *__restrict__ fb_count, const int32_t *__restrict__ fb_rows, float *__restrict__ scratch,
                 int64_t scratch_ld, int32_t *__restrict__ sel, int next_n)
 {
+    pdl_enter();
     extern __shared__ uint32_t smem_sel[];
     __shared__ SelScratch sc;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -828,6 +829,7 @@ refine_select_kernel(const float *__restrict__ approx, int64_t ld, const __nv_bf
                      int32_t *__restrict__ sel, int32_t *__restrict__ fb_count, int32_t *__restrict__ fb_rows,
                      int next_n)
 {
+    pdl_enter();
     extern __shared__ uint32_t smem_sel[];
     uint32_t *regA = smem_sel;                                        // kSegWords words
     uint2 *cand = reinterpret_cast<uint2 *>(smem_sel + kSegWords);    // kRefCap (key, index)
@@ -1026,7 +1028,11 @@ refine_select_kernel(const float *__restrict__ approx, int64_t ld, const __nv_bf
     select_from_list<kRefThreads>(cand, nw, bt, k, out, regA, sc, nf);
 }
 
-__global__ void clear_count_kernel(int32_t *c) { *c = 0; }
+__global__ void clear_count_kernel(int32_t *c)
+{
+    pdl_enter();
+    *c = 0;
+}
 
 }  // namespace
 
@@ -1156,18 +1162,17 @@ cudaError_t launch_decode_index_select(const IndexArgs &a, int k, void *ws, int 
         return launch_select(sa, stream);
     }
     if ((e = launch_index_rowwise_hi(a2, stream)) != cudaSuccess) return e;
-    clear_count_kernel<<<1, 1, 0, stream>>>(fb_count);
+    if ((e = launch_pdl(clear_count_kernel, dim3(1), dim3(1), 0, stream, fb_count)) != cudaSuccess) return e;
     if ((e = set_smem_attr_once(reinterpret_cast<const void *>(refine_select_kernel), kRefSmem)) != cudaSuccess)
         return e;
     if (rows > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    refine_select_kernel<<<(unsigned)rows, kRefThreads, kRefSmem, stream>>>(
-        scores, a.ld, a.q_idx, a.w, a.kc, a.cu_q, a.cu_k, a.cu_blocks, a.batch, a.row_begin, k, a.r, sel, fb_count,
-        fb_rows, next_n);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    fallback_kernel<<<(unsigned)grid, kFbThreads, sel_smem_bytes<kFbThreads>(), stream>>>(
-        a.q_idx, a.w, a.kc, a.cu_q, a.cu_k, a.cu_blocks, a.batch, a.row_begin, k, a.r, fb_count, fb_rows, scratch,
-        a.ld, sel, next_n);
-    return cudaGetLastError();
+    if ((e = launch_pdl(refine_select_kernel, dim3((unsigned)rows), dim3(kRefThreads), kRefSmem, stream,
+                        (const float *)scores, a.ld, a.q_idx, a.w, a.kc, a.cu_q, a.cu_k, a.cu_blocks, a.batch,
+                        a.row_begin, k, a.r, sel, fb_count, fb_rows, next_n)) != cudaSuccess)
+        return e;
+    return launch_pdl(fallback_kernel, dim3((unsigned)grid), dim3(kFbThreads), sel_smem_bytes<kFbThreads>(), stream,
+                      a.q_idx, a.w, a.kc, a.cu_q, a.cu_k, a.cu_blocks, a.batch, a.row_begin, k, a.r,
+                      (const int32_t *)fb_count, (const int32_t *)fb_rows, scratch, a.ld, sel, next_n);
 }
 
 }  // namespace qsa

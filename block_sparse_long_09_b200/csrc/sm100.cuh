@@ -127,6 +127,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with launch_pdl may be scheduled
+// while the previous kernel of its stream still runs.  pdl_wait blocks until that kernel
+// has completed and its writes are visible (it returns at once for a normal launch);
+// every kernel that launch_pdl starts calls it before its first global-memory access.
+// pdl_trigger, issued after the wait, lets the next kernel of the stream be scheduled:
+// by then every kernel before this one has completed, and no CTA waits while holding
+// tensor memory.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_enter()
+{
+    pdl_wait();
+    pdl_trigger();
+}
+
+// ---------------------------------------------------------------------------
 // TMA (tensor maps are kernel parameters: __grid_constant__ const CUtensorMap)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map)
