@@ -983,7 +983,7 @@ refine_select_kernel(const float *__restrict__ approx, int64_t ld, const __nv_bf
         if (tid == 0) fb_rows[atomicAdd(fb_count, 1)] = (int32_t)rl;
         return;
     }
-    uint32_t prefix, mask;
+    uint32_t prefix, mask, tau_hi;
     int need, in_bin;
     {
         uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
@@ -1000,32 +1000,49 @@ refine_select_kernel(const float *__restrict__ approx, int64_t ld, const __nv_bf
                 for (int c = tid; c < nw; c += kRefThreads) f(cand[c].x - kmin);
             },
             nw, need_total, span != 0u ? 31 - __clz(span) : 0, regA, &sc, &prefix, &mask, &need, &in_bin);
-        prefix += kmin;  // tau (or its bin's floor, a lower bound) as an absolute key
+        tau_hi = min(prefix | ~mask, span) + kmin;  // the bin's largest key: an upper bound of tau
+        prefix += kmin;                             // tau (or its bin's floor, a lower bound) as an absolute key
     }
-    //    the window W = {b : approx_b >= tau - 2E}: its block ids, compacted
+    //    the window W = {b : approx_b >= tau - 2E}.  tau_exact, the exact (k-1)-th best,
+    //    lies in [tau - E, tau + E] (k - 1 blocks have approx >= tau, at most k - 2 have
+    //    approx > tau), so a block with approx > tau + 2E has exact > tau_exact: a certain
+    //    winner, not rescored.  The band's block ids are compacted from the front of widx,
+    //    the certain winners' from the back.
     const uint32_t kw = order_key(key_value(prefix) - 2.f * e_row);
-    if (tid == 0) wcount = 0;
+    const uint32_t kw_hi = order_key(key_value(tau_hi) + 2.f * e_row);
+    __shared__ int ccount;
+    if (tid == 0) {
+        wcount = 0;
+        ccount = 0;
+    }
     __syncthreads();
     for (int c0 = 0; c0 < nw; c0 += kRefThreads) {
         const int c = c0 + tid;
-        const bool hit = c < nw && cand[c].x >= kw;
-        const uint32_t m = __ballot_sync(0xffffffffu, hit);
-        int base = 0;
-        if (lane == 0 && m != 0u) base = atomicAdd(&wcount, __popc(m));
-        base = __shfl_sync(0xffffffffu, base, 0);
-        if (hit) widx[base + __popc(m & lt_mask)] = (int32_t)cand[c].y;
+        const uint32_t key = c < nw ? cand[c].x : 0u;
+        const bool sure = c < nw && key > kw_hi;
+        const bool band = c < nw && !sure && key >= kw;
+        const uint32_t mb = __ballot_sync(0xffffffffu, band), ms = __ballot_sync(0xffffffffu, sure);
+        int bb = 0, bs = 0;
+        if (lane == 0 && mb != 0u) bb = atomicAdd(&wcount, __popc(mb));
+        if (lane == 0 && ms != 0u) bs = atomicAdd(&ccount, __popc(ms));
+        bb = __shfl_sync(0xffffffffu, bb, 0);
+        bs = __shfl_sync(0xffffffffu, bs, 0);
+        if (band) widx[bb + __popc(mb & lt_mask)] = (int32_t)cand[c].y;
+        if (sure) widx[kRefCap - 1 - (bs + __popc(ms & lt_mask))] = (int32_t)cand[c].y;
     }
     __syncthreads();
-    nw = wcount;
-    // 3. exact scores of the window, then its exact top k - 1
+    const int nb = wcount, ncs = ccount;
+    // 3. exact scores of the band, then the exact top k - 1 of band and certain winners
+    //    (these with the largest key, which no finite score reaches)
     const __nv_bfloat16 *kc_seq = kc + (int64_t)cu_blocks[s] * 256;
     index_row_cuda_at<2>(q_idx + i * 512, w + i * 4,
-                         [=](int64_t p) { return kc_seq + (int64_t)widx[p] * 256; }, 0, nw, exact, warp,
+                         [=](int64_t p) { return kc_seq + (int64_t)widx[p] * 256; }, 0, nb, exact, warp,
                          kRefThreads / 32, lane);
     __syncthreads();
-    for (int c = tid; c < nw; c += kRefThreads) cand[c] = make_uint2(order_key(exact[c]), (uint32_t)widx[c]);
+    for (int c = tid; c < nb; c += kRefThreads) cand[c] = make_uint2(order_key(exact[c]), (uint32_t)widx[c]);
+    for (int c = tid; c < ncs; c += kRefThreads) cand[nb + c] = make_uint2(0xFFFFFFFFu, (uint32_t)widx[kRefCap - 1 - c]);
     __syncthreads();
-    select_from_list<kRefThreads>(cand, nw, bt, k, out, regA, sc, nf);
+    select_from_list<kRefThreads>(cand, nb + ncs, bt, k, out, regA, sc, nf);
 }
 
 __global__ void clear_count_kernel(int32_t *c)

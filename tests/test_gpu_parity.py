@@ -13,7 +13,8 @@ import torch
 
 import oracle
 from block_sparse_long_09_b200 import inputs
-from parity_common import (SCALE, check_attn, check_scores, check_selection_near_threshold, kth_best,
+from parity_common import (SCALE, check_attn, check_scores, check_selection_invariants,
+                           check_selection_near_threshold, kth_best,
                            sampled_rows)
 
 pytestmark = pytest.mark.gpu
@@ -465,6 +466,36 @@ def test_dense_n8192_matches_full_budget_sparse(qsa):
     rows = sample_rows(n, 64)
     ref_o, _ = oracle.dense(x.q, x.k, x.v, n, n, SCALE, rows)
     check_attn(od.float().cpu().numpy()[rows], ref_o)
+    status_ok(qsa)
+
+
+@pytest.mark.parametrize("lengths,distinct,k", [([70001, 33000, 20000, 5], 300, 512), ([65540, 40000], 40, 512),
+                                                 ([131072], 2000, 2048), ([9000, 17000], 3, 16)])
+def test_decode_refine_with_repeated_blocks(qsa, lengths, distinct, k):
+    """The decode selection (hi-plane scan, exact rescoring of the near-threshold band,
+    certain winners above it) against the exact scan and the plain selector, bit for bit,
+    on caches whose blocks repeat a few patterns: equal scores by the hundreds sit at the
+    threshold, so the tie rule (lower block first) decides most of the selection."""
+    batch = len(lengths)
+    cfg = qsa.default_config(budget_blocks=k)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(77)
+    pats = torch.randn((distinct, 4, 128), generator=g, device="cuda").to(torch.bfloat16)
+    k_idx = torch.cat([pats[torch.randint(0, distinct, ((L + 3) // 4,), generator=g, device="cuda")]
+                       .reshape(-1, 128)[:L] for L in lengths])
+    q_idx = torch.randn((batch, 4, 128), generator=g, device="cuda").to(torch.bfloat16)
+    w = torch.rand((batch, 4), generator=g, device="cuda")
+    cu_k, cu_b = cu(lengths)
+    cu_q = torch.arange(batch + 1, dtype=torch.int32, device="cuda")
+    kc = qsa.compress_keys(k_idx, cu_k, cu_b, n_blocks=int(cu_b[-1]), cfg=cfg)
+    fused = qsa.index_select(q_idx, w, kc, cu_q, cu_k, cu_b, 1, max(lengths), cfg=cfg)
+    ld = max(4, ((max(lengths) - 1) // 4 + 3) // 4 * 4)
+    scores = qsa.index_scores(q_idx, w, kc, cu_q, cu_k, cu_b, 1, ld, cfg=cfg)
+    plain = qsa.select_blocks(scores, cu_q, cu_k, batch, cfg=cfg)
+    torch.cuda.synchronize()
+    assert torch.equal(fused, plain)
+    sel = fused.cpu().numpy()
+    check_selection_invariants(sel, [(L - 1) // 4 for L in lengths], k)
     status_ok(qsa)
 
 
