@@ -271,15 +271,16 @@ def run_qsa(args, rank, world, device):
     def mtp_attend():
         qsa.sparse_attn_decode_mtp(q4, d.k_cache, d.v_cache, cu_k, sel4, o=o4, ws=ws4a, cfg=cfg)
 
-    def mtp_step():
-        mtp_select()
-        mtp_attend()
-
-    mtp_step_us = timed(mtp_step, reps=10) * 1e3
+    # the step as a CUDA graph (qsa.MtpStep): refresh of the block the 4 new tokens
+    # completed, the shared selection and the attention; its parts launched eagerly
+    mtp = qsa.MtpStep(q4, dec.q_idx, dec.w, d.k_cache, d.v_cache, d.k_idx, dec.kc, cu_k, dec.cu_b, DEC_LEN,
+                      refresh_blocks=torch.tensor([(L - MTP_NEXT_N) // 4 for L in d.seqlens], dtype=torch.int32,
+                                                  device=device), cfg=cfg, graph=True)
+    mtp_step_us = timed(mtp, reps=10) * 1e3
     mtp_select_us = timed(mtp_select, reps=10) * 1e3
     mtp_attn_us = timed(mtp_attend, reps=10) * 1e3
     assert qsa.device_status() == 0
-    del q4, sel4, o4, ws4s, ws4a
+    del q4, sel4, o4, ws4s, ws4a, mtp
 
     # decode at 262144 tokens per sequence: the step, and the attention kernel alone
     del d, dec
@@ -369,7 +370,8 @@ def run_qsa(args, rank, world, device):
     if attn_src_hash() == ATTN_SMALL_TRAFFIC["src_sha256_16"] and world == 1:
         traffic = ATTN_SMALL_TRAFFIC["bytes"] * gather / ATTN_SMALL_TRAFFIC["gather_bytes"]
     attn_tflops = attn_flops / (attn_ms / 1e3) / 1e12
-    launches_prefill = 1 + 5 * n_chunks + 1  # compress; 5 launches of the fused index -> select per chunk; attention
+    # compress; 5 launches of the fused index -> select per chunk; the attention per pre.attn_rows rows
+    launches_prefill = 1 + 5 * n_chunks + (N_PREFILL + pre.attn_rows - 1) // pre.attn_rows
     launches_decode = 1 + 4 + 2               # refresh; hi-plane scan, count reset, refine, fallback; attention + merge
     kern = {
         "sparse_attn_prefill": {
@@ -395,7 +397,7 @@ def run_qsa(args, rank, world, device):
             "us_per_token": mtp_step_us / MTP_NEXT_N,
             "index_select_us": mtp_select_us, "attn_us": mtp_attn_us, "attn_bytes": dec_gather,
             "attn_frac": dec_gather / (mtp_attn_us / 1e6) / 1e9 / hbm,
-            "note": "eager launches: one shared selection and one K/V gather for the 4 queries of a sequence"},
+            "note": "step: qsa.MtpStep graph replay (refresh, shared selection, attention); parts: eager launches; one shared selection and one K/V gather serve the 4 queries of a sequence"},
         "decode_262k": {
             "step_us": step262_us, "step_bytes": step262_bytes,
             "step_frac": step262_bytes / (step262_us / 1e6) / 1e9 / hbm,

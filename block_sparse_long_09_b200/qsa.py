@@ -463,7 +463,7 @@ class Prefill:
     chunk's scores (qsa_index_scores) and selects on them (qsa_select_blocks)."""
 
     def __init__(self, seqlens, chunk_rows: int = 16384, cfg: Optional[Config] = None, device="cuda",
-                 fused: bool = True):
+                 fused: bool = True, attn_rows: int = 16384):
         self.cfg = _cfg(cfg)
         r = self.cfg.r
         self.seqlens = [int(x) for x in seqlens]
@@ -472,6 +472,9 @@ class Prefill:
         self.n_blocks = sum(L // r for L in self.seqlens)
         self.ld = max(4, ((self.max_len - 1) // r + 3) // 4 * 4)  # a multiple of 4
         self.chunk = int(chunk_rows)
+        self.attn_rows = int(attn_rows)
+        if self.chunk <= 0 or self.attn_rows <= 0:
+            raise ValueError("chunk_rows and attn_rows must be positive")
         self.fused = bool(fused)
         self.device = torch.device(device)
         cu = [0]
@@ -496,11 +499,13 @@ class Prefill:
         self.ws = torch.empty((need,), dtype=torch.uint8, device=self.device) if need > 0 else None
 
     def attend(self, q, k, v, o=None, lse=None):
-        """Sparse attention of every row: one launch over all rows (persistent CTAs), or,
-        with the key-chunked schedule (its workspace is sized per chunk), chunk by chunk."""
+        """Sparse attention of every row, one launch per attn_rows rows (persistent CTAs over
+        each launch's rows; on B200, launches of 16384 rows ran the 262144-row prefill about
+        8% faster than one launch over all rows), or, with the key-chunked schedule (its
+        workspace is sized per chunk_rows), chunk by chunk."""
         if o is None:
             o = torch.empty_like(q)
-        step = self.chunk if self.ws is not None else self.total
+        step = self.chunk if self.ws is not None else self.attn_rows
         for r0 in range(0, self.total, step):
             r1 = min(self.total, r0 + step)
             sparse_attn_prefill(q, k, v, self.sel, self.cu, self.cu, r0, r1, o=o, lse=lse, cfg=self.cfg, ws=self.ws,
@@ -600,6 +605,64 @@ class Prefill:
             done = d2h.record_event()
         cur.wait_event(done)
         return o
+
+
+class MtpStep:
+    """One multi-token decode step for a fixed batch: next_n new queries per sequence
+    (q [batch, next_n, 24, 256]; q_idx [batch, 4, 128] and w [batch, 4] of the last of
+    them) attend one shared selection.  The step recomputes the compressed blocks its
+    tokens may have completed (refresh_blocks [batch] int32: the first block to
+    recompute per sequence, then refresh_count blocks; blocks not yet complete are
+    skipped), makes the shared selection (qsa_index_select_mtp) and attends
+    (qsa_sparse_attn_decode_mtp).  The launches can be captured once in a CUDA graph
+    and replayed (graph=True): the tensors passed here are the graph's fixed inputs,
+    refreshed in place by the caller."""
+
+    def __init__(self, q, q_idx, w, k_cache, v_cache, k_idx, kc, cu_seqlens_k, cu_blocks, max_len_k: int,
+                 refresh_blocks=None, refresh_count: Optional[int] = None, cfg: Optional[Config] = None,
+                 graph: bool = True):
+        self.cfg = _cfg(cfg)
+        if q.dim() != 4:
+            raise ValueError("q must be [batch, next_n, heads, head_dim]")
+        self.q, self.q_idx, self.w = q, q_idx, w
+        self.k_cache, self.v_cache, self.k_idx, self.kc = k_cache, v_cache, k_idx, kc
+        self.cu_k, self.cu_b = cu_seqlens_k, cu_blocks
+        self.batch, self.next_n = q.shape[0], q.shape[1]
+        self.max_len_k = int(max_len_k)
+        self.refresh = refresh_blocks
+        r = self.cfg.r
+        self.refresh_count = int(refresh_count) if refresh_count is not None else (self.next_n + r - 1) // r + 1
+        dev = q.device
+        self.sel = torch.empty((self.batch, self.cfg.budget_blocks), dtype=torch.int32, device=dev)
+        self.ws_sel = torch.empty((max(workspace_size(OP_INDEX_SELECT, self.batch, self.batch, max_len_k, self.cfg),
+                                       16),), dtype=torch.uint8, device=dev)
+        self.ws = torch.empty((max(workspace_size(OP_DECODE_MTP, self.batch, self.batch, 0, self.cfg), 16),),
+                              dtype=torch.uint8, device=dev)
+        self.o = torch.empty_like(q)
+        self.graph = None
+        self.run()  # first call outside any capture (one-time kernel attribute setup)
+        if graph:
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.run()
+            self.graph = g
+
+    def run(self):
+        if self.refresh is not None:
+            compress_keys(self.k_idx, self.cu_k, self.cu_b, kc=self.kc, blk_begin=self.refresh,
+                          max_new_blocks=self.refresh_count, cfg=self.cfg)
+        index_select_mtp(self.q_idx, self.w, self.kc, self.cu_k, self.cu_b, self.next_n, self.max_len_k, sel=self.sel,
+                         ws=self.ws_sel, cfg=self.cfg)
+        sparse_attn_decode_mtp(self.q, self.k_cache, self.v_cache, self.cu_k, self.sel, o=self.o, ws=self.ws,
+                               cfg=self.cfg)
+        return self.o
+
+    def __call__(self):
+        if self.graph is not None:
+            self.graph.replay()
+            return self.o
+        return self.run()
 
 
 def prefill_copy_plan(total: int, select_rows: int, attend_rows: int, r: int = 4):

@@ -27,6 +27,8 @@ from typing import Callable, List, Optional, Sequence, Tuple
 
 import torch
 
+ATTN_ROWS = 16384  # query rows per attention launch
+
 # relative cost of a row: attention (about constant) and indexer pairs (per earlier block),
 # from the measured B200 times of the 262144-token prefill (about 0.43 us of attention per
 # row and 1.2 ps per (row, block) pair of the fused indexer)
@@ -131,8 +133,9 @@ class ShardedPrefill:
             b = min(self.n_local, a + self.chunk)
             qsa.index_select(q_idx, w, kc_pre, self.cu_q, self.cu_k, self.cu_b, self.n_local, self.r1, a, b,
                              sel=self.sel, ws=self.ws, cfg=self.cfg)
-        qsa.sparse_attn_prefill(q, k_pre, v_pre, self.sel, self.cu_q, self.cu_k, o=o, cfg=self.cfg,
-                                max_len_k=self.r1)
+        for a in range(0, self.n_local, ATTN_ROWS):  # launches of ATTN_ROWS rows, as qsa.Prefill.attend
+            qsa.sparse_attn_prefill(q, k_pre, v_pre, self.sel, self.cu_q, self.cu_k, a, min(self.n_local, a + ATTN_ROWS),
+                                    o=o, cfg=self.cfg, max_len_k=self.r1)
         return o
 
     def __call__(self, q, k, v, q_idx, w, k_idx, o=None):

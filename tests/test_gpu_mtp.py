@@ -93,3 +93,36 @@ def test_mtp_next_n_1_selection_equals_decode(qsa):
     torch.cuda.synchronize()
     assert torch.equal(a, b)
     assert qsa.device_status(clear=True) == 0
+
+
+def test_mtp_step_cuda_graph(qsa):
+    """qsa.MtpStep: the CUDA-graph replay of a multi-token step (compressed-block refresh,
+    shared selection, attention) equals the same calls launched eagerly, bit for bit, and
+    the refreshed blocks equal a full compression of the cache."""
+    next_n = 4
+    d = inputs.make_decode(6, 3000, 20000, seed=41, device="cuda", next_n=next_n)
+    cu_k, cu_b = d.cu_seqlens_k, d.cu_blocks
+    cfg = qsa.default_config()
+    kc_full = qsa.compress_keys(d.k_idx, cu_k, cu_b, n_blocks=int(cu_b[-1]), cfg=cfg)
+    # the blocks the step's tokens touched start stale: the refresh must recompute them
+    first = torch.tensor([(L - next_n) // 4 for L in d.seqlens], dtype=torch.int32, device="cuda")
+    kcs = []
+    for graph in (False, True):
+        kc = kc_full.clone()
+        for s in range(len(d.seqlens)):
+            b0, nb = int(cu_b[s]), int(cu_b[s + 1]) - int(cu_b[s])
+            lo = b0 + int(first[s])
+            kc[lo:b0 + nb] = 0
+        step = qsa.MtpStep(d.q, d.q_idx, d.w, d.k_cache, d.v_cache, d.k_idx, kc, cu_k, cu_b, max(d.seqlens),
+                           refresh_blocks=first, cfg=cfg, graph=graph)
+        for _ in range(2):
+            o = step()
+        torch.cuda.synchronize()
+        kcs.append((kc, step.sel.clone(), o.clone()))
+    assert torch.equal(kcs[0][0], kc_full) and torch.equal(kcs[1][0], kc_full)
+    assert torch.equal(kcs[0][1], kcs[1][1])
+    assert torch.equal(kcs[0][2], kcs[1][2])
+    sel = qsa.index_select_mtp(d.q_idx, d.w, kc_full, cu_k, cu_b, next_n, max(d.seqlens), cfg=cfg)
+    torch.cuda.synchronize()
+    assert torch.equal(sel, kcs[0][1])
+    assert qsa.device_status(clear=True) == 0

@@ -42,3 +42,24 @@ def test_from_host_equals_resident_prefill(qsa, lengths, k, chunk, pipe):
         assert torch.equal(o, o_ref.cpu())
         assert torch.equal(lse, lse_ref.cpu())
     assert qsa.device_status(clear=True) == 0
+
+
+def test_attention_launch_chunks_do_not_change_the_output(qsa):
+    """Prefill.attend launches the attention per attn_rows rows; every row's arithmetic is
+    its own, so one launch over all rows and launches of any size give the same bits."""
+    lengths = [20000, 7, 9001]
+    cfg = qsa.default_config(budget_blocks=128)
+    x = inputs.make_prefill(lengths, seed=92, device="cuda")
+    outs = []
+    for attn_rows in (sum(lengths), 16384, 1000, 333):
+        pre = qsa.Prefill(lengths, chunk_rows=8192, cfg=cfg, attn_rows=attn_rows)
+        o = torch.full_like(x.q, float("nan"))
+        lse = torch.full((x.q.shape[0], 24), float("nan"), dtype=torch.float32, device="cuda")
+        pre(x.q, x.k, x.v, x.q_idx, x.w, x.k_idx, o=o, lse=lse)
+        torch.cuda.synchronize()
+        outs.append((pre.sel.clone(), o, lse))
+    for sel, o, lse in outs[1:]:
+        assert torch.equal(sel, outs[0][0])
+        assert torch.equal(o, outs[0][1])
+        assert torch.equal(lse, outs[0][2])
+    assert qsa.device_status(clear=True) == 0
