@@ -325,7 +325,8 @@ def run_qsa(args, rank, world, device):
         e2e = {"value": ranks.job_throughput(world, N_PREFILL, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                "scope": "prefill 262144 via qsa.Prefill.from_host (pinned host in and out, copies overlapped "
-                        "with the compute in chunks of %d rows)" % args.e2e_rows}
+                        "with the compute in chunks of %d rows, attention launches of %d rows)" % (
+                            args.e2e_rows, pre.attn_rows)}
         # the same rows as the device-resident path of the timed steps, bit for bit
         assert torch.equal(o_host, o.cpu()), "the copy-overlapped prefill differs from the resident one"
         del host, o_host

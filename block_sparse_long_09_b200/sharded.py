@@ -27,7 +27,7 @@ from typing import Callable, List, Optional, Sequence, Tuple
 
 import torch
 
-ATTN_ROWS = 16384  # query rows per attention launch
+ATTN_ROWS = 4096  # query rows per attention launch
 
 # relative cost of a row: attention (about constant) and indexer pairs (per earlier block),
 # from the measured B200 times of the 262144-token prefill (about 0.43 us of attention per
