@@ -190,7 +190,7 @@ def run_qsa(args, rank, world, device):
                 ev["ix"].append((e0, e1))
         if record:
             e["a0"].record(stream)
-        pre.attend(x.q, x.k, x.v, o=o)  # one pass per query
+        pre.attend(x.q, x.k, x.v, o=o)  # one pass over the keys per query, 4096 rows per launch
         if record:
             e["a1"].record(stream)
             e["p1"].record(stream)
@@ -588,7 +588,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="qsa", choices=["qsa", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--e2e-rows", type=int, default=16384, help="attention rows per copy chunk of the e2e leg")
+    ap.add_argument("--e2e-rows", type=int, default=16384, help="query rows per copy chunk of the e2e leg (q, k, v in, o out)")
     ap.add_argument("--chunk-rows", type=int, default=CHUNK,
                     help="query rows per fused index -> select launch of the prefill")
     ap.add_argument("--no-cpu-baseline", action="store_true")

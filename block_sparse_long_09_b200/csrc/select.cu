@@ -44,6 +44,10 @@ constexpr int kSegWords = 2048;              // bitmap segment: 65536 candidates
 constexpr int kSegElems = kSegWords * 32;
 constexpr int kCandCap = 2048;               // candidate lists (and the sample)
 constexpr int kSampleMin = 1024;
+// Radix passes of a select that only needs a bound of its key (a threshold below which
+// no winner lies, or the bin around tau): two 8-bit digits below the keys' highest
+// differing bit leave a bin of 2^-16 of their span, and stopping there saves the rest.
+constexpr int kBoundPasses = 2;
 
 // shared memory: region A (kSegWords words: histogram, then the winner bitmap)
 // and region C (kCandCap (score bits, index) pairs; before them the sample keys,
@@ -646,8 +650,9 @@ threshold_kernel(const float *__restrict__ sample, int64_t sample_ld, int stride
         [&](auto f) {
             for (int p = tid; p < ns; p += kThrThreads) f(keys[p] - kmin);
         },
-        ns, r_lo, span != 0u ? 31 - __clz(span) : 0, hist, &sc, &prefix, &mask, &need, &in_bin);
-    // prefix + kmin is the r_lo-th largest key, or (bin taken whole) a lower bound of it
+        ns, r_lo, span != 0u ? 31 - __clz(span) : 0, hist, &sc, &prefix, &mask, &need, &in_bin, kBoundPasses);
+    // prefix + kmin is the r_lo-th largest key, or (bin taken whole, or the passes spent) a
+    // lower bound of it
     if (tid == 0) theta[rl] = key_value(prefix + kmin);
 }
 
@@ -917,7 +922,7 @@ refine_select_kernel(const float *__restrict__ approx, int64_t ld, const __nv_bf
             [&](auto f) {
                 for (int q = tid; q < ns; q += kRefThreads) f(skeys[q] - kmin);
             },
-            ns, r_lo, span != 0u ? 31 - __clz(span) : 0, regA, &sc, &sp, &sm, &sn, &sb);
+            ns, r_lo, span != 0u ? 31 - __clz(span) : 0, regA, &sc, &sp, &sm, &sn, &sb, kBoundPasses);
         theta_s = key_value(sp + kmin);  // the sample's r_lo-th largest, or its bin's floor
     }
     __syncthreads();
@@ -999,7 +1004,8 @@ refine_select_kernel(const float *__restrict__ approx, int64_t ld, const __nv_bf
             [&](auto f) {
                 for (int c = tid; c < nw; c += kRefThreads) f(cand[c].x - kmin);
             },
-            nw, need_total, span != 0u ? 31 - __clz(span) : 0, regA, &sc, &prefix, &mask, &need, &in_bin);
+            nw, need_total, span != 0u ? 31 - __clz(span) : 0, regA, &sc, &prefix, &mask, &need, &in_bin,
+            kBoundPasses);
         tau_hi = min(prefix | ~mask, span) + kmin;  // the bin's largest key: an upper bound of tau
         prefix += kmin;                             // tau (or its bin's floor, a lower bound) as an absolute key
     }

@@ -211,8 +211,9 @@ qsa_status qsa_select_blocks(const qsa_config *cfg, const float *scores, int64_t
  * score is within E = sum_h |w_h| ||q_h|| sqrt(idx_dim) (2^-8 1.01 + 1e-4) of the
  * exact one; the blocks within 2E of the row's (k-1)-th best are rescored exactly
  * (hi + lo) and the row's exact top k - 1 is taken among them -- the same selection
- * as qsa_index_scores + qsa_select_blocks.  A window of more than 4096 blocks, or
- * QSA_COMPRESS_NO_NORM, takes the exact scan of the whole row instead.
+ * as qsa_index_scores + qsa_select_blocks.  A row whose candidate list exceeds 4096
+ * blocks or whose sampled bound fails, and every row under QSA_COMPRESS_NO_NORM, takes
+ * the exact scan of the whole row instead (same selection).
  *   max_len_k  host: an upper bound of every L_k,s (sizes the samples and scratch)
  *   sel        [total_q, k] int32 as qsa_select_blocks writes it
  * Workspace: qsa_workspace_size(cfg, QSA_OP_INDEX_SELECT, batch, row_end - row_begin,

@@ -126,3 +126,28 @@ def test_mtp_step_cuda_graph(qsa):
     torch.cuda.synchronize()
     assert torch.equal(sel, kcs[0][1])
     assert qsa.device_status(clear=True) == 0
+
+
+def test_mtp_selection_when_every_block_ties(qsa):
+    """Every compressed key equal: the candidate list overflows, the row is selected from
+    its exact scores in the same CTA, and the tie rule leaves a closed form: every query's
+    own block (b_first .. b_last) forced, then the lowest blocks below b_first."""
+    next_n, k = 4, 512
+    lengths = [30002, 20001, 9, 2050]
+    cfg = qsa.default_config(budget_blocks=k)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(78)
+    pat = torch.randn((4, 128), generator=g, device="cuda").to(torch.bfloat16)
+    k_idx = torch.cat([pat.repeat((L + 3) // 4, 1)[:L] for L in lengths])
+    q_idx = torch.randn((len(lengths), 4, 128), generator=g, device="cuda").to(torch.bfloat16)
+    w = torch.rand((len(lengths), 4), generator=g, device="cuda")
+    cu_k, cu_b = cu(lengths)
+    kc = qsa.compress_keys(k_idx, cu_k, cu_b, n_blocks=int(cu_b[-1]), cfg=cfg)
+    sel = qsa.index_select_mtp(q_idx, w, kc, cu_k, cu_b, next_n, max(lengths), cfg=cfg).cpu().numpy()
+    for s, L in enumerate(lengths):
+        b_first, b_last = max(L - next_n, 0) // 4, (L - 1) // 4
+        nf = b_last - b_first + 1
+        want = list(range(min(k - nf, b_first))) + list(range(b_first, b_first + nf))
+        want += [-1] * (k - len(want))
+        np.testing.assert_array_equal(sel[s], np.array(want, dtype=np.int32))
+    assert qsa.device_status(clear=True) == 0

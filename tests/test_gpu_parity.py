@@ -470,12 +470,15 @@ def test_dense_n8192_matches_full_budget_sparse(qsa):
 
 
 @pytest.mark.parametrize("lengths,distinct,k", [([70001, 33000, 20000, 5], 300, 512), ([65540, 40000], 40, 512),
-                                                 ([131072], 2000, 2048), ([9000, 17000], 3, 16)])
+                                                 ([131072], 2000, 2048), ([9000, 17000], 3, 16),
+                                                 ([30000, 20001, 7], 1, 512)])
 def test_decode_refine_with_repeated_blocks(qsa, lengths, distinct, k):
     """The decode selection (hi-plane scan, exact rescoring of the near-threshold band,
     certain winners above it) against the exact scan and the plain selector, bit for bit,
     on caches whose blocks repeat a few patterns: equal scores by the hundreds sit at the
-    threshold, so the tie rule (lower block first) decides most of the selection."""
+    threshold, so the tie rule (lower block first) decides most of the selection.  With a
+    single pattern every block ties, the candidate list overflows and the row is selected
+    from its exact scores inside the same CTA."""
     batch = len(lengths)
     cfg = qsa.default_config(budget_blocks=k)
     g = torch.Generator(device="cuda")
@@ -496,6 +499,11 @@ def test_decode_refine_with_repeated_blocks(qsa, lengths, distinct, k):
     assert torch.equal(fused, plain)
     sel = fused.cpu().numpy()
     check_selection_invariants(sel, [(L - 1) // 4 for L in lengths], k)
+    if distinct == 1:  # every block ties (and the list overflows): the lowest k - 1 blocks and the own block
+        for s_, L in enumerate(lengths):
+            bt = (L - 1) // 4
+            want = list(range(min(k - 1, bt))) + [bt] + [-1] * max(0, k - 1 - bt)
+            np.testing.assert_array_equal(sel[s_], np.array(want[:k], dtype=np.int32))
     status_ok(qsa)
 
 
