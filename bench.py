@@ -446,6 +446,18 @@ def run_qsa(args, rank, world, device):
     return res
 
 
+def cpu_model() -> str:
+    """The host CPU's model string (from /proc/cpuinfo), for the baseline's record."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(seconds: float = 12.0, rows_hint: int = 16):
     """The fp64 oracle, as it stands, on a bounded sample of the prefill workload:
     for each sampled query row the whole chain (scores against every earlier
@@ -482,7 +494,8 @@ def cpu_baseline(seconds: float = 12.0, rows_hint: int = 16):
     if t < seconds / 3:
         n = max(n, int(n * seconds / max(t, 1e-3)))
         t = run(rng.integers(N_PREFILL // 2, N_PREFILL, n))
-    return {"value": n / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+    return {"value": n / t, "unit": "tokens/s", "cores": cores, "kind": "oracle", "cpu": cpu_model(),
+            "nproc": os.cpu_count(),
             "sample": "%d random query rows from the second half of the 262144-token prefill: compress of all "
                       "keys once, then per row scores, top-512 select and attention, fp64, %.1f s" % (n, t)}
 
@@ -490,7 +503,8 @@ def cpu_baseline(seconds: float = 12.0, rows_hint: int = 16):
 def run_extra_configs(steps: int = 5, warmup: int = 3):
     """The other workloads of the measurement plan, one line each on stderr (the bench's
     own JSON line on stdout is unchanged): prefill of 2 x 65536 tokens with peaked indexer
-    keys, and decode steps at 262144 tokens and at mixed lengths U{32768 .. 262144}."""
+    keys, decode steps at 262144 tokens and at mixed lengths U{32768 .. 262144}, and the
+    1M-token context of the pages' comparison (run_context_1m)."""
     from block_sparse_long_09_b200 import inputs, qsa
 
     torch.cuda.set_device(0)
@@ -537,6 +551,64 @@ def run_extra_configs(steps: int = 5, warmup: int = 3):
               file=sys.stderr)
         del d, kc, dec
         torch.cuda.empty_cache()
+    run_context_1m(timed, cfg, dev)
+
+
+def run_context_1m(timed, cfg, dev):
+    """The regime of the pages' kernel-level comparison (1M-token context): the prefill of
+    one 1048576-token sequence against this build's dense causal kernel, and decode at
+    batch 4 (the pages' decode batch, with next_n = 4) against the dense split-K decode of
+    one query per sequence -- a lower bound of any dense step, which reads every cached
+    token at least once."""
+    from block_sparse_long_09_b200 import inputs, qsa
+
+    n = 1 << 20
+    x = inputs.make_prefill([n], seed=0, device=dev)
+    pre = qsa.Prefill([n], chunk_rows=CHUNK, cfg=cfg, device=dev)
+    o = torch.empty_like(x.q)
+    qsa_ms = timed(lambda: pre(x.q, x.k, x.v, x.q_idx, x.w, x.k_idx, o=o))
+    att_ms = timed(lambda: pre.attend(x.q, x.k, x.v, o=o))
+    qsa.dense_attn_prefill(x.q, x.k, x.v, pre.cu, pre.cu, n, o=o, cfg=cfg, max_len_k=n)  # warm-up
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    qsa.dense_attn_prefill(x.q, x.k, x.v, pre.cu, pre.cu, n, o=o, cfg=cfg, max_len_k=n)
+    e1.record()
+    torch.cuda.synchronize()
+    dense_ms = e0.elapsed_time(e1)
+    assert qsa.device_status() == 0
+    print(json.dumps({"workload": "prefill 1 x 1048576 (k = 512)", "prefill_ms": qsa_ms,
+                      "tokens_per_s": n / (qsa_ms / 1e3), "attn_ms": att_ms, "dense_prefill_ms": dense_ms,
+                      "qsa_layer_speedup": dense_ms / qsa_ms, "qsa_attention_only_speedup": dense_ms / att_ms,
+                      "pages": "7.6x prefill at 1M context, kernel level, hardware not stated"}), file=sys.stderr)
+    del x, pre, o
+    torch.cuda.empty_cache()
+
+    batch, next_n = 4, MTP_NEXT_N
+    d = inputs.make_decode(batch, n, None, seed=0, device=dev, next_n=next_n)
+    kc = qsa.compress_keys(d.k_idx, d.cu_seqlens_k, d.cu_blocks, n_blocks=int(d.cu_blocks[-1]), cfg=cfg)
+    q1 = d.q[:, -1].contiguous()  # the last query of each sequence: plain decode
+    last = torch.tensor([L // 4 - 1 for L in d.seqlens], dtype=torch.int32, device=dev)
+    dec = qsa.DecodeStep(q1, d.q_idx, d.w, d.k_cache, d.v_cache, d.k_idx, kc, d.cu_seqlens_k, d.cu_blocks, n,
+                         refresh_blocks=last, cfg=cfg, graph=True)
+    dec_us = timed(dec) * 1e3
+    mtp = qsa.MtpStep(d.q, d.q_idx, d.w, d.k_cache, d.v_cache, d.k_idx, kc, d.cu_seqlens_k, d.cu_blocks, n,
+                      refresh_blocks=torch.tensor([(L - next_n) // 4 for L in d.seqlens], dtype=torch.int32,
+                                                  device=dev), cfg=cfg, graph=True)
+    mtp_us = timed(mtp) * 1e3
+    cu_q = torch.arange(batch + 1, dtype=torch.int32, device=dev)
+    dws = torch.empty((qsa.workspace_size(qsa.OP_DENSE, batch, batch, n, cfg),), dtype=torch.uint8, device=dev)
+    od = torch.empty_like(q1)
+    dense_us = timed(lambda: qsa.dense_attn_prefill(q1, d.k_cache, d.v_cache, cu_q, d.cu_seqlens_k, 1, o=od,
+                                                    cfg=cfg, max_len_k=n, ws=dws)) * 1e3
+    print(json.dumps({"workload": "decode batch 4 at 1048576 tokens", "step_us": dec_us,
+                      "mtp_next_n": next_n, "mtp_step_us": mtp_us, "mtp_us_per_token": mtp_us / next_n,
+                      "dense_decode_us": dense_us, "qsa_decode_speedup": dense_us / dec_us,
+                      "qsa_mtp_speedup_per_token": dense_us / (mtp_us / next_n),
+                      "pages": "4.9x decode at 1M context with next_n = 4, kernel level, hardware not stated"}),
+          file=sys.stderr)
+    del d, kc, dec, mtp, dws, od
+    torch.cuda.empty_cache()
 
 
 def run_profile_case(case: str, reps: int = 3):
@@ -630,7 +702,7 @@ def main():
                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                "data": "synthetic", "config": {"workload": "QSA prefill batch 1 n=262144, sampled rows (fp64 oracle)"},
                "cpu_baseline": {"value": val, "unit": "tokens/s", "kind": "oracle", "cores": b[0]["cores"],
-                                "sample": b[0]["sample"]},
+                                "cpu": b[0]["cpu"], "nproc": b[0]["nproc"], "sample": b[0]["sample"]},
                "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(res))
         return

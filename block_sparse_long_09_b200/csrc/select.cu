@@ -891,7 +891,12 @@ refine_select_kernel(const float *__restrict__ approx, int64_t ld, const __nv_bf
     //    row fits the list
     float theta_s = -INFINITY;
     if (n > kRefCap) {
-        const int runs = kCandCap / 8;
+        // about n / 32 keys (runs of 8, at least 2048, at most the 8192 the list area holds):
+        // some 16 expected winners fall in the sample, so the bound stays tight on long rows
+        // (with 2048 keys a 262143-block row keeps only 4, and its list overflows); every run
+        // starts at least 16 keys before the row's end
+        int runs = n / 256;
+        runs = runs < kCandCap / 8 ? kCandCap / 8 : (runs > kRefCap / 4 ? kRefCap / 4 : runs);
         const int ns = runs * 8;
         uint32_t *skeys = reinterpret_cast<uint32_t *>(cand);  // the list area, free until step 2
         for (int g = tid; g < runs; g += kRefThreads) {

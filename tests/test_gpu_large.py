@@ -11,9 +11,10 @@ micro-block.  The GPU side runs exactly as the benchmark does (the same inputs,
   selection  the GPU's top-k against the oracle's under the near-threshold rule
   attention  the GPU's output against the oracle's attention on the GPU's selection
 
-Workloads: prefill of one 262 144-token sequence (N(0,1) inputs), prefill of two
-65 536-token sequences with peaked indexer keys, and decode steps at batch 64
-with every cache at 131 072 tokens and with lengths U{32 768 .. 262 144}.
+Workloads: prefill of one 262 144-token sequence (N(0,1) inputs) and of one
+1 048 576-token sequence, prefill of two 65 536-token sequences with peaked indexer
+keys, and decode steps at batch 64 with every cache at 131 072 tokens and with
+lengths U{32 768 .. 262 144}.
 """
 import os
 from concurrent.futures import ThreadPoolExecutor
@@ -112,6 +113,13 @@ def prefill_case(qsa, lengths, peaked, seed):
 def test_prefill_262144_sampled_rows(qsa):
     """Batch 1, n = 262 144, N(0,1) inputs, budget 512 blocks (the benchmark's prefill)."""
     prefill_case(qsa, [262144], peaked=False, seed=0)
+
+
+def test_prefill_1048576_sampled_rows(qsa):
+    """Batch 1, n = 1 048 576 (the context of the pages' kernel-level comparison, which
+    the benchmark's extra workloads time): the sample stride of the fused selection
+    doubles past 524 288 tokens, so its bounds and lists run in another regime."""
+    prefill_case(qsa, [1 << 20], peaked=False, seed=3)
 
 
 def test_prefill_2x65536_peaked_sampled_rows(qsa):
