@@ -13,8 +13,8 @@ micro-block.  The GPU side runs exactly as the benchmark does (the same inputs,
 
 Workloads: prefill of one 262 144-token sequence (N(0,1) inputs) and of one
 1 048 576-token sequence, prefill of two 65 536-token sequences with peaked indexer
-keys, and decode steps at batch 64 with every cache at 131 072 tokens and with
-lengths U{32 768 .. 262 144}.
+keys, decode steps at batch 64 with every cache at 131 072 tokens and with lengths
+U{32 768 .. 262 144}, and a decode step at batch 4 with 1 048 576-token caches.
 """
 import os
 from concurrent.futures import ThreadPoolExecutor
@@ -127,12 +127,11 @@ def test_prefill_2x65536_peaked_sampled_rows(qsa):
     prefill_case(qsa, [65536, 65536], peaked=True, seed=0)
 
 
-def decode_case(qsa, lo, hi, seed):
-    """One decode step at batch 64 exactly as the benchmark runs it (CUDA graph of
-    compress refresh, indexer, select, attention, merge); every sequence checked."""
+def decode_case(qsa, lo, hi, seed, batch=64):
+    """One decode step as the benchmark runs it (CUDA graph of compress refresh, indexer,
+    select, attention, merge); every sequence checked."""
     from block_sparse_long_09_b200 import ranks
     dev = torch.device("cuda")
-    batch = 64
     d = inputs.make_decode(batch, lo, hi, seed=seed, device=dev)
     cfg = qsa.default_config(budget_blocks=K)
     kc = qsa.compress_keys(d.k_idx, d.cu_seqlens_k, d.cu_blocks, n_blocks=int(d.cu_blocks[-1]), cfg=cfg)
@@ -168,6 +167,12 @@ def decode_case(qsa, lo, hi, seed):
     assert agree >= 0.75 * batch, agree
     del step
     assert ranks.rank_seeds(0)["decode"] == 100  # the benchmark's decode seed
+
+
+def test_decode_b4_ctx1048576(qsa):
+    """Batch 4 with every cache at 1 048 576 tokens (the pages' decode batch and context):
+    262 143 candidate blocks per row, where the refine's bound needs its larger sample."""
+    decode_case(qsa, 1 << 20, None, seed=4, batch=4)
 
 
 def test_decode_b64_ctx131072(qsa):
