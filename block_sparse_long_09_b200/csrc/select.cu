@@ -826,13 +826,200 @@ constexpr int kRefThreads = 512;
 constexpr int kRefCap = 4096;
 constexpr int kRefSmem = kSegWords * 4 + kRefCap * (8 + 4 + 4);
 
+// E of a decode row (called by one warp; every lane returns it): the head dots move by at
+// most ||q_h|| ||lo_b|| with ||lo_b|| <= 2^-8 ||kc_b|| = 2^-8 sqrt(128)
+__device__ __forceinline__ float row_error_bound(const __nv_bfloat16 *__restrict__ q_row,
+                                                 const float *__restrict__ w_row, int lane)
+{
+    float e = 0.f;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const uint2 raw = *reinterpret_cast<const uint2 *>(q_row + h * 128 + lane * 4);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+        float ss = a.x * a.x + a.y * a.y + b.x * b.x + b.y * b.y;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        e += fabsf(__ldg(w_row + h)) * sqrtf(ss);
+    }
+    return e * 11.3137085f * (1.01f * 0.00390625f + 1e-4f) * 1.01f;  // sqrt(128) (2^-8 1.01 + 1e-4)
+}
+
+// theta_s, a lower bound of tau (the (k-1)-th largest of the n > kRefCap approximate
+// scores srow[0 .. n)): the r_lo-th largest of a sample of the row (runs of 8 keys spread
+// over it), r_lo = mu + 4 sqrt(mu) + 8 for mu expected winners in the sample.  The whole
+// CTA calls it; every thread returns theta_s.  skeys: 8192 words of shared memory.
+__device__ __forceinline__ float sample_bound(const float *__restrict__ srow, int n, int need_total,
+                                              uint32_t *skeys, uint32_t *hist, SelScratch &sc)
+{
+    const int tid = threadIdx.x;
+    // about n / 32 keys (runs of 8, at least 2048, at most 8192): some 16 expected winners
+    // fall in the sample, so the bound stays tight on long rows (with 2048 keys a
+    // 262143-block row keeps only 4, and its list overflows); every run starts at least
+    // 16 keys before the row's end
+    int runs = n / 256;
+    runs = runs < kCandCap / 8 ? kCandCap / 8 : (runs > kRefCap / 4 ? kRefCap / 4 : runs);
+    const int ns = runs * 8;
+    for (int g = tid; g < runs; g += kRefThreads) {
+        const int at = (int)(((int64_t)g * n) / runs) & ~3;
+        const float4 x0 = __ldg(reinterpret_cast<const float4 *>(srow + at));
+        const float4 x1 = __ldg(reinterpret_cast<const float4 *>(srow + at + 4));
+        const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) skeys[g * 8 + e] = order_key(xs[e]);
+    }
+    __syncthreads();
+    const float mu = (float)need_total * (float)ns / (float)n;
+    int r_lo = (int)ceilf(mu + 4.f * sqrtf(mu) + 8.f);
+    if (r_lo > ns) r_lo = ns;
+    // keys relative to the sample's smallest: the radix starts at their highest differing bit
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int q = tid; q < ns; q += kRefThreads) {
+        kmin = min(kmin, skeys[q]);
+        kmax = max(kmax, skeys[q]);
+    }
+    kmin = ~kmin;
+    block_max2<kRefThreads>(kmin, kmax, &sc);
+    kmin = ~kmin;
+    const uint32_t span = kmax - kmin;
+    uint32_t sp, sm;
+    int sn, sb;
+    radix_select<kRefThreads, 8>(
+        [&](auto f) {
+            for (int q = tid; q < ns; q += kRefThreads) f(skeys[q] - kmin);
+        },
+        ns, r_lo, span != 0u ? 31 - __clz(span) : 0, hist, &sc, &sp, &sm, &sn, &sb, kBoundPasses);
+    return key_value(sp + kmin);  // the sample's r_lo-th largest, or its bin's floor
+}
+
+// The decode row's position and the counts of its selection (k - nf slots for the best
+// candidates 0 .. bt - 1); false when the row is not a valid decode row.
+__device__ __forceinline__ bool refine_row(const int32_t *cu_q, const int32_t *cu_k, int batch, int64_t i, int r,
+                                           int next_n, int64_t ld, int k, int *s, int64_t *bt, int *nf)
+{
+    const int64_t t = row_position(cu_q, cu_k, batch, i, s);
+    if (t < 0) return false;
+    *bt = t / r;
+    *nf = 1;
+    if (next_n > 1) mtp_blocks(t + 1, next_n, r, bt, nf);
+    return !(*bt > ld || *bt > 0x7FFFFFFF || *nf > k);
+}
+
+// Batches too small to fill the GPU with one refine CTA per row build the candidate
+// lists W' in two launches before the refine: refine_bound_kernel (E and theta_s per
+// row, the list counter reset) and refine_list_kernel (CTAs over (row chunk, row) append
+// the approximate scores >= theta_s - 2E to the row's list in global memory).
+constexpr int kListChunk = 4096;  // approximate scores scanned by one list CTA
+constexpr int kListThreads = 256;
+constexpr int kBoundSmem = (kSegWords + 2 * kRefCap) * 4;
+
+__global__ void __launch_bounds__(kRefThreads, 1)
+refine_bound_kernel(const float *__restrict__ approx, int64_t ld, const __nv_bfloat16 *__restrict__ q_idx,
+                    const float *__restrict__ w, const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
+                    int batch, int64_t row_begin, int k, int r, int next_n, float2 *__restrict__ bound,
+                    int32_t *__restrict__ count)
+{
+    pdl_enter();
+    extern __shared__ uint32_t smem_sel[];
+    __shared__ SelScratch sc;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t rl = blockIdx.x, i = row_begin + rl;
+    if (tid == 0) count[rl] = 0;
+    int s, nf;
+    int64_t bt;
+    if (!refine_row(cu_q, cu_k, batch, i, r, next_n, ld, k, &s, &bt, &nf)) return;  // the refine flags it
+    const int need_total = k - nf;
+    if (bt <= need_total) return;  // every candidate wins: the refine writes it
+    const int n = (int)bt;
+    float theta_s = -INFINITY;
+    if (n > kRefCap) theta_s = sample_bound(approx + rl * ld, n, need_total, smem_sel + kSegWords, smem_sel, sc);
+    if (warp == 0) {
+        const float e = row_error_bound(q_idx + i * 512, w + i * 4, lane);
+        if (lane == 0) bound[rl] = make_float2(theta_s, e);
+    }
+}
+
+__global__ void __launch_bounds__(kListThreads)
+refine_list_kernel(const float *__restrict__ approx, int64_t ld, const int32_t *__restrict__ cu_q,
+                   const int32_t *__restrict__ cu_k, int batch, int64_t row_begin, int k, int r, int next_n,
+                   const float2 *__restrict__ bound, uint2 *__restrict__ lists, int32_t *__restrict__ count)
+{
+    pdl_enter();
+    constexpr int kW = kListThreads / 32, kPer = kListChunk / (4 * kListThreads);  // float4 groups per thread
+    __shared__ int warp_hits[kW];
+    __shared__ int cta_base;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t rl = blockIdx.y, i = row_begin + rl;
+    int s, nf;
+    int64_t bt;
+    if (!refine_row(cu_q, cu_k, batch, i, r, next_n, ld, k, &s, &bt, &nf)) return;  // uniform per CTA
+    if (bt <= k - nf) return;
+    const int n = (int)bt;
+    const int c0 = blockIdx.x * kListChunk;
+    if (c0 >= n) return;
+    const float2 b = bound[rl];
+    const float lo_bound = b.x - 2.f * b.y;
+    const float4 *srow4 = reinterpret_cast<const float4 *>(approx + rl * ld + c0);
+    const int len = n - c0 < kListChunk ? n - c0 : kListChunk;
+    const int n4 = (len + 3) / 4;
+    float4 x4[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int g = u * kListThreads + tid;
+        x4[u] = g < n4 ? __ldg(srow4 + g) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    }
+    uint32_t m[kPer * 4];
+    int hits = 0;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int g = u * kListThreads + tid;
+        const float xs[4] = {x4[u].x, x4[u].y, x4[u].z, x4[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            m[u * 4 + e] = __ballot_sync(0xffffffffu, 4 * g + e < len && xs[e] >= lo_bound);
+            hits += __popc(m[u * 4 + e]);
+        }
+    }
+    // one reservation of list slots per CTA: the warps' counts, their prefix, one atomic
+    if (lane == 0) warp_hits[warp] = hits;
+    __syncthreads();
+    if (tid == 0) {
+        int tot = 0;
+        for (int x = 0; x < kW; ++x) {
+            const int h = warp_hits[x];
+            warp_hits[x] = tot;
+            tot += h;
+        }
+        cta_base = tot > 0 ? atomicAdd(count + rl, tot) : 0;
+    }
+    __syncthreads();
+    if (hits == 0) return;  // warp-uniform
+    int base = cta_base + warp_hits[warp];
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    uint2 *lrow = lists + rl * kRefCap;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int g = u * kListThreads + tid;
+        const float xs[4] = {x4[u].x, x4[u].y, x4[u].z, x4[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const uint32_t mk = m[u * 4 + e];
+            const int pos = base + __popc(mk & lt_mask);
+            if (((mk >> lane) & 1u) && pos < kRefCap) lrow[pos] = make_uint2(order_key(xs[e]), (uint32_t)(c0 + 4 * g + e));
+            base += __popc(mk);
+        }
+    }
+}
+
+template <bool kListed>
 __global__ void __launch_bounds__(kRefThreads, 1)
 refine_select_kernel(const float *__restrict__ approx, int64_t ld, const __nv_bfloat16 *__restrict__ q_idx,
                      const float *__restrict__ w, const __nv_bfloat16 *__restrict__ kc,
                      const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
                      const int32_t *__restrict__ cu_blocks, int batch, int64_t row_begin, int k, int r,
                      int32_t *__restrict__ sel, int32_t *__restrict__ fb_count, int32_t *__restrict__ fb_rows,
-                     int next_n)
+                     int next_n, const float2 *__restrict__ bound, const uint2 *__restrict__ lists,
+                     const int32_t *__restrict__ count)
 {
     pdl_enter();
     extern __shared__ uint32_t smem_sel[];
@@ -845,16 +1032,9 @@ refine_select_kernel(const float *__restrict__ approx, int64_t ld, const __nv_bf
     __shared__ float e_row;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t rl = blockIdx.x, i = row_begin + rl;
-    int s;
-    const int64_t t = row_position(cu_q, cu_k, batch, i, &s);
-    if (t < 0) {
-        if (tid == 0) set_device_status(QSA_ERR_DEVICE_CHECK);
-        return;
-    }
-    int64_t bt = t / r;
-    int nf = 1;
-    if (next_n > 1) mtp_blocks(t + 1, next_n, r, &bt, &nf);
-    if (bt > ld || bt > 0x7FFFFFFF || nf > k) {
+    int s, nf;
+    int64_t bt;
+    if (!refine_row(cu_q, cu_k, batch, i, r, next_n, ld, k, &s, &bt, &nf)) {
         if (tid == 0) set_device_status(QSA_ERR_DEVICE_CHECK);
         return;
     }
@@ -865,76 +1045,36 @@ refine_select_kernel(const float *__restrict__ approx, int64_t ld, const __nv_bf
         return;
     }
     const int n = (int)bt;
-    const float *srow = approx + rl * ld;
-    // the error bound E of the row
-    if (warp == 0) {
-        const __nv_bfloat16 *qr = q_idx + i * 512;
-        float e = 0.f;
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const uint2 raw = *reinterpret_cast<const uint2 *>(qr + h * 128 + lane * 4);
-            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
-            const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
-            float ss = a.x * a.x + a.y * a.y + b.x * b.x + b.y * b.y;
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-            e += fabsf(__ldg(w + i * 4 + h)) * sqrtf(ss);
-        }
-        if (lane == 0) {
-            e_row = e * 11.3137085f * (1.01f * 0.00390625f + 1e-4f) * 1.01f;  // sqrt(128) (2^-8 1.01 + 1e-4)
-            wcount = 0;
-        }
-    }
-    // 1. a lower bound theta_s of tau, the (k-1)-th largest approximate score: the
-    //    r_lo-th largest of a sample of the row (runs of 8 keys spread over it), r_lo =
-    //    mu + 4 sqrt(mu) + 8 for mu expected winners in the sample; every block when the
-    //    row fits the list
+    const uint32_t lt_mask = (1u << lane) - 1u;
     float theta_s = -INFINITY;
-    if (n > kRefCap) {
-        // about n / 32 keys (runs of 8, at least 2048, at most the 8192 the list area holds):
-        // some 16 expected winners fall in the sample, so the bound stays tight on long rows
-        // (with 2048 keys a 262143-block row keeps only 4, and its list overflows); every run
-        // starts at least 16 keys before the row's end
-        int runs = n / 256;
-        runs = runs < kCandCap / 8 ? kCandCap / 8 : (runs > kRefCap / 4 ? kRefCap / 4 : runs);
-        const int ns = runs * 8;
-        uint32_t *skeys = reinterpret_cast<uint32_t *>(cand);  // the list area, free until step 2
-        for (int g = tid; g < runs; g += kRefThreads) {
-            const int at = (int)(((int64_t)g * n) / runs) & ~3;
-            const float4 x0 = __ldg(reinterpret_cast<const float4 *>(srow + at));
-            const float4 x1 = __ldg(reinterpret_cast<const float4 *>(srow + at + 4));
-            const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-            for (int e = 0; e < 8; ++e) skeys[g * 8 + e] = order_key(xs[e]);
+    if constexpr (kListed) {
+        // the bound and the list W' come from refine_bound_kernel and refine_list_kernel
+        const float2 b = bound[rl];
+        theta_s = b.x;
+        if (tid == 0) {
+            e_row = b.y;
+            wcount = __ldcg(count + rl);
         }
         __syncthreads();
-        const float mu = (float)need_total * (float)ns / (float)n;
-        int r_lo = (int)ceilf(mu + 4.f * sqrtf(mu) + 8.f);
-        if (r_lo > ns) r_lo = ns;
-        // keys relative to the sample's smallest: the radix starts at their highest differing bit
-        uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-        for (int q = tid; q < ns; q += kRefThreads) {
-            kmin = min(kmin, skeys[q]);
-            kmax = max(kmax, skeys[q]);
+        const int cnt = wcount;
+        if (cnt <= kRefCap)
+            for (int c = tid; c < cnt; c += kRefThreads) cand[c] = __ldcg(lists + rl * kRefCap + c);
+    } else {
+        const float *srow = approx + rl * ld;
+        // the error bound E of the row
+        if (warp == 0) {
+            const float e = row_error_bound(q_idx + i * 512, w + i * 4, lane);
+            if (lane == 0) {
+                e_row = e;
+                wcount = 0;
+            }
         }
-        kmin = ~kmin;
-        block_max2<kRefThreads>(kmin, kmax, &sc);
-        kmin = ~kmin;
-        const uint32_t span = kmax - kmin;
-        uint32_t sp, sm;
-        int sn, sb;
-        radix_select<kRefThreads, 8>(
-            [&](auto f) {
-                for (int q = tid; q < ns; q += kRefThreads) f(skeys[q] - kmin);
-            },
-            ns, r_lo, span != 0u ? 31 - __clz(span) : 0, regA, &sc, &sp, &sm, &sn, &sb, kBoundPasses);
-        theta_s = key_value(sp + kmin);  // the sample's r_lo-th largest, or its bin's floor
-    }
-    __syncthreads();
-    // 2. the candidates W' = {b : approx_b >= theta_s - 2E} (with their approximate keys)
-    const float lo_bound = theta_s - 2.f * e_row;
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    {
+        // 1. a lower bound theta_s of tau, the (k-1)-th largest approximate score, from a
+        //    sample; every block when the row fits the list
+        if (n > kRefCap) theta_s = sample_bound(srow, n, need_total, reinterpret_cast<uint32_t *>(cand), regA, sc);
+        __syncthreads();
+        // 2. the candidates W' = {b : approx_b >= theta_s - 2E} (with their approximate keys)
+        const float lo_bound = theta_s - 2.f * e_row;
         // rows are 16-byte aligned with ld a multiple of 4: float4 groups, kRefUnroll of
         // them in flight per thread; keys past n (inside the last group) are masked
         constexpr int kRefUnroll = 4;
@@ -1163,10 +1303,17 @@ cudaError_t launch_index_select(const IndexArgs &a, int k, void *ws, int grid, i
     return cudaGetLastError();
 }
 
+// Below this many rows the candidate lists are built by their own launches (most SMs
+// would otherwise idle while one CTA per row scans its row).
+constexpr int64_t kListedRows = 32;
+
 size_t decode_select_workspace_bytes(int64_t rows, int64_t ld, int grid)
 {
     auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    return al((size_t)rows * ld * 4) + al((size_t)(rows + 1) * 4) + al((size_t)grid * ld * 4);
+    // approximate scores, fallback rows, fallback scratch, then the listed path's bounds,
+    // list counters and lists
+    return al((size_t)rows * ld * 4) + al((size_t)(rows + 1) * 4) + al((size_t)grid * ld * 4) +
+           al((size_t)rows * 8) + al((size_t)rows * 4) + al((size_t)rows * kRefCap * 8);
 }
 
 cudaError_t launch_decode_index_select(const IndexArgs &a, int k, void *ws, int grid, bool refine, int32_t *sel,
@@ -1176,10 +1323,19 @@ cudaError_t launch_decode_index_select(const IndexArgs &a, int k, void *ws, int 
     if (rows <= 0) return cudaSuccess;
     auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
     uint8_t *base = static_cast<uint8_t *>(ws);
+    size_t off = 0;
     float *scores = reinterpret_cast<float *>(base);
-    int32_t *fb_count = reinterpret_cast<int32_t *>(base + al((size_t)rows * a.ld * 4));
+    off += al((size_t)rows * a.ld * 4);
+    int32_t *fb_count = reinterpret_cast<int32_t *>(base + off);
     int32_t *fb_rows = fb_count + 1;
-    float *scratch = reinterpret_cast<float *>(base + al((size_t)rows * a.ld * 4) + al((size_t)(rows + 1) * 4));
+    off += al((size_t)(rows + 1) * 4);
+    float *scratch = reinterpret_cast<float *>(base + off);
+    off += al((size_t)grid * a.ld * 4);
+    float2 *bound = reinterpret_cast<float2 *>(base + off);
+    off += al((size_t)rows * 8);
+    int32_t *count = reinterpret_cast<int32_t *>(base + off);
+    off += al((size_t)rows * 4);
+    uint2 *lists = reinterpret_cast<uint2 *>(base + off);
     IndexArgs a2 = a;
     a2.scores = scores;
     cudaError_t e;
@@ -1191,12 +1347,28 @@ cudaError_t launch_decode_index_select(const IndexArgs &a, int k, void *ws, int 
     }
     if ((e = launch_index_rowwise_hi(a2, stream)) != cudaSuccess) return e;
     if ((e = launch_pdl(clear_count_kernel, dim3(1), dim3(1), 0, stream, fb_count)) != cudaSuccess) return e;
-    if ((e = set_smem_attr_once(reinterpret_cast<const void *>(refine_select_kernel), kRefSmem)) != cudaSuccess)
-        return e;
     if (rows > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    if ((e = launch_pdl(refine_select_kernel, dim3((unsigned)rows), dim3(kRefThreads), kRefSmem, stream,
-                        (const float *)scores, a.ld, a.q_idx, a.w, a.kc, a.cu_q, a.cu_k, a.cu_blocks, a.batch,
-                        a.row_begin, k, a.r, sel, fb_count, fb_rows, next_n)) != cudaSuccess)
+    const bool listed = rows < kListedRows;
+    if (listed) {
+        if ((e = set_smem_attr_once(reinterpret_cast<const void *>(refine_bound_kernel), kBoundSmem)) != cudaSuccess)
+            return e;
+        if ((e = launch_pdl(refine_bound_kernel, dim3((unsigned)rows), dim3(kRefThreads), kBoundSmem, stream,
+                            (const float *)scores, a.ld, a.q_idx, a.w, a.cu_q, a.cu_k, a.batch, a.row_begin, k, a.r,
+                            next_n, bound, count)) != cudaSuccess)
+            return e;
+        const int64_t chunks = (a.ld + kListChunk - 1) / kListChunk;
+        if (chunks > 0x7FFFFFFF || rows > 65535) return cudaErrorInvalidValue;
+        if ((e = launch_pdl(refine_list_kernel, dim3((unsigned)chunks, (unsigned)rows), dim3(kListThreads), 0, stream,
+                            (const float *)scores, a.ld, a.cu_q, a.cu_k, a.batch, a.row_begin, k, a.r, next_n,
+                            (const float2 *)bound, lists, count)) != cudaSuccess)
+            return e;
+    }
+    auto kern = listed ? refine_select_kernel<true> : refine_select_kernel<false>;
+    if ((e = set_smem_attr_once(reinterpret_cast<const void *>(kern), kRefSmem)) != cudaSuccess) return e;
+    if ((e = launch_pdl(kern, dim3((unsigned)rows), dim3(kRefThreads), kRefSmem, stream, (const float *)scores, a.ld,
+                        a.q_idx, a.w, a.kc, a.cu_q, a.cu_k, a.cu_blocks, a.batch, a.row_begin, k, a.r, sel, fb_count,
+                        fb_rows, next_n, (const float2 *)bound, (const uint2 *)lists, (const int32_t *)count)) !=
+        cudaSuccess)
         return e;
     return launch_pdl(fallback_kernel, dim3((unsigned)grid), dim3(kFbThreads), sel_smem_bytes<kFbThreads>(), stream,
                       a.q_idx, a.w, a.kc, a.cu_q, a.cu_k, a.cu_blocks, a.batch, a.row_begin, k, a.r,
