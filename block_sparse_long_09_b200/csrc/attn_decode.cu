@@ -557,10 +557,39 @@ even_combine_kernel(const float *__restrict__ ws, int grid, int64_t row_begin, i
         const bool mine = is_piece(c);
         const float lc = mine ? lbase[c * kHQ + h] : -INFINITY;
         uint32_t m = __ballot_sync(0xffffffffu, mine);
-        while (m != 0u) {  // in share order
-            const int src = __ffs(m) - 1;
-            m &= m - 1u;
-            add(cb + src, __shfl_sync(0xffffffffu, lc, src));
+        // in share order, the partial outputs of up to four pieces loaded before they are
+        // added (a small batch cuts a row into tens of pieces): the sums keep their order
+        while (m != 0u) {
+            constexpr int kAhead = 4;
+            int src[kAhead];
+            int cnt = 0;
+#pragma unroll
+            for (int j = 0; j < kAhead; ++j) {
+                src[j] = m != 0u ? __ffs(m) - 1 : 0;
+                if (m != 0u) {
+                    m &= m - 1u;
+                    ++cnt;
+                }
+            }
+            float o[kAhead][kD / 32];
+#pragma unroll
+            for (int j = 0; j < kAhead; ++j) {
+                if (j < cnt) {
+                    const float *p = ws + ((cb + src[j]) * kHQ + h) * kD + lane;
+#pragma unroll
+                    for (int i = 0; i < kD / 32; ++i) o[j][i] = __ldcs(p + i * 32);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kAhead; ++j) {
+                const float l = __shfl_sync(0xffffffffu, lc, src[j]);
+                if (j < cnt) {
+                    const float wgt = (l == -INFINITY) ? 0.f : __expf(l - mx);
+                    tot += wgt;
+#pragma unroll
+                    for (int i = 0; i < kD / 32; ++i) acc[i] += wgt * o[j][i];
+                }
+            }
         }
     }
     const float inv = tot > 0.f ? 1.f / tot : 0.f;
