@@ -480,6 +480,7 @@ mtp_combine_kernel(const float *__restrict__ ws, int64_t n_items, int nsplit, in
     float tot = 0.f, acc[kD / 32];
 #pragma unroll
     for (int i = 0; i < kD / 32; ++i) acc[i] = 0.f;
+#pragma unroll 4
     for (int sp = 0; sp < nsplit; ++sp) {  // the splits in order
         const float w = __shfl_sync(0xffffffffu, wgt, sp);
         tot += w;
