@@ -660,7 +660,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="qsa", choices=["qsa", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--e2e-rows", type=int, default=16384, help="query rows per copy chunk of the e2e leg (q, k, v in, o out)")
+    ap.add_argument("--e2e-rows", type=int, default=8192, help="query rows per copy chunk of the e2e leg (q, k, v in, o out)")
     ap.add_argument("--chunk-rows", type=int, default=CHUNK,
                     help="query rows per fused index -> select launch of the prefill")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -534,7 +534,7 @@ class Prefill:
         self.index_select(q_idx, w, k_idx)
         return self.attend(q, k, v, o=o, lse=lse)
 
-    def from_host(self, q, k, v, q_idx, w, k_idx, o, lse=None, pipe_rows: int = 16384):
+    def from_host(self, q, k, v, q_idx, w, k_idx, o, lse=None, pipe_rows: int = 8192):
         """The whole prefill from host memory, copies overlapped with the compute.
 
         q, k, v, q_idx, w, k_idx are host tensors and o (and lse) host outputs, all
