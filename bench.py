@@ -552,6 +552,61 @@ def run_extra_configs(steps: int = 5, warmup: int = 3):
         del d, kc, dec
         torch.cuda.empty_cache()
     run_context_1m(timed, cfg, dev)
+    run_sharded_emulation(cfg, dev)
+
+
+def run_sharded_emulation(cfg, dev, worlds=(2, 4, 8), reps=3):
+    """The row-sharded prefill of 262144 tokens (block_sparse_long_09_b200.sharded) with
+    its N ranks emulated one after another on this GPU: each rank's fused index -> select
+    and attention over its own rows against the gathered prefix, timed alone (no rank
+    waits for another).  The slowest rank bounds an N-GPU step; the all-gathers of the
+    compressed keys and K/V rows are not run here and are estimated at the measured
+    770 GB/s peer bandwidth per direction (each rank receives the others' rows)."""
+    from block_sparse_long_09_b200 import inputs, qsa
+    from block_sparse_long_09_b200.sharded import ShardedPrefill, row_partition
+
+    n = N_PREFILL
+    x = inputs.make_prefill([n], seed=0, device=dev)
+    one = qsa.Prefill([n], chunk_rows=CHUNK, cfg=cfg, device=dev)
+    o = torch.empty_like(x.q)
+
+    def ev_time(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    one_ms = ev_time(lambda: one(x.q, x.k, x.v, x.q_idx, x.w, x.k_idx, o=o))
+    kv_row_bytes = 2 * (2 * 256 * 2) + (2 * 128 * 2) // 4  # a token's K and V rows, a quarter of a compressed key
+    for world in worlds:
+        parts = row_partition(n, world)
+        shards = [ShardedPrefill(n, j, world, chunk_rows=CHUNK, cfg=cfg, parts=parts, device=dev)
+                  for j in range(world)]
+        kc_all = torch.cat([sh.local_blocks(x.k_idx[a:b].contiguous()) for sh, (a, b) in zip(shards, parts)])
+        rank_ms = []
+        for sh, (a, b) in zip(shards, parts):
+            qa, qia, wa = x.q[a:b].contiguous(), x.q_idx[a:b].contiguous(), x.w[a:b].contiguous()
+            oa = torch.empty_like(qa)
+            rank_ms.append(ev_time(lambda: sh.attend(qa, qia, wa, kc_all, x.k, x.v, o=oa)))
+            del qa, qia, wa, oa
+        gather_ms = max((n - (b - a)) * kv_row_bytes for a, b in parts) / 770e9 * 1e3
+        assert qsa.device_status() == 0
+        print(json.dumps({"workload": "row-sharded prefill of %d tokens, %d ranks emulated on one GPU" % (n, world),
+                          "rows_per_rank": [b - a for a, b in parts], "rank_ms": rank_ms,
+                          "slowest_rank_ms": max(rank_ms), "balance": min(rank_ms) / max(rank_ms),
+                          "one_gpu_ms": one_ms, "gather_ms_estimated": gather_ms,
+                          "projected_speedup": one_ms / (max(rank_ms) + gather_ms),
+                          "note": "ranks timed one after another; the all-gathers estimated, not run"}),
+              file=sys.stderr)
+        del shards, kc_all
+        torch.cuda.empty_cache()
+    del x, one, o
+    torch.cuda.empty_cache()
 
 
 def run_context_1m(timed, cfg, dev):
@@ -667,8 +722,11 @@ def main():
     ap.add_argument("--no-dense", dest="dense", action="store_false",
                     help="skip the dense causal-attention comparison")
     ap.add_argument("--extra-configs", action="store_true",
-                    help="also time the other workloads (peaked 2 x 65536 prefill, decode at 262144 and mixed "
-                         "lengths) and print them on stderr")
+                    help="time the other workloads instead (peaked 2 x 65536 prefill, decode at 262144 and mixed "
+                         "lengths, the 1M-token comparison, the sharded-prefill emulation) and print them on stderr")
+    ap.add_argument("--sharded-emulation", action="store_true",
+                    help="time the row-sharded prefill's ranks one after another on this GPU (also part of "
+                         "--extra-configs) and print one line per rank count on stderr")
     ap.add_argument("--profile-case", choices=["attn", "index", "select", "index_select", "decode", "decode64k", "decode131k", "mtp"],
                     default=None,
                     help="run one small case for an ncu capture and exit")
@@ -682,6 +740,13 @@ def main():
         import block_sparse_long_09_b200.build as bld
         bld.build()
         run_extra_configs(args.steps, args.warmup)
+        return
+    if args.sharded_emulation:
+        import block_sparse_long_09_b200.build as bld
+        from block_sparse_long_09_b200 import qsa
+        bld.build()
+        torch.cuda.set_device(0)
+        run_sharded_emulation(qsa.default_config(budget_blocks=BUDGET), torch.device("cuda", 0))
         return
 
     from block_sparse_long_09_b200 import ranks

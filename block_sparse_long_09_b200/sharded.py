@@ -14,9 +14,10 @@ previous layer leaves them), and
      prefill with L_q = r1_j - r0_j queries against L_k = r1_j keys (the C ABI's
      bottom-right alignment puts query i of the shard at t = r0_j + i).
 
-Rows cost unequal work: the attention is about constant per row (2048 tokens),
-the indexer grows with the number of earlier blocks.  row_partition balances a
-cost a + b * floor(t / r) per row, so later ranks get fewer rows.
+Rows cost unequal work: the attention gathers 2048 tokens per row (from a prefix,
+and so an L2 hit rate, that depends on the row), the indexer grows with the number
+of earlier blocks.  row_partition balances a cost a + b * floor(t / r) per row, so
+later ranks get fewer rows.
 
 The arithmetic of a row does not depend on which shard holds it, so the sharded
 result equals the one-process result bit for bit.
@@ -29,11 +30,12 @@ import torch
 
 ATTN_ROWS = 4096  # query rows per attention launch
 
-# relative cost of a row: attention (about constant) and indexer pairs (per earlier block),
-# from the measured B200 times of the 262144-token prefill (about 0.43 us of attention per
-# row and 1.2 ps per (row, block) pair of the fused indexer)
-ATTN_ROW_COST = 0.43e-6
-INDEX_PAIR_COST = 1.2e-12
+# relative cost of a row: a constant part and a part per earlier block, fitted to the
+# per-rank times of a 262144-token prefill sharded over 2 ranks on one B200 (0.38 us per
+# row and 4.5 ps per (row, block) pair; the second term holds the fused indexer's pairs
+# and the attention's falling L2 hit rate, its prefix of K/V growing with the row)
+ATTN_ROW_COST = 0.38e-6
+INDEX_PAIR_COST = 4.5e-12
 
 
 def row_partition(n: int, world: int, r: int = 4, attn_cost: float = ATTN_ROW_COST,
