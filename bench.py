@@ -691,6 +691,17 @@ def run_profile_case(case: str, reps: int = 3):
         for _ in range(reps):
             sel = qsa.index_select_mtp(d.q_idx, d.w, kc, d.cu_seqlens_k, d.cu_blocks, MTP_NEXT_N, L, cfg=cfg)
             qsa.sparse_attn_decode_mtp(d.q, d.k_cache, d.v_cache, d.cu_seqlens_k, sel, cfg=cfg)
+    elif case == "decode1m":
+        # decode steps at batch 4 with 1048576-token caches (the pages' decode regime): the
+        # small-batch selection path (bound and list launches before the refine); 10 GB
+        L, B = 1 << 20, 4
+        d = inputs.make_decode(B, L, None, seed=1, device=dev)
+        cu_q = torch.arange(B + 1, dtype=torch.int32, device=dev)
+        kc = qsa.compress_keys(d.k_idx, d.cu_seqlens_k, d.cu_blocks, n_blocks=int(d.cu_blocks[-1]), cfg=cfg)
+        ws = torch.empty((qsa.workspace_size(qsa.OP_INDEX_SELECT, B, B, L, cfg),), dtype=torch.uint8, device=dev)
+        for _ in range(reps):
+            sel = qsa.index_select(d.q_idx, d.w, kc, cu_q, d.cu_seqlens_k, d.cu_blocks, 1, L, ws=ws, cfg=cfg)
+            qsa.sparse_attn_decode(d.q, d.k_cache, d.v_cache, d.cu_seqlens_k, sel, cfg=cfg)
     elif case in ("decode", "decode64k", "decode131k"):
         # decode steps of batch 64 (16384-token caches: small; 65536: kc hi planes of 268 MB,
         # above L2, 5.5 GB on the device; 131072: the benchmark's, 11 GB)
@@ -727,7 +738,8 @@ def main():
     ap.add_argument("--sharded-emulation", action="store_true",
                     help="time the row-sharded prefill's ranks one after another on this GPU (also part of "
                          "--extra-configs) and print one line per rank count on stderr")
-    ap.add_argument("--profile-case", choices=["attn", "index", "select", "index_select", "decode", "decode64k", "decode131k", "mtp"],
+    ap.add_argument("--profile-case", choices=["attn", "index", "select", "index_select", "decode", "decode64k", "decode131k", "decode1m",
+                             "mtp"],
                     default=None,
                     help="run one small case for an ncu capture and exit")
     args = ap.parse_args()
