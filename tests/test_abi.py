@@ -177,3 +177,21 @@ def test_prefill_copy_plan_covers_every_row_once_and_in_time(qsa, total, sel_row
         assert kv_hi >= min(total, r1 - 1 + r)          # the micro-block holding row r1 - 1, loaded whole
     with pytest.raises(ValueError):
         qsa.prefill_copy_plan(10, 0, 4)
+
+
+def test_binding_constants_match_the_header(qsa):
+    """Every status code, flag and workspace op the binding hard-codes equals the value
+    include/qsa.h defines (the binding passes them to the library as plain integers)."""
+    text = open(os.path.join(ROOT, "include", "qsa.h")).read()
+    defs = {}
+    for name, value in re.findall(r"#define\s+(QSA_[A-Z_]+)\s+\(?([0-9x]+)u?", text):
+        defs[name] = int(value, 0)
+    assert defs["QSA_STATIC_SCRATCH_BYTES"] == 16  # "(16u * 1024u * 1024u)": the first factor
+    assert qsa.STATIC_SCRATCH_BYTES == 16 * 1024 * 1024
+    for name in ("QSA_OK", "QSA_ERR_INVALID_ARG", "QSA_ERR_UNSUPPORTED", "QSA_ERR_WORKSPACE_TOO_SMALL",
+                 "QSA_ERR_CUDA", "QSA_ERR_TIMEOUT", "QSA_ERR_DEVICE_CHECK", "QSA_ERR_SCRATCH_LIMIT",
+                 "QSA_COMPRESS_NO_NORM", "QSA_INDEX_ROPE"):
+        assert getattr(qsa, name) == defs[name], name
+    for name in ("COMPRESS", "INDEX", "SELECT", "PREFILL", "DECODE", "DENSE", "DECODE_PAGED", "INDEX_SELECT",
+                 "INDEX_SELECT_PAGED", "DECODE_MTP"):
+        assert getattr(qsa, "OP_" + name) == defs["QSA_OP_" + name], name
